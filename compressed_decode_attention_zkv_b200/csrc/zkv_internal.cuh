@@ -1,0 +1,145 @@
+// Internal helpers shared by the libzkv kernels (sm_100a).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "zkv.h"
+
+namespace zkv {
+
+constexpr int kCodebook = ZKV_CODEBOOK_SIZE;   // 256 codewords per stage
+constexpr int kMaxStages = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+inline bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
+
+#define ZKV_CHECK_LAUNCH()                                   \
+  do {                                                       \
+    if (cudaGetLastError() != cudaSuccess) return ZKV_ERR_CUDA; \
+  } while (0)
+
+// ------------------------------------------------------------------------------------------
+// Walsh-Hadamard transform of one vector held by a warp, float64.
+// Lane l holds elements j*32 + l for j < E = D/32 (strided: coalesced loads, conflict-free
+// shared-memory stores).  Butterfly pairs (i, i+h) map to (x_i + x_{i+h}, x_i - x_{i+h}) for
+// every h = 1, 2, ..., D/2 (Sylvester order): h < 32 pairs lanes l and l^h, h >= 32 pairs the
+// lane's own registers j and j ^ (h/32).  For fp16 inputs every partial sum is exact in float64,
+// so the result does not depend on the order in which the levels are applied.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void fwht_warp_f64(double (&v)[D / 32], int lane) {
+  constexpr int E = D / 32;
+#pragma unroll
+  for (int lm = 1; lm < 32; lm <<= 1) {
+    const bool upper = (lane & lm) != 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const double o = __shfl_xor_sync(0xffffffffu, v[j], lm);
+      v[j] = upper ? (o - v[j]) : (v[j] + o);
+    }
+  }
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      if ((j & h) == 0) {
+        const double a = v[j], b = v[j + h];
+        v[j] = a + b;
+        v[j + h] = a - b;
+      }
+    }
+  }
+}
+
+// Load the E strided elements (j*32 + lane) of a row (fp16 or fp32) as doubles.
+template <int E>
+__device__ __forceinline__ void load_row_f64(const void* base, int dtype, int64_t off, int lane,
+                                             double (&v)[E]) {
+  if (dtype == ZKV_DTYPE_F16) {
+    const __half* p = reinterpret_cast<const __half*>(base) + off + lane;
+#pragma unroll
+    for (int j = 0; j < E; ++j) v[j] = (double)__half2float(p[j * 32]);
+  } else {
+    const float* p = reinterpret_cast<const float*>(base) + off + lane;
+#pragma unroll
+    for (int j = 0; j < E; ++j) v[j] = (double)p[j * 32];
+  }
+}
+
+__device__ __forceinline__ double warp_sum_f64(double x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_sum_f32(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_max_f32(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+__device__ __forceinline__ float warp_min_f32(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// 2^x via the PTX approximate base-2 exponential (relative error about 2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void set_error(int32_t* flag, int bits) {
+  if (flag) atomicOr(flag, bits);
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device); later calls are
+// plain launches (so they can be captured into CUDA graphs).  Keyed by the kernel's address:
+// every template instantiation has its own entry.
+inline cudaError_t ensure_smem_limit_raw(const void* kernel, size_t bytes) {
+  struct Entry { const void* fn; int dev; size_t bytes; };
+  static std::mutex mu;
+  static Entry table[512];
+  static int n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  int slot = -1;
+  for (int i = 0; i < n; ++i)
+    if (table[i].fn == kernel && table[i].dev == dev) { slot = i; break; }
+  if (slot >= 0 && table[slot].bytes >= bytes) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (slot < 0) {
+    if (n == 512) return cudaSuccess;   // table full: the attribute is set, just not cached
+    slot = n++;
+    table[slot].fn = kernel;
+    table[slot].dev = dev;
+  }
+  table[slot].bytes = bytes;
+  return cudaSuccess;
+}
+
+template <class F>
+inline cudaError_t ensure_smem_limit(F* kernel, size_t bytes) {
+  return ensure_smem_limit_raw(reinterpret_cast<const void*>(kernel), bytes);
+}
+
+// Round-up helpers for workspace carving.
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace zkv

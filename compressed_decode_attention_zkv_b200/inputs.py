@@ -177,6 +177,23 @@ def kv_tokens(wl: Workload, kind: str, b: int, t0: int, t1: int,
     return out.astype(np.float16)
 
 
+def window_tokens(wl: Workload, kind: str, lengths: np.ndarray,
+                  seed: int = SEED_DATA) -> np.ndarray:
+    """The W newest tokens of every sequence, fp16 [B][Hkv][W][d], drawn from a stream of
+    their own (cheap for long contexts); keys get RoPE at positions len-W .. len-1."""
+    tag = 41 if kind == "k" else 42
+    out = np.empty((wl.B, wl.Hkv, wl.W, wl.d), np.float16)
+    scales = channel_scales(wl, kind, seed)
+    for b in range(wl.B):
+        z = _rng(seed, tag, b).standard_normal((wl.Hkv, wl.W, wl.d), dtype=np.float32)
+        z *= scales[:, None, :]
+        if kind == "k" and wl.rope_theta is not None:
+            pos = np.arange(int(lengths[b]) - wl.W, int(lengths[b]))
+            z = apply_rope(z, pos, wl.rope_theta)
+        out[b] = z.astype(np.float16)
+    return out
+
+
 def queries(wl: Workload, seed: int = SEED_DATA, step: int = 0) -> np.ndarray:
     """Decode queries, fp16 N(0, 1), [B][Hq][d]."""
     z = _rng(seed, _TAG_Q, step).standard_normal((wl.B, wl.Hq, wl.d), dtype=np.float32)

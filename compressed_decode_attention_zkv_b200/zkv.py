@@ -1,0 +1,390 @@
+"""Thin ctypes binding of libzkv (include/zkv.h): argument marshalling only.
+
+Every computation runs in the library's CUDA kernels; PyTorch supplies device memory and the
+current CUDA stream.  If the library is missing or a call fails, an exception is raised -- there
+is no fallback path.
+
+Entry points (same names as the C ABI):
+  fwht, rvq_encode, rvq_reconstruct, decode_workspace_size, rvq_decode_attn, rvq_append
+plus ``RVQKVCache``, a small owner of one layer's compressed cache built on them
+(prefill -> append -> attend, the append/attend cache interface of the VeloxQuant-MLX page).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from ctypes import POINTER, c_float, c_int, c_int64, c_size_t, c_void_p
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libzkv.so")
+
+ZKV_OK, ZKV_ERR_INVALID_ARG, ZKV_ERR_UNSUPPORTED, ZKV_ERR_WORKSPACE, ZKV_ERR_CUDA = range(5)
+ZKV_DEVERR_COMP_LEN = 1
+ZKV_DEVERR_WIN_LEN = 2
+ZKV_DTYPE_F16, ZKV_DTYPE_F32 = 0, 1
+CODEBOOK_SIZE = 256
+
+
+class ZkvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+class EncodeParams(ctypes.Structure):
+    _fields_ = [("n_batch", c_int64), ("n_tok", c_int64), ("n_head", c_int64),
+                ("d", c_int), ("S", c_int), ("rotate", c_int), ("x_dtype", c_int),
+                ("x", c_void_p), ("x_sb", c_int64), ("x_st", c_int64), ("x_sh", c_int64),
+                ("codebooks", c_void_p),
+                ("codes", c_void_p), ("c_sb", c_int64), ("c_st", c_int64), ("c_sh", c_int64),
+                ("norms", c_void_p), ("n_sb", c_int64), ("n_st", c_int64), ("n_sh", c_int64)]
+
+
+class ReconstructParams(ctypes.Structure):
+    _fields_ = [("n_batch", c_int64), ("n_tok", c_int64), ("n_head", c_int64),
+                ("d", c_int), ("S", c_int), ("unrotate", c_int),
+                ("codes", c_void_p), ("c_sb", c_int64), ("c_st", c_int64), ("c_sh", c_int64),
+                ("codebooks", c_void_p),
+                ("out", c_void_p), ("o_sb", c_int64), ("o_st", c_int64), ("o_sh", c_int64)]
+
+
+class DecodeParams(ctypes.Structure):
+    _fields_ = [("B", c_int), ("Hq", c_int), ("Hkv", c_int), ("d", c_int), ("Sk", c_int),
+                ("Sv", c_int), ("Tcap", c_int64), ("Wcap", c_int64), ("max_comp_len", c_int64),
+                ("softmax_scale", c_float),
+                ("q", c_void_p), ("k_codes", c_void_p), ("v_codes", c_void_p),
+                ("comp_len", c_void_p), ("k_codebooks", c_void_p), ("v_codebooks", c_void_p),
+                ("win_k", c_void_p), ("win_v", c_void_p), ("win_len", c_void_p),
+                ("out", c_void_p), ("lse", c_void_p), ("error_flag", c_void_p),
+                ("trace_events", c_void_p)]
+
+
+class AppendParams(ctypes.Structure):
+    _fields_ = [("B", c_int), ("Hkv", c_int), ("d", c_int), ("Sk", c_int), ("Sv", c_int),
+                ("Tcap", c_int64), ("Wcap", c_int64),
+                ("new_k", c_void_p), ("new_v", c_void_p), ("win_k", c_void_p),
+                ("win_v", c_void_p), ("win_len", c_void_p), ("win_head", c_void_p),
+                ("comp_len", c_void_p), ("k_codes", c_void_p), ("v_codes", c_void_p),
+                ("k_codebooks", c_void_p), ("v_codebooks", c_void_p), ("error_flag", c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libzkv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libzkv.so not found at {LIB_PATH}; build it with "
+                              "`python -m compressed_decode_attention_zkv_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.zkv_status_string.restype = ctypes.c_char_p
+        L.zkv_status_string.argtypes = [c_int]
+        L.zkv_version.restype = c_int
+        L.zkv_fwht.restype = c_int
+        L.zkv_fwht.argtypes = [c_void_p, c_int, c_void_p, c_int64, c_int, c_float, c_void_p]
+        L.zkv_rvq_encode.restype = c_int
+        L.zkv_rvq_encode.argtypes = [POINTER(EncodeParams), c_void_p]
+        L.zkv_rvq_reconstruct.restype = c_int
+        L.zkv_rvq_reconstruct.argtypes = [POINTER(ReconstructParams), c_void_p]
+        L.zkv_decode_workspace_size.restype = c_size_t
+        L.zkv_decode_workspace_size.argtypes = [POINTER(DecodeParams)]
+        L.zkv_rvq_decode_attn.restype = c_int
+        L.zkv_rvq_decode_attn.argtypes = [POINTER(DecodeParams), c_void_p, c_size_t, c_void_p]
+        L.zkv_rvq_append.restype = c_int
+        L.zkv_rvq_append.argtypes = [POINTER(AppendParams), c_void_p]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().zkv_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != ZKV_OK:
+        raise ZkvError(fn, status)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype, contiguous=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# --------------------------------------------------------------------------------------------
+# Entry points
+# --------------------------------------------------------------------------------------------
+
+def fwht(x: torch.Tensor, scale: float, out: torch.Tensor | None = None) -> torch.Tensor:
+    """out = float32(scale * H_d x) for every row of x ([..., d], fp16 or fp32)."""
+    if x.dtype not in (torch.float16, torch.float32):
+        raise TypeError("x must be fp16 or fp32")
+    _need(x, "x", x.dtype)
+    d = x.shape[-1]
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32)
+    dt = ZKV_DTYPE_F16 if x.dtype == torch.float16 else ZKV_DTYPE_F32
+    _check("zkv_fwht", lib().zkv_fwht(_ptr(x), dt, _ptr(out), x.numel() // d, d,
+                                      float(scale), _stream()))
+    return out
+
+
+def _as4(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dim() == 2:
+        return t[None, :, None, :]
+    if t.dim() == 3:
+        return t[None]
+    if t.dim() == 4:
+        return t
+    raise ValueError(f"{name} must be [N, X], [T, H, X] or [B, T, H, X]")
+
+
+def rvq_encode(x: torch.Tensor, codebooks: torch.Tensor, codes: torch.Tensor | None = None,
+               norms: torch.Tensor | None = None, rotate: bool = True,
+               with_norms: bool = True):
+    """Greedy RVQ of x rows.  x: [B, T, H, d] view (any strides, d contiguous), or [T, H, d],
+    or [N, d] (one head).  codebooks: [H, S, 256, d] float32 contiguous.
+    Returns (codes uint8 [B, T, H, S] view, norms float32 [B, T, H, S] or None)."""
+    if x.dtype not in (torch.float16, torch.float32):
+        raise TypeError("x must be fp16 or fp32")
+    _need(x, "x", x.dtype, contiguous=False)
+    _need(codebooks, "codebooks", torch.float32)
+    x4 = _as4(x, "x")
+    if x4.stride(-1) != 1:
+        raise ValueError("x rows must be contiguous")
+    Bn, T, H, d = x4.shape
+    S = codebooks.shape[1]
+    if codebooks.shape != (H, S, CODEBOOK_SIZE, d):
+        raise ValueError(f"codebooks must be [H={H}, S, 256, d={d}], got {tuple(codebooks.shape)}")
+    if codes is None:
+        codes = torch.empty((Bn, T, H, S), dtype=torch.uint8, device=x.device)
+    if norms is None and with_norms:
+        norms = torch.empty((Bn, T, H, S), dtype=torch.float32, device=x.device)
+    _need(codes, "codes", torch.uint8, contiguous=False)
+    c4 = _as4(codes, "codes")
+    if c4.shape != (Bn, T, H, S) or c4.stride(-1) != 1:
+        raise ValueError("codes must be a [B, T, H, S] view with contiguous S")
+    p = EncodeParams(n_batch=Bn, n_tok=T, n_head=H, d=d, S=S, rotate=int(bool(rotate)),
+                     x_dtype=ZKV_DTYPE_F16 if x.dtype == torch.float16 else ZKV_DTYPE_F32,
+                     x=_ptr(x4), x_sb=x4.stride(0), x_st=x4.stride(1), x_sh=x4.stride(2),
+                     codebooks=_ptr(codebooks), codes=_ptr(c4), c_sb=c4.stride(0),
+                     c_st=c4.stride(1), c_sh=c4.stride(2))
+    if norms is not None:
+        _need(norms, "norms", torch.float32, contiguous=False)
+        n4 = _as4(norms, "norms")
+        if n4.shape != (Bn, T, H, S) or n4.stride(-1) != 1:
+            raise ValueError("norms must be a [B, T, H, S] view with contiguous S")
+        p.norms, p.n_sb, p.n_st, p.n_sh = _ptr(n4), n4.stride(0), n4.stride(1), n4.stride(2)
+    _check("zkv_rvq_encode", lib().zkv_rvq_encode(ctypes.byref(p), _stream()))
+    return codes, norms
+
+
+def rvq_reconstruct(codes: torch.Tensor, codebooks: torch.Tensor, unrotate: bool = False,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """x_hat = sum_s C[h][s][z_s] for codes [B, T, H, S] (views allowed); returns float32
+    [B, T, H, d] (rotated back by H/sqrt(d) when ``unrotate``)."""
+    _need(codes, "codes", torch.uint8, contiguous=False)
+    _need(codebooks, "codebooks", torch.float32)
+    c4 = _as4(codes, "codes")
+    Bn, T, H, S = c4.shape
+    d = codebooks.shape[-1]
+    if codebooks.shape != (H, S, CODEBOOK_SIZE, d):
+        raise ValueError("codebooks must be [H, S, 256, d]")
+    if out is None:
+        out = torch.empty((Bn, T, H, d), dtype=torch.float32, device=codes.device)
+    _need(out, "out", torch.float32, contiguous=False)
+    o4 = _as4(out, "out")
+    p = ReconstructParams(n_batch=Bn, n_tok=T, n_head=H, d=d, S=S, unrotate=int(bool(unrotate)),
+                          codes=_ptr(c4), c_sb=c4.stride(0), c_st=c4.stride(1), c_sh=c4.stride(2),
+                          codebooks=_ptr(codebooks), out=_ptr(o4), o_sb=o4.stride(0),
+                          o_st=o4.stride(1), o_sh=o4.stride(2))
+    _check("zkv_rvq_reconstruct", lib().zkv_rvq_reconstruct(ctypes.byref(p), _stream()))
+    return out
+
+
+def _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
+                   win_len, out, lse, max_comp_len, softmax_scale, error_flag) -> DecodeParams:
+    _need(q, "q", torch.float16)
+    _need(k_codes, "k_codes", torch.uint8)
+    _need(v_codes, "v_codes", torch.uint8)
+    _need(comp_len, "comp_len", torch.int32)
+    _need(win_len, "win_len", torch.int32)
+    _need(k_codebooks, "k_codebooks", torch.float32)
+    _need(v_codebooks, "v_codebooks", torch.float32)
+    _need(win_k, "win_k", torch.float16)
+    _need(win_v, "win_v", torch.float16)
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, Sk = k_codes.shape
+    Sv = v_codes.shape[3]
+    Wcap = win_k.shape[2]
+    if out is not None:
+        _need(out, "out", torch.float32)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+    if error_flag is not None:
+        _need(error_flag, "error_flag", torch.int32)
+    return DecodeParams(B=B, Hq=Hq, Hkv=Hkv, d=d, Sk=Sk, Sv=Sv, Tcap=Tcap, Wcap=Wcap,
+                        max_comp_len=Tcap if max_comp_len is None else int(max_comp_len),
+                        softmax_scale=0.0 if softmax_scale is None else float(softmax_scale),
+                        q=_ptr(q), k_codes=_ptr(k_codes), v_codes=_ptr(v_codes),
+                        comp_len=_ptr(comp_len), k_codebooks=_ptr(k_codebooks),
+                        v_codebooks=_ptr(v_codebooks), win_k=_ptr(win_k), win_v=_ptr(win_v),
+                        win_len=_ptr(win_len), out=_ptr(out), lse=_ptr(lse),
+                        error_flag=_ptr(error_flag))
+
+
+def decode_workspace_size(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
+                          win_v, win_len, max_comp_len=None) -> int:
+    p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
+                       win_len, None, None, max_comp_len, None, None)
+    n = lib().zkv_decode_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise ZkvError("zkv_decode_workspace_size", ZKV_ERR_INVALID_ARG)
+    return n
+
+
+def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
+                    win_len, out=None, lse=None, max_comp_len=None, softmax_scale=None,
+                    workspace: torch.Tensor | None = None, error_flag=None, trace_events=None):
+    """Decode attention over the compressed prefix plus the fp16 window (see include/zkv.h).
+    ``trace_events``: optional 4 torch.cuda.Event(enable_timing=True) recorded around the
+    library's three kernels.  Returns (out float32 [B, Hq, d], lse float32 [B, Hq])."""
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
+                       win_len, out, lse, max_comp_len, softmax_scale, error_flag)
+    ev_arr = None
+    if trace_events is not None:
+        if len(trace_events) != 4:
+            raise ValueError("trace_events needs 4 events")
+        ev_arr = (c_void_p * 4)(*[e.cuda_event for e in trace_events])
+        p.trace_events = ctypes.cast(ev_arr, c_void_p)
+    need = lib().zkv_decode_workspace_size(ctypes.byref(p))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8)
+    _check("zkv_rvq_decode_attn",
+           lib().zkv_rvq_decode_attn(ctypes.byref(p), _ptr(workspace), workspace.numel(),
+                                     _stream()))
+    return out, lse
+
+
+def rvq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
+               k_codebooks, v_codebooks, error_flag=None):
+    """One serving step of cache maintenance (see include/zkv.h); state updated in place."""
+    _need(new_k, "new_k", torch.float16)
+    _need(new_v, "new_v", torch.float16)
+    for n, t in (("win_k", win_k), ("win_v", win_v)):
+        _need(t, n, torch.float16)
+    for n, t in (("win_len", win_len), ("win_head", win_head), ("comp_len", comp_len)):
+        _need(t, n, torch.int32)
+    _need(k_codes, "k_codes", torch.uint8)
+    _need(v_codes, "v_codes", torch.uint8)
+    _need(k_codebooks, "k_codebooks", torch.float32)
+    _need(v_codebooks, "v_codebooks", torch.float32)
+    if error_flag is not None:
+        _need(error_flag, "error_flag", torch.int32)
+    B, Hkv, Tcap, Sk = k_codes.shape
+    p = AppendParams(B=B, Hkv=Hkv, d=new_k.shape[-1], Sk=Sk, Sv=v_codes.shape[3], Tcap=Tcap,
+                     Wcap=win_k.shape[2], new_k=_ptr(new_k), new_v=_ptr(new_v),
+                     win_k=_ptr(win_k), win_v=_ptr(win_v), win_len=_ptr(win_len),
+                     win_head=_ptr(win_head), comp_len=_ptr(comp_len), k_codes=_ptr(k_codes),
+                     v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
+                     v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag))
+    _check("zkv_rvq_append", lib().zkv_rvq_append(ctypes.byref(p), _stream()))
+
+
+# --------------------------------------------------------------------------------------------
+# A layer's compressed cache
+# --------------------------------------------------------------------------------------------
+
+class RVQKVCache:
+    """Compressed KV cache of one attention layer: RVQ codes for old tokens, an fp16 window for
+    the newest ones.  prefill() encodes a prompt, append() inserts one token per sequence
+    (evicting and encoding the oldest window token when the window is full), attend() runs one
+    decode step of attention.  All state lives on the GPU; lengths never leave the device."""
+
+    def __init__(self, k_codebooks: torch.Tensor, v_codebooks: torch.Tensor, batch: int,
+                 capacity: int, window: int, device="cuda"):
+        Hkv, Sk, _, d = k_codebooks.shape
+        Sv = v_codebooks.shape[1]
+        self.Ck, self.Cv = k_codebooks.contiguous(), v_codebooks.contiguous()
+        self.B, self.Hkv, self.d, self.Sk, self.Sv = batch, Hkv, d, Sk, Sv
+        self.Tcap = (capacity + 15) // 16 * 16
+        self.Wcap = window
+        dev = torch.device(device)
+        self.k_codes = torch.zeros((batch, Hkv, self.Tcap, Sk), dtype=torch.uint8, device=dev)
+        self.v_codes = torch.zeros((batch, Hkv, self.Tcap, Sv), dtype=torch.uint8, device=dev)
+        self.win_k = torch.zeros((batch, Hkv, window, d), dtype=torch.float16, device=dev)
+        self.win_v = torch.zeros((batch, Hkv, window, d), dtype=torch.float16, device=dev)
+        self.comp_len = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.win_len = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.win_head = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.error_flag = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.max_comp_len = 0      # host-side bound used to size decode launches
+        self._ws = None
+
+    def prefill(self, k: torch.Tensor, v: torch.Tensor):
+        """k, v: fp16 [B, Hkv, T, d] (same T for every sequence).  The last min(T, window)
+        tokens go to the window, the rest are encoded."""
+        T = k.shape[2]
+        W = min(T, self.Wcap)
+        Tc = T - W
+        if Tc > self.Tcap:
+            raise ValueError("prompt longer than capacity + window")
+        if Tc > 0:
+            rvq_encode(k[:, :, :Tc].permute(0, 2, 1, 3), self.Ck,
+                       codes=self.k_codes[:, :, :Tc].permute(0, 2, 1, 3), with_norms=False)
+            rvq_encode(v[:, :, :Tc].permute(0, 2, 1, 3), self.Cv,
+                       codes=self.v_codes[:, :, :Tc].permute(0, 2, 1, 3), with_norms=False)
+        self.win_k[:, :, :W].copy_(k[:, :, Tc:])
+        self.win_v[:, :, :W].copy_(v[:, :, Tc:])
+        self.comp_len.fill_(Tc)
+        self.win_len.fill_(W)
+        self.win_head.zero_()
+        self.max_comp_len = Tc
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor):
+        """k_new, v_new: fp16 [B, Hkv, d]."""
+        rvq_append(k_new.contiguous(), v_new.contiguous(), self.win_k, self.win_v, self.win_len,
+                   self.win_head, self.comp_len, self.k_codes, self.v_codes, self.Ck, self.Cv,
+                   self.error_flag)
+        self.max_comp_len = min(self.max_comp_len + 1, self.Tcap)
+
+    def attend(self, q: torch.Tensor, softmax_scale=None, out=None, lse=None):
+        """q: fp16 [B, Hq, d] -> (out float32 [B, Hq, d], lse float32 [B, Hq])."""
+        args = (q, self.k_codes, self.v_codes, self.comp_len, self.Ck, self.Cv, self.win_k,
+                self.win_v, self.win_len)
+        need = decode_workspace_size(*args, max_comp_len=self.max_comp_len)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        return rvq_decode_attn(*args, out=out, lse=lse, max_comp_len=self.max_comp_len,
+                               softmax_scale=softmax_scale, workspace=self._ws,
+                               error_flag=self.error_flag)
+
+    def memory_bytes(self) -> int:
+        """Bytes held by codes and window (codebooks are shared across layers' caches)."""
+        return sum(t.numel() * t.element_size() for t in
+                   (self.k_codes, self.v_codes, self.win_k, self.win_v))

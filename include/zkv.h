@@ -1,0 +1,236 @@
+/*
+ * zkv.h -- C ABI of libzkv: RVQ KV-cache encode and compressed decode attention on B200.
+ *
+ * The method (web pages this library follows):
+ *   - "VQKV: High-Fidelity and High-Ratio Cache Compression via Vector-Quantization"
+ *     (gist.science summary of arXiv 2603.16435), section 2.1 "Residual Simple Vector
+ *     Quantization": greedy residual stages and reconstruction x_hat = sum_s Q_s[z_s];
+ *     section 2.3 "Inference Integration": codes stored at prefill, on-demand reconstruction
+ *     inside attention at decode, a local window of recent tokens kept uncompressed.
+ *   - "zerokv-neo 4.0.0", "Architecture": FWHT energy spreading before quantisation.
+ *   - "VeloxQuant-MLX 0.5.1", "VecInfer": Walsh-Hadamard rotation absorbed into the query.
+ *   - "Differential-KV", "Decode & Prefill Innovations": flash-style fp32 log-sum-exp combine
+ *     of the compressed part with a dense recency window.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates
+ *     nothing and keeps no state between calls.  fp16 tensors are passed as uint16_t bit
+ *     patterns (IEEE binary16).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream).  Argument validation is synchronous and happens before any launch; a
+ *     failed validation returns an error and launches nothing.  A launch failure returns
+ *     ZKV_ERR_CUDA.  No C++ exception crosses this boundary.
+ *   - Codebooks hold K = 256 float32 codewords per stage in the ROTATED domain
+ *     (y = H_d x / sqrt(d), Sylvester-ordered Hadamard), layout [n_head][S][256][d].  Codeword
+ *     0 of every stage should be the zero vector (then residual norms never increase).
+ *   - Head dimension d must be 64, 128 or 256; stage counts 1..8.
+ *   - GQA: query head h reads kv head h / (Hq / Hkv).
+ *   - Device-side conditions that cannot be checked on the host (a length beyond capacity)
+ *     are reported by OR-ing ZKV_DEVERR_* bits into an optional caller-owned device word
+ *     (`error_flag`, may be NULL); the offending sequence is clamped or skipped, never read
+ *     or written out of bounds.  No kernel waits on another.
+ */
+#ifndef ZKV_H
+#define ZKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+  ZKV_OK = 0,
+  ZKV_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shapes, misalignment */
+  ZKV_ERR_UNSUPPORTED = 2, /* d not in {64,128,256}, S not in 1..8, GQA group > 8, ...     */
+  ZKV_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the size query returned     */
+  ZKV_ERR_CUDA = 4         /* a CUDA launch or attribute call failed                        */
+} zkv_status;
+
+/* Bits OR-ed into a caller's device error word. */
+#define ZKV_DEVERR_COMP_LEN 1   /* comp_len[b] > Tcap (clamped) or append at Tcap (skipped) */
+#define ZKV_DEVERR_WIN_LEN 2    /* win_len[b] > Wcap (clamped)                              */
+
+#define ZKV_DTYPE_F16 0
+#define ZKV_DTYPE_F32 1
+
+#define ZKV_CODEBOOK_SIZE 256
+
+/* Human-readable name of a status code (static string). */
+const char* zkv_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int zkv_version(void);
+
+/*
+ * zkv_fwht -- Walsh-Hadamard transform of n_vec vectors of length d.
+ * Passage: zerokv-neo "Architecture" (FWHT energy spreading); VeloxQuant "Highlights"
+ * (O(d log d) Hadamard rotation).
+ *   out[n][i] = float32( scale * sum_j H_d[i][j] * in[n][j] ),  H_d Sylvester-ordered (+-1).
+ * The sum is accumulated in float64 (exact for fp16 inputs), multiplied by `scale` in float64
+ * and rounded once to float32.  scale = 1/sqrt(d) gives the orthonormal, self-inverse rotation.
+ *   in      device, [n_vec][d], dtype ZKV_DTYPE_F16 or ZKV_DTYPE_F32, contiguous rows
+ *   out     device, [n_vec][d] float32; may alias `in` only when in_dtype is F32
+ *   n_vec   >= 0 (0 launches nothing); d in {64,128,256}
+ * Errors: INVALID_ARG (null with n_vec>0, bad dtype), UNSUPPORTED (d), CUDA.
+ */
+int zkv_fwht(const void* in, int in_dtype, float* out, int64_t n_vec, int d, float scale,
+             void* stream);
+
+/*
+ * zkv_rvq_encode -- greedy residual vector quantisation of KV head vectors.
+ * Passage: VQKV section 2.1 "Process" steps 1-4 (nearest codeword per stage, residual passed
+ * on), section 2.3 "Prefilling Stage" (store only integer codes); rotation: zerokv-neo
+ * "Architecture".
+ * Rows are addressed as (b, t, h) for b < n_batch, t < n_tok, h < n_head.  For each row:
+ *   y = rotate ? float32(H_d x / sqrt(d)) : x        (float64 accumulate, one rounding)
+ *   r = y; for s in 0..S-1:
+ *     z_s = argmin_c ||r - C[h][s][c]||^2   decided in float64, ties -> lowest c
+ *     r   = r - C[h][s][z_s]                 (float32, elementwise)
+ *     norms[s] = float32(||r||_2)            (float64 accumulate)
+ * Layouts (strides in ELEMENTS of each tensor's type; the innermost index is contiguous):
+ *   x      fp16 or fp32 (x_dtype), element (b,t,h,i) at x[b*x_sb + t*x_st + h*x_sh + i]
+ *   codes  uint8, code s of (b,t,h) at codes[b*c_sb + t*c_st + h*c_sh + s]
+ *   norms  float32 or NULL, norm s of (b,t,h) at norms[b*n_sb + t*n_st + n_sh*h + s]
+ *   codebooks float32 [n_head][S][256][d]
+ * Alignment: x rows 16-byte aligned (x base and strides multiples of 8 fp16 / 4 fp32 elements).
+ * Errors: INVALID_ARG, UNSUPPORTED (d, S), CUDA.
+ */
+typedef struct {
+  int64_t n_batch, n_tok, n_head;
+  int d, S;
+  int rotate;   /* 1: apply the Hadamard rotation first; 0: x is already rotated */
+  int x_dtype;  /* ZKV_DTYPE_F16 or ZKV_DTYPE_F32 */
+  const void* x;
+  int64_t x_sb, x_st, x_sh;
+  const float* codebooks;
+  uint8_t* codes;
+  int64_t c_sb, c_st, c_sh;
+  float* norms;
+  int64_t n_sb, n_st, n_sh;
+} zkv_encode_params;
+
+int zkv_rvq_encode(const zkv_encode_params* p, void* stream);
+
+/*
+ * zkv_rvq_reconstruct -- x_hat = sum_s C[h][s][z_s] (float32, s ascending), optionally
+ * rotated back: out = H_d x_hat / sqrt(d) (float64 transform, one rounding).
+ * Passage: VQKV section 2.1 "Reconstruction".  Same row addressing as zkv_rvq_encode; `out`
+ * is float32 with strides o_sb, o_st, o_sh (elements) and contiguous d.
+ */
+typedef struct {
+  int64_t n_batch, n_tok, n_head;
+  int d, S;
+  int unrotate;
+  const uint8_t* codes;
+  int64_t c_sb, c_st, c_sh;
+  const float* codebooks;
+  float* out;
+  int64_t o_sb, o_st, o_sh;
+} zkv_reconstruct_params;
+
+int zkv_rvq_reconstruct(const zkv_reconstruct_params* p, void* stream);
+
+/*
+ * zkv_rvq_decode_attn -- one decode step of attention over an RVQ-compressed prefix plus an
+ * fp16 recency window, for every (sequence, query head) in one call.
+ * Passages: VQKV section 2.3 "Decoding Stage" (on-demand reconstruction inside attention;
+ * local sliding window); VeloxQuant "VecInfer" (q_tilde . k_tilde = q . k: the rotation is
+ * applied to the query); Differential-KV "Flash-Style LSE Combine" (fp32 log-sum-exp merge).
+ * Computes, for b < B, h < Hq, kvh = h / (Hq/Hkv):
+ *   keys   = { H (sum_s Ck[kvh][s][zk[b][kvh][t][s]]) / sqrt(d) : t < comp_len[b] }
+ *            U { win_k[b][kvh][w] : w < win_len[b] }                (values likewise)
+ *   out[b][h] = softmax(softmax_scale * q[b][h] . keys) . values    (float32)
+ *   lse[b][h] = natural log of sum exp(softmax_scale * q . k)        (float32, may be NULL)
+ * An empty context gives out = 0 and lse = -inf.
+ * Internally: q_tilde = H q / sqrt(d); per-stage tables LUT_s[c] = q_tilde . Ck_s[c]; scores
+ * are sums of table entries; values are accumulated as per-codeword weight histograms that are
+ * contracted with Cv once per (sequence, kv head); window and compressed part are joined by
+ * the log-sum-exp combine.
+ * Layouts:
+ *   q        fp16  [B][Hq][d]
+ *   k_codes  uint8 [B][Hkv][Tcap][Sk]      v_codes uint8 [B][Hkv][Tcap][Sv]
+ *   comp_len int32 [B] (device)             compressed tokens of each sequence, <= Tcap
+ *   k_codebooks float32 [Hkv][Sk][256][d]   v_codebooks float32 [Hkv][Sv][256][d]
+ *   win_k, win_v fp16 [B][Hkv][Wcap][d]     slots 0..win_len[b]-1 are valid (any order)
+ *   win_len  int32 [B] (device), <= Wcap
+ *   out      float32 [B][Hq][d]             lse float32 [B][Hq] or NULL
+ * max_comp_len: host-side upper bound on every comp_len[b] (<= Tcap); it sizes the launch.
+ *   Tokens beyond it are not read.
+ * softmax_scale: <= 0 selects 1/sqrt(d).
+ * The first call on a device sets kernel shared-memory attributes; make it before capturing
+ * calls into a CUDA graph.
+ * Workspace: device buffer of at least zkv_decode_workspace_size(p) bytes, 256-byte aligned,
+ *   no initial contents required; it must not be shared by calls that run concurrently.
+ * Errors: INVALID_ARG, UNSUPPORTED (d, S, Hq/Hkv > 8), WORKSPACE, CUDA.
+ */
+typedef struct {
+  int B, Hq, Hkv, d, Sk, Sv;
+  int64_t Tcap, Wcap;
+  int64_t max_comp_len;
+  float softmax_scale;
+  const uint16_t* q;
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const int32_t* comp_len;
+  const float* k_codebooks;
+  const float* v_codebooks;
+  const uint16_t* win_k;
+  const uint16_t* win_v;
+  const int32_t* win_len;
+  float* out;
+  float* lse;
+  int32_t* error_flag;
+  /* Optional tracing: NULL, or 4 cudaEvent_t handles (as void*) recorded on `stream` before
+   * the lookup-table kernel, before the scan kernel, before the merge kernel and after it. */
+  void* const* trace_events;
+} zkv_decode_params;
+
+/* Workspace bytes for a call with these shapes (data pointers are not read); 0 if the shapes
+ * are invalid or unsupported. */
+size_t zkv_decode_workspace_size(const zkv_decode_params* p);
+int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * zkv_rvq_append -- one serving step of cache maintenance: each sequence's new token enters
+ * the fp16 window; when the window is full, its oldest token is evicted, RVQ-encoded (same
+ * rule as zkv_rvq_encode, rotate = 1) and appended to the compressed prefix.
+ * Passages: VQKV section 2.3 "Local Sliding Window" (recent tokens uncompressed, middle tokens
+ * compressed); VeloxQuant "Quick start" (cache.append then cache.attend).
+ * Per sequence b (device-side state, updated in place):
+ *   if win_len[b] < Wcap:  slot = win_len[b]; win_len[b] += 1
+ *   else: slot = win_head[b]; encode win_k/win_v[b][:][slot] into k_codes/v_codes at position
+ *         comp_len[b]; comp_len[b] += 1; win_head[b] = (slot + 1) % Wcap
+ *   win_k[b][:][slot] = new_k[b]; win_v[b][:][slot] = new_v[b]
+ * If comp_len[b] == Tcap when an eviction is due, sequence b is left unchanged and
+ * ZKV_DEVERR_COMP_LEN is set.  Layouts as in zkv_rvq_decode_attn; new_k/new_v fp16 [B][Hkv][d];
+ * win_head int32 [B].  No workspace.  Two kernels are launched (encode+write, then the length
+ * update), so the state is consistent for any later work on the same stream.
+ */
+typedef struct {
+  int B, Hkv, d, Sk, Sv;
+  int64_t Tcap, Wcap;
+  const uint16_t* new_k;
+  const uint16_t* new_v;
+  uint16_t* win_k;
+  uint16_t* win_v;
+  int32_t* win_len;
+  int32_t* win_head;
+  int32_t* comp_len;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  const float* k_codebooks;
+  const float* v_codebooks;
+  int32_t* error_flag;
+} zkv_append_params;
+
+int zkv_rvq_append(const zkv_append_params* p, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZKV_H */

@@ -343,9 +343,12 @@ def append_step(state: dict, new_k: np.ndarray, new_v: np.ndarray) -> dict:
     is full); Ck, Cv codebooks.  new_k / new_v: [B][Hkv][d] fp16.
     While win_len < Wcap the token goes to slot win_len.  Otherwise slot win_head is evicted
     (its key and value are encoded to position comp_len), overwritten, and win_head advances.
+    If an eviction is due while comp_len == Tcap, that sequence is left unchanged and the
+    returned state's "error" entry is set to True (the prefix has no room).
     Returns a new state dict (inputs are not modified).
     """
     st = {k: (np.array(v, copy=True) if isinstance(v, np.ndarray) else v) for k, v in state.items()}
+    st["error"] = bool(state.get("error", False))
     B, Hkv, Wcap, d = st["win_k"].shape
     Tcap = st["k_codes"].shape[2]
     for b in range(B):
@@ -357,7 +360,8 @@ def append_step(state: dict, new_k: np.ndarray, new_v: np.ndarray) -> dict:
             slot = int(st["win_head"][b])
             pos = int(st["comp_len"][b])
             if pos >= Tcap:
-                raise ValueError("compressed prefix is at capacity")
+                st["error"] = True
+                continue
             for h in range(Hkv):
                 zk, _, _, _ = rvq_encode(st["win_k"][b, h, slot][None], st["Ck"][h])
                 zv, _, _, _ = rvq_encode(st["win_v"][b, h, slot][None], st["Cv"][h])

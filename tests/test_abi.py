@@ -1,0 +1,122 @@
+"""The C-ABI library loads and exports every function include/zkv.h declares; host-side
+argument validation rejects bad calls before any launch.  No GPU needed: every call below
+returns during validation, before the CUDA runtime is touched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_decode_attention_zkv_b200 import build as B
+from compressed_decode_attention_zkv_b200 import zkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return zkv.lib()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "zkv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(zkv_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("zkv_fwht", "zkv_rvq_encode", "zkv_rvq_decode_attn", "zkv_rvq_reconstruct",
+              "zkv_decode_workspace_size", "zkv_rvq_append", "zkv_status_string", "zkv_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in _declared_functions():
+        assert hasattr(L, n), f"{n} not exported"
+
+
+def test_status_strings_and_version(L):
+    assert zkv.status_string(0) == "ZKV_OK"
+    assert zkv.status_string(3) == "ZKV_ERR_WORKSPACE"
+    assert zkv.status_string(99) == "ZKV_ERR_UNKNOWN"
+    assert L.zkv_version() >= 100
+
+
+def test_fwht_validation(L):
+    assert L.zkv_fwht(None, 0, None, -1, 128, 1.0, None) == zkv.ZKV_ERR_INVALID_ARG
+    assert L.zkv_fwht(None, 7, None, 4, 128, 1.0, None) == zkv.ZKV_ERR_INVALID_ARG
+    assert L.zkv_fwht(None, 0, None, 4, 96, 1.0, None) == zkv.ZKV_ERR_UNSUPPORTED
+    assert L.zkv_fwht(None, 0, None, 0, 128, 1.0, None) == zkv.ZKV_OK
+    assert L.zkv_fwht(None, 0, None, 4, 128, 1.0, None) == zkv.ZKV_ERR_INVALID_ARG
+
+
+def test_encode_validation(L):
+    p = zkv.EncodeParams(n_batch=1, n_tok=4, n_head=1, d=128, S=4, rotate=1, x_dtype=0)
+    assert L.zkv_rvq_encode(ctypes.byref(p), None) == zkv.ZKV_ERR_INVALID_ARG   # null pointers
+    p.S = 9
+    assert L.zkv_rvq_encode(ctypes.byref(p), None) == zkv.ZKV_ERR_UNSUPPORTED
+    p.S, p.d = 4, 100
+    assert L.zkv_rvq_encode(ctypes.byref(p), None) == zkv.ZKV_ERR_UNSUPPORTED
+    p.d, p.x_dtype = 128, 5
+    assert L.zkv_rvq_encode(ctypes.byref(p), None) == zkv.ZKV_ERR_INVALID_ARG
+    p.x_dtype, p.n_tok = 0, 0
+    assert L.zkv_rvq_encode(ctypes.byref(p), None) == zkv.ZKV_OK               # empty: no-op
+    p.n_tok, p.x, p.codebooks, p.codes = 4, 0x1002, 0x1000, 0x1000              # misaligned x
+    assert L.zkv_rvq_encode(ctypes.byref(p), None) == zkv.ZKV_ERR_INVALID_ARG
+    assert L.zkv_rvq_encode(None, None) == zkv.ZKV_ERR_INVALID_ARG
+
+
+def _decode_params(**kw):
+    base = dict(B=2, Hq=8, Hkv=2, d=128, Sk=4, Sv=4, Tcap=64, Wcap=16, max_comp_len=64,
+                softmax_scale=0.0, q=0x1000, k_codes=0x2000, v_codes=0x3000, comp_len=0x4000,
+                k_codebooks=0x5000, v_codebooks=0x6000, win_k=0x7000, win_v=0x8000,
+                win_len=0x9000, out=0xa000)
+    base.update(kw)
+    return zkv.DecodeParams(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=6, Hkv=4), zkv.ZKV_ERR_INVALID_ARG),        # Hq not a multiple of Hkv
+    (dict(Hq=32, Hkv=2), zkv.ZKV_ERR_UNSUPPORTED),       # GQA group of 16
+    (dict(d=96), zkv.ZKV_ERR_UNSUPPORTED),
+    (dict(Sk=0), zkv.ZKV_ERR_UNSUPPORTED),
+    (dict(Sv=9), zkv.ZKV_ERR_UNSUPPORTED),
+    (dict(Tcap=60, max_comp_len=60), zkv.ZKV_ERR_INVALID_ARG),  # Tcap not a multiple of 16
+    (dict(max_comp_len=65), zkv.ZKV_ERR_INVALID_ARG),
+    (dict(q=0), zkv.ZKV_ERR_INVALID_ARG),
+    (dict(win_k=0), zkv.ZKV_ERR_INVALID_ARG),
+    (dict(k_codes=0x2008), zkv.ZKV_ERR_INVALID_ARG),     # misaligned
+])
+def test_decode_validation(L, kw, status):
+    p = _decode_params(**kw)
+    assert L.zkv_rvq_decode_attn(ctypes.byref(p), None, 0, None) == status
+    shape_error = not any(k in kw for k in ("q", "win_k", "k_codes"))
+    assert (L.zkv_decode_workspace_size(ctypes.byref(p)) == 0) == shape_error
+
+
+def test_decode_workspace_is_required(L):
+    p = _decode_params()
+    need = L.zkv_decode_workspace_size(ctypes.byref(p))
+    assert need > 0
+    assert L.zkv_rvq_decode_attn(ctypes.byref(p), None, need, None) == zkv.ZKV_ERR_WORKSPACE
+    assert L.zkv_rvq_decode_attn(ctypes.byref(p), 0x10000, need - 1, None) == zkv.ZKV_ERR_WORKSPACE
+    assert L.zkv_rvq_decode_attn(ctypes.byref(p), 0x10010, need, None) == zkv.ZKV_ERR_WORKSPACE
+
+
+def test_append_validation(L):
+    p = zkv.AppendParams(B=2, Hkv=2, d=128, Sk=4, Sv=4, Tcap=64, Wcap=0)
+    assert L.zkv_rvq_append(ctypes.byref(p), None) == zkv.ZKV_ERR_INVALID_ARG  # no window
+    p.Wcap, p.d = 8, 32
+    assert L.zkv_rvq_append(ctypes.byref(p), None) == zkv.ZKV_ERR_UNSUPPORTED
+    p.d = 128
+    assert L.zkv_rvq_append(ctypes.byref(p), None) == zkv.ZKV_ERR_INVALID_ARG  # null pointers
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        zkv.fwht(x, 1.0)

@@ -409,3 +409,18 @@ def test_append_step_window_then_eviction():
     np.testing.assert_array_equal(out["win_v"][1, :, 1], nv[1])
     # The caller's state is untouched.
     assert st["comp_len"][1] == 5
+
+
+def test_append_step_at_capacity_leaves_sequence_unchanged():
+    rng = np.random.default_rng(31)
+    B, Hkv, Wcap, d, Tcap, S, K = 1, 1, 2, 64, 4, 1, 8
+    C = _tiny_books(rng, S, K, d)[None]
+    st = dict(k_codes=np.zeros((B, Hkv, Tcap, S), np.uint8),
+              v_codes=np.zeros((B, Hkv, Tcap, S), np.uint8), comp_len=np.array([Tcap]),
+              win_k=rng.standard_normal((B, Hkv, Wcap, d)).astype(np.float16),
+              win_v=rng.standard_normal((B, Hkv, Wcap, d)).astype(np.float16),
+              win_len=np.array([Wcap]), win_head=np.array([1]), Ck=C, Cv=C)
+    out = O.append_step(st, np.ones((B, Hkv, d), np.float16), np.ones((B, Hkv, d), np.float16))
+    assert out["error"]
+    for k in ("k_codes", "v_codes", "comp_len", "win_k", "win_v", "win_len", "win_head"):
+        np.testing.assert_array_equal(out[k], st[k])
