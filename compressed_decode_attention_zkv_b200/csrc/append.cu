@@ -43,7 +43,9 @@ constexpr int kAppendR = 8;
 
 template <int D>
 __global__ void __launch_bounds__(256) append_encode_kernel(zkv_append_params p, double rot) {
-  __shared__ RowsSmem<D, kAppendR> sm;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  RowsSmem<D, kAppendR>& sm = *reinterpret_cast<RowsSmem<D, kAppendR>*>(smem_raw);
+  float* cb = reinterpret_cast<float*>(smem_raw + ((sizeof(RowsSmem<D, kAppendR>) + 15) / 16) * 16);
   const int kind = blockIdx.z;   // 0 = keys, 1 = values
   const int h = blockIdx.y;
   const int64_t row0 = (int64_t)blockIdx.x * kAppendR;
@@ -60,7 +62,7 @@ __global__ void __launch_bounds__(256) append_encode_kernel(zkv_append_params p,
   map.comp_len = p.comp_len;
   const int S = kind ? p.Sv : p.Sk;
   const float* books = kind ? p.v_codebooks : p.k_codebooks;
-  encode_rows_body<D, kAppendR>(map, books, S, rot, row0, h, sm);
+  encode_rows_body<D, kAppendR>(map, books, S, rot, row0, h, sm, cb);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < kAppendR) {
     const int64_t j = row0 + tid;
@@ -124,10 +126,15 @@ extern "C" int zkv_rvq_append(const zkv_append_params* p, void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const double rot = 1.0 / std::sqrt((double)p->d);
   const dim3 grid((unsigned)((p->B + kAppendR - 1) / kAppendR), (unsigned)p->Hkv, 2);
+  const bool ok =
+      ensure_smem_limit(append_encode_kernel<64>, rows_smem_bytes<64, kAppendR>()) == cudaSuccess &&
+      ensure_smem_limit(append_encode_kernel<128>, rows_smem_bytes<128, kAppendR>()) == cudaSuccess &&
+      ensure_smem_limit(append_encode_kernel<256>, rows_smem_bytes<256, kAppendR>()) == cudaSuccess;
+  if (!ok) return ZKV_ERR_CUDA;
   switch (p->d) {
-    case 64: append_encode_kernel<64><<<grid, 256, 0, st>>>(*p, rot); break;
-    case 128: append_encode_kernel<128><<<grid, 256, 0, st>>>(*p, rot); break;
-    default: append_encode_kernel<256><<<grid, 256, 0, st>>>(*p, rot); break;
+    case 64: append_encode_kernel<64><<<grid, 256, rows_smem_bytes<64, kAppendR>(), st>>>(*p, rot); break;
+    case 128: append_encode_kernel<128><<<grid, 256, rows_smem_bytes<128, kAppendR>(), st>>>(*p, rot); break;
+    default: append_encode_kernel<256><<<grid, 256, rows_smem_bytes<256, kAppendR>(), st>>>(*p, rot); break;
   }
   ZKV_CHECK_LAUNCH();
   append_lengths_kernel<<<(p->B + 127) / 128, 128, 0, st>>>(p->B, p->Tcap, p->Wcap, p->win_len,

@@ -40,9 +40,10 @@
 
 namespace zkv {
 
-constexpr int kScanSub = 1024;      // tokens per scan sub-chunk (4 per thread)
-constexpr int kScanThreads = 256;
+constexpr int kScanSub = 512;       // tokens per scan sub-chunk (1 per thread)
+constexpr int kScanThreads = 512;
 constexpr int kColCap = 8176;       // tokens per histogram column per segment (sum < 2^32)
+constexpr float kHeadroom = 8.f;    // log2 units added to the running maximum on growth
 constexpr size_t kSmemMax = 227 * 1024;
 
 static int sm_count() {
@@ -83,12 +84,13 @@ struct DecodePlan {
       off_cnt, total;
 };
 
-static size_t scan_smem_bytes(int Rk, int Sk, int GP, const VMap& v) {
+static size_t scan_smem_bytes(int Rk, int Sk, int Sv, int GP, const VMap& v) {
   size_t b = (size_t)Rk * Sk * kCodebook * GP * 4;            // key tables
+  b += (size_t)Sv * kCodebook * GP * 4;                         // fp32 master histograms
   b += 2ull * kCodebook * v.VW * 4;                            // value histograms (hi, lo)
-  b += (size_t)v.J * GP * (v.rounds + 4) * 4;                   // p staging
+  b += 2ull * v.J * GP * (v.rounds + 4) * 4;                    // fixed-point p staging (hi, lo)
   b += (size_t)v.J * (v.rounds + 4) * v.codew * 4;              // value-code staging
-  b += (size_t)9 * GP * 4 + 16;                                 // reductions
+  b += (size_t)(kScanThreads / 32 + 1) * GP * 4 + 16;           // reductions
   return b;
 }
 
@@ -101,9 +103,9 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   const VMap v = vmap(pl.SVP, pl.GP);
   // replication that makes the key gathers conflict-free, reduced until shared memory fits
   int Rk = pl.GP == 1 ? 32 : pl.GP == 2 ? 16 : pl.GP == 4 ? 8 : 4;
-  while (Rk > 1 && scan_smem_bytes(Rk, p->Sk, pl.GP, v) > kSmemMax) Rk >>= 1;
+  while (Rk > 1 && scan_smem_bytes(Rk, p->Sk, p->Sv, pl.GP, v) > kSmemMax) Rk >>= 1;
   pl.Rk = Rk;
-  pl.scan_smem = scan_smem_bytes(Rk, p->Sk, pl.GP, v);
+  pl.scan_smem = scan_smem_bytes(Rk, p->Sk, p->Sv, pl.GP, v);
   const int64_t pairs = (int64_t)p->B * p->Hkv;
   pl.cap = (int64_t)kColCap * v.J;
   const int64_t bound = pairs * p->max_comp_len;
@@ -183,90 +185,130 @@ struct LutSmem {
   float cT[D][kLutC + 1];     // codebook slice, k-major
 };
 
+// Ask the memory system to stage [p, p + bytes) in L2 (no data returned to the SM).  p and
+// bytes are rounded outward to 16-byte granules inside [lo, hi), the caller's allocation.
+__device__ __forceinline__ void prefetch_l2(const uint8_t* lo, const uint8_t* hi, const uint8_t* p,
+                                            int64_t bytes) {
+  uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(15);
+  uintptr_t e = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t(15);
+  if (a < reinterpret_cast<uintptr_t>(lo)) a = reinterpret_cast<uintptr_t>(lo);
+  if (e > reinterpret_cast<uintptr_t>(hi)) e = reinterpret_cast<uintptr_t>(hi);
+  while (a < e) {
+    const uint32_t n = (uint32_t)((e - a) < 65536 ? (e - a) : 65536);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
+    a += n;
+  }
+}
+
+// Dense attention of the GP heads of one (sequence, kv head) over its fp16 window (base-2
+// logits, online maximum over 256-token tiles).  Warps take tokens, lanes split the head
+// dimension, so every load is an independent coalesced row fragment.
 template <int D, int GP>
 __device__ void window_item(const DecodeArgs& a, int b, int kvh, float* smem) {
-  float* qs = smem;                 // [GP][D]   query * scale * log2 e
-  float* ps = qs + GP * D;          // [256][GP] probabilities of the current tile
-  float* red = ps + 256 * GP;       // [8][GP]
-  float* alph = red + 8 * GP;       // [GP]      rescale factor of the current tile
+  constexpr int PL = D / 32;        // head dims per lane
+  float* sc = smem;                 // [256][GP] scores, then probabilities, of the tile
+  float* red = sc + 256 * GP;       // [8][GP]
+  float* part = red + 8 * GP;       // [8][GP][D] per-warp partial outputs
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pair = (int64_t)b * a.Hkv + kvh;
   const int64_t wl = clamp_win_len(a, b);
-  for (int f = tid; f < GP * D; f += 256) {
-    const int g = f / D, i = f % D;
-    qs[f] = g < a.G ? __half2float(a.q[((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D + i]) *
-                          a.scale_log2
-                    : 0.f;
+  float qf[GP][PL];
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int e = 0; e < PL; ++e)
+      qf[g][e] = g < a.G ? __half2float(a.q[((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D +
+                                            lane * PL + e]) * a.scale_log2
+                         : 0.f;
+  float m_run[GP], l_run[GP], acc[GP][PL];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    m_run[g] = -INFINITY;
+    l_run[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < PL; ++e) acc[g][e] = 0.f;
   }
-  float m_run[GP], l_run[GP];
-#pragma unroll
-  for (int g = 0; g < GP; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
-  constexpr int OPT = (GP * D + 255) / 256;   // output elements (g, i) owned per thread
-  float oacc[OPT];
-#pragma unroll
-  for (int r = 0; r < OPT; ++r) oacc[r] = 0.f;
-  __syncthreads();
   const __half* Kb = a.win_k + pair * a.Wcap * D;
   const __half* Vb = a.win_v + pair * a.Wcap * D;
   for (int64_t base = 0; base < wl; base += 256) {
-    const int64_t t = base + tid;
-    float sc[GP];
+    const int n = (int)(wl - base < 256 ? wl - base : 256);
+    // scores
+#pragma unroll 2
+    for (int tt = warp; tt < n; tt += 8) {
+      const __half* kr = Kb + (base + tt) * D + lane * PL;
+      float kf[PL];
 #pragma unroll
-    for (int g = 0; g < GP; ++g) sc[g] = t < wl ? 0.f : -INFINITY;
-    if (t < wl) {
-      const __half* kr = Kb + t * D;
-      for (int i = 0; i < D; i += 8) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(kr + i));
-        const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+      for (int e = 0; e < PL; e += 2) {
+        const float2 v = __half22float2(*reinterpret_cast<const __half2*>(kr + e));
+        kf[e] = v.x;
+        kf[e + 1] = v.y;
+      }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 kv = __half22float2(h2[e]);
+      for (int g = 0; g < GP; ++g) {
+        float d = 0.f;
 #pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            sc[g] = fmaf(qs[g * D + i + 2 * e], kv.x, sc[g]);
-            sc[g] = fmaf(qs[g * D + i + 2 * e + 1], kv.y, sc[g]);
-          }
-        }
+        for (int e = 0; e < PL; ++e) d = fmaf(qf[g][e], kf[e], d);
+        d = warp_sum_f32(d);
+        if (lane == 0) sc[tt * GP + g] = d;
       }
     }
+    __syncthreads();
+    // tile maximum, probabilities
+    float mt[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
-      const float m = warp_max_f32(sc[g]);
+      const float v = tid < n ? sc[tid * GP + g] : -INFINITY;
+      const float m = warp_max_f32(v);
       if (lane == 0) red[warp * GP + g] = m;
     }
     __syncthreads();
+    float alpha[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       float m = red[g];
 #pragma unroll
       for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w * GP + g]);
       const float mn = fmaxf(m_run[g], m);
-      const float alpha = m_run[g] == -INFINITY ? 0.f : ex2_approx(m_run[g] - mn);
-      l_run[g] *= alpha;
+      alpha[g] = m_run[g] == -INFINITY ? 0.f : ex2_approx(m_run[g] - mn);
       m_run[g] = mn;
-      const float pv = t < wl ? ex2_approx(sc[g] - mn) : 0.f;
-      ps[tid * GP + g] = pv;
-      l_run[g] += pv;
-      if (tid == 0) alph[g] = alpha;
-    }
-    __syncthreads();
-    const int64_t nt = wl - base < 256 ? wl - base : 256;
+      mt[g] = mn;
+      l_run[g] *= alpha[g];
 #pragma unroll
-    for (int r = 0; r < OPT; ++r) {
-      const int f = tid + 256 * r;
-      if (f < GP * D) {
-        const int g = f / D, i = f % D;
-        float acc = oacc[r] * alph[g];
-#pragma unroll 4
-        for (int64_t tt = 0; tt < nt; ++tt)
-          acc = fmaf(ps[tt * GP + g], __half2float(Vb[(base + tt) * D + i]), acc);
-        oacc[r] = acc;
+      for (int e = 0; e < PL; ++e) acc[g][e] *= alpha[g];
+    }
+    if (tid < n) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float pv = ex2_approx(sc[tid * GP + g] - mt[g]);
+        sc[tid * GP + g] = pv;
+        l_run[g] += pv;
       }
     }
     __syncthreads();
+    // values
+#pragma unroll 2
+    for (int tt = warp; tt < n; tt += 8) {
+      const __half* vr = Vb + (base + tt) * D + lane * PL;
+      float vf[PL];
+#pragma unroll
+      for (int e = 0; e < PL; e += 2) {
+        const float2 v = __half22float2(*reinterpret_cast<const __half2*>(vr + e));
+        vf[e] = v.x;
+        vf[e + 1] = v.y;
+      }
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float pv = sc[tt * GP + g];
+#pragma unroll
+        for (int e = 0; e < PL; ++e) acc[g][e] = fmaf(pv, vf[e], acc[g][e]);
+      }
+    }
+    __syncthreads();   // sc is rewritten by the next tile
   }
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
+#pragma unroll
+    for (int e = 0; e < PL; ++e) part[(warp * GP + g) * D + lane * PL + e] = acc[g][e];
     const float l = warp_sum_f32(l_run[g]);
     if (lane == 0) red[warp * GP + g] = l;
   }
@@ -277,10 +319,11 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, float* smem) {
     a.wm[pair * GP + tid] = m_run[tid];
     a.wl[pair * GP + tid] = l;
   }
+  for (int f = tid; f < GP * D; f += 256) {
+    float v = 0.f;
 #pragma unroll
-  for (int r = 0; r < OPT; ++r) {
-    const int f = tid + 256 * r;
-    if (f < GP * D) a.wo[pair * GP * D + f] = oacc[r];
+    for (int w = 0; w < 8; ++w) v += part[w * GP * D + f];
+    a.wo[pair * GP * D + f] = v;
   }
 }
 
@@ -295,25 +338,55 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
     return;
   }
   if (blockIdx.x == 0) {
+    // exclusive prefix sums of the clamped compressed lengths, 256 pairs per round
+    __shared__ int64_t warp_tot[8];
+    __shared__ int64_t carry_s;
     const int npairs = a.B * a.Hkv;
     for (int i = tid; i < npairs; i += blockDim.x) a.cnt[i] = 0u;
     if (tid == 0) {
-      int64_t acc = 0;
+      carry_s = 0;
       a.pre[0] = 0;
-      for (int pr = 0; pr < npairs; ++pr) {
-        int64_t c = a.comp_len[pr / a.Hkv];
+    }
+    __syncthreads();
+    for (int base = 0; base < npairs; base += 256) {
+      const int pr = base + tid;
+      int64_t c = 0;
+      if (pr < npairs) {
+        c = a.comp_len[pr / a.Hkv];
         if (c < 0 || c > a.Tcap) {
           set_error(a.err, ZKV_DEVERR_COMP_LEN);
           c = c < 0 ? 0 : a.Tcap;
         }
         c = c < a.max_comp ? c : a.max_comp;
-        acc += c;
-        a.pre[pr + 1] = acc;
       }
+      int64_t x = c;   // inclusive warp scan
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) warp_tot[warp] = x;
+      __syncthreads();
+      int64_t off = carry_s;
+      for (int w = 0; w < warp; ++w) off += warp_tot[w];
+      if (pr < npairs) a.pre[pr + 1] = off + x;
+      __syncthreads();
+      if (tid == 255) carry_s = off + x;
+      __syncthreads();
+    }
+    if (tid == 0) {
+      const int64_t acc = carry_s;
       int64_t sh = (acc + a.grid - 1) / a.grid;
       sh = (sh + 15) / 16 * 16;
       *a.share = sh < 16 ? 16 : sh;
     }
+  }
+  if ((int)blockIdx.x < a.Hkv * a.Sv && tid == 0) {
+    // the merge kernel reads every value codebook; stream them into L2 meanwhile
+    const uint8_t* cv0 = reinterpret_cast<const uint8_t*>(a.Cv);
+    const int64_t bytes = (int64_t)kCodebook * D * sizeof(float);
+    const uint8_t* p = cv0 + (int64_t)blockIdx.x * bytes;
+    prefetch_l2(p, p + bytes, p, bytes);
   }
   LutSmem<D>& sm = *reinterpret_cast<LutSmem<D>*>(smem_raw);
   const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
@@ -385,86 +458,137 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
 // 2. Scan of the compressed tokens.
 // ------------------------------------------------------------------------------------------
 
+// 32-bit shared-memory address operations (the hot loop keeps precomputed addresses).
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float2 lds64f(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds32f(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128u(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts32u(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v));
+}
+__device__ __forceinline__ void sts64u(uint32_t a, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y));
+}
+// hi at a, lo at a + LO_OFF bytes (the lo table follows the hi table)
+template <int LO_OFF>
+__device__ __forceinline__ void red_pair(uint32_t a, uint32_t hi, uint32_t lo) {
+  asm volatile("red.shared.add.u32 [%0], %1;\n\tred.shared.add.u32 [%0+%3], %2;"
+               ::"r"(a), "r"(hi), "r"(lo), "n"(LO_OFF));
+}
+
 // Codes of one token (S <= 8 bytes, little-endian in up to two words).
 template <int SP>
 struct Code {
   uint32_t w[SP <= 4 ? 1 : 2];
   __device__ __forceinline__ int byte(int s) const {
-    if constexpr (SP <= 4) return (w[0] >> (8 * s)) & 0xff;
-    else return (w[s >> 2] >> (8 * (s & 3))) & 0xff;
+    return (int)__byte_perm(w[SP <= 4 ? 0 : (s >> 2)], 0u, 0x4440u | (unsigned)(s & 3));
   }
 };
 
-// Codes of the 4 consecutive tokens t0..t0+3 (t0 a multiple of 4, below Tcap).  When S equals
-// its padded size SP one naturally aligned vector load covers all four; otherwise byte loads.
+// Codes of token t (0 when t >= tend).  When S equals its padded size SP a single naturally
+// aligned 2-, 4- or 8-byte load reads them; otherwise byte loads.
 template <int SP>
-__device__ __forceinline__ void load_codes4(const uint8_t* base, int S, int64_t t0, int64_t tend,
-                                            Code<SP> (&out)[4]) {
+__device__ __forceinline__ Code<SP> load_code1(const uint8_t* base, int S, uint32_t t, uint32_t tend) {
+  // t is a pair-local token index (Tcap * S < 2^32 bytes per pair)
+  Code<SP> r;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-#pragma unroll
-    for (int q = 0; q < (SP <= 4 ? 1 : 2); ++q) out[u].w[q] = 0u;
-  }
-  if (t0 >= tend) return;
+  for (int q = 0; q < (SP <= 4 ? 1 : 2); ++q) r.w[q] = 0u;
+  if (t >= tend) return r;
   if (S == SP) {
-    const uint8_t* p = base + t0 * SP;
+    const uint8_t* p = base + t * SP;
     if constexpr (SP == 2) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-      out[0].w[0] = v.x & 0xffffu; out[1].w[0] = v.x >> 16;
-      out[2].w[0] = v.y & 0xffffu; out[3].w[0] = v.y >> 16;
+      r.w[0] = __ldg(reinterpret_cast<const unsigned short*>(p));
     } else if constexpr (SP == 4) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-      out[0].w[0] = v.x; out[1].w[0] = v.y; out[2].w[0] = v.z; out[3].w[0] = v.w;
+      r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
     } else {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(p + 16));
-      out[0].w[0] = v.x; out[0].w[1] = v.y; out[1].w[0] = v.z; out[1].w[1] = v.w;
-      out[2].w[0] = u.x; out[2].w[1] = u.y; out[3].w[0] = u.z; out[3].w[1] = u.w;
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+      r.w[0] = v.x;
+      r.w[1] = v.y;
     }
   } else {
+    const uint8_t* p = base + t * S;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (t0 + u < tend) {
-        const uint8_t* p = base + (t0 + u) * S;
-#pragma unroll
-        for (int s = 0; s < SP; ++s)
-          if (s < S) out[u].w[s >> 2] |= (uint32_t)p[s] << (8 * (s & 3));
-      }
-    }
+    for (int s = 0; s < SP; ++s)
+      if (s < S) r.w[s >> 2] |= (uint32_t)__ldg(p + s) << (8 * (s & 3));
   }
+  return r;
 }
 
 // Key score of one token: sum over stages of the token's table entries (GP heads).
+// sbase[s] is the shared address of this lane's copy of stage s codeword 0; codeword c is
+// (c << csh) bytes further.
 template <int GP, int SKP>
-__device__ __forceinline__ void key_score(const float* lut, int Sk, int Rk, int copy, int lane,
-                                          const Code<SKP>& kc, float (&sc)[GP]) {
+__device__ __forceinline__ void key_score(const uint32_t (&sbase)[SKP], int Sk, uint32_t csh,
+                                          int lane, const Code<SKP>& kc, float (&sc)[GP]) {
 #pragma unroll
   for (int g = 0; g < GP; ++g) sc[g] = 0.f;
 #pragma unroll
   for (int s = 0; s < SKP; ++s) {
     if (s < Sk) {
-      const int c = kc.byte(s);
-      const float* e = lut + ((size_t)(s * kCodebook + c) * Rk + copy) * GP;
+      const uint32_t e = sbase[s] + ((uint32_t)kc.byte(s) << csh);
       if constexpr (GP == 8) {
         // the two halves are read in lane-dependent order: lanes 4-7 of each 8-lane phase
         // start with the upper half, which puts all 8 lanes of a phase in distinct banks
-        const int h0 = (lane >> 2) & 1;
-        const float4 v0 = *reinterpret_cast<const float4*>(e + 4 * h0);
-        const float4 v1 = *reinterpret_cast<const float4*>(e + 4 * (h0 ^ 1));
+        const uint32_t h0 = ((uint32_t)lane >> 2) & 1u;
+        const float4 v0 = lds128f(e + 16u * h0);
+        const float4 v1 = lds128f(e + 16u * (h0 ^ 1u));
         const float4 lo4 = h0 ? v1 : v0, hi4 = h0 ? v0 : v1;
         sc[0] += lo4.x; sc[1] += lo4.y; sc[2] += lo4.z; sc[3] += lo4.w;
         sc[4] += hi4.x; sc[5] += hi4.y; sc[6] += hi4.z; sc[7] += hi4.w;
       } else if constexpr (GP == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(e);
+        const float4 v = lds128f(e);
         sc[0] += v.x; sc[1] += v.y; sc[2] += v.z; sc[3] += v.w;
       } else if constexpr (GP == 2) {
-        const float2 v = *reinterpret_cast<const float2*>(e);
+        const float2 v = lds64f(e);
         sc[0] += v.x; sc[1] += v.y;
       } else {
-        sc[0] += e[0];
+        sc[0] += lds32f(e);
       }
     }
   }
+}
+
+// p in [0, 1] as p * 2^38 = hi * 2^19 + lo with hi = round(p * 2^19) in [0, 2^19] and
+// lo = round((p * 2^19 - hi) * 2^19) in [-2^18, 2^18] (two's complement).  Each FMA below is
+// exact except the roundings to an integer (|error of p * 2^38| <= 1/2); rounding uses the
+// 1.5 * 2^23 addend, so only FMA-pipe and integer instructions are involved.
+__device__ __forceinline__ void split_fixed38(float p, uint32_t& hi, uint32_t& lo) {
+  const float magic = 12582912.0f;                          // 1.5 * 2^23
+  const float xr = __fmaf_rn(p, 524288.0f, magic);          // round(p * 2^19) + magic
+  hi = __float_as_uint(xr) - 0x4B400000u;
+  const float h = __fsub_rn(xr, magic);                     // round(p * 2^19), exact
+  const float d = __fmaf_rn(p, 524288.0f, -h);              // p * 2^19 - h, exact
+  lo = __float_as_uint(__fmaf_rn(d, 524288.0f, magic)) - 0x4B400000u;
+}
+
+// Order-preserving map of a float to an unsigned key (for integer max reductions).
+__device__ __forceinline__ uint32_t ord_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_val(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 __device__ __forceinline__ void red_add_u32(uint32_t* p, uint32_t v) {
@@ -478,10 +602,46 @@ struct ScanCfg {
   static constexpr int J = COMBOS >= 32 ? 1 : 32 / COMBOS;
   static constexpr int PASSES = COMBOS > 32 ? COMBOS / 32 : 1;
   static constexpr int VW = 32 * PASSES;
+  static constexpr int VWSH = PASSES == 1 ? 5 : 6;   // log2(VW)
   static constexpr int ROUNDS = kScanSub / J;
-  static constexpr int PR = ROUNDS + 4;          // padded staging row (floats / words)
+  static constexpr int PR = ROUNDS + 4;          // padded staging row (words)
   static constexpr int CODEW = SVP <= 4 ? 1 : 2;
+  static constexpr int NW = kScanThreads / 32;
 };
+
+// master[(s, c, g)] = (master (if any) + histogram value) * scale[g], where the histogram
+// value of (s, c, g) is the sum over token slots j of hi * 2^-19 + lo * 2^-38 in column
+// j * COMBOS + s * GP + g of code row c.  Threads walk the tables row by row (consecutive
+// threads, consecutive words: no bank conflicts); the J columns of one (s, g) are combined
+// with xor-shuffles (they are COMBOS lanes apart).
+template <class C, int GP>
+__device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t* vlo,
+                                            float* master, int Sv, bool has_master,
+                                            const float (&scale)[GP], int tid) {
+  const int lane = tid & 31;
+  const int total = kCodebook * C::VW;           // words per table
+  for (int w0 = tid - lane; w0 < total; w0 += kScanThreads) {
+    const int wi = w0 + lane;                      // total is a multiple of 32
+    const int cc = wi / C::VW, col = wi % C::VW;
+    double v = (double)vhi[wi] * (1.0 / 524288.0) + (double)(int32_t)vlo[wi] * (1.0 / 274877906944.0);
+    if constexpr (C::PASSES == 1) {
+#pragma unroll
+      for (int o = C::COMBOS; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    }
+    const int combo = C::PASSES == 1 ? col % C::COMBOS : col;
+    const int ss = combo / GP, g = combo % GP;
+    const bool writer = (C::PASSES == 1 ? col < C::COMBOS : true) && ss < Sv;
+    if (writer) {
+      float sc = 1.f;
+#pragma unroll
+      for (int q = 0; q < GP; ++q)
+        if (q == g) sc = scale[q];
+      const size_t f = ((size_t)ss * kCodebook + cc) * GP + g;
+      const float old = has_master ? master[f] : 0.f;
+      master[f] = (old + (float)v) * sc;
+    }
+  }
+}
 
 template <int GP, int SKP, int SVP>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
@@ -489,12 +649,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) unsigned char smraw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Rk = a.Rk, Sk = a.Sk, Sv = a.Sv, G = a.G;
+  const int ntab = Sv * kCodebook * GP;           // histogram entries (s, c, g)
   float* lut = reinterpret_cast<float*>(smraw);                                 // [Sk][256][Rk][GP]
-  uint32_t* vhi = reinterpret_cast<uint32_t*>(lut + (size_t)Rk * Sk * kCodebook * GP);  // [256][VW]
+  float* master = lut + (size_t)Rk * Sk * kCodebook * GP;                       // [Sv][256][GP]
+  uint32_t* vhi = reinterpret_cast<uint32_t*>(master + ntab);                   // [256][VW]
   uint32_t* vlo = vhi + kCodebook * C::VW;
-  float* pst = reinterpret_cast<float*>(vlo + kCodebook * C::VW);               // [J][GP][PR]
-  uint32_t* cst = reinterpret_cast<uint32_t*>(pst + C::J * GP * C::PR);         // [J][PR][CODEW]
-  float* red = reinterpret_cast<float*>(cst + C::J * C::PR * C::CODEW);         // [8][GP]
+  uint32_t* hst = vlo + kCodebook * C::VW;                                      // [J][GP][PR]
+  uint32_t* lst = hst + C::J * GP * C::PR;                                      // [J][GP][PR]
+  uint32_t* cst = lst + C::J * GP * C::PR;                                      // [J][PR][CODEW]
+  uint32_t* redk = cst + C::J * C::PR * C::CODEW;                               // [NW][GP]
+  float* red = reinterpret_cast<float*>(redk);
 
   const int npairs = a.B * a.Hkv;
   const int64_t share = *a.share;
@@ -513,8 +677,22 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     pfirst = l;
   }
   const int copy = lane & (Rk - 1);
+  const int cshift = __ffs(Rk * GP) - 1;          // Rk * GP is a power of two
+  const int sstride = kCodebook * Rk * GP;
+  // shared addresses used by the token loop
+  uint32_t sbase[SKP];
+#pragma unroll
+  for (int q = 0; q < SKP; ++q) sbase[q] = smem_u32(lut) + 4u * (uint32_t)(q * sstride + copy * GP);
+  const uint32_t csh = (uint32_t)cshift + 2u;
   // value-side lane roles (PASSES == 1: lane = j * COMBOS + s * GP + g)
   const int vj = C::PASSES == 1 ? lane / C::COMBOS : 0;
+  // staging slot of this thread's token
+  const int sj = tid % C::J, sk = tid / C::J;
+  const uint32_t hst_base = smem_u32(hst), cst_base = smem_u32(cst);
+  const uint32_t hst_a = hst_base + 4u * (uint32_t)(sj * GP * C::PR + sk);
+  const uint32_t cst_a = cst_base + 4u * C::CODEW * (uint32_t)(sj * C::PR + sk);
+  const uint32_t vtab_base = smem_u32(vhi);
+  const uint32_t redk_a = smem_u32(redk);
 
   for (int pr = pfirst; pr < npairs && a.pre[pr] < hi; ++pr) {
     const int64_t seg0 = lo > a.pre[pr] ? lo : a.pre[pr];
@@ -526,133 +704,163 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     const uint8_t* kcb = a.k_codes + (int64_t)pr * a.Tcap * Sk;
     const uint8_t* vcb = a.v_codes + (int64_t)pr * a.Tcap * Sv;
 
+    if (tid == 0) {
+      // the segment's codes stream into L2 while the tables are filled; the per-thread loads
+      // below then find them there
+      const int64_t pbytes_k = (int64_t)a.Tcap * Sk, pbytes_v = (int64_t)a.Tcap * Sv;
+      prefetch_l2(kcb, kcb + pbytes_k, kcb + (s0 & ~int64_t(15)) * Sk, (s1 - (s0 & ~int64_t(15))) * Sk);
+      prefetch_l2(vcb, vcb + pbytes_v, vcb + (s0 & ~int64_t(15)) * Sv, (s1 - (s0 & ~int64_t(15))) * Sv);
+    }
     __syncthreads();   // previous segment's shared memory is free
     {
+      // the pair's G x Sk x 256 table entries: coalesced loads into a staging area (the
+      // histogram region, 2 * 256 * VW >= 16384 words), stored (s, c)-major with a padded
+      // head stride, then replicated into the lane-group copies with linear stores
       const float* src = a.lut + ((int64_t)b * a.Hq + (int64_t)kvh * G) * Sk * kCodebook;
-      const int n = Sk * kCodebook * GP;
+      float* stage = reinterpret_cast<float*>(vhi);
+      const int nsc = Sk * kCodebook;
+      const int str = (nsc * (GP + 1) <= 2 * kCodebook * C::VW) ? GP + 1 : GP;
+      for (int g = 0; g < G; ++g)
+        for (int sc = tid; sc < nsc; sc += kScanThreads) stage[sc * str + g] = __ldg(src + g * nsc + sc);
+      __syncthreads();
+      const int n = nsc * Rk * GP;    // replicated table, written linearly
       for (int f = tid; f < n; f += kScanThreads) {
-        const int g = f % GP, sc = f / GP;       // sc = s*256 + c
-        const float v = g < G ? __ldg(src + (int64_t)g * Sk * kCodebook + sc) : 0.f;
-        float* dst = lut + (size_t)sc * Rk * GP + g;
-        for (int cp = 0; cp < Rk; ++cp) dst[cp * GP] = v;
+        const int g = f & (GP - 1), sc = f >> cshift;   // sc = s*256 + c
+        lut[f] = g < G ? stage[sc * str + g] : 0.f;
       }
+      __syncthreads();
       uint4* z = reinterpret_cast<uint4*>(vhi);
       const int nz = 2 * kCodebook * C::VW / 4;
       for (int f = tid; f < nz; f += kScanThreads) z[f] = make_uint4(0u, 0u, 0u, 0u);
     }
-    __syncthreads();
+    // (the first __syncthreads of the token loop orders the zeroing before any reduction)
 
-    const int64_t abase = s0 & ~int64_t(3);
-    // ---- pass 1: maximum score per head
-    float mloc[GP];
+    float mref[GP], lacc[GP];
 #pragma unroll
-    for (int g = 0; g < GP; ++g) mloc[g] = -INFINITY;
-    for (int64_t base = abase; base < s1; base += kScanSub) {
-      const int64_t t0 = base + 4 * tid;
-      Code<SKP> kc[4];
-      load_codes4<SKP>(kcb, Sk, t0, s1, kc);
+    for (int g = 0; g < GP; ++g) {
+      mref[g] = -INFINITY;
+      lacc[g] = 0.f;
+    }
+    bool dirty = false, has_master = false;   // uniform across the block
+    const uint32_t u0 = (uint32_t)s0, u1 = (uint32_t)s1;
+    Code<SKP> kn = load_code1<SKP>(kcb, Sk, u0 + tid, u1);
+    Code<SVP> vn = load_code1<SVP>(vcb, Sv, u0 + tid, u1);
+    for (uint32_t ubase = u0; ubase < u1; ubase += kScanSub) {
+      const uint32_t t = ubase + tid;
+      const Code<SKP> kc = kn;
+      const Code<SVP> vc = vn;
+      kn = load_code1<SKP>(kcb, Sk, t + kScanSub, u1);   // next sub-chunk in flight
+      vn = load_code1<SVP>(vcb, Sv, t + kScanSub, u1);
+      const bool ok = t < u1;
+      float sc[GP];
+      key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
+      // sub-chunk maximum per head (integer reduction on order-preserving keys)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t t = t0 + u;
-        if (t >= s0 && t < s1) {
-          float sc[GP];
-          key_score<GP, SKP>(lut, Sk, Rk, copy, lane, kc[u], sc);
+      for (int g = 0; g < GP; ++g) {
+        const uint32_t k = __reduce_max_sync(0xffffffffu, ok ? ord_key(sc[g]) : 0u);
+        if (lane == 0) sts32u(redk_a + 4u * (uint32_t)(warp * GP + g), k);
+      }
+      __syncthreads();   // also: the previous sub-chunk's staging has been consumed
+      // every warp combines the NW x GP partial maxima: lanes read them (entry w * GP + g sits
+      // in lane (w * GP + g) % 32), fold over w with xor-shuffles, then broadcast each head
+      float mn[GP];
+      {
+        uint32_t k = 0u;
 #pragma unroll
-          for (int g = 0; g < GP; ++g) mloc[g] = fmaxf(mloc[g], sc[g]);
+        for (int e = 0; e < C::NW * GP; e += 32)
+          if (e + lane < C::NW * GP) {
+            uint32_t v;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(redk_a + 4u * (uint32_t)(e + lane)));
+            k = max(k, v);
+          }
+#pragma unroll
+        for (int o = GP; o < 32 && o < C::NW * GP; o <<= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+#pragma unroll
+        for (int g = 0; g < GP; ++g) mn[g] = ord_val(__shfl_sync(0xffffffffu, k, g));
+      }
+      bool grow = false;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) grow |= mn[g] > mref[g];
+      if (grow) {   // uniform: every thread read the same maxima
+        // New reference = maximum + kHeadroom: later sub-chunks rarely exceed it, so folds
+        // stay rare.  Precision: the segment's largest p is >= 2^-kHeadroom and the
+        // fixed-point error is <= 8176 * 2^-39 = 2^-26 absolute, i.e. <= 2^(kHeadroom - 26)
+        // relative to the segment's mass.
+        float alpha[GP];
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float m2 = mn[g] > mref[g] ? mn[g] + kHeadroom : mref[g];
+          alpha[g] = mref[g] == -INFINITY ? 0.f : ex2_approx(mref[g] - m2);
+          mref[g] = m2;
+          lacc[g] *= alpha[g];
+        }
+        if (dirty) {
+          // fold the integer histograms (relative to the old maximum) into the fp32 master
+          // and rescale it to the new maximum
+          fold_tables<C, GP>(vhi, vlo, master, Sv, has_master, alpha, tid);
+          __syncthreads();
+          uint4* z = reinterpret_cast<uint4*>(vhi);
+          const int nz = 2 * kCodebook * C::VW / 4;
+          for (int f = tid; f < nz; f += kScanThreads) z[f] = make_uint4(0u, 0u, 0u, 0u);
+          has_master = true;
+          dirty = false;
         }
       }
-    }
 #pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      const float m = warp_max_f32(mloc[g]);
-      if (lane == 0) red[warp * GP + g] = m;
-    }
-    __syncthreads();
-    float mseg[GP];
-#pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      float m = red[g];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w * GP + g]);
-      mseg[g] = m;
-    }
-
-    // ---- pass 2: probabilities and value histograms
-    float lacc[GP];
-#pragma unroll
-    for (int g = 0; g < GP; ++g) lacc[g] = 0.f;
-    for (int64_t base = abase; base < s1; base += kScanSub) {
-      const int64_t t0 = base + 4 * tid;
-      Code<SKP> kc[4];
-      Code<SVP> vc[4];
-      load_codes4<SKP>(kcb, Sk, t0, s1, kc);
-      load_codes4<SVP>(vcb, Sv, t0, s1, vc);
-      __syncthreads();   // staging of the previous sub-chunk (and red) has been consumed
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t t = t0 + u;
-        const bool ok = t >= s0 && t < s1;
-        float p[GP];
+      for (int g = 0; g < GP; ++g) {
+        uint32_t hv = 0u, lv = 0u;
         if (ok) {
-          float sc[GP];
-          key_score<GP, SKP>(lut, Sk, Rk, copy, lane, kc[u], sc);
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            p[g] = ex2_approx(sc[g] - mseg[g]);
-            lacc[g] += p[g];
-          }
-        } else {
-#pragma unroll
-          for (int g = 0; g < GP; ++g) p[g] = 0.f;
+          const float pv = ex2_approx(sc[g] - mref[g]);
+          lacc[g] += pv;
+          if (g < G) split_fixed38(pv, hv, lv);
         }
-        // staging position: u * 256 + tid  ->  slot j, round k
-        const int pos = u * kScanThreads + tid;
-        const int j = pos % C::J, k = pos / C::J;
-#pragma unroll
-        for (int g = 0; g < GP; ++g) pst[(j * GP + g) * C::PR + k] = p[g];
-        if constexpr (C::CODEW == 1) {
-          cst[j * C::PR + k] = ok ? vc[u].w[0] : 0u;
-        } else {
-          reinterpret_cast<uint2*>(cst)[j * C::PR + k] =
-              ok ? make_uint2(vc[u].w[0], vc[u].w[1]) : make_uint2(0u, 0u);
-        }
+        sts32u(hst_a + 4u * (uint32_t)(g * C::PR), hv);
+        sts32u(hst_a + 4u * (uint32_t)((C::J * GP + g) * C::PR), lv);   // lo staging follows
+      }
+      if constexpr (C::CODEW == 1) {
+        sts32u(cst_a, vc.w[0]);
+      } else {
+        sts64u(cst_a, vc.w[0], vc.w[1]);
       }
       __syncthreads();
-      // value side: batches of 4 rounds, warp-strided
+      // value side: batches of 4 rounds, warp-strided.  Padded heads carry p = 0 and padded
+      // stages read code byte 0 of a stage that is never output, so no lane needs masking.
 #pragma unroll
       for (int ps = 0; ps < C::PASSES; ++ps) {
         const int combo = C::PASSES == 1 ? lane % C::COMBOS : ps * 32 + lane;
         const int vs = combo / GP, vg = combo % GP;
-        const bool active = vs < Sv && vg < G;
-        const int col = ps * 32 + lane;
-        const float* prow = pst + (vj * GP + vg) * C::PR;
-        for (int bt = warp; bt < C::ROUNDS / 4; bt += 8) {
-          const int k0 = bt * 4;
-          const float4 pv = *reinterpret_cast<const float4*>(prow + k0);
+        const uint32_t hrow = hst_base + 4u * (uint32_t)((vj * GP + vg) * C::PR);
+        const uint32_t lrow = hrow + 4u * (uint32_t)(C::J * GP * C::PR);
+        const uint32_t crow = cst_base + 4u * C::CODEW * (uint32_t)(vj * C::PR);
+        const unsigned sel = 0x4440u | (unsigned)(vs & 3);
+        const uint32_t tab = vtab_base + 4u * (uint32_t)(ps * 32 + lane);
+        for (int bt = warp; bt < C::ROUNDS / 4; bt += C::NW) {
+          const uint32_t k0b = 16u * (uint32_t)bt;   // 4 rounds of 4-byte words
+          const uint4 h4 = lds128u(hrow + k0b);
+          const uint4 l4 = lds128u(lrow + k0b);
           uint32_t cw[4];
           if constexpr (C::CODEW == 1) {
-            const uint4 c4 = *reinterpret_cast<const uint4*>(cst + vj * C::PR + k0);
+            const uint4 c4 = lds128u(crow + k0b);
             cw[0] = c4.x; cw[1] = c4.y; cw[2] = c4.z; cw[3] = c4.w;
           } else {
-            const uint4 c01 = *reinterpret_cast<const uint4*>(cst + 2 * (vj * C::PR + k0));
-            const uint4 c23 = *reinterpret_cast<const uint4*>(cst + 2 * (vj * C::PR + k0) + 4);
+            const uint4 c01 = lds128u(crow + 2u * k0b);
+            const uint4 c23 = lds128u(crow + 2u * k0b + 16u);
             const int hw = vs >> 2;
             cw[0] = hw ? c01.y : c01.x; cw[1] = hw ? c01.w : c01.z;
             cw[2] = hw ? c23.y : c23.x; cw[3] = hw ? c23.w : c23.z;
           }
-          const float pr4[4] = {pv.x, pv.y, pv.z, pv.w};
+          const uint32_t hh[4] = {h4.x, h4.y, h4.z, h4.w};
+          const uint32_t ll[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            if (!active || pr4[r] == 0.f) continue;
-            const int c = (cw[r] >> (8 * (vs & 3))) & 0xff;
-            const unsigned long long fx = __float2ull_rn(pr4[r] * 274877906944.0f);  // p * 2^38
-            red_add_u32(vhi + c * C::VW + col, (uint32_t)(fx >> 19));
-            red_add_u32(vlo + c * C::VW + col, (uint32_t)(fx & 0x7ffffull));
+            const uint32_t adr = tab + (__byte_perm(cw[r], 0u, sel) << (C::VWSH + 2));
+            red_pair<kCodebook * C::VW * 4>(adr, hh[r], ll[r]);
           }
         }
       }
+      dirty = true;
     }
-    // ---- segment partial: maximum, sum of p, histograms in float
+    // ---- segment partial: maximum, sum of p, fp32 histograms (master + integer tables)
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       const float l = warp_sum_f32(lacc[g]);
@@ -662,26 +870,20 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     if (tid < GP) {
       float l = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) l += red[w * GP + tid];
-      a.pm[slot * GP + tid] = mseg[tid];
+      for (int w = 0; w < C::NW; ++w) l += red[w * GP + tid];
+      a.pm[slot * GP + tid] = mref[tid];
       a.pl[slot * GP + tid] = l;
     }
     {
-      float* dst = a.pw + slot * (int64_t)Sv * kCodebook * GP;
-      const int n = Sv * kCodebook * GP;
-      for (int f = tid; f < n; f += kScanThreads) {
-        const int g = f % GP, c = (f / GP) % kCodebook, s = f / (GP * kCodebook);
-        const int combo = s * GP + g;
-        unsigned long long h = 0, l = 0;
+      float one[GP];
 #pragma unroll
-        for (int j = 0; j < C::J; ++j) {
-          const int col = C::PASSES == 1 ? j * C::COMBOS + combo : combo;
-          h += vhi[c * C::VW + col];
-          l += vlo[c * C::VW + col];
-        }
-        dst[f] = (float)((double)h * (1.0 / 524288.0) + (double)l * (1.0 / 274877906944.0));
-      }
+      for (int g = 0; g < GP; ++g) one[g] = 1.f;
+      fold_tables<C, GP>(vhi, vlo, master, Sv, has_master, one, tid);
     }
+    __syncthreads();
+    float4* dst = reinterpret_cast<float4*>(a.pw + slot * (int64_t)ntab);
+    const float4* srcm = reinterpret_cast<const float4*>(master);
+    for (int f = tid; f < ntab / 4; f += kScanThreads) dst[f] = srcm[f];
   }
 }
 
@@ -733,11 +935,16 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
     float acc[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) acc[g] = 0.f;
-#pragma unroll 4
-    for (int c = part; c < kCodebook; c += PARTS) {
-      const float cv = __ldg(Cs + (size_t)c * D + e);
+    constexpr int UB = 16;   // loads in flight per thread
+#pragma unroll 1
+    for (int c0 = part; c0 < kCodebook; c0 += PARTS * UB) {
+      float cv[UB];
 #pragma unroll
-      for (int g = 0; g < GP; ++g) acc[g] = fmaf(Ws[c * GP + g], cv, acc[g]);
+      for (int u = 0; u < UB; ++u) cv[u] = __ldg(Cs + (size_t)(c0 + u * PARTS) * D + e);
+#pragma unroll
+      for (int u = 0; u < UB; ++u)
+#pragma unroll
+        for (int g = 0; g < GP; ++g) acc[g] = fmaf(Ws[(c0 + u * PARTS) * GP + g], cv[u], acc[g]);
     }
     if constexpr (PARTS > 1) {
 #pragma unroll
@@ -840,7 +1047,7 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
   trace(ev, 0, st);
   {
     const size_t lut_smem = sizeof(LutSmem<D>);
-    const size_t win_smem = ((size_t)GP * D + 256 * GP + 9 * GP) * sizeof(float);
+    const size_t win_smem = ((size_t)256 * GP + 8 * GP + 8 * (size_t)GP * D) * sizeof(float);
     const size_t smem = lut_smem > win_smem ? lut_smem : win_smem;
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
@@ -898,6 +1105,7 @@ static int validate_decode_shapes(const zkv_decode_params* p) {
   if (p->Tcap < 0 || p->Wcap < 0 || p->max_comp_len < 0 || p->max_comp_len > p->Tcap)
     return ZKV_ERR_INVALID_ARG;
   if (p->Tcap % 16) return ZKV_ERR_INVALID_ARG;
+  if (p->Tcap > (int64_t(1) << 28)) return ZKV_ERR_UNSUPPORTED;   // 32-bit in-pair offsets
   return ZKV_OK;
 }
 

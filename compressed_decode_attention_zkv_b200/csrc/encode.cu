@@ -58,10 +58,12 @@ template <int D, int R>
 __global__ void __launch_bounds__(256) encode_rows_kernel(StridedRows map,
                                                           const float* __restrict__ books, int S,
                                                           double rot_scale) {
-  __shared__ RowsSmem<D, R> sm;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  RowsSmem<D, R>& sm = *reinterpret_cast<RowsSmem<D, R>*>(smem_raw);
+  float* cb = reinterpret_cast<float*>(smem_raw + ((sizeof(RowsSmem<D, R>) + 15) / 16) * 16);
   const int h = blockIdx.y;
   const int64_t row0 = (int64_t)blockIdx.x * R;
-  encode_rows_body<D, R>(map, books, S, rot_scale, row0, h, sm);
+  encode_rows_body<D, R>(map, books, S, rot_scale, row0, h, sm, cb);
   if (threadIdx.x < R) {
     const int64_t j = row0 + threadIdx.x;
     if (map.valid(j, h)) map.store(j, h, S, sm.code[threadIdx.x], sm.nrm[threadIdx.x]);
@@ -321,10 +323,14 @@ int launch_encode(const StridedRows& map, int64_t n_head, int d, int S, const fl
   if (n_rows * n_head <= 4096) {
     constexpr int R = 8;
     const dim3 grid((unsigned)((n_rows + R - 1) / R), (unsigned)n_head);
+    const bool ok = ensure_smem_limit(encode_rows_kernel<64, R>, rows_smem_bytes<64, R>()) == cudaSuccess &&
+                    ensure_smem_limit(encode_rows_kernel<128, R>, rows_smem_bytes<128, R>()) == cudaSuccess &&
+                    ensure_smem_limit(encode_rows_kernel<256, R>, rows_smem_bytes<256, R>()) == cudaSuccess;
+    if (!ok) return ZKV_ERR_CUDA;
     switch (d) {
-      case 64: encode_rows_kernel<64, R><<<grid, 256, 0, st>>>(map, books, S, rot); break;
-      case 128: encode_rows_kernel<128, R><<<grid, 256, 0, st>>>(map, books, S, rot); break;
-      case 256: encode_rows_kernel<256, R><<<grid, 256, 0, st>>>(map, books, S, rot); break;
+      case 64: encode_rows_kernel<64, R><<<grid, 256, rows_smem_bytes<64, R>(), st>>>(map, books, S, rot); break;
+      case 128: encode_rows_kernel<128, R><<<grid, 256, rows_smem_bytes<128, R>(), st>>>(map, books, S, rot); break;
+      case 256: encode_rows_kernel<256, R><<<grid, 256, rows_smem_bytes<256, R>(), st>>>(map, books, S, rot); break;
     }
   } else {
     const bool ok = ensure_smem_limit(encode_tile_kernel<64>, sizeof(TileSmem<64>)) == cudaSuccess &&

@@ -20,7 +20,10 @@ __device__ __forceinline__ double candidate_margin(double rnorm, float cn_max, i
 // ------------------------------------------------------------------------------------------
 // Row-group encoder: R rows of one head per CTA, thread c owns codeword c (256 threads).
 // Used for small batches (window evictions, short prefills): few rows, latency matters more
-// than codebook reuse.
+// than codebook reuse.  Each stage's codebook is staged through shared memory in slices of
+// KC dims with cp.async (all requests in flight at once).  Slice layout: codeword c's 16-byte
+// piece q is stored at position q ^ (c & 7), so the 8 lanes of a 128-bit read phase (8
+// consecutive codewords, same q) hit 8 distinct bank groups; the row operands are broadcasts.
 // ------------------------------------------------------------------------------------------
 template <int D, int R>
 struct RowsSmem {
@@ -36,11 +39,34 @@ struct RowsSmem {
   float nrm[R][kMaxStages];
 };
 
+template <int D>
+struct RowsSlice {
+  static constexpr int KC = D < 128 ? D : 128;   // dims per staged slice
+};
+
+template <int D, int R>
+constexpr size_t rows_smem_bytes() {
+  return ((sizeof(RowsSmem<D, R>) + 15) / 16) * 16 +
+         (size_t)kCodebook * RowsSlice<D>::KC * sizeof(float);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (unsigned)__cvta_generic_to_shared(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 template <int D, int R, class Map>
 __device__ __forceinline__ void encode_rows_body(const Map& map, const float* __restrict__ books,
                                                  int S, double rot_scale, int64_t row0, int h,
-                                                 RowsSmem<D, R>& sm) {
+                                                 RowsSmem<D, R>& sm, float* cb) {
   constexpr int E = D / 32;
+  constexpr int KC = RowsSlice<D>::KC;
+  constexpr int NQ = KC / 4;           // 16-byte pieces per codeword slice
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (warp < R) {
@@ -67,30 +93,39 @@ __device__ __forceinline__ void encode_rows_body(const Map& map, const float* __
     ss = warp_sum_f64(ss);
     if (lane == 0) sm.rn[warp] = sqrt(ss);
   }
-  __syncthreads();
 
   const float* CB = books + (size_t)h * S * kCodebook * D;
   for (int s = 0; s < S; ++s) {
     const float* C = CB + (size_t)s * kCodebook * D;
-    const float* crow = C + (size_t)tid * D;
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
     float cn = 0.f;
-#pragma unroll 2
-    for (int i = 0; i < D; i += 4) {
-      const float4 c4 = __ldg(reinterpret_cast<const float4*>(crow + i));
-      cn = fmaf(c4.x, c4.x, cn);
-      cn = fmaf(c4.y, c4.y, cn);
-      cn = fmaf(c4.z, c4.z, cn);
-      cn = fmaf(c4.w, c4.w, cn);
+    for (int k0 = 0; k0 < D; k0 += KC) {
+      __syncthreads();   // previous slice (and the rows) are ready / consumed
+      for (int f = tid; f < kCodebook * NQ; f += 256) {
+        const int c = f / NQ, q = f % NQ;
+        cp_async16(cb + c * KC + 4 * (q ^ (c & 7)), C + (size_t)c * D + k0 + 4 * q);
+      }
+      cp_async_wait_all();
+      __syncthreads();
+      const float* row = cb + tid * KC;
+      const int sw = tid & 7;
+#pragma unroll 4
+      for (int q = 0; q < NQ; ++q) {
+        const float4 c4 = *reinterpret_cast<const float4*>(row + 4 * (q ^ sw));
+        cn = fmaf(c4.x, c4.x, cn);
+        cn = fmaf(c4.y, c4.y, cn);
+        cn = fmaf(c4.z, c4.z, cn);
+        cn = fmaf(c4.w, c4.w, cn);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float4 x4 = *reinterpret_cast<const float4*>(&sm.r[r][i]);
-        acc[r] = fmaf(x4.x, c4.x, acc[r]);
-        acc[r] = fmaf(x4.y, c4.y, acc[r]);
-        acc[r] = fmaf(x4.z, c4.z, acc[r]);
-        acc[r] = fmaf(x4.w, c4.w, acc[r]);
+        for (int r = 0; r < R; ++r) {
+          const float4 x4 = *reinterpret_cast<const float4*>(&sm.r[r][k0 + 4 * q]);
+          acc[r] = fmaf(x4.x, c4.x, acc[r]);
+          acc[r] = fmaf(x4.y, c4.y, acc[r]);
+          acc[r] = fmaf(x4.z, c4.z, acc[r]);
+          acc[r] = fmaf(x4.w, c4.w, acc[r]);
+        }
       }
     }
     float dist[R];
@@ -175,8 +210,9 @@ __device__ __forceinline__ void encode_rows_body(const Map& map, const float* __
         sm.nrm[warp][s] = (float)nn;
       }
     }
-    __syncthreads();
+    // the next stage's first __syncthreads orders these writes before their use
   }
+  __syncthreads();
 }
 
 }  // namespace zkv
