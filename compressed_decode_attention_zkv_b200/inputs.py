@@ -245,12 +245,18 @@ def _kmeans_zero_pinned(X: np.ndarray, K: int, iters: int,
                         rng: np.random.Generator) -> tuple[np.ndarray, np.ndarray]:
     """Lloyd k-means with codeword 0 held at the zero vector.
 
-    Init: K-1 distinct samples chosen by ``rng``.  Empty clusters keep their centroid.
+    Init: K-1 samples chosen by ``rng`` among the distinct nonzero rows of X (residual stages
+    contain exact zeros where an earlier centroid was a single sample; seeding from those would
+    create duplicate zero codewords).  Empty clusters keep their centroid.
     Returns (centroids float32 [K][d], final assignment int64 [n]).
     """
     n, d = X.shape
     C = np.zeros((K, d), np.float32)
-    C[1:] = X[rng.choice(n, K - 1, replace=False)]
+    nz = np.nonzero(np.any(X != 0, axis=1))[0]
+    _, first = np.unique(X[nz], axis=0, return_index=True)
+    pool = nz[np.sort(first)]
+    pick = rng.choice(pool, min(K - 1, len(pool)), replace=False)
+    C[1:1 + len(pick)] = X[pick]
 
     def assign(C):
         score = (C.astype(np.float32) ** 2).sum(1)[None, :] - 2.0 * (X @ C.T)
