@@ -167,7 +167,9 @@ __device__ __forceinline__ void encode_rows_body(const Map& map, const float* __
 #pragma unroll
       for (int q = 0; q < E; ++q) {
         const int i = q * 32 + lane;
-        const double df = (double)sm.r[r][i] - (double)__ldg(cw + i);
+        // the staged slice holds the whole codeword when KC == D (swizzled 16-byte pieces)
+        const float cv = KC == D ? cb[c * KC + 4 * ((i >> 2) ^ (c & 7)) + (i & 3)] : __ldg(cw + i);
+        const double df = (double)sm.r[r][i] - (double)cv;
         a = fma(df, df, a);
       }
       a = warp_sum_f64(a);
