@@ -1171,3 +1171,49 @@ extern "C" int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace,
     default: return launch_decode_g<256>(a, pl, p->trace_events, st);
   }
 }
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free variant: the workspace is a fixed module-scope device array.
+//
+// For callers that cannot hand the library a device buffer: a host program that links only
+// this library and the CUDA runtime and keeps no device allocator of its own, or an engine
+// that reserves all of its device memory up front and has no pool to carve a per-call
+// workspace from.  Such callers get one resident array of ZKV_DECODE_SCRATCH_BYTES per device
+// (allocated by the driver when the module loads) instead of a buffer they own.
+//
+// Nothing in the array has to start at zero: every word a call reads is written earlier in
+// the same call (the first kernel clears the completion counters).  There is one array per
+// device, so calls on one device that overlap in time (two streams, two host threads) race
+// on it; the caller orders them.
+// ------------------------------------------------------------------------------------------
+namespace zkv {
+
+static __device__ __align__(256) unsigned char g_decode_scratch[ZKV_DECODE_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_scratch_mu;
+static void* g_scratch_addr[kMaxDevices];
+
+// Device address of g_decode_scratch on the current device, looked up once per device.
+static void* decode_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_decode_scratch) != cudaSuccess) return nullptr;
+    g_scratch_addr[dev] = a;
+  }
+  return g_scratch_addr[dev];
+}
+
+}  // namespace zkv
+
+extern "C" int zkv_rvq_decode_attn_noalloc(const zkv_decode_params* p, void* stream) {
+  const int v = validate_decode(p);
+  if (v != ZKV_OK) return v;
+  if (make_plan(p).total > (size_t)ZKV_DECODE_SCRATCH_BYTES) return ZKV_ERR_WORKSPACE;
+  void* ws = decode_scratch_address();
+  if (!ws) return ZKV_ERR_CUDA;
+  return zkv_rvq_decode_attn(p, ws, (size_t)ZKV_DECODE_SCRATCH_BYTES, stream);
+}

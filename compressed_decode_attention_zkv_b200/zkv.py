@@ -5,7 +5,8 @@ current CUDA stream.  If the library is missing or a call fails, an exception is
 is no fallback path.
 
 Entry points (same names as the C ABI):
-  fwht, rvq_encode, rvq_reconstruct, decode_workspace_size, rvq_decode_attn, rvq_append
+  fwht, rvq_encode, rvq_reconstruct, decode_workspace_size, rvq_decode_attn,
+  rvq_decode_attn_noalloc, rvq_append
 plus ``RVQKVCache``, a small owner of one layer's compressed cache built on them
 (prefill -> append -> attend, the append/attend cache interface of the VeloxQuant-MLX page).
 """
@@ -26,11 +27,13 @@ ZKV_DEVERR_COMP_LEN = 1
 ZKV_DEVERR_WIN_LEN = 2
 ZKV_DTYPE_F16, ZKV_DTYPE_F32 = 0, 1
 CODEBOOK_SIZE = 256
+DECODE_SCRATCH_BYTES = 8 << 20   # ZKV_DECODE_SCRATCH_BYTES: the no-allocation decode's array
 
 
 class ZkvError(RuntimeError):
-    def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})"
+                         + (f": {detail}" if detail else ""))
         self.status = status
 
 
@@ -95,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.zkv_decode_workspace_size.argtypes = [POINTER(DecodeParams)]
         L.zkv_rvq_decode_attn.restype = c_int
         L.zkv_rvq_decode_attn.argtypes = [POINTER(DecodeParams), c_void_p, c_size_t, c_void_p]
+        L.zkv_rvq_decode_attn_noalloc.restype = c_int
+        L.zkv_rvq_decode_attn_noalloc.argtypes = [POINTER(DecodeParams), c_void_p]
         L.zkv_rvq_append.restype = c_int
         L.zkv_rvq_append.argtypes = [POINTER(AppendParams), c_void_p]
         _lib = L
@@ -288,6 +293,29 @@ def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win
     _check("zkv_rvq_decode_attn",
            lib().zkv_rvq_decode_attn(ctypes.byref(p), _ptr(workspace), workspace.numel(),
                                      _stream()))
+    return out, lse
+
+
+def rvq_decode_attn_noalloc(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
+                            win_v, win_len, out=None, lse=None, max_comp_len=None,
+                            softmax_scale=None, error_flag=None):
+    """rvq_decode_attn with the library's fixed device scratch array as workspace
+    (zkv_rvq_decode_attn_noalloc).  Calls on one device must not overlap in time.  Raises
+    ZkvError(ZKV_ERR_WORKSPACE) when the shapes need more than DECODE_SCRATCH_BYTES."""
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
+                       win_len, out, lse, max_comp_len, softmax_scale, error_flag)
+    status = lib().zkv_rvq_decode_attn_noalloc(ctypes.byref(p), _stream())
+    if status == ZKV_ERR_WORKSPACE:
+        need = lib().zkv_decode_workspace_size(ctypes.byref(p))
+        raise ZkvError("zkv_rvq_decode_attn_noalloc", status,
+                       f"these shapes need {need} bytes of workspace; the library's scratch "
+                       f"array holds {DECODE_SCRATCH_BYTES}; use rvq_decode_attn")
+    _check("zkv_rvq_decode_attn_noalloc", status)
     return out, lse
 
 

@@ -195,6 +195,29 @@ int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace, size_t work
                         void* stream);
 
 /*
+ * zkv_rvq_decode_attn_noalloc -- zkv_rvq_decode_attn without a caller workspace.  The web
+ * pages have no counterpart: this is a library convenience for callers that cannot allocate
+ * device memory per call (a host program with no device allocator of its own, or an engine
+ * whose device memory is fully reserved up front).
+ * Computes exactly what zkv_rvq_decode_attn computes, with the same parameters, layouts and
+ * errors, using as workspace a device array inside this library of ZKV_DECODE_SCRATCH_BYTES
+ * bytes (one per device, allocated when the library's device code is loaded; nothing is
+ * allocated or freed by the call).
+ *   - A call whose zkv_decode_workspace_size(p) exceeds ZKV_DECODE_SCRATCH_BYTES returns
+ *     ZKV_ERR_WORKSPACE and launches nothing (8 x 32K-token GQA batches need about 5 MiB;
+ *     64 sequences x 16K tokens need about 30 MiB and are refused).
+ *   - Nothing in the array must start at zero: each call writes every word it reads.
+ *   - There is ONE array per device: calls on the same device that overlap in time (different
+ *     streams or host threads) race on it and give wrong results.  Order them (same stream,
+ *     or events).  Calls on different devices do not interact.
+ *   - The first call on each device looks up the array's device address (once) and sets
+ *     kernel attributes; make that first call before any stream capture.
+ * Errors: as zkv_rvq_decode_attn; ZKV_ERR_CUDA if the array's address cannot be obtained.
+ */
+#define ZKV_DECODE_SCRATCH_BYTES (8u << 20)
+int zkv_rvq_decode_attn_noalloc(const zkv_decode_params* p, void* stream);
+
+/*
  * zkv_rvq_append -- one serving step of cache maintenance: each sequence's new token enters
  * the fp16 window; when the window is full, its oldest token is evicted, RVQ-encoded (same
  * rule as zkv_rvq_encode, rotate = 1) and appended to the compressed prefix.
