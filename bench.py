@@ -37,7 +37,10 @@ WORKLOAD = "llama3_8b_32k"
 
 # DRAM traffic of one scan-kernel launch from an ncu capture (see profiles/), valid only while
 # the scan kernel source is unchanged (hash of decode.cu at capture time).
-SCAN_TRAFFIC = {"decode_cu_sha1": None, "bytes_per_launch": None}
+# DRAM bytes (read + write) of one scan_kernel launch on this workload, from one ncu capture
+# (profiles/scan_kernel_llama3_8b_32k.md), valid while the scan's source is unchanged.
+SCAN_TRAFFIC = {"scan_src_sha1": "37851bd740c0e6e896734acff1aad85385092be5",
+                "bytes_per_launch": 17798144}
 
 
 def parse():
@@ -270,6 +273,17 @@ def run_reference(args):
 # Our implementation
 # --------------------------------------------------------------------------------------------
 
+def scan_src_sha1():
+    """sha1 of the parts of decode.cu the scan kernel is built from: the shared constants and
+    launch plan (up to the lookup-table section), the scan section, and the launchers."""
+    text = open(os.path.join(ROOT, "compressed_decode_attention_zkv_b200", "csrc",
+                             "decode.cu")).read()
+    head = text.split("// 1. Query rotation")[0]
+    scan = text.split("// 2. Scan of the compressed tokens.")[1].split("// 3. Merge:")[0]
+    launch = text.split("// Launch\n")[1].split("// Shapes only")[0]
+    return hashlib.sha1((head + scan + launch).encode()).hexdigest()
+
+
 def sha1_of(path):
     with open(path, "rb") as f:
         return hashlib.sha1(f.read()).hexdigest()
@@ -470,14 +484,15 @@ def run_ours(args):
     per = {"append": t_append, "lut": t_lut, "scan": t_scan, "merge": t_merge}
     dominant = max(per, key=lambda k: per[k] if per[k] == per[k] else -1)
     Tc_avg = tokens / (wl.B * args.steps)
-    # algorithmic bytes (counted once per distinct byte)
-    scan_bytes = wl.B * wl.Hkv * (Tc_avg * (wl.Sk + wl.Sv) + wl.W * wl.d * 2 * 2)
-    call_bytes = (scan_bytes + wl.Hkv * (wl.Sk + wl.Sv) * 256 * wl.d * 4
+    # algorithmic bytes (counted once per distinct byte).  The scan kernel reads the codes of
+    # every compressed token: (Sk + Sv) bytes per (token, kv head).
+    scan_bytes = wl.B * wl.Hkv * Tc_avg * (wl.Sk + wl.Sv)
+    call_bytes = (scan_bytes + wl.B * wl.Hkv * wl.W * wl.d * 2 * 2
+                  + wl.Hkv * (wl.Sk + wl.Sv) * 256 * wl.d * 4
                   + wl.B * wl.Hq * wl.d * 2 + wl.B * wl.Hq * (wl.d + 1) * 4)
     decode_time = t_lut + t_scan + t_merge
-    src_hash = sha1_of(os.path.join(ROOT, "compressed_decode_attention_zkv_b200", "csrc", "decode.cu"))
     traffic = (SCAN_TRAFFIC["bytes_per_launch"]
-               if SCAN_TRAFFIC["decode_cu_sha1"] == src_hash else None)
+               if SCAN_TRAFFIC["scan_src_sha1"] == scan_src_sha1() else None)
     roof = {"bound": "hbm", "kernel": "scan_kernel", "achieved": scan_bytes / t_scan / 1e9,
             "peak": hbm_peak, "unit": "GB/s", "frac": scan_bytes / t_scan / 1e9 / hbm_peak,
             "traffic": traffic, "peak_kind": f"{peak_kind} (hbm_gbs copy, burst)",
