@@ -562,7 +562,7 @@ def run_ours(args):
                        "l2": f"{R} rotating replicas x {rep_mb:.1f} MB = {R * rep_mb:.0f} MB > 126 MB L2",
                        "parallelism": f"replicas x{world}, no collective",
                        "graph": "one CUDA graph per replica step"},
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": 6 * args.steps,   # append (2), lut, scan, merge, finalize
             "roofline": roof,
             "kernels_s": per,
             "decode_call": {"seconds": decode_time, "algorithmic_bytes": call_bytes,

@@ -7,22 +7,23 @@
 // q . k).  Differential-KV README, "Decode & Prefill Innovations": flash-style fp32
 // log-sum-exp combine of the compressed part with the dense recency window.
 //
-// Three kernels per call:
+// Four kernels per call:
 //   1. lut_kernel    q_tilde = H q / sqrt(d) (float64, one rounding), per stage
 //                    LUT_s[c] = (scale * log2 e) * q_tilde . Ck_s[c] -> workspace; the dense
 //                    window attention of every (sequence, kv head); prefix sums of the
 //                    compressed lengths that partition the token space among scan CTAs.
 //   2. scan_kernel   one CTA per SM walks a contiguous range of the concatenated compressed
-//                    tokens of all (sequence, kv head) pairs.  Per pair segment: pass 1 takes
-//                    score_t = sum_s LUT_s[zk_{t,s}] (base-2 logits) and their maximum m; pass 2
-//                    recomputes the scores, p_t = 2^(score_t - m), and accumulates per-stage
-//                    codeword weight histograms W_s[c] = sum over tokens with zv_{t,s} = c of p_t.
+//                    tokens of all (sequence, kv head) pairs.  Per pair segment it takes
+//                    score_t = sum_s LUT_s[zk_{t,s}] (base-2 logits), keeps a running reference
+//                    maximum m, and accumulates p_t = 2^(score_t - m) into per-stage codeword
+//                    weight histograms W_s[c] = sum over tokens with zv_{t,s} = c of p_t.
 //                    sum_t p_t sum_s Cv_s[zv_{t,s}] = sum_s sum_c W_s[c] Cv_s[c]: the value
 //                    reconstruction regrouped by codeword.
-//   3. merge_kernel  grid (value stage, kv head, sequence): merges the segment histograms by
-//                    their maxima, contracts W_s with Cv_s, and the last stage CTA of each
-//                    (sequence, kv head) sums the stages, rotates back, and merges with the
-//                    window by log-sum-exp.  "Last CTA" is an atomic ticket; no CTA waits.
+//   3. merge_kernel  grid (codeword quarter, value stage, kv head): merges the segment
+//                    histograms by their maxima and contracts W_s with its Cv_s codewords for
+//                    every sequence (Cv_s is read once per call).
+//   4. finalize_kernel  one block per (sequence, kv head): sums the partials, rotates back, and
+//                    merges with the window by log-sum-exp.
 //
 // Shared-memory design of the scan (shared memory bandwidth, not HBM, bounds this kernel):
 //  * key tables are replicated per lane group so that the 8 (or 16, 32) lanes of a 128-bit
@@ -44,6 +45,9 @@ constexpr int kScanSub = 512;       // tokens per scan sub-chunk (1 per thread)
 constexpr int kScanThreads = 512;
 constexpr int kColCap = 8176;       // tokens per histogram column per segment (sum < 2^32)
 constexpr float kHeadroom = 8.f;    // log2 units added to the running maximum on growth
+constexpr int kMergeQ = 4;          // codeword quarters (64 codewords each) per value stage
+constexpr int kMergeC = kCodebook / kMergeQ;
+constexpr int kMergeRows = 32;      // (sequence, head) rows per merge pass
 constexpr size_t kSmemMax = 227 * 1024;
 
 static int sm_count() {
@@ -81,7 +85,7 @@ struct DecodePlan {
   int64_t cap, slots;
   size_t scan_smem;
   size_t off_lut, off_pre, off_share, off_pm, off_pl, off_pw, off_wm, off_wl, off_wo, off_so,
-      off_cnt, total;
+      total;
 };
 
 static size_t scan_smem_bytes(int Rk, int Sk, int Sv, int GP, const VMap& v) {
@@ -127,8 +131,7 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   pl.off_wm = o;    o = align256(o + (size_t)pairs * pl.GP * f);
   pl.off_wl = o;    o = align256(o + (size_t)pairs * pl.GP * f);
   pl.off_wo = o;    o = align256(o + (size_t)pairs * pl.GP * p->d * f);
-  pl.off_so = o;    o = align256(o + (size_t)pairs * p->Sv * pl.GP * p->d * f);
-  pl.off_cnt = o;   o = align256(o + (size_t)pairs * sizeof(unsigned));
+  pl.off_so = o;    o = align256(o + (size_t)pairs * p->Sv * kMergeQ * pl.GP * p->d * f);
   pl.total = o;
   return pl;
 }
@@ -159,8 +162,7 @@ struct DecodeArgs {
   float* wm;         // [B*Hkv][GP]
   float* wl;         // [B*Hkv][GP]
   float* wo;         // [B*Hkv][GP][d]
-  float* so;         // [B*Hkv][Sv][GP][d]
-  unsigned* cnt;     // [B*Hkv]
+  float* so;         // [B*Hkv][Sv][kMergeQ][GP][d] partial stage outputs
 };
 
 __device__ __forceinline__ int64_t clamp_win_len(const DecodeArgs& a, int b) {
@@ -182,7 +184,7 @@ constexpr int kLutH = 32;     // attached query heads per block (b * G + g)
 template <int D>
 struct LutSmem {
   float qT[D][kLutH + 4];     // rotated queries, k-major
-  float cT[D][kLutC + 1];     // codebook slice, k-major
+  float cb[kLutC * D];        // codebook slice, row-major; 16-byte piece q of codeword c at q ^ (c & 7)
 };
 
 // Ask the memory system to stage [p, p + bytes) in L2 (no data returned to the SM).  p and
@@ -201,17 +203,41 @@ __device__ __forceinline__ void prefetch_l2(const uint8_t* lo, const uint8_t* hi
 }
 
 // Dense attention of the GP heads of one (sequence, kv head) over its fp16 window (base-2
-// logits, online maximum over 256-token tiles).  Warps take tokens, lanes split the head
-// dimension, so every load is an independent coalesced row fragment.
+// logits, online maximum over tiles).  Each tile's K and V rows are copied to shared memory
+// with cp.async in one round (64 KB); warps then take tokens and lanes split the head
+// dimension.
+template <int D>
+constexpr int win_tile() { return 16384 / D; }   // tokens per tile: K + V tiles = 64 KB
+
 template <int D, int GP>
-__device__ void window_item(const DecodeArgs& a, int b, int kvh, float* smem) {
+constexpr size_t window_smem_bytes() {
+  return (size_t)2 * win_tile<D>() * D * sizeof(__half) + (size_t)win_tile<D>() * GP * 4 +
+         (size_t)8 * GP * 4;
+}
+
+template <int D, int GP>
+__device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* smem) {
   constexpr int PL = D / 32;        // head dims per lane
-  float* sc = smem;                 // [256][GP] scores, then probabilities, of the tile
-  float* red = sc + 256 * GP;       // [8][GP]
-  float* part = red + 8 * GP;       // [8][GP][D] per-warp partial outputs
+  constexpr int WT = win_tile<D>();
+  __half* kt = reinterpret_cast<__half*>(smem);                     // [WT][D]
+  __half* vt = kt + WT * D;                                         // [WT][D]
+  float* sc = reinterpret_cast<float*>(vt + WT * D);                // [WT][GP] scores, then p
+  float* red = sc + WT * GP;                                        // [8][GP]
+  float* part = reinterpret_cast<float*>(smem);                     // [8][GP][D], after the tiles
+  static_assert((size_t)8 * GP * D * 4 <= (size_t)2 * WT * D * 2, "partials fit in the tiles");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pair = (int64_t)b * a.Hkv + kvh;
   const int64_t wl = clamp_win_len(a, b);
+  const __half* Kb = a.win_k + pair * a.Wcap * D;
+  const __half* Vb = a.win_v + pair * a.Wcap * D;
+  auto stage = [&](int64_t base) {   // rows [base, base + n) as 16-byte pieces
+    const int n = (int)(wl - base < WT ? wl - base : WT);
+    for (int f = tid; f < n * D / 8; f += 256) {
+      cp_async16(kt + f * 8, Kb + base * D + f * 8);
+      cp_async16(vt + f * 8, Vb + base * D + f * 8);
+    }
+  };
+  if (wl > 0) stage(0);   // in flight while the query is loaded
   float qf[GP][PL];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
@@ -228,14 +254,15 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, float* smem) {
 #pragma unroll
     for (int e = 0; e < PL; ++e) acc[g][e] = 0.f;
   }
-  const __half* Kb = a.win_k + pair * a.Wcap * D;
-  const __half* Vb = a.win_v + pair * a.Wcap * D;
-  for (int64_t base = 0; base < wl; base += 256) {
-    const int n = (int)(wl - base < 256 ? wl - base : 256);
+  for (int64_t base = 0; base < wl; base += WT) {
+    const int n = (int)(wl - base < WT ? wl - base : WT);
+    if (base > 0) stage(base);
+    cp_async_wait_all();
+    __syncthreads();
     // scores
 #pragma unroll 2
     for (int tt = warp; tt < n; tt += 8) {
-      const __half* kr = Kb + (base + tt) * D + lane * PL;
+      const __half* kr = kt + tt * D + lane * PL;
       float kf[PL];
 #pragma unroll
       for (int e = 0; e < PL; e += 2) {
@@ -257,30 +284,30 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, float* smem) {
     float mt[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
-      const float v = tid < n ? sc[tid * GP + g] : -INFINITY;
+      float v = -INFINITY;
+      for (int t2 = tid; t2 < n; t2 += 256) v = fmaxf(v, sc[t2 * GP + g]);
       const float m = warp_max_f32(v);
       if (lane == 0) red[warp * GP + g] = m;
     }
     __syncthreads();
-    float alpha[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       float m = red[g];
 #pragma unroll
       for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w * GP + g]);
       const float mn = fmaxf(m_run[g], m);
-      alpha[g] = m_run[g] == -INFINITY ? 0.f : ex2_approx(m_run[g] - mn);
+      const float alpha = m_run[g] == -INFINITY ? 0.f : ex2_approx(m_run[g] - mn);
       m_run[g] = mn;
       mt[g] = mn;
-      l_run[g] *= alpha[g];
+      l_run[g] *= alpha;
 #pragma unroll
-      for (int e = 0; e < PL; ++e) acc[g][e] *= alpha[g];
+      for (int e = 0; e < PL; ++e) acc[g][e] *= alpha;
     }
-    if (tid < n) {
+    for (int t2 = tid; t2 < n; t2 += 256) {
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
-        const float pv = ex2_approx(sc[tid * GP + g] - mt[g]);
-        sc[tid * GP + g] = pv;
+        const float pv = ex2_approx(sc[t2 * GP + g] - mt[g]);
+        sc[t2 * GP + g] = pv;
         l_run[g] += pv;
       }
     }
@@ -288,7 +315,7 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, float* smem) {
     // values
 #pragma unroll 2
     for (int tt = warp; tt < n; tt += 8) {
-      const __half* vr = Vb + (base + tt) * D + lane * PL;
+      const __half* vr = vt + tt * D + lane * PL;
       float vf[PL];
 #pragma unroll
       for (int e = 0; e < PL; e += 2) {
@@ -303,7 +330,7 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, float* smem) {
         for (int e = 0; e < PL; ++e) acc[g][e] = fmaf(pv, vf[e], acc[g][e]);
       }
     }
-    __syncthreads();   // sc is rewritten by the next tile
+    __syncthreads();   // the tiles and sc are rewritten by the next tile (or by part below)
   }
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
@@ -334,7 +361,7 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if ((int)blockIdx.x >= a.n_lut_blocks) {
     const int pair = blockIdx.x - a.n_lut_blocks;
-    window_item<D, GP>(a, pair / a.Hkv, pair % a.Hkv, reinterpret_cast<float*>(smem_raw));
+    window_item<D, GP>(a, pair / a.Hkv, pair % a.Hkv, smem_raw);
     return;
   }
   if (blockIdx.x == 0) {
@@ -342,7 +369,6 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
     __shared__ int64_t warp_tot[8];
     __shared__ int64_t carry_s;
     const int npairs = a.B * a.Hkv;
-    for (int i = tid; i < npairs; i += blockDim.x) a.cnt[i] = 0u;
     if (tid == 0) {
       carry_s = 0;
       a.pre[0] = 0;
@@ -398,50 +424,67 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
   const int hg = rest % n_hg;
   const int kvh = rest / n_hg;
   const int c0 = cblk * kLutC;
-  // rotated queries of the attached heads j = b*G + g
-  for (int jl = warp; jl < kLutH; jl += 8) {
-    const int j = hg * kLutH + jl;
-    double v[E];
-    if (j < a.B * a.G) {
-      const int b = j / a.G, g = j % a.G;
-      const int64_t off = ((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D;
-      load_row_f64<E>(a.q, ZKV_DTYPE_F16, off, lane, v);
-      fwht_warp_f64<D>(v, lane);
+  // codebook slice C[kvh][s][c0 .. c0+63][:] -> shared memory, in flight during the rotation
+  {
+    const float* C = a.Ck + (((size_t)kvh * a.Sk + s) * kCodebook + c0) * D;
+    for (int f = tid; f < kLutC * D / 4; f += 256) {
+      const int c = f / (D / 4), qq = f % (D / 4);
+      cp_async16(sm.cb + c * D + 4 * (qq ^ (c & 7)), C + (size_t)c * D + 4 * qq);
+    }
+    cp_async_commit();
+  }
+  // rotated queries of the attached heads j = b*G + g: this warp's rows are loaded first
+  // (independent loads), then transformed
+  {
+    constexpr int NR = kLutH / 8;
+    double v[NR][E];
 #pragma unroll
-      for (int q = 0; q < E; ++q) sm.qT[q * 32 + lane][jl] = (float)(v[q] * a.rot);
-    } else {
+    for (int k = 0; k < NR; ++k) {
+      const int j = hg * kLutH + warp + 8 * k;
+      if (j < a.B * a.G) {
+        const int b = j / a.G, g = j % a.G;
+        const int64_t off = ((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D;
+        load_row_f64<E>(a.q, ZKV_DTYPE_F16, off, lane, v[k]);
+      } else {
 #pragma unroll
-      for (int q = 0; q < E; ++q) sm.qT[q * 32 + lane][jl] = 0.f;
+        for (int q = 0; q < E; ++q) v[k][q] = 0.0;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      fwht_warp_f64<D>(v[k], lane);
+#pragma unroll
+      for (int q = 0; q < E; ++q) sm.qT[q * 32 + lane][warp + 8 * k] = (float)(v[k][q] * a.rot);
     }
   }
-  // codebook slice C[kvh][s][c0 .. c0+63][:]
-  const float* C = a.Ck + (((size_t)kvh * a.Sk + s) * kCodebook + c0) * D;
-  for (int f = tid; f < kLutC * D / 4; f += 256) {
-    const int c = f / (D / 4), i = (f % (D / 4)) * 4;
-    const float4 v = __ldg(reinterpret_cast<const float4*>(C + (size_t)c * D + i));
-    sm.cT[i + 0][c] = v.x;
-    sm.cT[i + 1][c] = v.y;
-    sm.cT[i + 2][c] = v.z;
-    sm.cT[i + 3][c] = v.w;
-  }
+  cp_async_wait_all();
   __syncthreads();
+  // thread (codeword cc, head group hq): 8 dot products; the codeword is read as 16-byte
+  // pieces (conflict-free thanks to the swizzle), the query columns are broadcasts
   const int cc = tid & (kLutC - 1), hq = tid >> 6;   // 4 groups of 8 heads
+  const float* row = sm.cb + cc * D;
+  const int sw = cc & 7;
   float acc[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < D; ++i) {
-    const float cv = sm.cT[i][cc];
-    const float4 q0 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8]);
-    const float4 q1 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8 + 4]);
-    acc[0] = fmaf(q0.x, cv, acc[0]);
-    acc[1] = fmaf(q0.y, cv, acc[1]);
-    acc[2] = fmaf(q0.z, cv, acc[2]);
-    acc[3] = fmaf(q0.w, cv, acc[3]);
-    acc[4] = fmaf(q1.x, cv, acc[4]);
-    acc[5] = fmaf(q1.y, cv, acc[5]);
-    acc[6] = fmaf(q1.z, cv, acc[6]);
-    acc[7] = fmaf(q1.w, cv, acc[7]);
+#pragma unroll 2
+  for (int qq = 0; qq < D / 4; ++qq) {
+    const float4 c4 = *reinterpret_cast<const float4*>(row + 4 * (qq ^ sw));
+    const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = 4 * qq + e;
+      const float4 q0 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8]);
+      const float4 q1 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8 + 4]);
+      acc[0] = fmaf(q0.x, cv[e], acc[0]);
+      acc[1] = fmaf(q0.y, cv[e], acc[1]);
+      acc[2] = fmaf(q0.z, cv[e], acc[2]);
+      acc[3] = fmaf(q0.w, cv[e], acc[3]);
+      acc[4] = fmaf(q1.x, cv[e], acc[4]);
+      acc[5] = fmaf(q1.y, cv[e], acc[5]);
+      acc[6] = fmaf(q1.z, cv[e], acc[6]);
+      acc[7] = fmaf(q1.w, cv[e], acc[7]);
+    }
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -888,106 +931,215 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------------------------------
-// 3. Merge: segment histograms -> W_s, contraction with Cv_s, stage sum, rotation back,
-//    log-sum-exp merge with the window.  grid (Sv, Hkv, B); 256 threads.
+// 3. Merge: segment histograms -> W_s, contraction with Cv_s, then (finalize) stage sum,
+//    rotation back, log-sum-exp merge with the window.
 // ------------------------------------------------------------------------------------------
+
+// Scan segments (slots) of a pair: scan CTA c covers the pair's tokens iff first <= c <= last;
+// its partial is in slot pair + c.
+__device__ __forceinline__ void pair_slots(const DecodeArgs& a, int64_t pair, int64_t share,
+                                           int64_t& first, int64_t& last) {
+  const int64_t p0 = a.pre[pair], p1 = a.pre[pair + 1];
+  first = p1 > p0 ? p0 / share : 1;
+  last = p1 > p0 ? (p1 - 1) / share : 0;
+}
+
+// grid (codeword quarter, value stage, kv head), 256 threads.  The block copies its 64
+// codewords of Cv_s once and, 32 (sequence, head) rows at a time, merges the segment
+// histograms of those codewords by their maxima (W_s[c] = sum over slots of
+// 2^(m_slot - m*) W_slot[c]) and contracts them: so[pair][s][quarter][g][:] =
+// sum_c W_s[c][g] Cv_s[c][:].  Each row's slot range, maximum m* and first kMergeW slot
+// weights are tabulated once, so the weight sums are runs of independent loads.
+constexpr int kMergeW = 32;   // slot weights tabulated per row
+
 template <int D, int GP>
 __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
-  constexpr int E = D / 32;
-  constexpr int PARTS = 256 / D;   // threads per output element
+  constexpr int TG = 256 / D;               // thread groups (one column e per thread)
+  constexpr int RPT = kMergeRows / TG;      // rows per thread
   extern __shared__ __align__(16) float sm[];
-  float* Ws = sm;                              // [256][GP]
-  float* oc = Ws + kCodebook * GP;             // [PARTS][GP][D]
-  __shared__ float mstar_s[GP], lstar_s[GP];
-  __shared__ int is_last;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int s = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int64_t pair = (int64_t)b * a.Hkv + kvh;
+  float* Cs = sm;                           // [64][D]
+  float* Ws = Cs + kMergeC * D;             // [64][32] (codeword, row)
+  __shared__ float mst[kMergeRows];
+  __shared__ int64_t rfirst[kMergeRows];
+  __shared__ int rcount[kMergeRows];
+  __shared__ float rw[kMergeW][kMergeRows];
+  __shared__ int nmax_s;
+  const int tid = threadIdx.x;
+  const int qtr = blockIdx.x, s = blockIdx.y, kvh = blockIdx.z;
+  const int c0 = qtr * kMergeC;
   const int64_t share = *a.share;
-  const int64_t p0 = a.pre[pair], p1 = a.pre[pair + 1];
-  // scan CTAs first..last covered this pair; CTA c wrote its segment to slot pair + c
-  const int64_t first = p1 > p0 ? p0 / share : 1, last = p1 > p0 ? (p1 - 1) / share : 0;
+  {
+    const float* src = a.Cv + (((size_t)kvh * a.Sv + s) * kCodebook + c0) * D;
+    for (int f = tid; f < kMergeC * D / 4; f += 256) cp_async16(Cs + 4 * f, src + 4 * f);
+    cp_async_commit();
+  }
+  const int nrows = a.B * GP;
+  const int e = tid % D, grp = tid / D;
+  for (int r0 = 0; r0 < nrows; r0 += kMergeRows) {
+    if (tid < kMergeRows) {   // warp 0: one row per lane
+      const int r = r0 + tid, b = r / GP, g = r % GP;
+      float m = -INFINITY;
+      int64_t first = 0;
+      int n = 0;
+      if (b < a.B) {
+        const int64_t pair = (int64_t)b * a.Hkv + kvh;
+        int64_t last;
+        pair_slots(a, pair, share, first, last);
+        n = last >= first ? (int)(last - first + 1) : 0;
+        first += pair;   // absolute slot index
+      }
+      // groups of 8 predicated loads: one round trip for up to 8 slots
+      for (int k0 = 0; k0 < n; k0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = k0 + i < n ? a.pm[(first + k0 + i) * GP + g] : -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, v[i]);
+      }
+      for (int k0 = 0; k0 < n && k0 < kMergeW; k0 += 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (k0 + i < n && k0 + i < kMergeW) rw[k0 + i][tid] = ex2_approx(a.pm[(first + k0 + i) * GP + g] - m);
+      }
+      mst[tid] = m;
+      rfirst[tid] = first;
+      rcount[tid] = n;
+      const int nm = __reduce_max_sync(0xffffffffu, n);
+      if (tid == 0) nmax_s = nm;
+    }
+    __syncthreads();
+    // W for (codeword c0 + c, row r): thread = (row lane, codewords warp + 8 k8).  Slots go in
+    // groups of 4 up to the pass's largest count; within a group all 8 x 4 loads are
+    // independent (predicated), so each group costs one round trip.
+    {
+      constexpr int NE = kMergeC * kMergeRows / 256;   // 8 entries per thread
+      const int rl = tid % kMergeRows, cw = tid / kMergeRows;
+      const int g = (r0 + rl) % GP, n = rcount[rl];
+      const int64_t stride = (int64_t)a.Sv * kCodebook * GP;   // one slot
+      const float* src = a.pw + (rfirst[rl] * a.Sv + s) * (int64_t)(kCodebook * GP) + (int64_t)c0 * GP + g;
+      float acc[NE];
+#pragma unroll
+      for (int k8 = 0; k8 < NE; ++k8) acc[k8] = 0.f;
+      const int nm = nmax_s;
+      for (int k0 = 0; k0 < nm; k0 += 4) {
+        float w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int k = k0 + i;
+          w[i] = k >= n ? 0.f : k < kMergeW ? rw[k][rl] : ex2_approx(a.pm[(rfirst[rl] + k) * GP + g] - mst[rl]);
+        }
+        float v[NE][4];
+#pragma unroll
+        for (int k8 = 0; k8 < NE; ++k8)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            v[k8][i] = k0 + i < n ? src[(k0 + i) * stride + (cw + 8 * k8) * GP] : 0.f;
+#pragma unroll
+        for (int k8 = 0; k8 < NE; ++k8)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[k8] = fmaf(w[i], v[k8][i], acc[k8]);
+      }
+#pragma unroll
+      for (int k8 = 0; k8 < NE; ++k8) Ws[(cw + 8 * k8) * kMergeRows + rl] = acc[k8];
+    }
+    cp_async_wait_all();   // the codeword slice (first pass only; later a no-op)
+    __syncthreads();
+    float acc[RPT];
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) acc[j] = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < kMergeC; ++c) {
+      const float cv = Cs[c * D + e];
+      const float4* w4 = reinterpret_cast<const float4*>(Ws + c * kMergeRows + grp * RPT);
+#pragma unroll
+      for (int j4 = 0; j4 < RPT / 4; ++j4) {
+        const float4 w = w4[j4];
+        acc[4 * j4 + 0] = fmaf(w.x, cv, acc[4 * j4 + 0]);
+        acc[4 * j4 + 1] = fmaf(w.y, cv, acc[4 * j4 + 1]);
+        acc[4 * j4 + 2] = fmaf(w.z, cv, acc[4 * j4 + 2]);
+        acc[4 * j4 + 3] = fmaf(w.w, cv, acc[4 * j4 + 3]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) {
+      const int r = r0 + grp * RPT + j, b = r / GP, g = r % GP;
+      if (b < a.B) {
+        const int64_t pair = (int64_t)b * a.Hkv + kvh;
+        a.so[(((pair * a.Sv + s) * kMergeQ + qtr) * GP + g) * D + e] = acc[j];
+      }
+    }
+    __syncthreads();   // the row tables and Ws are rewritten by the next pass
+  }
+}
 
+// One block per (sequence, kv head): sum of the stage / quarter partials (rotated domain,
+// unnormalised), rotation back one head per warp, log-sum-exp merge with the window.
+template <int D, int GP>
+__global__ void __launch_bounds__(256) finalize_kernel(DecodeArgs a) {
+  constexpr int E = D / 32;
+  __shared__ __align__(16) float oc[GP * D];
+  __shared__ float mstar_s[GP], lstar_s[GP];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t pair = blockIdx.x;
+  const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
   if (tid < GP) {
+    int64_t first, last;
+    pair_slots(a, pair, *a.share, first, last);
+    const int n = last >= first ? (int)(last - first + 1) : 0;
+    const float* pmp = a.pm + (pair + first) * GP + tid;
+    const float* plp = a.pl + (pair + first) * GP + tid;
     float m = -INFINITY, l = 0.f;
-    for (int64_t c = first; c <= last; ++c) m = fmaxf(m, a.pm[(pair + c) * GP + tid]);
-    for (int64_t c = first; c <= last; ++c)
-      l += ex2_approx(a.pm[(pair + c) * GP + tid] - m) * a.pl[(pair + c) * GP + tid];
+    for (int k0 = 0; k0 < n; k0 += 8) {   // groups of 8 predicated loads
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = k0 + i < n ? pmp[(k0 + i) * GP] : -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, v[i]);
+    }
+    for (int k0 = 0; k0 < n; k0 += 8) {
+      float v[8], w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = k0 + i < n ? pmp[(k0 + i) * GP] : -INFINITY;
+        w[i] = k0 + i < n ? plp[(k0 + i) * GP] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) l += k0 + i < n ? ex2_approx(v[i] - m) * w[i] : 0.f;
+    }
     mstar_s[tid] = m;
     lstar_s[tid] = l;
   }
-  __syncthreads();
-  // W_s[c][g] = sum_slots 2^(m_slot - m*) W_slot[s][c][g]
-  for (int f = tid; f < kCodebook * GP; f += 256) {
-    const int g = f % GP;
-    float acc = 0.f;
-    for (int64_t c = first; c <= last; ++c) {
-      const float w = ex2_approx(a.pm[(pair + c) * GP + g] - mstar_s[g]);
-      acc = fmaf(w, a.pw[((pair + c) * a.Sv + s) * kCodebook * GP + f], acc);
-    }
-    Ws[f] = acc;
+  // window terms of this warp's first head, loaded before the barrier
+  const int g0 = warp;
+  float mw0 = -INFINITY, lw0 = 0.f, ow0[E];
+  if (g0 < a.G) {
+    mw0 = a.wm[pair * GP + g0];
+    lw0 = a.wl[pair * GP + g0];
+#pragma unroll
+    for (int q = 0; q < E; ++q) ow0[q] = a.wo[(pair * GP + g0) * D + q * 32 + lane];
   }
-  __syncthreads();
-  // o_s[g][e] = sum_c W_s[c][g] Cv_s[c][e]
-  {
-    const int e = tid % D, part = tid / D;
-    const float* Cs = a.Cv + ((size_t)kvh * a.Sv + s) * kCodebook * D;
-    float acc[GP];
-#pragma unroll
-    for (int g = 0; g < GP; ++g) acc[g] = 0.f;
-    constexpr int UB = 16;   // loads in flight per thread
-#pragma unroll 1
-    for (int c0 = part; c0 < kCodebook; c0 += PARTS * UB) {
-      float cv[UB];
-#pragma unroll
-      for (int u = 0; u < UB; ++u) cv[u] = __ldg(Cs + (size_t)(c0 + u * PARTS) * D + e);
-#pragma unroll
-      for (int u = 0; u < UB; ++u)
-#pragma unroll
-        for (int g = 0; g < GP; ++g) acc[g] = fmaf(Ws[(c0 + u * PARTS) * GP + g], cv[u], acc[g]);
-    }
-    if constexpr (PARTS > 1) {
-#pragma unroll
-      for (int g = 0; g < GP; ++g) oc[(part * GP + g) * D + e] = acc[g];
-      __syncthreads();
-      if (part == 0) {
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          float v = acc[g];
-          for (int q = 1; q < PARTS; ++q) v += oc[(q * GP + g) * D + e];
-          acc[g] = v;
-        }
-      }
-    }
-    if (part == 0) {
-#pragma unroll
-      for (int g = 0; g < GP; ++g) a.so[((pair * a.Sv + s) * GP + g) * D + e] = acc[g];
-    }
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned ticket = atomicAdd(&a.cnt[pair], 1u);
-    is_last = (ticket == (unsigned)a.Sv - 1u);
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  // sum of the stage contributions (rotated domain, unnormalised)
+  const int nparts = a.Sv * kMergeQ;   // a multiple of 4, at most 32
   for (int f = tid; f < GP * D; f += 256) {
+    const float* src = a.so + pair * nparts * GP * D + f;
     float v = 0.f;
-    for (int q = 0; q < a.Sv; ++q) v += __ldcg(a.so + (pair * a.Sv + q) * GP * D + f);
+    for (int q0 = 0; q0 < nparts; q0 += 16) {   // 16 predicated loads per round trip
+      float t[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) t[i] = q0 + i < nparts ? src[(q0 + i) * GP * D] : 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v += t[i];
+    }
     oc[f] = v;
   }
   __syncthreads();
-  // rotate back one head per warp, merge with the window, write out
   for (int g = warp; g < a.G; g += 8) {
     double v[E];
 #pragma unroll
     for (int q = 0; q < E; ++q) v[q] = (double)oc[g * D + q * 32 + lane];
     fwht_warp_f64<D>(v, lane);
     const float mc = mstar_s[g], lc = lstar_s[g];
-    const float mw = __ldcg(a.wm + pair * GP + g), lw = __ldcg(a.wl + pair * GP + g);
+    const float mw = g == g0 ? mw0 : a.wm[pair * GP + g];
+    const float lw = g == g0 ? lw0 : a.wl[pair * GP + g];
     const float M = fmaxf(mc, mw);
     const float wc = (mc == -INFINITY) ? 0.f : ex2_approx(mc - M);
     const float ww = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
@@ -998,14 +1150,13 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
 #pragma unroll
     for (int q = 0; q < E; ++q) {
       const int i = q * 32 + lane;
-      const float ow = __ldcg(a.wo + (pair * GP + g) * D + i);
+      const float ow = g == g0 ? ow0[q] : a.wo[(pair * GP + g) * D + i];
       o[i] = (wc * (float)(v[q] * a.rot) + ww * ow) * inv;
     }
     if (lane == 0 && a.lse) {
       a.lse[(int64_t)b * a.Hq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
   }
-  if (tid == 0) a.cnt[pair] = 0u;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1047,7 +1198,7 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
   trace(ev, 0, st);
   {
     const size_t lut_smem = sizeof(LutSmem<D>);
-    const size_t win_smem = ((size_t)256 * GP + 8 * GP + 8 * (size_t)GP * D) * sizeof(float);
+    const size_t win_smem = window_smem_bytes<D, GP>();
     const size_t smem = lut_smem > win_smem ? lut_smem : win_smem;
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
@@ -1069,14 +1220,15 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     }
     if (rc != ZKV_OK) return rc;
   }
-  // 3. merge
+  // 3. merge, finalize
   trace(ev, 2, st);
   {
-    const size_t smem = ((size_t)kCodebook * GP + (size_t)GP * D * (256 / D > 1 ? 256 / D : 1)) *
-                        sizeof(float);
+    const size_t smem = ((size_t)kMergeC * D + (size_t)kMergeC * kMergeRows) * sizeof(float);
     if (ensure_smem_limit(merge_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
-    const dim3 grid((unsigned)a.Sv, (unsigned)a.Hkv, (unsigned)a.B);
+    const dim3 grid((unsigned)kMergeQ, (unsigned)a.Sv, (unsigned)a.Hkv);
     merge_kernel<D, GP><<<grid, 256, smem, st>>>(a);
+    ZKV_CHECK_LAUNCH();
+    finalize_kernel<D, GP><<<(unsigned)(a.B * a.Hkv), 256, 0, st>>>(a);
     ZKV_CHECK_LAUNCH();
   }
   trace(ev, 3, st);
@@ -1163,7 +1315,6 @@ extern "C" int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace,
   a.wl = reinterpret_cast<float*>(ws + pl.off_wl);
   a.wo = reinterpret_cast<float*>(ws + pl.off_wo);
   a.so = reinterpret_cast<float*>(ws + pl.off_so);
-  a.cnt = reinterpret_cast<unsigned*>(ws + pl.off_cnt);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (p->d) {
     case 64: return launch_decode_g<64>(a, pl, p->trace_events, st);

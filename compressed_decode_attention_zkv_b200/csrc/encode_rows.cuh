@@ -50,16 +50,6 @@ constexpr size_t rows_smem_bytes() {
          (size_t)kCodebook * RowsSlice<D>::KC * sizeof(float);
 }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   (unsigned)__cvta_generic_to_shared(smem_dst)),
-               "l"(gmem_src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
 template <int D, int R, class Map>
 __device__ __forceinline__ void encode_rows_body(const Map& map, const float* __restrict__ books,
                                                  int S, double rot_scale, int64_t row0, int h,

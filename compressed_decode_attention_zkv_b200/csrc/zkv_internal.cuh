@@ -23,6 +23,21 @@ inline bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
     if (cudaGetLastError() != cudaSuccess) return ZKV_ERR_CUDA; \
   } while (0)
 
+// 16-byte asynchronous global -> shared copy (both addresses 16-byte aligned).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (unsigned)__cvta_generic_to_shared(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Commit the copies issued so far and wait for all of this thread's copies.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // Walsh-Hadamard transform of one vector held by a warp, float64.
 // Lane l holds elements j*32 + l for j < E = D/32 (strided: coalesced loads, conflict-free

@@ -271,8 +271,9 @@ def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win
                     win_len, out=None, lse=None, max_comp_len=None, softmax_scale=None,
                     workspace: torch.Tensor | None = None, error_flag=None, trace_events=None):
     """Decode attention over the compressed prefix plus the fp16 window (see include/zkv.h).
-    ``trace_events``: optional 4 torch.cuda.Event(enable_timing=True) recorded around the
-    library's three kernels.  Returns (out float32 [B, Hq, d], lse float32 [B, Hq])."""
+    ``trace_events``: optional 4 torch.cuda.Event(enable_timing=True) recorded before the
+    table, scan and merge stages and after the last kernel.
+    Returns (out float32 [B, Hq, d], lse float32 [B, Hq])."""
     B, Hq, d = q.shape
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)

@@ -184,7 +184,8 @@ typedef struct {
   float* lse;
   int32_t* error_flag;
   /* Optional tracing: NULL, or 4 cudaEvent_t handles (as void*) recorded on `stream` before
-   * the lookup-table kernel, before the scan kernel, before the merge kernel and after it. */
+   * the lookup-table kernel, before the scan kernel, before the two merge kernels and after
+   * them. */
   void* const* trace_events;
 } zkv_decode_params;
 
