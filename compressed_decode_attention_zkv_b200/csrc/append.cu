@@ -5,70 +5,277 @@
 // Window" (recent tokens uncompressed, older "middle" tokens compressed to codes); VeloxQuant-
 // MLX 0.5.1 "Quick start" (cache.append(k, v) per token, then cache.attend(q)).
 //
-// Kernel 1 (grid: sequence groups x kv heads x {K, V}) encodes the evicted rows with the
-// row-group encoder and writes the new token into its slot; kernel 2 advances the lengths.
-// Both read the same pre-step lengths, so their decisions agree.
+// Kernel 1 encodes the evicted rows and writes each new token into its window slot; kernel 2
+// advances the lengths.  Both read the same pre-step lengths, so their decisions agree.
+//
+// Kernel 1 is a cluster of 8 CTAs per (group of 8 sequences, kv head, K or V).  CTA k of the
+// cluster owns codewords [32k, 32k + 32) of every stage: it copies its slices with cp.async
+// into a ring of kAppendNB buffers (up to kAppendNB - 1 stages ahead; all of them when
+// S <= kAppendNB) and computes its 32 x 8 float32 distances.  Its candidates
+// are the codewords within the rounding margin (the row encoder's bound, taken with this
+// slice's largest codeword norm) of its own row minimum: a superset of the slice's codewords
+// within the margin of the global minimum, so the exact argmin is always among them.  Each CTA
+// publishes, per row, its best (float64 distance, index) and after one cluster barrier every
+// CTA reduces the 8 published bests the same way (decided in float64, ties to the lowest
+// index).  Every CTA keeps an identical copy of the residuals and reads the chosen codeword
+// from its owner's shared memory.
+#include <cooperative_groups.h>
+
 #include "encode_rows.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace zkv {
 
-struct AppendRows {
-  int B, Hkv, d;
-  int64_t Tcap, Wcap;
-  const __half* win;
-  uint8_t* codes;
-  const int32_t* win_len;
-  const int32_t* win_head;
-  const int32_t* comp_len;
-
-  // Row j (a sequence) is encoded iff its window is full and the prefix has room.
-  __device__ bool valid(int64_t j, int) const {
-    if (j >= B) return false;
-    const int64_t wl = win_len[j], hd = win_head[j], c = comp_len[j];
-    return wl == Wcap && hd >= 0 && hd < Wcap && c >= 0 && c < Tcap;
-  }
-  __device__ const void* src() const { return win; }
-  __device__ int dtype() const { return ZKV_DTYPE_F16; }
-  __device__ bool do_rotate() const { return true; }
-  __device__ int64_t x_off(int64_t j, int h) const {
-    return (((int64_t)j * Hkv + h) * Wcap + win_head[j]) * d;
-  }
-  __device__ void store(int64_t j, int h, int S, const uint8_t* code, const float*) const {
-    uint8_t* c = codes + (((int64_t)j * Hkv + h) * Tcap + comp_len[j]) * S;
-    for (int s = 0; s < S; ++s) c[s] = code[s];
-  }
-};
-
-constexpr int kAppendR = 8;
+constexpr int kAppendR = 8;        // sequences per cluster
+constexpr int kAppendCl = 8;       // CTAs per cluster
+constexpr int kAppendCw = kCodebook / kAppendCl;   // codewords per CTA
+constexpr int kAppendNB = 4;       // codeword slice buffers (stages in flight)
 
 template <int D>
-__global__ void __launch_bounds__(256) append_encode_kernel(zkv_append_params p, double rot) {
+struct AppendSmem {
+  static constexpr int LD = D + 4;            // padded row stride (conflict-free 16-byte reads)
+  float cb[kAppendNB][kAppendCw * LD];        // this CTA's codeword slices, ring of stages
+  float rows[kAppendR * LD];                  // residuals (identical in every CTA)
+  double rn[kAppendR];                        // residual norms
+  float dist[kAppendCw][kAppendR];            // float32 distances of this CTA's codewords
+  float cnorm[kAppendCw];                     // their squared norms
+  float lmin[kAppendR];                       // this CTA's per-row minima
+  float lcmax;                                // this CTA's largest codeword norm
+  int ncand;
+  uint16_t cand[kAppendCw * kAppendR];        // (local codeword << 3) | row
+  double cand_d[kAppendCw * kAppendR];        // their float64 distances
+  double best_d[2][kAppendR];                 // published per-row best, by stage parity
+  int best_c[2][kAppendR];
+  int zsel[kAppendR];
+  uint8_t code[kAppendR][kMaxStages];
+};
+
+template <int D>
+__global__ void __cluster_dims__(kAppendCl, 1, 1) __launch_bounds__(256)
+    append_cluster_kernel(zkv_append_params p, double rot) {
+  constexpr int E = D / 32;
+  constexpr int LD = AppendSmem<D>::LD;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  RowsSmem<D, kAppendR>& sm = *reinterpret_cast<RowsSmem<D, kAppendR>*>(smem_raw);
-  float* cb = reinterpret_cast<float*>(smem_raw + ((sizeof(RowsSmem<D, kAppendR>) + 15) / 16) * 16);
+  AppendSmem<D>& sm = *reinterpret_cast<AppendSmem<D>*>(smem_raw);
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kind = blockIdx.z;   // 0 = keys, 1 = values
   const int h = blockIdx.y;
-  const int64_t row0 = (int64_t)blockIdx.x * kAppendR;
-  AppendRows map;
-  map.B = p.B;
-  map.Hkv = p.Hkv;
-  map.d = D;
-  map.Tcap = p.Tcap;
-  map.Wcap = p.Wcap;
-  map.win = reinterpret_cast<const __half*>(kind ? p.win_v : p.win_k);
-  map.codes = kind ? p.v_codes : p.k_codes;
-  map.win_len = p.win_len;
-  map.win_head = p.win_head;
-  map.comp_len = p.comp_len;
+  const int64_t row0 = (int64_t)(blockIdx.x / kAppendCl) * kAppendR;
   const int S = kind ? p.Sv : p.Sk;
-  const float* books = kind ? p.v_codebooks : p.k_codebooks;
-  encode_rows_body<D, kAppendR>(map, books, S, rot, row0, h, sm, cb);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* CB = (kind ? p.v_codebooks : p.k_codebooks) + (size_t)h * S * kCodebook * D;
+  const __half* win = reinterpret_cast<const __half*>(kind ? p.win_v : p.win_k);
+  uint8_t* codes = kind ? p.v_codes : p.k_codes;
+
+  auto row_valid = [&](int64_t j) {   // sequence j evicts a token into a prefix with room
+    if (j >= p.B) return false;
+    const int64_t wl = p.win_len[j], hd = p.win_head[j], c = p.comp_len[j];
+    return wl == p.Wcap && hd >= 0 && hd < p.Wcap && c >= 0 && c < p.Tcap;
+  };
+  auto load_slice = [&](int s) {      // stage s, codewords [32 rank, 32 rank + 32)
+    const float* src = CB + ((size_t)s * kCodebook + (size_t)rank * kAppendCw) * D;
+    float* dst = sm.cb[s % kAppendNB];
+    for (int f = tid; f < kAppendCw * D / 4; f += 256) {
+      const int cl = f / (D / 4), q = f % (D / 4);
+      cp_async16(dst + cl * LD + 4 * q, src + (size_t)cl * D + 4 * q);
+    }
+    cp_async_commit();
+  };
+
+  // the first slices; every later one is issued (one commit group per stage) after the cluster
+  // barrier of the stage whose buffer it reuses has been passed
+  for (int q = 0; q < kAppendNB - 1 && q < S; ++q) load_slice(q);
+  // rotated rows (every CTA of the cluster computes the same values)
+  if (warp < kAppendR) {
+    const int64_t j = row0 + warp;
+    double ss = 0.0;
+    if (row_valid(j)) {
+      double v[E];
+      load_row_f64<E>(win, ZKV_DTYPE_F16, ((j * p.Hkv + h) * p.Wcap + p.win_head[j]) * D, lane, v);
+      fwht_warp_f64<D>(v, lane);
+#pragma unroll
+      for (int q = 0; q < E; ++q) {
+        const float y = (float)(v[q] * rot);
+        sm.rows[warp * LD + q * 32 + lane] = y;
+        ss += (double)y * (double)y;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < E; ++q) sm.rows[warp * LD + q * 32 + lane] = 0.f;
+    }
+    ss = warp_sum_f64(ss);
+    if (lane == 0) sm.rn[warp] = sqrt(ss);
+  }
+
+  // distance pass: thread = (codeword pair, row half, dimension slice); slice ks holds the
+  // 16-byte chunks 4 ks + 32 j of every vector (conflict-free 16-byte reads)
+  const int ks = tid & 7, cpair = (tid >> 3) & 15, rhalf = tid >> 7;
+  for (int s = 0; s < S; ++s) {
+    // groups committed so far: stages 0 .. min(s + NB - 2, S - 1); stage s must be complete
+    const int later = (s + kAppendNB - 2 < S - 1 ? s + kAppendNB - 2 : S - 1) - s;
+    if (later >= 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
+    else if (later == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();   // slice s and the residuals are ready
+    const float* slice = sm.cb[s % kAppendNB];
+    {
+      float acc[2][4], cn[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        cn[u] = 0.f;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        const int off = 4 * ks + 32 * j;
+        float4 c4[2], x4[4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) c4[u] = *reinterpret_cast<const float4*>(slice + (2 * cpair + u) * LD + off);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) x4[v] = *reinterpret_cast<const float4*>(sm.rows + (4 * rhalf + v) * LD + off);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          cn[u] = fmaf(c4[u].x, c4[u].x, cn[u]);
+          cn[u] = fmaf(c4[u].y, c4[u].y, cn[u]);
+          cn[u] = fmaf(c4[u].z, c4[u].z, cn[u]);
+          cn[u] = fmaf(c4[u].w, c4[u].w, cn[u]);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            acc[u][v] = fmaf(x4[v].x, c4[u].x, acc[u][v]);
+            acc[u][v] = fmaf(x4[v].y, c4[u].y, acc[u][v]);
+            acc[u][v] = fmaf(x4[v].z, c4[u].z, acc[u][v]);
+            acc[u][v] = fmaf(x4[v].w, c4[u].w, acc[u][v]);
+          }
+        }
+      }
+      // sum over the 8 slices (lanes differing in bits 0-2); the rounding bound used for the
+      // margin holds for any summation order
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          cn[u] += __shfl_xor_sync(0xffffffffu, cn[u], o);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[u][v] += __shfl_xor_sync(0xffffffffu, acc[u][v], o);
+        }
+      }
+      if (ks == 0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (rhalf == 0) sm.cnorm[2 * cpair + u] = cn[u];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) sm.dist[2 * cpair + u][4 * rhalf + v] = cn[u] - 2.f * acc[u][v];
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < kAppendR) {
+      float v = sm.dist[0][tid];
+      for (int c = 1; c < kAppendCw; ++c) v = fminf(v, sm.dist[c][tid]);
+      sm.lmin[tid] = v;
+    } else if (tid == 32) {
+      float v = sm.cnorm[0];
+      for (int c = 1; c < kAppendCw; ++c) v = fmaxf(v, sm.cnorm[c]);
+      sm.lcmax = v;
+      sm.ncand = 0;
+    }
+    __syncthreads();
+    // local candidates: within the margin of this CTA's row minimum
+    {
+      const int c = tid >> 3, r = tid & 7;
+      if ((double)sm.dist[c][r] <= (double)sm.lmin[r] + candidate_margin(sm.rn[r], sm.lcmax, D)) {
+        const int k = atomicAdd(&sm.ncand, 1);
+        sm.cand[k] = (uint16_t)((c << 3) | r);
+      }
+    }
+    __syncthreads();
+    // exact float64 distance of each candidate, one warp per candidate
+    const int nc = sm.ncand;
+    for (int k = warp; k < nc; k += 8) {
+      const int c = sm.cand[k] >> 3, r = sm.cand[k] & 7;
+      double a = 0.0;
+#pragma unroll
+      for (int q = 0; q < E; ++q) {
+        const int i = q * 32 + lane;
+        const double df = (double)sm.rows[r * LD + i] - (double)slice[c * LD + i];
+        a = fma(df, df, a);
+      }
+      a = warp_sum_f64(a);
+      if (lane == 0) sm.cand_d[k] = a;
+    }
+    __syncthreads();
+    if (tid < kAppendR) {   // this CTA's best per row, published for the cluster
+      double d = DBL_MAX;
+      int bc = kCodebook;
+      for (int k = 0; k < nc; ++k) {
+        if ((sm.cand[k] & 7) != tid) continue;
+        const int c = rank * kAppendCw + (sm.cand[k] >> 3);
+        const double dd = sm.cand_d[k];
+        if (dd < d || (dd == d && c < bc)) {
+          d = dd;
+          bc = c;
+        }
+      }
+      sm.best_d[s & 1][tid] = d;
+      sm.best_c[s & 1][tid] = bc;
+    }
+    // every CTA's bests are visible; every read of stage s-1's slices and bests is done
+    cluster.sync();
+    // the buffer of stage s-1 is free (its remote reads are done): refill it NB - 1 stages ahead
+    if (s + kAppendNB - 1 < S) load_slice(s + kAppendNB - 1);
+    if (tid < kAppendR) {
+      double d[kAppendCl];
+      int c[kAppendCl];
+#pragma unroll
+      for (int k = 0; k < kAppendCl; ++k) {
+        const AppendSmem<D>* o = cluster.map_shared_rank(&sm, k);
+        d[k] = o->best_d[s & 1][tid];
+        c[k] = o->best_c[s & 1][tid];
+      }
+      double bd2 = d[0];
+      int bc2 = c[0];
+#pragma unroll
+      for (int k = 1; k < kAppendCl; ++k)
+        if (d[k] < bd2 || (d[k] == bd2 && c[k] < bc2)) {
+          bd2 = d[k];
+          bc2 = c[k];
+        }
+      // non-finite rows match no candidate; never index past the stage's codebook
+      sm.zsel[tid] = bc2 < kCodebook ? bc2 : 0;
+    }
+    __syncthreads();
+    // residual update with the chosen codeword, read from its owner's slice
+    if (warp < kAppendR) {
+      const int z = sm.zsel[warp];
+      const float* src = cluster.map_shared_rank(&sm.cb[s % kAppendNB][0], z / kAppendCw) + (z % kAppendCw) * LD;
+      double ss = 0.0;
+#pragma unroll
+      for (int q = 0; q < E; ++q) {
+        const int i = q * 32 + lane;
+        const float nr = sm.rows[warp * LD + i] - src[i];
+        sm.rows[warp * LD + i] = nr;
+        ss += (double)nr * (double)nr;
+      }
+      ss = warp_sum_f64(ss);
+      if (lane == 0) {
+        sm.rn[warp] = sqrt(ss);
+        sm.code[warp][s] = (uint8_t)z;
+      }
+    }
+  }
+  cluster.sync();   // no CTA leaves while another may still read its shared memory
+  if (rank != 0) return;
   if (tid < kAppendR) {
     const int64_t j = row0 + tid;
-    if (map.valid(j, h)) map.store(j, h, S, sm.code[tid], sm.nrm[tid]);
+    if (row_valid(j)) {
+      uint8_t* c = codes + ((j * p.Hkv + h) * p.Tcap + p.comp_len[j]) * S;
+      for (int s = 0; s < S; ++s) c[s] = sm.code[tid][s];
+    }
   }
-  __syncthreads();   // every read of an evicted slot precedes the overwrite below
+  // every CTA read the evicted slots before its first cluster barrier
   if (warp < kAppendR) {
     const int64_t j = row0 + warp;
     if (j >= p.B) return;
@@ -83,10 +290,8 @@ __global__ void __launch_bounds__(256) append_encode_kernel(zkv_append_params p,
       set_error(p.error_flag, ZKV_DEVERR_WIN_LEN);
     }
     if (slot < 0) return;
-    const __half* src = reinterpret_cast<const __half*>(kind ? p.new_v : p.new_k) +
-                        ((int64_t)j * p.Hkv + h) * D;
-    __half* dst = reinterpret_cast<__half*>(kind ? p.win_v : p.win_k) +
-                  (((int64_t)j * p.Hkv + h) * p.Wcap + slot) * D;
+    const __half* src = reinterpret_cast<const __half*>(kind ? p.new_v : p.new_k) + (j * p.Hkv + h) * D;
+    __half* dst = reinterpret_cast<__half*>(kind ? p.win_v : p.win_k) + ((j * p.Hkv + h) * p.Wcap + slot) * D;
     for (int i = lane; i < D; i += 32) dst[i] = src[i];
   }
 }
@@ -125,16 +330,17 @@ extern "C" int zkv_rvq_append(const zkv_append_params* p, void* stream) {
   if (al & 15) return ZKV_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const double rot = 1.0 / std::sqrt((double)p->d);
-  const dim3 grid((unsigned)((p->B + kAppendR - 1) / kAppendR), (unsigned)p->Hkv, 2);
+  const unsigned groups = (unsigned)((p->B + kAppendR - 1) / kAppendR);
+  const dim3 grid(groups * kAppendCl, (unsigned)p->Hkv, 2);
   const bool ok =
-      ensure_smem_limit(append_encode_kernel<64>, rows_smem_bytes<64, kAppendR>()) == cudaSuccess &&
-      ensure_smem_limit(append_encode_kernel<128>, rows_smem_bytes<128, kAppendR>()) == cudaSuccess &&
-      ensure_smem_limit(append_encode_kernel<256>, rows_smem_bytes<256, kAppendR>()) == cudaSuccess;
+      ensure_smem_limit(append_cluster_kernel<64>, sizeof(AppendSmem<64>)) == cudaSuccess &&
+      ensure_smem_limit(append_cluster_kernel<128>, sizeof(AppendSmem<128>)) == cudaSuccess &&
+      ensure_smem_limit(append_cluster_kernel<256>, sizeof(AppendSmem<256>)) == cudaSuccess;
   if (!ok) return ZKV_ERR_CUDA;
   switch (p->d) {
-    case 64: append_encode_kernel<64><<<grid, 256, rows_smem_bytes<64, kAppendR>(), st>>>(*p, rot); break;
-    case 128: append_encode_kernel<128><<<grid, 256, rows_smem_bytes<128, kAppendR>(), st>>>(*p, rot); break;
-    default: append_encode_kernel<256><<<grid, 256, rows_smem_bytes<256, kAppendR>(), st>>>(*p, rot); break;
+    case 64: append_cluster_kernel<64><<<grid, 256, sizeof(AppendSmem<64>), st>>>(*p, rot); break;
+    case 128: append_cluster_kernel<128><<<grid, 256, sizeof(AppendSmem<128>), st>>>(*p, rot); break;
+    default: append_cluster_kernel<256><<<grid, 256, sizeof(AppendSmem<256>), st>>>(*p, rot); break;
   }
   ZKV_CHECK_LAUNCH();
   append_lengths_kernel<<<(p->B + 127) / 128, 128, 0, st>>>(p->B, p->Tcap, p->Wcap, p->win_len,

@@ -189,14 +189,15 @@ def test_decode_full_size_sampled(name):
 
 # ------------------------------------------------------------------ serving step
 
-def _state(seed, B_, Hkv, d, S, Tcap, Wcap, win_len, win_head, comp_len):
+def _state(seed, B_, Hkv, d, S, Tcap, Wcap, win_len, win_head, comp_len, Sv=None):
     rng = np.random.default_rng(seed)
+    Sv = S if Sv is None else Sv
     Ck = (rng.standard_normal((Hkv, S, 256, d)) * 0.3).astype(np.float32)
-    Cv = (rng.standard_normal((Hkv, S, 256, d)) * 0.3).astype(np.float32)
+    Cv = (rng.standard_normal((Hkv, Sv, 256, d)) * 0.3).astype(np.float32)
     Ck[:, :, 0] = 0
     Cv[:, :, 0] = 0
     return dict(k_codes=rng.integers(0, 256, (B_, Hkv, Tcap, S)).astype(np.uint8),
-                v_codes=rng.integers(0, 256, (B_, Hkv, Tcap, S)).astype(np.uint8),
+                v_codes=rng.integers(0, 256, (B_, Hkv, Tcap, Sv)).astype(np.uint8),
                 comp_len=np.array(comp_len), win_len=np.array(win_len),
                 win_head=np.array(win_head),
                 win_k=rng.standard_normal((B_, Hkv, Wcap, d)).astype(np.float16),
@@ -214,6 +215,35 @@ def test_append_steps_match_oracle():
     for step in range(4):
         nk = rng.standard_normal((5, 2, 128)).astype(np.float16)
         nv = rng.standard_normal((5, 2, 128)).astype(np.float16)
+        st = O.append_step(st, nk, nv)
+        zkv.rvq_append(_cuda(nk), _cuda(nv), g["win_k"], g["win_v"], g["win_len"],
+                       g["win_head"], g["comp_len"], g["k_codes"], g["v_codes"], g["Ck"],
+                       g["Cv"], error_flag=flag)
+        torch.cuda.synchronize()
+        for key in ("comp_len", "win_len", "win_head", "k_codes", "v_codes", "win_k", "win_v"):
+            np.testing.assert_array_equal(g[key].cpu().numpy(), st[key], err_msg=f"{key} step {step}")
+    assert st["error"] and (int(flag.item()) & zkv.ZKV_DEVERR_COMP_LEN)
+
+
+@pytest.mark.parametrize("B_,Hkv,d,Sk,Sv", [(11, 3, 64, 2, 5), (17, 1, 256, 4, 3),
+                                           (9, 2, 128, 8, 1)])
+def test_append_row_groups_and_shapes(B_, Hkv, d, Sk, Sv):
+    """Several 8-sequence groups per head (the last one ragged), every head dimension, Sk != Sv,
+    windows filling and full, one prefix at capacity."""
+    Tcap, Wcap = 16, 3
+    rng = np.random.default_rng(50 + B_)
+    win_len = rng.integers(0, Wcap + 1, B_)
+    win_len[: B_ // 2] = Wcap
+    comp_len = rng.integers(0, Tcap - 2, B_)
+    comp_len[1] = Tcap
+    st = _state(60 + B_, B_=B_, Hkv=Hkv, d=d, S=Sk, Sv=Sv, Tcap=Tcap, Wcap=Wcap,
+                win_len=win_len, win_head=rng.integers(0, Wcap, B_), comp_len=comp_len)
+    g = {k: _cuda(v.astype(np.int32) if k in ("comp_len", "win_len", "win_head") else v)
+         for k, v in st.items()}
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for step in range(3):
+        nk = rng.standard_normal((B_, Hkv, d)).astype(np.float16)
+        nv = rng.standard_normal((B_, Hkv, d)).astype(np.float16)
         st = O.append_step(st, nk, nv)
         zkv.rvq_append(_cuda(nk), _cuda(nv), g["win_k"], g["win_v"], g["win_len"],
                        g["win_head"], g["comp_len"], g["k_codes"], g["v_codes"], g["Ck"],
