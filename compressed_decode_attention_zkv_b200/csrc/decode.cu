@@ -92,9 +92,9 @@ static size_t scan_smem_bytes(int Rk, int Sk, int Sv, int GP, const VMap& v) {
   size_t b = (size_t)Rk * Sk * kCodebook * GP * 4;            // key tables
   b += (size_t)Sv * kCodebook * GP * 4;                         // fp32 master histograms
   b += 2ull * kCodebook * v.VW * 4;                            // value histograms (hi, lo)
-  b += 2ull * v.J * GP * (v.rounds + 4) * 4;                    // fixed-point p staging (hi, lo)
-  b += (size_t)v.J * (v.rounds + 4) * v.codew * 4;              // value-code staging
-  b += (size_t)(kScanThreads / 32 + 1) * GP * 4 + 16;           // reductions
+  b += 2ull * 2 * v.J * GP * (v.rounds + 4) * 4;                // p staging (2 buffers x hi, lo)
+  b += 2ull * v.J * (v.rounds + 4) * v.codew * 4;               // value-code staging (2 buffers)
+  b += (size_t)(2 * (kScanThreads / 32) + kScanThreads / 32) * GP * 4 + 16;   // maxima (2), sums
   return b;
 }
 
@@ -122,7 +122,7 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   pl.slots = pairs + grid;
   const size_t f = sizeof(float);
   size_t o = 0;
-  pl.off_lut = o;   o = align256(o + (size_t)p->B * p->Hq * p->Sk * kCodebook * f);
+  pl.off_lut = o;   o = align256(o + (size_t)pairs * p->Sk * kCodebook * pl.GP * f);
   pl.off_pre = o;   o = align256(o + (size_t)(pairs + 1) * sizeof(int64_t));
   pl.off_share = o; o = align256(o + sizeof(int64_t));
   pl.off_pm = o;    o = align256(o + (size_t)pl.slots * pl.GP * f);
@@ -153,7 +153,7 @@ struct DecodeArgs {
   float* out;
   float* lse;
   int32_t* err;
-  float* lut;        // [B][Hq][Sk][256]
+  float* lut;        // [B][Hkv][Sk][256][GP] (heads g >= G unwritten)
   int64_t* pre;      // [B*Hkv + 1] exclusive prefix sums of compressed lengths
   int64_t* share;    // tokens per scan CTA
   float* pm;         // [slots][GP] segment maxima
@@ -491,8 +491,8 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
     const int j = hg * kLutH + hq * 8 + k;
     if (j < a.B * a.G) {
       const int b = j / a.G, g = j % a.G;
-      const int64_t h = (int64_t)kvh * a.G + g;
-      a.lut[(((int64_t)b * a.Hq + h) * a.Sk + s) * kCodebook + c0 + cc] = acc[k] * a.scale_log2;
+      a.lut[((((int64_t)b * a.Hkv + kvh) * a.Sk + s) * kCodebook + c0 + cc) * GP + g] =
+          acc[k] * a.scale_log2;
     }
   }
 }
@@ -650,6 +650,8 @@ struct ScanCfg {
   static constexpr int PR = ROUNDS + 4;          // padded staging row (words)
   static constexpr int CODEW = SVP <= 4 ? 1 : 2;
   static constexpr int NW = kScanThreads / 32;
+  static constexpr int BUFW = 2 * J * GP * PR;   // words of one p staging buffer (hi, lo)
+  static constexpr int CBUFW = J * PR * CODEW;   // words of one code staging buffer
 };
 
 // master[(s, c, g)] = (master (if any) + histogram value) * scale[g], where the histogram
@@ -663,6 +665,7 @@ __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t*
                                             const float (&scale)[GP], int tid) {
   const int lane = tid & 31;
   const int total = kCodebook * C::VW;           // words per table
+#pragma unroll 4
   for (int w0 = tid - lane; w0 < total; w0 += kScanThreads) {
     const int wi = w0 + lane;                      // total is a multiple of 32
     const int cc = wi / C::VW, col = wi % C::VW;
@@ -686,6 +689,13 @@ __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t*
   }
 }
 
+// The token loop is software-pipelined with one barrier per sub-chunk.  In interval i every
+// thread (a) reads the partial maxima of sub-chunk i and decides whether the reference grows,
+// (b) adds the staged p of sub-chunk i-1 to the integer histograms, (c) computes and stages
+// the p of sub-chunk i, and (d) gathers the key scores and partial maxima of sub-chunk i+1.
+// Staging buffers and partial maxima alternate between two copies, so no interval reads what
+// the same interval writes.  A growth of the reference with non-empty histograms takes a
+// slow path (barrier, fold, barrier, zero, barrier) after (b), uniformly across the block.
 template <int GP, int SKP, int SVP>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   using C = ScanCfg<GP, SKP, SVP>;
@@ -697,11 +707,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   float* master = lut + (size_t)Rk * Sk * kCodebook * GP;                       // [Sv][256][GP]
   uint32_t* vhi = reinterpret_cast<uint32_t*>(master + ntab);                   // [256][VW]
   uint32_t* vlo = vhi + kCodebook * C::VW;
-  uint32_t* hst = vlo + kCodebook * C::VW;                                      // [J][GP][PR]
-  uint32_t* lst = hst + C::J * GP * C::PR;                                      // [J][GP][PR]
-  uint32_t* cst = lst + C::J * GP * C::PR;                                      // [J][PR][CODEW]
-  uint32_t* redk = cst + C::J * C::PR * C::CODEW;                               // [NW][GP]
-  float* red = reinterpret_cast<float*>(redk);
+  uint32_t* stg = vlo + kCodebook * C::VW;        // [2][hi, lo][J][GP][PR]
+  uint32_t* cst = stg + 2 * C::BUFW;              // [2][J][PR][CODEW]
+  uint32_t* redk = cst + 2 * C::CBUFW;            // [2][NW][GP] partial maxima (keys)
+  float* red = reinterpret_cast<float*>(redk + 2 * C::NW * GP);   // [NW][GP]
 
   const int npairs = a.B * a.Hkv;
   const int64_t share = *a.share;
@@ -709,13 +718,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   const int64_t lo = (int64_t)blockIdx.x * share;
   const int64_t hi = lo + share < tot ? lo + share : tot;
   if (lo >= hi) return;
-  // last pair whose prefix start is <= lo
+  // last pair whose prefix start is <= lo: block-parallel search, one round of loads per
+  // factor of kScanThreads (pre is non-decreasing, so the sampled predicate is a prefix)
   int pfirst = 0;
   {
     int l = 0, r = npairs;   // invariant: pre[l] <= lo < pre[r] (pre[npairs] = tot > lo)
     while (r - l > 1) {
-      const int m = (l + r) >> 1;
-      if (a.pre[m] <= lo) l = m; else r = m;
+      const int step = (r - l + kScanThreads - 1) / kScanThreads;
+      const int k = l + tid * step;
+      const int cnt = __syncthreads_count(k < r && a.pre[k] <= lo);
+      l = l + (cnt - 1) * step;
+      r = l + step < r ? l + step : r;
     }
     pfirst = l;
   }
@@ -731,18 +744,65 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   const int vj = C::PASSES == 1 ? lane / C::COMBOS : 0;
   // staging slot of this thread's token
   const int sj = tid % C::J, sk = tid / C::J;
-  const uint32_t hst_base = smem_u32(hst), cst_base = smem_u32(cst);
-  const uint32_t hst_a = hst_base + 4u * (uint32_t)(sj * GP * C::PR + sk);
+  const uint32_t stg_base = smem_u32(stg), cst_base = smem_u32(cst);
+  const uint32_t hst_a = stg_base + 4u * (uint32_t)(sj * GP * C::PR + sk);
   const uint32_t cst_a = cst_base + 4u * C::CODEW * (uint32_t)(sj * C::PR + sk);
   const uint32_t vtab_base = smem_u32(vhi);
   const uint32_t redk_a = smem_u32(redk);
+
+  // integer histograms += staged p of one sub-chunk (buffer bf).  Batches of 4 rounds,
+  // warp-strided.  Padded heads carry p = 0 and padded stages read code byte 0 of a stage that
+  // is never output, so no lane needs masking.
+  auto accumulate = [&](int bf) {
+#pragma unroll
+    for (int ps = 0; ps < C::PASSES; ++ps) {
+      const int combo = C::PASSES == 1 ? lane % C::COMBOS : ps * 32 + lane;
+      const int vs = combo / GP, vg = combo % GP;
+      const uint32_t hrow = stg_base + 4u * (uint32_t)(bf * C::BUFW + (vj * GP + vg) * C::PR);
+      const uint32_t lrow = hrow + 4u * (uint32_t)(C::J * GP * C::PR);
+      const uint32_t crow = cst_base + 4u * (uint32_t)(bf * C::CBUFW + C::CODEW * vj * C::PR);
+      const unsigned sel = 0x4440u | (unsigned)(vs & 3);
+      const uint32_t tab = vtab_base + 4u * (uint32_t)(ps * 32 + lane);
+      for (int bt = warp; bt < C::ROUNDS / 4; bt += C::NW) {
+        const uint32_t k0b = 16u * (uint32_t)bt;   // 4 rounds of 4-byte words
+        const uint4 h4 = lds128u(hrow + k0b);
+        const uint4 l4 = lds128u(lrow + k0b);
+        uint32_t cw[4];
+        if constexpr (C::CODEW == 1) {
+          const uint4 c4 = lds128u(crow + k0b);
+          cw[0] = c4.x; cw[1] = c4.y; cw[2] = c4.z; cw[3] = c4.w;
+        } else {
+          const uint4 c01 = lds128u(crow + 2u * k0b);
+          const uint4 c23 = lds128u(crow + 2u * k0b + 16u);
+          const int hw = vs >> 2;
+          cw[0] = hw ? c01.y : c01.x; cw[1] = hw ? c01.w : c01.z;
+          cw[2] = hw ? c23.y : c23.x; cw[3] = hw ? c23.w : c23.z;
+        }
+        const uint32_t hh[4] = {h4.x, h4.y, h4.z, h4.w};
+        const uint32_t ll[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint32_t adr = tab + (__byte_perm(cw[r], 0u, sel) << (C::VWSH + 2));
+          red_pair<kCodebook * C::VW * 4>(adr, hh[r], ll[r]);
+        }
+      }
+    }
+  };
+  // key scores of this thread's token of a sub-chunk and the warp's partial maxima -> redk[bf]
+  auto score = [&](const Code<SKP>& kc, bool ok, int bf, float (&sc)[GP]) {
+    key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const uint32_t k = __reduce_max_sync(0xffffffffu, ok ? ord_key(sc[g]) : 0u);
+      if (lane == 0) sts32u(redk_a + 4u * (uint32_t)((bf * C::NW + warp) * GP + g), k);
+    }
+  };
 
   for (int pr = pfirst; pr < npairs && a.pre[pr] < hi; ++pr) {
     const int64_t seg0 = lo > a.pre[pr] ? lo : a.pre[pr];
     const int64_t seg1 = hi < a.pre[pr + 1] ? hi : a.pre[pr + 1];
     if (seg0 >= seg1) continue;
     const int64_t s0 = seg0 - a.pre[pr], s1 = seg1 - a.pre[pr];   // pair-local token range
-    const int b = pr / a.Hkv, kvh = pr % a.Hkv;
     const int64_t slot = (int64_t)pr + blockIdx.x;
     const uint8_t* kcb = a.k_codes + (int64_t)pr * a.Tcap * Sk;
     const uint8_t* vcb = a.v_codes + (int64_t)pr * a.Tcap * Sv;
@@ -754,30 +814,53 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       prefetch_l2(kcb, kcb + pbytes_k, kcb + (s0 & ~int64_t(15)) * Sk, (s1 - (s0 & ~int64_t(15))) * Sk);
       prefetch_l2(vcb, vcb + pbytes_v, vcb + (s0 & ~int64_t(15)) * Sv, (s1 - (s0 & ~int64_t(15))) * Sv);
     }
+    const uint32_t u0 = (uint32_t)s0, u1 = (uint32_t)s1;
+    // codes of sub-chunks 0 and 1 in flight during the table fill
+    Code<SKP> kc = load_code1<SKP>(kcb, Sk, u0 + tid, u1);
+    Code<SVP> vc = load_code1<SVP>(vcb, Sv, u0 + tid, u1);
+    Code<SKP> kn = load_code1<SKP>(kcb, Sk, u0 + kScanSub + tid, u1);
+    Code<SVP> vn = load_code1<SVP>(vcb, Sv, u0 + kScanSub + tid, u1);
     __syncthreads();   // previous segment's shared memory is free
     {
-      // the pair's G x Sk x 256 table entries: coalesced loads into a staging area (the
-      // histogram region, 2 * 256 * VW >= 16384 words), stored (s, c)-major with a padded
-      // head stride, then replicated into the lane-group copies with linear stores
-      const float* src = a.lut + ((int64_t)b * a.Hq + (int64_t)kvh * G) * Sk * kCodebook;
-      float* stage = reinterpret_cast<float*>(vhi);
-      const int nsc = Sk * kCodebook;
-      const int str = (nsc * (GP + 1) <= 2 * kCodebook * C::VW) ? GP + 1 : GP;
-      for (int g = 0; g < G; ++g)
-        for (int sc = tid; sc < nsc; sc += kScanThreads) stage[sc * str + g] = __ldg(src + g * nsc + sc);
-      __syncthreads();
-      const int n = nsc * Rk * GP;    // replicated table, written linearly
-      for (int f = tid; f < n; f += kScanThreads) {
-        const int g = f & (GP - 1), sc = f >> cshift;   // sc = s*256 + c
-        lut[f] = g < G ? stage[sc * str + g] : 0.f;
-      }
-      __syncthreads();
+      // zero the histograms, then copy the pair's table entries (s, c) -> every lane-group
+      // copy: item f = (entry, copy) with the copy fastest, so consecutive lanes store
+      // consecutive GP-wide entries; heads g >= G are zero
       uint4* z = reinterpret_cast<uint4*>(vhi);
       const int nz = 2 * kCodebook * C::VW / 4;
       for (int f = tid; f < nz; f += kScanThreads) z[f] = make_uint4(0u, 0u, 0u, 0u);
+      const float* src = a.lut + (int64_t)pr * Sk * kCodebook * GP;
+      const int rsh = __ffs(Rk) - 1;
+      const int n = Sk * kCodebook * Rk;
+      for (int f0 = 0; f0 < n; f0 += 4 * kScanThreads) {
+        float v[4][GP];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int f = f0 + u * kScanThreads + tid;
+          const int sc = f >> rsh;
+#pragma unroll
+          for (int g = 0; g < GP; ++g) v[u][g] = (f < n && g < G) ? __ldg(src + (int64_t)sc * GP + g) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int f = f0 + u * kScanThreads + tid;
+          if (f < n) {
+            float* dst = lut + (size_t)f * GP;   // (sc * Rk + copy) * GP
+            if constexpr (GP >= 4) {
+#pragma unroll
+              for (int g = 0; g < GP; g += 4)
+                *reinterpret_cast<float4*>(dst + g) = make_float4(v[u][g], v[u][g + 1], v[u][g + 2], v[u][g + 3]);
+            } else if constexpr (GP == 2) {
+              *reinterpret_cast<float2*>(dst) = make_float2(v[u][0], v[u][1]);
+            } else {
+              dst[0] = v[u][0];
+            }
+          }
+        }
+      }
     }
-    // (the first __syncthreads of the token loop orders the zeroing before any reduction)
+    __syncthreads();   // tables and zeroed histograms are ready
 
+    const int nsub = (int)((u1 - u0 + kScanSub - 1) / kScanSub);   // same on every thread
     float mref[GP], lacc[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -785,27 +868,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       lacc[g] = 0.f;
     }
     bool dirty = false, has_master = false;   // uniform across the block
-    const uint32_t u0 = (uint32_t)s0, u1 = (uint32_t)s1;
-    Code<SKP> kn = load_code1<SKP>(kcb, Sk, u0 + tid, u1);
-    Code<SVP> vn = load_code1<SVP>(vcb, Sv, u0 + tid, u1);
-    for (uint32_t ubase = u0; ubase < u1; ubase += kScanSub) {
-      const uint32_t t = ubase + tid;
-      const Code<SKP> kc = kn;
-      const Code<SVP> vc = vn;
-      kn = load_code1<SKP>(kcb, Sk, t + kScanSub, u1);   // next sub-chunk in flight
-      vn = load_code1<SVP>(vcb, Sv, t + kScanSub, u1);
+    // prologue: scores of sub-chunk 0
+    float sc[GP];
+    score(kc, u0 + tid < u1, 0, sc);
+    __syncthreads();
+    for (int i = 0; i < nsub; ++i) {
+      const int bf = i & 1;
+      const uint32_t t = u0 + (uint32_t)i * kScanSub + tid;
       const bool ok = t < u1;
-      float sc[GP];
-      key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
-      // sub-chunk maximum per head (integer reduction on order-preserving keys)
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const uint32_t k = __reduce_max_sync(0xffffffffu, ok ? ord_key(sc[g]) : 0u);
-        if (lane == 0) sts32u(redk_a + 4u * (uint32_t)(warp * GP + g), k);
-      }
-      __syncthreads();   // also: the previous sub-chunk's staging has been consumed
-      // every warp combines the NW x GP partial maxima: lanes read them (entry w * GP + g sits
-      // in lane (w * GP + g) % 32), fold over w with xor-shuffles, then broadcast each head
+      // (a) maxima of sub-chunk i: lanes read the NW x GP partial maxima (entry w * GP + g in
+      // lane (w * GP + g) % 32), fold over w with xor-shuffles, broadcast each head
       float mn[GP];
       {
         uint32_t k = 0u;
@@ -813,7 +885,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
         for (int e = 0; e < C::NW * GP; e += 32)
           if (e + lane < C::NW * GP) {
             uint32_t v;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(redk_a + 4u * (uint32_t)(e + lane)));
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(redk_a + 4u * (uint32_t)(bf * C::NW * GP + e + lane)));
             k = max(k, v);
           }
 #pragma unroll
@@ -824,6 +896,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       bool grow = false;
 #pragma unroll
       for (int g = 0; g < GP; ++g) grow |= mn[g] > mref[g];
+      // (b) histograms += p of sub-chunk i-1
+      if (i > 0) {
+        accumulate(bf ^ 1);
+        dirty = true;
+      }
       if (grow) {   // uniform: every thread read the same maxima
         // New reference = maximum + kHeadroom: later sub-chunks rarely exceed it, so folds
         // stay rare.  Precision: the segment's largest p is >= 2^-kHeadroom and the
@@ -838,17 +915,20 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
           lacc[g] *= alpha[g];
         }
         if (dirty) {
-          // fold the integer histograms (relative to the old maximum) into the fp32 master
-          // and rescale it to the new maximum
+          // fold the integer histograms (relative to the old reference) into the fp32
+          // master and rescale it to the new reference
+          __syncthreads();   // every reduction so far has landed
           fold_tables<C, GP>(vhi, vlo, master, Sv, has_master, alpha, tid);
           __syncthreads();
           uint4* z = reinterpret_cast<uint4*>(vhi);
           const int nz = 2 * kCodebook * C::VW / 4;
           for (int f = tid; f < nz; f += kScanThreads) z[f] = make_uint4(0u, 0u, 0u, 0u);
+          __syncthreads();
           has_master = true;
           dirty = false;
         }
       }
+      // (c) p of sub-chunk i -> staging buffer bf
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         uint32_t hv = 0u, lv = 0u;
@@ -857,52 +937,26 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
           lacc[g] += pv;
           if (g < G) split_fixed38(pv, hv, lv);
         }
-        sts32u(hst_a + 4u * (uint32_t)(g * C::PR), hv);
-        sts32u(hst_a + 4u * (uint32_t)((C::J * GP + g) * C::PR), lv);   // lo staging follows
+        sts32u(hst_a + 4u * (uint32_t)(bf * C::BUFW + g * C::PR), hv);
+        sts32u(hst_a + 4u * (uint32_t)(bf * C::BUFW + (C::J * GP + g) * C::PR), lv);   // lo follows hi
       }
       if constexpr (C::CODEW == 1) {
-        sts32u(cst_a, vc.w[0]);
+        sts32u(cst_a + 4u * (uint32_t)(bf * C::CBUFW), vc.w[0]);
       } else {
-        sts64u(cst_a, vc.w[0], vc.w[1]);
+        sts64u(cst_a + 4u * (uint32_t)(bf * C::CBUFW), vc.w[0], vc.w[1]);
+      }
+      // (d) scores of sub-chunk i+1; codes of sub-chunk i+2 in flight
+      if (i + 1 < nsub) {
+        kc = kn;
+        vc = vn;
+        kn = load_code1<SKP>(kcb, Sk, t + 2 * kScanSub, u1);
+        vn = load_code1<SVP>(vcb, Sv, t + 2 * kScanSub, u1);
+        score(kc, t + kScanSub < u1, bf ^ 1, sc);
       }
       __syncthreads();
-      // value side: batches of 4 rounds, warp-strided.  Padded heads carry p = 0 and padded
-      // stages read code byte 0 of a stage that is never output, so no lane needs masking.
-#pragma unroll
-      for (int ps = 0; ps < C::PASSES; ++ps) {
-        const int combo = C::PASSES == 1 ? lane % C::COMBOS : ps * 32 + lane;
-        const int vs = combo / GP, vg = combo % GP;
-        const uint32_t hrow = hst_base + 4u * (uint32_t)((vj * GP + vg) * C::PR);
-        const uint32_t lrow = hrow + 4u * (uint32_t)(C::J * GP * C::PR);
-        const uint32_t crow = cst_base + 4u * C::CODEW * (uint32_t)(vj * C::PR);
-        const unsigned sel = 0x4440u | (unsigned)(vs & 3);
-        const uint32_t tab = vtab_base + 4u * (uint32_t)(ps * 32 + lane);
-        for (int bt = warp; bt < C::ROUNDS / 4; bt += C::NW) {
-          const uint32_t k0b = 16u * (uint32_t)bt;   // 4 rounds of 4-byte words
-          const uint4 h4 = lds128u(hrow + k0b);
-          const uint4 l4 = lds128u(lrow + k0b);
-          uint32_t cw[4];
-          if constexpr (C::CODEW == 1) {
-            const uint4 c4 = lds128u(crow + k0b);
-            cw[0] = c4.x; cw[1] = c4.y; cw[2] = c4.z; cw[3] = c4.w;
-          } else {
-            const uint4 c01 = lds128u(crow + 2u * k0b);
-            const uint4 c23 = lds128u(crow + 2u * k0b + 16u);
-            const int hw = vs >> 2;
-            cw[0] = hw ? c01.y : c01.x; cw[1] = hw ? c01.w : c01.z;
-            cw[2] = hw ? c23.y : c23.x; cw[3] = hw ? c23.w : c23.z;
-          }
-          const uint32_t hh[4] = {h4.x, h4.y, h4.z, h4.w};
-          const uint32_t ll[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const uint32_t adr = tab + (__byte_perm(cw[r], 0u, sel) << (C::VWSH + 2));
-            red_pair<kCodebook * C::VW * 4>(adr, hh[r], ll[r]);
-          }
-        }
-      }
-      dirty = true;
     }
+    // histograms += p of the last sub-chunk
+    accumulate((nsub - 1) & 1);
     // ---- segment partial: maximum, sum of p, fp32 histograms (master + integer tables)
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -914,7 +968,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       float l = 0.f;
 #pragma unroll
       for (int w = 0; w < C::NW; ++w) l += red[w * GP + tid];
-      a.pm[slot * GP + tid] = mref[tid];
+      float mr = 0.f;
+#pragma unroll
+      for (int g = 0; g < GP; ++g)
+        if (g == tid) mr = mref[g];
+      a.pm[slot * GP + tid] = mr;
       a.pl[slot * GP + tid] = l;
     }
     {
