@@ -44,7 +44,7 @@ namespace zkv {
 constexpr int kScanSub = 512;       // tokens per scan sub-chunk (1 per thread)
 constexpr int kScanThreads = 512;
 constexpr int kColCap = 8176;       // tokens per histogram column per segment (sum < 2^32)
-constexpr float kHeadroom = 8.f;    // log2 units added to the running maximum on growth
+constexpr float kHeadroom = 10.f;   // log2 units added to the running maximum on growth
 constexpr int kMergeQ = 4;          // codeword quarters (64 codewords each) per value stage
 constexpr int kMergeC = kCodebook / kMergeQ;
 constexpr int kMergeRows = 32;      // (sequence, head) rows per merge pass
@@ -654,15 +654,15 @@ struct ScanCfg {
   static constexpr int CBUFW = J * PR * CODEW;   // words of one code staging buffer
 };
 
-// master[(s, c, g)] = (master (if any) + histogram value) * scale[g], where the histogram
+// dst[(s, c, g)] = (master (if any) + histogram value) * scale[g], where the histogram
 // value of (s, c, g) is the sum over token slots j of hi * 2^-19 + lo * 2^-38 in column
 // j * COMBOS + s * GP + g of code row c.  Threads walk the tables row by row (consecutive
 // threads, consecutive words: no bank conflicts); the J columns of one (s, g) are combined
 // with xor-shuffles (they are COMBOS lanes apart).
 template <class C, int GP>
 __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t* vlo,
-                                            float* master, int Sv, bool has_master,
-                                            const float (&scale)[GP], int tid) {
+                                            const float* master, float* dst, int Sv,
+                                            bool has_master, const float (&scale)[GP], int tid) {
   const int lane = tid & 31;
   const int total = kCodebook * C::VW;           // words per table
 #pragma unroll 4
@@ -684,7 +684,7 @@ __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t*
         if (q == g) sc = scale[q];
       const size_t f = ((size_t)ss * kCodebook + cc) * GP + g;
       const float old = has_master ? master[f] : 0.f;
-      master[f] = (old + (float)v) * sc;
+      dst[f] = (old + (float)v) * sc;
     }
   }
 }
@@ -903,9 +903,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       }
       if (grow) {   // uniform: every thread read the same maxima
         // New reference = maximum + kHeadroom: later sub-chunks rarely exceed it, so folds
-        // stay rare.  Precision: the segment's largest p is >= 2^-kHeadroom and the
-        // fixed-point error is <= 8176 * 2^-39 = 2^-26 absolute, i.e. <= 2^(kHeadroom - 26)
-        // relative to the segment's mass.
+        // stay rare.  Precision: the segment's largest p is >= 2^-kHeadroom and its
+        // fixed-point error is <= (tokens <= 2^14) * 2^-39 = 2^-25 absolute, i.e.
+        // <= 2^(kHeadroom - 25) = 2^-15 relative to the segment's mass.
         float alpha[GP];
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
@@ -918,7 +918,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
           // fold the integer histograms (relative to the old reference) into the fp32
           // master and rescale it to the new reference
           __syncthreads();   // every reduction so far has landed
-          fold_tables<C, GP>(vhi, vlo, master, Sv, has_master, alpha, tid);
+          fold_tables<C, GP>(vhi, vlo, master, master, Sv, has_master, alpha, tid);
           __syncthreads();
           uint4* z = reinterpret_cast<uint4*>(vhi);
           const int nz = 2 * kCodebook * C::VW / 4;
@@ -979,12 +979,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       float one[GP];
 #pragma unroll
       for (int g = 0; g < GP; ++g) one[g] = 1.f;
-      fold_tables<C, GP>(vhi, vlo, master, Sv, has_master, one, tid);
+      // straight into the segment's slot (the next segment's first barrier orders these reads
+      // of the shared tables before they are reused)
+      fold_tables<C, GP>(vhi, vlo, master, a.pw + slot * (int64_t)ntab, Sv, has_master, one, tid);
     }
-    __syncthreads();
-    float4* dst = reinterpret_cast<float4*>(a.pw + slot * (int64_t)ntab);
-    const float4* srcm = reinterpret_cast<const float4*>(master);
-    for (int f = tid; f < ntab / 4; f += kScanThreads) dst[f] = srcm[f];
   }
 }
 
