@@ -8,7 +8,7 @@
 // log-sum-exp combine of the compressed part with the dense recency window.
 //
 // Four kernels per call:
-//   1. lut_kernel    q_tilde = H q / sqrt(d) (float64, one rounding), per stage
+//   1. lut_kernel    q_tilde = H q / sqrt(d) (float32 transform), per stage
 //                    LUT_s[c] = (scale * log2 e) * q_tilde . Ck_s[c] -> workspace; the dense
 //                    window attention of every (sequence, kv head); prefix sums of the
 //                    compressed lengths that partition the token space among scan CTAs.
@@ -178,7 +178,7 @@ __device__ __forceinline__ int64_t clamp_win_len(const DecodeArgs& a, int b) {
 // 1. Query rotation + lookup tables; window attention; length prefix sums.
 //    1-D grid: [0, n_lut_blocks) tables, then one block per (sequence, kv head) window.
 // ------------------------------------------------------------------------------------------
-constexpr int kLutC = 64;     // codewords per block
+constexpr int kLutC = 128;    // codewords per block (2 per thread)
 constexpr int kLutH = 32;     // attached query heads per block (b * G + g)
 
 template <int D>
@@ -270,14 +270,16 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
         kf[e] = v.x;
         kf[e + 1] = v.y;
       }
+      float d[GP];
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
-        float d = 0.f;
+        d[g] = 0.f;
 #pragma unroll
-        for (int e = 0; e < PL; ++e) d = fmaf(qf[g][e], kf[e], d);
-        d = warp_sum_f32(d);
-        if (lane == 0) sc[tt * GP + g] = d;
+        for (int e = 0; e < PL; ++e) d[g] = fmaf(qf[g][e], kf[e], d[g]);
       }
+      int hd = 0;
+      const float tot = TransposeSum<GP, GP, 16>::run(d, lane, hd);
+      if ((lane & (32 / GP - 1)) == 0) sc[tt * GP + hd] = tot;
     }
     __syncthreads();
     // tile maximum, probabilities
@@ -343,7 +345,11 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
   if (tid < GP) {
     float l = 0.f;
     for (int w = 0; w < 8; ++w) l += red[w * GP + tid];
-    a.wm[pair * GP + tid] = m_run[tid];
+    float mr = 0.f;
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+      if (g == tid) mr = m_run[g];
+    a.wm[pair * GP + tid] = mr;
     a.wl[pair * GP + tid] = l;
   }
   for (int f = tid; f < GP * D; f += 256) {
@@ -433,57 +439,60 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
     }
     cp_async_commit();
   }
-  // rotated queries of the attached heads j = b*G + g: this warp's rows are loaded first
-  // (independent loads), then transformed
+  // rotated queries of the attached heads j = b*G + g (float32 transform): this warp's rows
+  // are loaded first (independent loads), then transformed
   {
     constexpr int NR = kLutH / 8;
-    double v[NR][E];
+    float v[NR][E];
 #pragma unroll
     for (int k = 0; k < NR; ++k) {
       const int j = hg * kLutH + warp + 8 * k;
       if (j < a.B * a.G) {
         const int b = j / a.G, g = j % a.G;
-        const int64_t off = ((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D;
-        load_row_f64<E>(a.q, ZKV_DTYPE_F16, off, lane, v[k]);
+        const __half* qr = a.q + ((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D + lane;
+#pragma unroll
+        for (int q = 0; q < E; ++q) v[k][q] = __half2float(qr[q * 32]);
       } else {
 #pragma unroll
-        for (int q = 0; q < E; ++q) v[k][q] = 0.0;
+        for (int q = 0; q < E; ++q) v[k][q] = 0.f;
       }
     }
+    const float rs = (float)a.rot;
 #pragma unroll
     for (int k = 0; k < NR; ++k) {
-      fwht_warp_f64<D>(v[k], lane);
+      fwht_warp_f32<D>(v[k], lane);
 #pragma unroll
-      for (int q = 0; q < E; ++q) sm.qT[q * 32 + lane][warp + 8 * k] = (float)(v[k][q] * a.rot);
+      for (int q = 0; q < E; ++q) sm.qT[q * 32 + lane][warp + 8 * k] = v[k][q] * rs;
     }
   }
   cp_async_wait_all();
   __syncthreads();
-  // thread (codeword cc, head group hq): 8 dot products; the codeword is read as 16-byte
-  // pieces (conflict-free thanks to the swizzle), the query columns are broadcasts
-  const int cc = tid & (kLutC - 1), hq = tid >> 6;   // 4 groups of 8 heads
-  const float* row = sm.cb + cc * D;
-  const int sw = cc & 7;
-  float acc[8];
+  // thread (codewords cc and cc + 64, head group hq): 16 dot products; the codewords are read
+  // as 16-byte pieces (conflict-free thanks to the swizzle), the query columns are broadcasts
+  const int cc = tid & 63, hq = tid >> 6;   // 4 groups of 8 heads
+  const float* row0 = sm.cb + cc * D;
+  const float* row1 = sm.cb + (cc + 64) * D;
+  const int sw = cc & 7;                   // (cc + 64) & 7 == cc & 7
+  float acc[2][8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[u][k] = 0.f;
 #pragma unroll 2
   for (int qq = 0; qq < D / 4; ++qq) {
-    const float4 c4 = *reinterpret_cast<const float4*>(row + 4 * (qq ^ sw));
-    const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+    const float4 ca = *reinterpret_cast<const float4*>(row0 + 4 * (qq ^ sw));
+    const float4 cb = *reinterpret_cast<const float4*>(row1 + 4 * (qq ^ sw));
+    const float cv[2][4] = {{ca.x, ca.y, ca.z, ca.w}, {cb.x, cb.y, cb.z, cb.w}};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int i = 4 * qq + e;
       const float4 q0 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8]);
       const float4 q1 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8 + 4]);
-      acc[0] = fmaf(q0.x, cv[e], acc[0]);
-      acc[1] = fmaf(q0.y, cv[e], acc[1]);
-      acc[2] = fmaf(q0.z, cv[e], acc[2]);
-      acc[3] = fmaf(q0.w, cv[e], acc[3]);
-      acc[4] = fmaf(q1.x, cv[e], acc[4]);
-      acc[5] = fmaf(q1.y, cv[e], acc[5]);
-      acc[6] = fmaf(q1.z, cv[e], acc[6]);
-      acc[7] = fmaf(q1.w, cv[e], acc[7]);
+      const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[u][k] = fmaf(qv[k], cv[u][e], acc[u][k]);
     }
   }
 #pragma unroll
@@ -491,8 +500,9 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
     const int j = hg * kLutH + hq * 8 + k;
     if (j < a.B * a.G) {
       const int b = j / a.G, g = j % a.G;
-      a.lut[((((int64_t)b * a.Hkv + kvh) * a.Sk + s) * kCodebook + c0 + cc) * GP + g] =
-          acc[k] * a.scale_log2;
+      float* dst = a.lut + ((((int64_t)b * a.Hkv + kvh) * a.Sk + s) * kCodebook + c0 + cc) * GP + g;
+      dst[0] = acc[0][k] * a.scale_log2;
+      dst[64 * GP] = acc[1][k] * a.scale_log2;
     }
   }
 }
@@ -656,7 +666,8 @@ struct ScanCfg {
 
 // dst[(s, c, g)] = (master (if any) + histogram value) * scale[g], where the histogram
 // value of (s, c, g) is the sum over token slots j of hi * 2^-19 + lo * 2^-38 in column
-// j * COMBOS + s * GP + g of code row c.  Threads walk the tables row by row (consecutive
+// j * COMBOS + s * GP + g of code row c.  The integer sums are exact; converting them to
+// float32 and adding costs a few roundings, <= 2^-21 relative per entry.  Threads walk the tables row by row (consecutive
 // threads, consecutive words: no bank conflicts); the J columns of one (s, g) are combined
 // with xor-shuffles (they are COMBOS lanes apart).
 template <class C, int GP>
@@ -669,7 +680,7 @@ __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t*
   for (int w0 = tid - lane; w0 < total; w0 += kScanThreads) {
     const int wi = w0 + lane;                      // total is a multiple of 32
     const int cc = wi / C::VW, col = wi % C::VW;
-    double v = (double)vhi[wi] * (1.0 / 524288.0) + (double)(int32_t)vlo[wi] * (1.0 / 274877906944.0);
+    float v = fmaf((float)(int32_t)vlo[wi], 0x1p-38f, (float)vhi[wi] * 0x1p-19f);
     if constexpr (C::PASSES == 1) {
 #pragma unroll
       for (int o = C::COMBOS; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -684,7 +695,7 @@ __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t*
         if (q == g) sc = scale[q];
       const size_t f = ((size_t)ss * kCodebook + cc) * GP + g;
       const float old = has_master ? master[f] : 0.f;
-      dst[f] = (old + (float)v) * sc;
+      dst[f] = (old + v) * sc;
     }
   }
 }
@@ -831,17 +842,33 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       const float* src = a.lut + (int64_t)pr * Sk * kCodebook * GP;
       const int rsh = __ffs(Rk) - 1;
       const int n = Sk * kCodebook * Rk;
-      for (int f0 = 0; f0 < n; f0 += 4 * kScanThreads) {
-        float v[4][GP];
+      constexpr int NB = GP >= 8 ? 4 : 8;   // items in flight per thread
+      for (int f0 = 0; f0 < n; f0 += NB * kScanThreads) {
+        float v[NB][GP];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < NB; ++u) {
           const int f = f0 + u * kScanThreads + tid;
-          const int sc = f >> rsh;
+          const float* e = src + (int64_t)(f >> rsh) * GP;   // 16-byte aligned for GP >= 4
+          if (f < n) {
+            if constexpr (GP >= 4) {
 #pragma unroll
-          for (int g = 0; g < GP; ++g) v[u][g] = (f < n && g < G) ? __ldg(src + (int64_t)sc * GP + g) : 0.f;
+              for (int g = 0; g < GP; g += 4) {
+                const float4 t4 = __ldg(reinterpret_cast<const float4*>(e + g));
+                v[u][g] = t4.x; v[u][g + 1] = t4.y; v[u][g + 2] = t4.z; v[u][g + 3] = t4.w;
+              }
+            } else if constexpr (GP == 2) {
+              const float2 t2 = __ldg(reinterpret_cast<const float2*>(e));
+              v[u][0] = t2.x; v[u][1] = t2.y;
+            } else {
+              v[u][0] = __ldg(e);
+            }
+          }
+#pragma unroll
+          for (int g = 0; g < GP; ++g)
+            if (g >= G) v[u][g] = 0.f;   // padded heads (not written by the table kernel)
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < NB; ++u) {
           const int f = f0 + u * kScanThreads + tid;
           if (f < n) {
             float* dst = lut + (size_t)f * GP;   // (sc * Rk + copy) * GP

@@ -71,6 +71,61 @@ __device__ __forceinline__ void fwht_warp_f64(double (&v)[D / 32], int lane) {
   }
 }
 
+// The same transform in float32 (each level rounds once), for operands that only feed float32
+// arithmetic afterwards (the decode-time query rotation).
+template <int D>
+__device__ __forceinline__ void fwht_warp_f32(float (&v)[D / 32], int lane) {
+  constexpr int E = D / 32;
+#pragma unroll
+  for (int lm = 1; lm < 32; lm <<= 1) {
+    const bool upper = (lane & lm) != 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[j], lm);
+      v[j] = upper ? (o - v[j]) : (v[j] + o);
+    }
+  }
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      if ((j & h) == 0) {
+        const float a = v[j], b = v[j + h];
+        v[j] = a + b;
+        v[j + h] = a - b;
+      }
+    }
+  }
+}
+
+// Warp sums of NT values per lane in NT - 1 + log2(32 / NT) shuffles (instead of 5 NT): at
+// each level a lane keeps half of its live values (x[0 .. N-1]) and sends the other half to its
+// partner.  Afterwards every lane holds the full sum of value `h` (accumulated into h).
+template <int NT, int N, int O>
+struct TransposeSum {
+  __device__ __forceinline__ static float run(float (&x)[NT], int lane, int& h) {
+    constexpr int H = N / 2;
+    const bool up = (lane & O) != 0;
+#pragma unroll
+    for (int k = 0; k < H; ++k) {
+      const float send = up ? x[k] : x[k + H];
+      const float keep = up ? x[k + H] : x[k];
+      x[k] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+    }
+    if (up) h += H;
+    return TransposeSum<NT, H, O / 2>::run(x, lane, h);
+  }
+};
+template <int NT, int O>
+struct TransposeSum<NT, 1, O> {
+  __device__ __forceinline__ static float run(float (&x)[NT], int, int&) {
+    float v = x[0];
+#pragma unroll
+    for (int o = O; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+  }
+};
+
 // Load the E strided elements (j*32 + lane) of a row (fp16 or fp32) as doubles.
 template <int E>
 __device__ __forceinline__ void load_row_f64(const void* base, int dtype, int64_t off, int lane,
