@@ -39,8 +39,8 @@ WORKLOAD = "llama3_8b_32k"
 # the scan kernel source is unchanged (hash of decode.cu at capture time).
 # DRAM bytes (read + write) of one scan_kernel launch on this workload, from one ncu capture
 # (profiles/scan_kernel_llama3_8b_32k.md), valid while the scan's source is unchanged.
-SCAN_TRAFFIC = {"scan_src_sha1": "f0f9744a4e31147197812ae385e253632f9d0c0c",
-                "bytes_per_launch": 17798144}
+SCAN_TRAFFIC = {"scan_src_sha1": "4059898c4288ecf49174cd5293ae938bc34b500d",
+                "bytes_per_launch": 17808896}
 
 
 def parse():
@@ -223,6 +223,14 @@ def oracle_rate(wl, seconds: float, n_tok_cap: int | None = None):
                             "cores": 1}
 
 
+def workload_config(wl):
+    """The workload fields both arms report."""
+    return {"workload": WORKLOAD, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
+            "head_dim": wl.d, "context": wl.T, "window": wl.W, "stages_k": wl.Sk,
+            "stages_v": wl.Sv, "codewords": 256,
+            "step": "append (evict+encode 1 token/seq) + decode attention"}
+
+
 def run_reference(args):
     from compressed_decode_attention_zkv_b200 import inputs as I
     wl = I.workload(WORKLOAD)
@@ -263,7 +271,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * total / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "sample": "bounded CPU sample per step"},
+            "config": dict(workload_config(wl), sample="bounded CPU sample per step"),
             "cpu_baseline": cpu,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -552,14 +560,10 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * elapsed / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
-                       "head_dim": wl.d, "context": wl.T, "window": wl.W,
-                       "stages_k": wl.Sk, "stages_v": wl.Sv, "codewords": 256,
-                       "compressed_tokens_per_seq_avg": Tc_avg,
-                       "step": "append (evict+encode 1 token/seq) + decode attention",
-                       "l2": f"{R} rotating replicas x {rep_mb:.1f} MB = {R * rep_mb:.0f} MB > 126 MB L2",
-                       "parallelism": f"replicas x{world}, no collective",
-                       "graph": "one CUDA graph per replica step"},
+            "config": dict(workload_config(wl), compressed_tokens_per_seq_avg=Tc_avg,
+                           l2=f"{R} rotating replicas x {rep_mb:.1f} MB = {R * rep_mb:.0f} MB > 126 MB L2",
+                           parallelism=f"replicas x{world}, no collective",
+                           graph="one CUDA graph per replica step"),
             "gpu_launches": 6 * args.steps,   # append (2), lut, scan, merge, finalize
             "roofline": roof,
             "kernels_s": per,
