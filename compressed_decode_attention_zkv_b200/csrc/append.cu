@@ -58,6 +58,7 @@ __global__ void __cluster_dims__(kAppendCl, 1, 1) __launch_bounds__(256)
   constexpr int LD = AppendSmem<D>::LD;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AppendSmem<D>& sm = *reinterpret_cast<AppendSmem<D>*>(smem_raw);
+  pdl_trigger();   // the length update may launch now; it waits for this kernel's completion
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -298,6 +299,7 @@ __global__ void __cluster_dims__(kAppendCl, 1, 1) __launch_bounds__(256)
 
 __global__ void append_lengths_kernel(int B, int64_t Tcap, int64_t Wcap, int32_t* win_len,
                                       int32_t* win_head, int32_t* comp_len) {
+  pdl_wait();   // the encode kernel read the pre-step lengths
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;
   const int64_t wl = win_len[b];
@@ -343,8 +345,8 @@ extern "C" int zkv_rvq_append(const zkv_append_params* p, void* stream) {
     default: append_cluster_kernel<256><<<grid, 256, sizeof(AppendSmem<256>), st>>>(*p, rot); break;
   }
   ZKV_CHECK_LAUNCH();
-  append_lengths_kernel<<<(p->B + 127) / 128, 128, 0, st>>>(p->B, p->Tcap, p->Wcap, p->win_len,
-                                                           p->win_head, p->comp_len);
-  ZKV_CHECK_LAUNCH();
+  if (launch_pdl(append_lengths_kernel, dim3((p->B + 127) / 128), dim3(128), 0, st, p->B, p->Tcap,
+                 p->Wcap, p->win_len, p->win_head, p->comp_len) != cudaSuccess)
+    return ZKV_ERR_CUDA;
   return ZKV_OK;
 }

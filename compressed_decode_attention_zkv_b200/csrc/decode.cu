@@ -711,6 +711,7 @@ template <int GP, int SKP, int SVP>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   using C = ScanCfg<GP, SKP, SVP>;
   extern __shared__ __align__(16) unsigned char smraw[];
+  pdl_wait();   // tables, prefix sums and codes
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Rk = a.Rk, Sk = a.Sk, Sv = a.Sv, G = a.G;
   const int ntab = Sv * kCodebook * GP;           // histogram entries (s, c, g)
@@ -1050,12 +1051,13 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
   const int tid = threadIdx.x;
   const int qtr = blockIdx.x, s = blockIdx.y, kvh = blockIdx.z;
   const int c0 = qtr * kMergeC;
-  const int64_t share = *a.share;
   {
     const float* src = a.Cv + (((size_t)kvh * a.Sv + s) * kCodebook + c0) * D;
     for (int f = tid; f < kMergeC * D / 4; f += 256) cp_async16(Cs + 4 * f, src + 4 * f);
     cp_async_commit();
   }
+  pdl_wait();   // segment partials of the scan
+  const int64_t share = *a.share;
   const int nrows = a.B * GP;
   const int e = tid % D, grp = tid / D;
   for (int r0 = 0; r0 < nrows; r0 += kMergeRows) {
@@ -1165,6 +1167,17 @@ __global__ void __launch_bounds__(256) finalize_kernel(DecodeArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pair = blockIdx.x;
   const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
+  // window terms of this warp's first head (written by the table kernel, which completed before
+  // the scan started): loaded before waiting for the merge
+  const int g0 = warp;
+  float mw0 = -INFINITY, lw0 = 0.f, ow0[E];
+  if (g0 < a.G) {
+    mw0 = a.wm[pair * GP + g0];
+    lw0 = a.wl[pair * GP + g0];
+#pragma unroll
+    for (int q = 0; q < E; ++q) ow0[q] = a.wo[(pair * GP + g0) * D + q * 32 + lane];
+  }
+  pdl_wait();   // stage partials of the merge
   if (tid < GP) {
     int64_t first, last;
     pair_slots(a, pair, *a.share, first, last);
@@ -1191,15 +1204,6 @@ __global__ void __launch_bounds__(256) finalize_kernel(DecodeArgs a) {
     }
     mstar_s[tid] = m;
     lstar_s[tid] = l;
-  }
-  // window terms of this warp's first head, loaded before the barrier
-  const int g0 = warp;
-  float mw0 = -INFINITY, lw0 = 0.f, ow0[E];
-  if (g0 < a.G) {
-    mw0 = a.wm[pair * GP + g0];
-    lw0 = a.wl[pair * GP + g0];
-#pragma unroll
-    for (int q = 0; q < E; ++q) ow0[q] = a.wo[(pair * GP + g0) * D + q * 32 + lane];
   }
   const int nparts = a.Sv * kMergeQ;   // a multiple of 4, at most 32
   for (int f = tid; f < GP * D; f += 256) {
@@ -1252,8 +1256,8 @@ static inline void trace(void* const* ev, int i, cudaStream_t st) {
 template <int GP, int SKP, int SVP>
 static int launch_scan(const DecodeArgs& a, size_t smem, cudaStream_t st) {
   if (ensure_smem_limit(scan_kernel<GP, SKP, SVP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
-  scan_kernel<GP, SKP, SVP><<<a.grid, kScanThreads, smem, st>>>(a);
-  ZKV_CHECK_LAUNCH();
+  if (launch_pdl(scan_kernel<GP, SKP, SVP>, dim3(a.grid), dim3(kScanThreads), smem, st, a) != cudaSuccess)
+    return ZKV_ERR_CUDA;
   return ZKV_OK;
 }
 
@@ -1288,6 +1292,8 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
     const int64_t blocks = (int64_t)a.n_lut_blocks + (int64_t)a.B * a.Hkv;
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
+    // a normal launch: the caller's preceding work (which may write q) must be complete, since
+    // the table blocks do not wait
     lut_kernel<D, GP><<<(unsigned)blocks, 256, smem, st>>>(a);
     ZKV_CHECK_LAUNCH();
   }
@@ -1309,10 +1315,9 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     const size_t smem = ((size_t)kMergeC * D + (size_t)kMergeC * kMergeRows) * sizeof(float);
     if (ensure_smem_limit(merge_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const dim3 grid((unsigned)kMergeQ, (unsigned)a.Sv, (unsigned)a.Hkv);
-    merge_kernel<D, GP><<<grid, 256, smem, st>>>(a);
-    ZKV_CHECK_LAUNCH();
-    finalize_kernel<D, GP><<<(unsigned)(a.B * a.Hkv), 256, 0, st>>>(a);
-    ZKV_CHECK_LAUNCH();
+    if (launch_pdl(merge_kernel<D, GP>, grid, dim3(256), smem, st, a) != cudaSuccess) return ZKV_ERR_CUDA;
+    if (launch_pdl(finalize_kernel<D, GP>, dim3((unsigned)(a.B * a.Hkv)), dim3(256), 0, st, a) != cudaSuccess)
+      return ZKV_ERR_CUDA;
   }
   trace(ev, 3, st);
   return ZKV_OK;

@@ -23,6 +23,34 @@ inline bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
     if (cudaGetLastError() != cudaSuccess) return ZKV_ERR_CUDA; \
   } while (0)
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may start before the
+// previous kernel on the stream has finished; pdl_wait() blocks until that kernel has
+// completed and its memory is visible (it returns at once for a normal launch).  A kernel's
+// blocks all pass their pdl_wait before they exit, so its completion implies the completion of
+// everything before it on the stream.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream launch now (its blocks that do not read this kernel's
+// results may run concurrently; the others pdl_wait).
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // 16-byte asynchronous global -> shared copy (both addresses 16-byte aligned).
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
