@@ -8,6 +8,38 @@
 
 namespace zkv {
 
+// ------------------------------------------------------------------------------------------
+// Row addressing: generic strided (b, t, h) rows of zkv_rvq_encode.
+// ------------------------------------------------------------------------------------------
+struct StridedRows {
+  int64_t n_tok, n_rows;  // n_rows = n_batch * n_tok rows per head
+  const void* x;
+  int x_dtype, rotate;
+  int64_t x_sb, x_st, x_sh;
+  uint8_t* codes;
+  int64_t c_sb, c_st, c_sh;
+  float* norms;
+  int64_t n_sb, n_st, n_sh;
+
+  __device__ bool valid(int64_t j, int) const { return j < n_rows; }
+  __device__ const void* src() const { return x; }
+  __device__ int dtype() const { return x_dtype; }
+  __device__ bool do_rotate() const { return rotate != 0; }
+  __device__ int64_t x_off(int64_t j, int h) const {
+    const int64_t b = j / n_tok, t = j - b * n_tok;
+    return b * x_sb + t * x_st + (int64_t)h * x_sh;
+  }
+  __device__ void store(int64_t j, int h, int S, const uint8_t* code, const float* nrm) const {
+    const int64_t b = j / n_tok, t = j - b * n_tok;
+    uint8_t* c = codes + b * c_sb + t * c_st + (int64_t)h * c_sh;
+    for (int s = 0; s < S; ++s) c[s] = code[s];
+    if (norms) {
+      float* n = norms + b * n_sb + t * n_st + (int64_t)h * n_sh;
+      for (int s = 0; s < S; ++s) n[s] = nrm[s];
+    }
+  }
+};
+
 __device__ __forceinline__ double candidate_margin(double rnorm, float cn_max, int D) {
   const double u = 1.0 / 16777216.0;
   const double g = (double)D * u / (1.0 - (double)D * u);

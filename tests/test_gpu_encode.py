@@ -169,3 +169,24 @@ def test_encode_then_reconstruct_plus_residual_identity():
     y = O.rotate_to_f32(x)
     resid = np.linalg.norm(y.astype(np.float64) - xh, axis=1)
     np.testing.assert_allclose(resid, norms[0, :, 0, -1].cpu().numpy(), rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("kind", ["k", "v"])
+def test_encode_full_size_sampled(kind):
+    """prefill_encode_64k at full size (65536 tokens x 8 kv heads, d = 128, S = 8), encoded in
+    the launch configuration the benchmark times; 256 sampled rows against the oracle, the
+    residual norms of every row non-increasing."""
+    wl = I.workload("prefill_encode_64k")
+    books = I.train_codebooks(wl, kind)                   # [8][8][256][128]
+    x = I.kv_tokens(wl, kind, 0, 0, wl.T)                 # [Hkv][T][d] fp16
+    codes, norms = zkv.rvq_encode(_cuda(x).permute(1, 0, 2), _cuda(books))
+    codes = codes[0].cpu().numpy()                        # [T, H, S]
+    norms = norms[0].cpu().numpy()
+    rng = np.random.default_rng(7)
+    for h in range(wl.Hkv):
+        rows = np.sort(rng.choice(wl.T, 32, replace=False))
+        rows[0], rows[-1] = 0, wl.T - 1
+        _check_codes(x[h, rows], books[h], codes[rows, h], norms[rows, h], f"{kind}/h{h}")
+    # every row: the norms after each stage never increase (codeword 0 is zero)
+    assert np.all(np.diff(norms.astype(np.float64), axis=2) <= 1e-5 * (1.0 + norms[..., :-1]))
+    assert np.all(np.isfinite(norms))
