@@ -31,7 +31,7 @@ namespace zkv {
 
 constexpr int kTcM = 128;          // rows per CTA (TMEM lanes)
 constexpr int kTcN = 256;          // codewords (TMEM columns)
-constexpr int kTcList = 32;        // candidates kept per row after filter 1
+constexpr int kTcList = 16;        // candidates kept per row after filter 1
 
 template <int D>
 struct TcSmem {
@@ -42,8 +42,12 @@ struct TcSmem {
   float cmax_w[16];
   double rn[kTcM];                                    // ||r|| (float64)
   double part[4][kTcM];                               // partial residual norms
-  float gmin[4][kTcM];                                // per column group row minima (filter 1)
+  float gmin[4][kTcM];                                // per column group row minima (filters 1, 2)
+  double gbest[4][kTcM];                              // per column group best float64 distance
+  int gbz[4][kTcM];
   int ncand[kTcM];
+  int nsurv[kTcM];
+  float d2[kTcM][kTcList];                            // filter-2 distances of the candidates
   uint8_t cand[kTcM][kTcList];                        // filter-1 candidates
   uint8_t code[kTcM][kMaxStages];
   float nrm[kTcM][kMaxStages];
@@ -234,10 +238,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows ma
   const float* CB = books + (size_t)h * S * kCodebook * D;
   for (int s = 0; s < S; ++s) {
     const float* C = CB + (size_t)s * kCodebook * D;
-    // codebook stage -> swizzled panels: chunk f = (codeword n, global chunk gc)
-    for (int f = tid; f < kTcN * D / 4; f += kTcThreads) {
-      const int n = f / (D / 4), gc = f % (D / 4);
-      cp_async16(&sm.b[gc >> 3][tc_chunk(n, gc & 7)], C + (size_t)n * D + gc * 4);
+    // codebook stage -> swizzled panels: chunk f = (codeword n, global chunk gc); a thread's
+    // chunks share gc and n & 7, so its destinations and sources advance by fixed strides
+    {
+      constexpr int CPR = D / 4;                      // chunks per codeword
+      constexpr int NSTEP = kTcThreads / CPR;         // codewords per pass
+      const int n0 = tid / CPR, gc = tid % CPR;
+      float* dst = &sm.b[gc >> 3][tc_chunk(n0, gc & 7)];
+      const float* src = C + (size_t)n0 * D + gc * 4;
+#pragma unroll 4
+      for (int i = 0; i < kTcN / NSTEP; ++i) cp_async16(dst + i * NSTEP * 32, src + (size_t)i * NSTEP * D);
     }
     cp_async_wait_all();
     // residual writes (previous stage) and the copies must be visible to the tensor cores
@@ -310,42 +320,90 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows ma
     __syncthreads();
     const double rn = sm.rn[r];
     {
+      // thresholds are compared in float32, rounded up: a superset of the exact comparison
       const float m1 = fminf(fminf(sm.gmin[0][r], sm.gmin[1][r]), fminf(sm.gmin[2][r], sm.gmin[3][r]));
       const double e1 = 1.02 * 0.00390625 * rn * sqrt((double)cmax) + 1.52587890625e-05 * (double)cmax;
-      const double thr1 = (double)m1 + 2.0 * e1;
+      const float thr1 = __double2float_ru((double)m1 + 2.0 * e1);
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         float dv[32];
         tc_ld32(taddr + 32u * h2, dv);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
+        for (int k = 0; k < 32; k += 4) {
           const int c = g * 64 + 32 * h2 + k;
-          if ((double)(sm.cn[c] - 2.f * dv[k]) <= thr1) {
-            const int slot = atomicAdd(&sm.ncand[r], 1);
-            if (slot < kTcList) sm.cand[r][slot] = (uint8_t)c;
+          const float4 c4 = *reinterpret_cast<const float4*>(&sm.cn[c]);
+          const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (cv[e] - 2.f * dv[k + e] <= thr1) {
+              const int slot = atomicAdd(&sm.ncand[r], 1);
+              if (slot < kTcList) sm.cand[r][slot] = (uint8_t)(c + e);
+            }
           }
         }
       }
     }
+    if (tid < kTcM) sm.nsurv[tid] = 0;
     tc_fence_before();
     __syncthreads();   // also: every TMEM read of this stage is done
-    // filters 2 and 3: one thread per row (column group 0)
-    if (g == 0) {
-      const int n1 = sm.ncand[r];
-      const bool all = n1 > kTcList;   // list overflowed: every codeword is a candidate
-      const int nl = all ? kTcN : n1;
+    // filters 2 and 3, each row's candidates split among its four column-group threads.
+    // Overflowed lists (never seen in practice) fall back to every codeword.
+    const int n1 = sm.ncand[r];
+    const bool all = n1 > kTcList;
+    const int nl = all ? kTcN : n1;
+    if (nl > 1) {
       float m2 = FLT_MAX;
-      for (int k = 0; k < nl; ++k) {
+      for (int k = g; k < nl; k += 4) {
         const int c = all ? k : sm.cand[r][k];
-        m2 = fminf(m2, tc_dist32<P>(sm.a, sm.b, sm.cn, r, c));
+        const float d2 = tc_dist32<P>(sm.a, sm.b, sm.cn, r, c);
+        if (!all) sm.d2[r][k] = d2;
+        m2 = fminf(m2, d2);
       }
-      const double thr2 = (double)m2 + candidate_margin(rn, cmax, D);
+      sm.gmin[g][r] = m2;
+    }
+    __syncthreads();
+    float thr2 = 0.f;
+    if (nl > 1) {
+      const float m2 = fminf(fminf(sm.gmin[0][r], sm.gmin[1][r]), fminf(sm.gmin[2][r], sm.gmin[3][r]));
+      thr2 = __double2float_ru((double)m2 + candidate_margin(rn, cmax, D));
+      int cnt = 0;
+      for (int k = g; k < nl; k += 4) {
+        const float d2 = all ? tc_dist32<P>(sm.a, sm.b, sm.cn, r, k) : sm.d2[r][k];
+        cnt += d2 <= thr2 ? 1 : 0;
+      }
+      if (cnt) atomicAdd(&sm.nsurv[r], cnt);
+    }
+    __syncthreads();
+    {
+      // one survivor: it is the argmin; several: float64 distances, ties to the lowest index
       double best = DBL_MAX;
       int bz = kCodebook;
-      for (int k = 0; k < nl; ++k) {
-        const int c = all ? k : sm.cand[r][k];
-        if (nl > 1 && (double)tc_dist32<P>(sm.a, sm.b, sm.cn, r, c) > thr2) continue;
-        const double dd = nl > 1 ? tc_dist64<P>(sm.a, sm.b, r, c) : 0.0;
+      if (nl == 1) {
+        if (g == 0) bz = sm.cand[r][0];
+      } else if (nl > 1) {
+        const bool exact = sm.nsurv[r] > 1;
+        for (int k = g; k < nl; k += 4) {
+          const int c = all ? k : sm.cand[r][k];
+          const float d2 = all ? tc_dist32<P>(sm.a, sm.b, sm.cn, r, k) : sm.d2[r][k];
+          if (d2 > thr2) continue;
+          const double dd = exact ? tc_dist64<P>(sm.a, sm.b, r, c) : 0.0;
+          if (dd < best || (dd == best && c < bz)) {
+            best = dd;
+            bz = c;
+          }
+        }
+      }
+      sm.gbest[g][r] = best;
+      sm.gbz[g][r] = bz;
+    }
+    __syncthreads();
+    if (g == 0) {
+      double best = sm.gbest[0][r];
+      int bz = sm.gbz[0][r];
+#pragma unroll
+      for (int q = 1; q < 4; ++q) {
+        const double dd = sm.gbest[q][r];
+        const int c = sm.gbz[q][r];
         if (dd < best || (dd == best && c < bz)) {
           best = dd;
           bz = c;
@@ -402,6 +460,7 @@ template <int D>
 constexpr size_t tc_smem_bytes() {
   return sizeof(TcSmem<D>) + 1024;   // + alignment of the operand panels
 }
+static_assert(sizeof(TcSmem<128>) + 1024 <= 227 * 1024, "tensor-core encode tile exceeds shared memory");
 
 int launch_encode_tc(const StridedRows& map, int64_t n_head, int d, int S, const float* books,
                      cudaStream_t st) {
