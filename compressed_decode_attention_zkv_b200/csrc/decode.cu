@@ -45,6 +45,10 @@ constexpr int kScanSub = 512;       // tokens per scan sub-chunk (1 per thread)
 constexpr int kScanThreads = 512;
 constexpr int kColCap = 8176;       // tokens per histogram column per segment (sum < 2^32)
 constexpr float kHeadroom = 10.f;   // log2 units added to the running maximum on growth
+// Setup cost of one scan segment (table fill, histogram zeroing, final fold: about 11K cycles)
+// in tokens of the scan loop (about 5.7 cycles per token): the token space is partitioned so
+// that tokens + kSegCost x segments is equal across scan CTAs.
+constexpr int64_t kSegCost = 1900;
 constexpr int kMergeQ = 4;          // codeword quarters (64 codewords each) per value stage
 constexpr int kMergeC = kCodebook / kMergeQ;
 constexpr int kMergeRows = 32;      // (sequence, head) rows per merge pass
@@ -84,8 +88,8 @@ struct DecodePlan {
   int G, GP, SKP, SVP, Rk, grid;
   int64_t cap, slots;
   size_t scan_smem;
-  size_t off_lut, off_pre, off_share, off_pm, off_pl, off_pw, off_wm, off_wl, off_wo, off_so,
-      total;
+  size_t off_lut, off_pre, off_bounds, off_vs, off_pfirst, off_plast, off_pm, off_pl, off_pw,
+      off_wm, off_wl, off_wo, off_so, total;
 };
 
 static size_t scan_smem_bytes(int Rk, int Sk, int Sv, int GP, const VMap& v) {
@@ -114,7 +118,8 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   pl.cap = (int64_t)kColCap * v.J;
   const int64_t bound = pairs * p->max_comp_len;
   const int sms = sm_count();
-  int64_t g1 = (bound + pl.cap - 1) / pl.cap;
+  // every CTA's virtual share (tokens + kSegCost per pair) stays below the column capacity
+  int64_t g1 = (bound + kSegCost * pairs + pl.cap - 1) / pl.cap;
   int64_t g2 = std::min<int64_t>(sms, (bound + 1023) / 1024);
   int64_t grid = std::max<int64_t>(1, std::max(g1, g2));
   if (grid > sms) grid = (grid + sms - 1) / sms * sms;
@@ -124,7 +129,10 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   size_t o = 0;
   pl.off_lut = o;   o = align256(o + (size_t)pairs * p->Sk * kCodebook * pl.GP * f);
   pl.off_pre = o;   o = align256(o + (size_t)(pairs + 1) * sizeof(int64_t));
-  pl.off_share = o; o = align256(o + sizeof(int64_t));
+  pl.off_bounds = o; o = align256(o + (size_t)(grid + 1) * sizeof(int64_t));
+  pl.off_vs = o;    o = align256(o + (size_t)(pairs + 1) * sizeof(int64_t));
+  pl.off_pfirst = o; o = align256(o + (size_t)pairs * sizeof(int32_t));
+  pl.off_plast = o; o = align256(o + (size_t)pairs * sizeof(int32_t));
   pl.off_pm = o;    o = align256(o + (size_t)pl.slots * pl.GP * f);
   pl.off_pl = o;    o = align256(o + (size_t)pl.slots * pl.GP * f);
   pl.off_pw = o;    o = align256(o + (size_t)pl.slots * p->Sv * kCodebook * pl.GP * f);
@@ -155,7 +163,10 @@ struct DecodeArgs {
   int32_t* err;
   float* lut;        // [B][Hkv][Sk][256][GP] (heads g >= G unwritten)
   int64_t* pre;      // [B*Hkv + 1] exclusive prefix sums of compressed lengths
-  int64_t* share;    // tokens per scan CTA
+  int64_t* bounds;   // [grid + 1] token range of each scan CTA
+  int64_t* vs;       // [B*Hkv + 1] virtual start of each pair (tokens + kSegCost per nonempty pair)
+  int32_t* pfirst;   // [B*Hkv] first scan CTA covering the pair (> plast when it has no tokens)
+  int32_t* plast;    // [B*Hkv] last scan CTA covering the pair
   float* pm;         // [slots][GP] segment maxima
   float* pl;         // [slots][GP] segment sums of p
   float* pw;         // [slots][Sv][256][GP] segment histograms
@@ -371,13 +382,16 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
     return;
   }
   if (blockIdx.x == 0) {
-    // exclusive prefix sums of the clamped compressed lengths, 256 pairs per round
-    __shared__ int64_t warp_tot[8];
-    __shared__ int64_t carry_s;
+    // exclusive prefix sums of the clamped compressed lengths (pre) and of the virtual lengths
+    // len + kSegCost * (len > 0) (vs), 256 pairs per round
+    __shared__ int64_t warp_tot[2][8];
+    __shared__ int64_t carry_s[2];
     const int npairs = a.B * a.Hkv;
     if (tid == 0) {
-      carry_s = 0;
+      carry_s[0] = 0;
+      carry_s[1] = 0;
       a.pre[0] = 0;
+      a.vs[0] = 0;
     }
     __syncthreads();
     for (int base = 0; base < npairs; base += 256) {
@@ -391,26 +405,82 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
         }
         c = c < a.max_comp ? c : a.max_comp;
       }
-      int64_t x = c;   // inclusive warp scan
+      int64_t x = c, y = c > 0 ? c + kSegCost : 0;   // inclusive warp scans
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+        const int64_t ux = __shfl_up_sync(0xffffffffu, x, o);
+        const int64_t uy = __shfl_up_sync(0xffffffffu, y, o);
+        if (lane >= o) {
+          x += ux;
+          y += uy;
+        }
       }
-      if (lane == 31) warp_tot[warp] = x;
+      if (lane == 31) {
+        warp_tot[0][warp] = x;
+        warp_tot[1][warp] = y;
+      }
       __syncthreads();
-      int64_t off = carry_s;
-      for (int w = 0; w < warp; ++w) off += warp_tot[w];
-      if (pr < npairs) a.pre[pr + 1] = off + x;
+      int64_t ox = carry_s[0], oy = carry_s[1];
+      for (int w = 0; w < warp; ++w) {
+        ox += warp_tot[0][w];
+        oy += warp_tot[1][w];
+      }
+      if (pr < npairs) {
+        a.pre[pr + 1] = ox + x;
+        a.vs[pr + 1] = oy + y;
+      }
       __syncthreads();
-      if (tid == 255) carry_s = off + x;
+      if (tid == 255) {
+        carry_s[0] = ox + x;
+        carry_s[1] = oy + y;
+      }
       __syncthreads();
     }
-    if (tid == 0) {
-      const int64_t acc = carry_s;
-      int64_t sh = (acc + a.grid - 1) / a.grid;
-      sh = (sh + 15) / 16 * 16;
-      *a.share = sh < 16 ? 16 : sh;
+    // scan CTA c covers virtual positions [c V / grid, (c+1) V / grid); a cut inside a pair's
+    // kSegCost gap moves to the pair's first token
+    const int64_t V = carry_s[1], tot = carry_s[0];
+    const int grid = a.grid;
+    for (int c = tid; c <= grid; c += 256) {
+      int64_t x;
+      if (c == 0) {
+        x = 0;
+      } else if (c == grid) {
+        x = tot;
+      } else {
+        const int64_t v = (V / grid) * c + ((V % grid) * c) / grid;
+        int l = 0, r = npairs;   // largest k with vs[k] <= v: vs[l] <= v < vs[r] (vs[npairs] = V > v)
+        while (r - l > 1) {
+          const int m = (l + r) >> 1;
+          if (a.vs[m] <= v) l = m; else r = m;
+        }
+        const int64_t off = v - a.vs[l];
+        const int64_t len = a.pre[l + 1] - a.pre[l];
+        x = off < kSegCost ? a.pre[l] : a.pre[l] + (off - kSegCost < len ? off - kSegCost : len);
+      }
+      a.bounds[c] = x;
+    }
+    __syncthreads();
+    // first and last scan CTA of every pair: the CTAs whose ranges hold its first / last token
+    for (int k = tid; k < npairs; k += 256) {
+      const int64_t p0 = a.pre[k], p1 = a.pre[k + 1];
+      int f = 1, t = 0;
+      if (p1 > p0) {
+        int l = 0, r = grid;   // largest c with bounds[c] <= p0
+        while (r - l > 1) {
+          const int m = (l + r) >> 1;
+          if (a.bounds[m] <= p0) l = m; else r = m;
+        }
+        f = l;
+        l = 0;
+        r = grid;              // largest c with bounds[c] <= p1 - 1
+        while (r - l > 1) {
+          const int m = (l + r) >> 1;
+          if (a.bounds[m] <= p1 - 1) l = m; else r = m;
+        }
+        t = l;
+      }
+      a.pfirst[k] = f;
+      a.plast[k] = t;
     }
   }
   if ((int)blockIdx.x < a.Hkv * a.Sv && tid == 0) {
@@ -725,10 +795,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   float* red = reinterpret_cast<float*>(redk + 2 * C::NW * GP);   // [NW][GP]
 
   const int npairs = a.B * a.Hkv;
-  const int64_t share = *a.share;
-  const int64_t tot = a.pre[npairs];
-  const int64_t lo = (int64_t)blockIdx.x * share;
-  const int64_t hi = lo + share < tot ? lo + share : tot;
+  const int64_t lo = a.bounds[blockIdx.x], hi = a.bounds[blockIdx.x + 1];
   if (lo >= hi) return;
   // last pair whose prefix start is <= lo: block-parallel search, one round of loads per
   // factor of kScanThreads (pre is non-decreasing, so the sampled predicate is a prefix)
@@ -1021,11 +1088,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
 
 // Scan segments (slots) of a pair: scan CTA c covers the pair's tokens iff first <= c <= last;
 // its partial is in slot pair + c.
-__device__ __forceinline__ void pair_slots(const DecodeArgs& a, int64_t pair, int64_t share,
-                                           int64_t& first, int64_t& last) {
-  const int64_t p0 = a.pre[pair], p1 = a.pre[pair + 1];
-  first = p1 > p0 ? p0 / share : 1;
-  last = p1 > p0 ? (p1 - 1) / share : 0;
+__device__ __forceinline__ void pair_slots(const DecodeArgs& a, int64_t pair, int64_t& first,
+                                           int64_t& last) {
+  first = a.pfirst[pair];
+  last = a.plast[pair];
 }
 
 // grid (codeword quarter, value stage, kv head), 256 threads.  The block copies its 64
@@ -1057,7 +1123,6 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
     cp_async_commit();
   }
   pdl_wait();   // segment partials of the scan
-  const int64_t share = *a.share;
   const int nrows = a.B * GP;
   const int e = tid % D, grp = tid / D;
   for (int r0 = 0; r0 < nrows; r0 += kMergeRows) {
@@ -1069,7 +1134,7 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
       if (b < a.B) {
         const int64_t pair = (int64_t)b * a.Hkv + kvh;
         int64_t last;
-        pair_slots(a, pair, share, first, last);
+        pair_slots(a, pair, first, last);
         n = last >= first ? (int)(last - first + 1) : 0;
         first += pair;   // absolute slot index
       }
@@ -1180,7 +1245,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(DecodeArgs a) {
   pdl_wait();   // stage partials of the merge
   if (tid < GP) {
     int64_t first, last;
-    pair_slots(a, pair, *a.share, first, last);
+    pair_slots(a, pair, first, last);
     const int n = last >= first ? (int)(last - first + 1) : 0;
     const float* pmp = a.pm + (pair + first) * GP + tid;
     const float* plp = a.pl + (pair + first) * GP + tid;
@@ -1395,7 +1460,10 @@ extern "C" int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace,
   a.win_len = p->win_len; a.out = p->out; a.lse = p->lse; a.err = p->error_flag;
   a.lut = reinterpret_cast<float*>(ws + pl.off_lut);
   a.pre = reinterpret_cast<int64_t*>(ws + pl.off_pre);
-  a.share = reinterpret_cast<int64_t*>(ws + pl.off_share);
+  a.bounds = reinterpret_cast<int64_t*>(ws + pl.off_bounds);
+  a.vs = reinterpret_cast<int64_t*>(ws + pl.off_vs);
+  a.pfirst = reinterpret_cast<int32_t*>(ws + pl.off_pfirst);
+  a.plast = reinterpret_cast<int32_t*>(ws + pl.off_plast);
   a.pm = reinterpret_cast<float*>(ws + pl.off_pm);
   a.pl = reinterpret_cast<float*>(ws + pl.off_pl);
   a.pw = reinterpret_cast<float*>(ws + pl.off_pw);
