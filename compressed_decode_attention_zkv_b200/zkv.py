@@ -7,7 +7,8 @@ is no fallback path.
 Entry points (same names as the C ABI):
   fwht, rvq_encode, rvq_reconstruct, decode_workspace_size, rvq_decode_attn,
   rvq_decode_attn_noalloc, rvq_append
-plus ``RVQKVCache``, a small owner of one layer's compressed cache built on them
+plus PreparedAppend / PreparedDecode (the same calls with their arguments marshalled once)
+and ``RVQKVCache``, a small owner of one layer's compressed cache built on them
 (prefill -> append -> attend, the append/attend cache interface of the VeloxQuant-MLX page).
 """
 from __future__ import annotations
@@ -343,6 +344,85 @@ def rvq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
                      v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
                      v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag))
     _check("zkv_rvq_append", lib().zkv_rvq_append(ctypes.byref(p), _stream()))
+
+
+class PreparedAppend:
+    """rvq_append with its arguments validated and marshalled once.  The tensors must keep their
+    storage (their contents may change between calls); calling the object runs one serving
+    step on the current stream with no per-call Python work beyond the library call."""
+
+    def __init__(self, new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
+                 v_codes, k_codebooks, v_codebooks, error_flag=None):
+        _need(new_k, "new_k", torch.float16)
+        _need(new_v, "new_v", torch.float16)
+        for n, t in (("win_k", win_k), ("win_v", win_v)):
+            _need(t, n, torch.float16)
+        for n, t in (("win_len", win_len), ("win_head", win_head), ("comp_len", comp_len)):
+            _need(t, n, torch.int32)
+        _need(k_codes, "k_codes", torch.uint8)
+        _need(v_codes, "v_codes", torch.uint8)
+        _need(k_codebooks, "k_codebooks", torch.float32)
+        _need(v_codebooks, "v_codebooks", torch.float32)
+        if error_flag is not None:
+            _need(error_flag, "error_flag", torch.int32)
+        B, Hkv, Tcap, Sk = k_codes.shape
+        self._keep = (new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
+                      k_codebooks, v_codebooks, error_flag)
+        self._p = AppendParams(B=B, Hkv=Hkv, d=new_k.shape[-1], Sk=Sk, Sv=v_codes.shape[3],
+                               Tcap=Tcap, Wcap=win_k.shape[2], new_k=_ptr(new_k),
+                               new_v=_ptr(new_v), win_k=_ptr(win_k), win_v=_ptr(win_v),
+                               win_len=_ptr(win_len), win_head=_ptr(win_head),
+                               comp_len=_ptr(comp_len), k_codes=_ptr(k_codes),
+                               v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
+                               v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag))
+        self._ref = ctypes.byref(self._p)
+        self._fn = lib().zkv_rvq_append
+
+    def __call__(self):
+        st = self._fn(self._ref, torch.cuda.current_stream().cuda_stream)
+        if st != ZKV_OK:
+            raise ZkvError("zkv_rvq_append", st)
+
+
+class PreparedDecode:
+    """rvq_decode_attn with its arguments validated and marshalled once (workspace included).
+    The tensors must keep their storage; max_comp_len must stay an upper bound of every
+    comp_len for as long as the object is used.  Calling it runs one decode step on the current
+    stream and returns (out, lse)."""
+
+    def __init__(self, q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
+                 win_len, out=None, lse=None, max_comp_len=None, softmax_scale=None,
+                 workspace: torch.Tensor | None = None, error_flag=None):
+        B, Hq, d = q.shape
+        if out is None:
+            out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+        if lse is None:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        self._p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
+                                 win_v, win_len, out, lse, max_comp_len, softmax_scale,
+                                 error_flag)
+        need = lib().zkv_decode_workspace_size(ctypes.byref(self._p))
+        if need == 0:
+            raise ZkvError("zkv_decode_workspace_size", ZKV_ERR_INVALID_ARG)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8)
+        if workspace.numel() < need:
+            raise ZkvError("zkv_rvq_decode_attn", ZKV_ERR_WORKSPACE,
+                           f"workspace holds {workspace.numel()} bytes, {need} needed")
+        self.out, self.lse = out, lse
+        self._keep = (q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
+                      win_len, workspace, error_flag)
+        self._ref = ctypes.byref(self._p)
+        self._ws = ctypes.c_void_p(workspace.data_ptr())
+        self._wsn = ctypes.c_size_t(workspace.numel())
+        self._fn = lib().zkv_rvq_decode_attn
+
+    def __call__(self):
+        st = self._fn(self._ref, self._ws, self._wsn, torch.cuda.current_stream().cuda_stream)
+        if st != ZKV_OK:
+            raise ZkvError("zkv_rvq_decode_attn", st)
+        return self.out, self.lse
 
 
 # --------------------------------------------------------------------------------------------

@@ -289,3 +289,46 @@ def test_serving_loop_matches_oracle():
                 st["win_v"], st["win_len"])
         _compare(case, out.cpu().numpy(), lse.cpu().numpy())
     assert int(cache.error_flag.item()) == 0
+
+
+def test_prepared_calls_match_the_plain_entry_points():
+    """PreparedAppend / PreparedDecode (arguments marshalled once) give bit-identical results
+    to rvq_append / rvq_decode_attn over several serving steps."""
+    st = _state(80, B_=3, Hkv=2, d=128, S=4, Tcap=64, Wcap=4, win_len=[4, 4, 2],
+                win_head=[1, 0, 0], comp_len=[10, 0, 33])
+    rng = np.random.default_rng(81)
+    sides = []
+    for _ in range(2):
+        g = {k: _cuda(v.astype(np.int32) if k in ("comp_len", "win_len", "win_head") else v)
+             for k, v in st.items()}
+        g["err"] = torch.zeros(1, dtype=torch.int32, device="cuda")
+        g["new_k"] = torch.zeros((3, 2, 128), dtype=torch.float16, device="cuda")
+        g["new_v"] = torch.zeros((3, 2, 128), dtype=torch.float16, device="cuda")
+        g["q"] = torch.zeros((3, 8, 128), dtype=torch.float16, device="cuda")
+        sides.append(g)
+    a, b = sides
+    app = zkv.PreparedAppend(b["new_k"], b["new_v"], b["win_k"], b["win_v"], b["win_len"],
+                             b["win_head"], b["comp_len"], b["k_codes"], b["v_codes"], b["Ck"],
+                             b["Cv"], error_flag=b["err"])
+    dec = zkv.PreparedDecode(b["q"], b["k_codes"], b["v_codes"], b["comp_len"], b["Ck"], b["Cv"],
+                             b["win_k"], b["win_v"], b["win_len"], max_comp_len=64,
+                             error_flag=b["err"])
+    for step in range(3):
+        nk = _cuda(rng.standard_normal((3, 2, 128)).astype(np.float16))
+        nv = _cuda(rng.standard_normal((3, 2, 128)).astype(np.float16))
+        q = _cuda(rng.standard_normal((3, 8, 128)).astype(np.float16))
+        zkv.rvq_append(nk, nv, a["win_k"], a["win_v"], a["win_len"], a["win_head"],
+                       a["comp_len"], a["k_codes"], a["v_codes"], a["Ck"], a["Cv"],
+                       error_flag=a["err"])
+        o1, l1 = zkv.rvq_decode_attn(q, a["k_codes"], a["v_codes"], a["comp_len"], a["Ck"],
+                                     a["Cv"], a["win_k"], a["win_v"], a["win_len"],
+                                     max_comp_len=64, error_flag=a["err"])
+        b["new_k"].copy_(nk)
+        b["new_v"].copy_(nv)
+        b["q"].copy_(q)
+        app()
+        o2, l2 = dec()
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {step}"
+        for key in ("k_codes", "v_codes", "win_k", "win_v", "comp_len", "win_len", "win_head"):
+            assert torch.equal(a[key], b[key]), f"{key} step {step}"
