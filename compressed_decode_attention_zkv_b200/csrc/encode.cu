@@ -285,13 +285,13 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(zkv_reconstruct_params
 // Launchers
 // ------------------------------------------------------------------------------------------
 int launch_encode_tc(const StridedRows& map, int64_t n_head, int d, int S, const float* books,
-                     cudaStream_t st);   // encode_tc.cu
+                     int* err, cudaStream_t st);   // encode_tc.cu
 
 int launch_encode(const StridedRows& map, int64_t n_head, int d, int S, const float* books,
-                  cudaStream_t st) {
+                  int* err, cudaStream_t st) {
   const double rot = 1.0 / std::sqrt((double)d);
   const int64_t n_rows = map.n_rows;
-  if (n_rows * n_head > 4096 && (d == 64 || d == 128)) return launch_encode_tc(map, n_head, d, S, books, st);
+  if (n_rows * n_head > 4096 && (d == 64 || d == 128)) return launch_encode_tc(map, n_head, d, S, books, err, st);
   if (n_rows * n_head <= 4096) {
     constexpr int R = 8;
     const dim3 grid((unsigned)((n_rows + R - 1) / R), (unsigned)n_head);
@@ -355,7 +355,7 @@ extern "C" int zkv_rvq_encode(const zkv_encode_params* p, void* stream) {
   m.n_sb = p->n_sb;
   m.n_st = p->n_st;
   m.n_sh = p->n_sh;
-  return launch_encode(m, p->n_head, p->d, p->S, p->codebooks,
+  return launch_encode(m, p->n_head, p->d, p->S, p->codebooks, p->error_flag,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -104,9 +104,9 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
   for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-// Bounded wait for phase `parity` of the MMA mbarrier (a lost completion leaves the stage's
-// codes wrong instead of hanging the device).
-__device__ __forceinline__ void tc_wait(uint32_t mbar, uint32_t parity) {
+// Bounded wait for phase `parity` of the MMA mbarrier; false when the limit ran out (the
+// caller then reports ZKV_DEVERR_TIMEOUT and stops instead of hanging the device).
+__device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
   for (uint32_t it = 0; it < (1u << 20); ++it) {
     uint32_t ok;
     asm volatile(
@@ -116,8 +116,9 @@ __device__ __forceinline__ void tc_wait(uint32_t mbar, uint32_t parity) {
         : "=r"(ok)
         : "r"(mbar), "r"(parity)
         : "memory");
-    if (ok) return;
+    if (ok) return true;
   }
+  return false;
 }
 
 // float32 dot-form distance ||c||^2 - 2 r.c of row r and codeword c (sequential-FMA error
@@ -165,7 +166,8 @@ constexpr int kTcThreads = 512;    // 16 warps: 4 per TMEM lane quarter, each 64
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows map,
                                                                   const float* __restrict__ books,
-                                                                  int S, double rot_scale) {
+                                                                  int S, double rot_scale,
+                                                                  int* __restrict__ err) {
   constexpr int E = D / 32;          // elements per lane in the row transform
   constexpr int P = TcSmem<D>::P;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -236,6 +238,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows ma
   const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * 64);
 
   const float* CB = books + (size_t)h * S * kCodebook * D;
+  int stalled = -1;                   // stage whose MMA completion never arrived
   for (int s = 0; s < S; ++s) {
     const float* C = CB + (size_t)s * kCodebook * D;
     // codebook stage -> swizzled panels: chunk f = (codeword n, global chunk gc); a thread's
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows ma
     float cmax = sm.cmax_w[0];
 #pragma unroll
     for (int w = 1; w < kTcN / 32; ++w) cmax = fmaxf(cmax, sm.cmax_w[w]);
-    tc_wait(mbar, (uint32_t)(s & 1));
+    const bool late = !tc_wait(mbar, (uint32_t)(s & 1));
     tc_fence_after();
 
     // filter 1: TF32 distances of this thread's 64 columns; pass 1 takes the minimum, pass 2
@@ -317,7 +320,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows ma
       }
     }
     sm.gmin[g][r] = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3]));
-    __syncthreads();
+    if (__syncthreads_or(late)) {      // uniform: every thread leaves the stage loop together
+      stalled = s;
+      break;
+    }
     const double rn = sm.rn[r];
     {
       // thresholds are compared in float32, rounded up: a superset of the exact comparison
@@ -441,8 +447,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows ma
     }
     // the next stage's first barrier orders these writes before their use
   }
+  if (stalled >= 0) {
+    // no codes are stored; one more bounded wait lets the stage's MMAs finish before the
+    // accumulator columns are freed
+    if (tid == 0 && err != nullptr) atomicOr(err, ZKV_DEVERR_TIMEOUT);
+    if (warp == 0) (void)tc_wait(mbar, (uint32_t)(stalled & 1));
+  }
   __syncthreads();
-  if (g == 0) {
+  if (g == 0 && stalled < 0) {
     const int64_t j = row0 + r;
     if (map.valid(j, h)) map.store(j, h, S, sm.code[r], sm.nrm[r]);
   }
@@ -463,17 +475,17 @@ constexpr size_t tc_smem_bytes() {
 static_assert(sizeof(TcSmem<128>) + 1024 <= 227 * 1024, "tensor-core encode tile exceeds shared memory");
 
 int launch_encode_tc(const StridedRows& map, int64_t n_head, int d, int S, const float* books,
-                     cudaStream_t st) {
+                     int* err, cudaStream_t st) {
   const double rot = 1.0 / std::sqrt((double)d);
   const dim3 grid((unsigned)((map.n_rows + kTcM - 1) / kTcM), (unsigned)n_head);
   switch (d) {
     case 64:
       if (ensure_smem_limit(encode_tc_kernel<64>, tc_smem_bytes<64>()) != cudaSuccess) return ZKV_ERR_CUDA;
-      encode_tc_kernel<64><<<grid, kTcThreads, tc_smem_bytes<64>(), st>>>(map, books, S, rot);
+      encode_tc_kernel<64><<<grid, kTcThreads, tc_smem_bytes<64>(), st>>>(map, books, S, rot, err);
       break;
     case 128:
       if (ensure_smem_limit(encode_tc_kernel<128>, tc_smem_bytes<128>()) != cudaSuccess) return ZKV_ERR_CUDA;
-      encode_tc_kernel<128><<<grid, kTcThreads, tc_smem_bytes<128>(), st>>>(map, books, S, rot);
+      encode_tc_kernel<128><<<grid, kTcThreads, tc_smem_bytes<128>(), st>>>(map, books, S, rot, err);
       break;
     default:
       return ZKV_ERR_UNSUPPORTED;

@@ -26,6 +26,7 @@ LIB_PATH = os.path.join(_PKG, "libzkv.so")
 ZKV_OK, ZKV_ERR_INVALID_ARG, ZKV_ERR_UNSUPPORTED, ZKV_ERR_WORKSPACE, ZKV_ERR_CUDA = range(5)
 ZKV_DEVERR_COMP_LEN = 1
 ZKV_DEVERR_WIN_LEN = 2
+ZKV_DEVERR_TIMEOUT = 4
 ZKV_DTYPE_F16, ZKV_DTYPE_F32 = 0, 1
 CODEBOOK_SIZE = 256
 DECODE_SCRATCH_BYTES = 8 << 20   # ZKV_DECODE_SCRATCH_BYTES: the no-allocation decode's array
@@ -44,7 +45,8 @@ class EncodeParams(ctypes.Structure):
                 ("x", c_void_p), ("x_sb", c_int64), ("x_st", c_int64), ("x_sh", c_int64),
                 ("codebooks", c_void_p),
                 ("codes", c_void_p), ("c_sb", c_int64), ("c_st", c_int64), ("c_sh", c_int64),
-                ("norms", c_void_p), ("n_sb", c_int64), ("n_st", c_int64), ("n_sh", c_int64)]
+                ("norms", c_void_p), ("n_sb", c_int64), ("n_st", c_int64), ("n_sh", c_int64),
+                ("error_flag", c_void_p)]
 
 
 class ReconstructParams(ctypes.Structure):
@@ -166,9 +168,10 @@ def _as4(t: torch.Tensor, name: str) -> torch.Tensor:
 
 def rvq_encode(x: torch.Tensor, codebooks: torch.Tensor, codes: torch.Tensor | None = None,
                norms: torch.Tensor | None = None, rotate: bool = True,
-               with_norms: bool = True):
+               with_norms: bool = True, error_flag: torch.Tensor | None = None):
     """Greedy RVQ of x rows.  x: [B, T, H, d] view (any strides, d contiguous), or [T, H, d],
-    or [N, d] (one head).  codebooks: [H, S, 256, d] float32 contiguous.
+    or [N, d] (one head).  codebooks: [H, S, 256, d] float32 contiguous.  error_flag: optional
+    int32 device word that receives ZKV_DEVERR_TIMEOUT.
     Returns (codes uint8 [B, T, H, S] view, norms float32 [B, T, H, S] or None)."""
     if x.dtype not in (torch.float16, torch.float32):
         raise TypeError("x must be fp16 or fp32")
@@ -200,6 +203,9 @@ def rvq_encode(x: torch.Tensor, codebooks: torch.Tensor, codes: torch.Tensor | N
         if n4.shape != (Bn, T, H, S) or n4.stride(-1) != 1:
             raise ValueError("norms must be a [B, T, H, S] view with contiguous S")
         p.norms, p.n_sb, p.n_st, p.n_sh = _ptr(n4), n4.stride(0), n4.stride(1), n4.stride(2)
+    if error_flag is not None:
+        _need(error_flag, "error_flag", torch.int32)
+        p.error_flag = _ptr(error_flag)
     _check("zkv_rvq_encode", lib().zkv_rvq_encode(ctypes.byref(p), _stream()))
     return codes, norms
 

@@ -28,7 +28,9 @@
  *   - Device-side conditions that cannot be checked on the host (a length beyond capacity)
  *     are reported by OR-ing ZKV_DEVERR_* bits into an optional caller-owned device word
  *     (`error_flag`, may be NULL); the offending sequence is clamped or skipped, never read
- *     or written out of bounds.  No kernel waits on another.
+ *     or written out of bounds.  No kernel waits on another.  The tensor-core encoder's wait
+ *     for its own matrix-multiply completion is bounded: if it ever ran out, that tile's codes
+ *     are not written and ZKV_DEVERR_TIMEOUT is set instead of the device hanging.
  */
 #ifndef ZKV_H
 #define ZKV_H
@@ -52,6 +54,7 @@ typedef enum {
 /* Bits OR-ed into a caller's device error word. */
 #define ZKV_DEVERR_COMP_LEN 1   /* comp_len[b] > Tcap (clamped) or append at Tcap (skipped) */
 #define ZKV_DEVERR_WIN_LEN 2    /* win_len[b] > Wcap (clamped)                              */
+#define ZKV_DEVERR_TIMEOUT 4    /* a bounded on-chip wait ran out (results of that tile absent) */
 
 #define ZKV_DTYPE_F16 0
 #define ZKV_DTYPE_F32 1
@@ -96,6 +99,7 @@ int zkv_fwht(const void* in, int in_dtype, float* out, int64_t n_vec, int d, flo
  *   norms  float32 or NULL, norm s of (b,t,h) at norms[b*n_sb + t*n_st + n_sh*h + s]
  *   codebooks float32 [n_head][S][256][d]
  * Alignment: x rows 16-byte aligned (x base and strides multiples of 8 fp16 / 4 fp32 elements).
+ * error_flag: optional device int32 that receives ZKV_DEVERR_TIMEOUT (see the conventions above).
  * Errors: INVALID_ARG, UNSUPPORTED (d, S), CUDA.
  */
 typedef struct {
@@ -110,6 +114,7 @@ typedef struct {
   int64_t c_sb, c_st, c_sh;
   float* norms;
   int64_t n_sb, n_st, n_sh;
+  int32_t* error_flag;
 } zkv_encode_params;
 
 int zkv_rvq_encode(const zkv_encode_params* p, void* stream);

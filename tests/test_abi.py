@@ -120,3 +120,34 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(4, 128, dtype=torch.float16)
     with pytest.raises(ValueError):
         zkv.fwht(x, 1.0)
+
+
+def test_ctypes_structs_match_the_header_layout(tmp_path):
+    """Every parameter struct the binding passes has the C compiler's size and field offsets
+    (a field added to the header but not to the binding would shift every later field)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    pairs = [("zkv_encode_params", zkv.EncodeParams), ("zkv_reconstruct_params", zkv.ReconstructParams),
+             ("zkv_decode_params", zkv.DecodeParams), ("zkv_append_params", zkv.AppendParams)]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zkv.h"', "int main(void) {"]
+    for cname, cls in pairs:
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict()
+    for ln in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n"):
+        if ln:
+            a, b, v = ln.split()
+            got[(a, b)] = int(v)
+    for cname, cls in pairs:
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for f, _ in cls._fields_:
+            assert got[(cname, f)] == getattr(cls, f).offset, f"{cname}.{f}"
