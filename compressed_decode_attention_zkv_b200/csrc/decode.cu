@@ -43,6 +43,7 @@ namespace zkv {
 
 constexpr int kScanSub = 512;       // tokens per scan sub-chunk (1 per thread)
 constexpr int kScanThreads = 512;
+static_assert(kScanSub == kScanThreads && kScanThreads % 32 == 0, "one token per thread and sub-chunk; 32 per warp");
 constexpr int kColCap = 8176;       // tokens per histogram column per segment (sum < 2^32)
 constexpr float kHeadroom = 10.f;   // log2 units added to the running maximum on growth
 // Setup cost of one scan segment (table fill, histogram zeroing, final fold: about 11K cycles)
@@ -894,11 +895,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       prefetch_l2(vcb, vcb + pbytes_v, vcb + (s0 & ~int64_t(15)) * Sv, (s1 - (s0 & ~int64_t(15))) * Sv);
     }
     const uint32_t u0 = (uint32_t)s0, u1 = (uint32_t)s1;
+    const int nsub = (int)((u1 - u0 + kScanSub - 1) / kScanSub);   // same on every thread
+    // Token order: warp w owns the contiguous run of nsub * 32 tokens starting at
+    // u0 + w * nsub * 32, and sub-chunk i takes block i of every warp's run.  A warp's codes are
+    // still one contiguous load per sub-chunk, while each sub-chunk samples the whole segment,
+    // so the first sub-chunk's maxima (the initial reference) are close to the segment's and
+    // later growth of the reference (a fold) is rare.  The histograms do not depend on order.
+    const uint32_t tw = u0 + (uint32_t)(warp * nsub) * 32u + (uint32_t)lane;   // token of sub-chunk 0
     // codes of sub-chunks 0 and 1 in flight during the table fill
-    Code<SKP> kc = load_code1<SKP>(kcb, Sk, u0 + tid, u1);
-    Code<SVP> vc = load_code1<SVP>(vcb, Sv, u0 + tid, u1);
-    Code<SKP> kn = load_code1<SKP>(kcb, Sk, u0 + kScanSub + tid, u1);
-    Code<SVP> vn = load_code1<SVP>(vcb, Sv, u0 + kScanSub + tid, u1);
+    Code<SKP> kc = load_code1<SKP>(kcb, Sk, tw, u1);
+    Code<SVP> vc = load_code1<SVP>(vcb, Sv, tw, u1);
+    Code<SKP> kn = load_code1<SKP>(kcb, Sk, tw + 32u, u1);
+    Code<SVP> vn = load_code1<SVP>(vcb, Sv, tw + 32u, u1);
     __syncthreads();   // previous segment's shared memory is free
     {
       // zero the histograms, then copy the pair's table entries (s, c) -> every lane-group
@@ -955,7 +963,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     }
     __syncthreads();   // tables and zeroed histograms are ready
 
-    const int nsub = (int)((u1 - u0 + kScanSub - 1) / kScanSub);   // same on every thread
     float mref[GP], lacc[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -965,11 +972,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     bool dirty = false, has_master = false;   // uniform across the block
     // prologue: scores of sub-chunk 0
     float sc[GP];
-    score(kc, u0 + tid < u1, 0, sc);
+    score(kc, tw < u1, 0, sc);
     __syncthreads();
     for (int i = 0; i < nsub; ++i) {
       const int bf = i & 1;
-      const uint32_t t = u0 + (uint32_t)i * kScanSub + tid;
+      const uint32_t t = tw + 32u * (uint32_t)i;
       const bool ok = t < u1;
       // (a) maxima of sub-chunk i: lanes read the NW x GP partial maxima (entry w * GP + g in
       // lane (w * GP + g) % 32), fold over w with xor-shuffles, broadcast each head
@@ -1044,9 +1051,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       if (i + 1 < nsub) {
         kc = kn;
         vc = vn;
-        kn = load_code1<SKP>(kcb, Sk, t + 2 * kScanSub, u1);
-        vn = load_code1<SVP>(vcb, Sv, t + 2 * kScanSub, u1);
-        score(kc, t + kScanSub < u1, bf ^ 1, sc);
+        kn = load_code1<SKP>(kcb, Sk, t + 64u, u1);
+        vn = load_code1<SVP>(vcb, Sv, t + 64u, u1);
+        score(kc, t + 32u < u1, bf ^ 1, sc);
       }
       __syncthreads();
     }
