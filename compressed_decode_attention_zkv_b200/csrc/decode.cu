@@ -998,12 +998,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       bool grow = false;
 #pragma unroll
       for (int g = 0; g < GP; ++g) grow |= mn[g] > mref[g];
-      // (b) histograms += p of sub-chunk i-1
-      if (i > 0) {
-        accumulate(bf ^ 1);
-        dirty = true;
-      }
+      // Phase order: even warps (b), (c), (d); odd warps (c), (d), (b) -- half of the block
+      // issues the reduction-heavy phase while the other half gathers, so the shared-memory
+      // pipe sees a mix.  (c) must precede (d) (it reads this sub-chunk's scores and value
+      // codes, which (d) replaces).  A growth takes (b) first on every warp, then the fold.
+      const bool odd = (warp & 1) != 0;
       if (grow) {   // uniform: every thread read the same maxima
+        if (i > 0) {
+          accumulate(bf ^ 1);
+          dirty = true;
+        }
         // New reference = maximum + kHeadroom: later sub-chunks rarely exceed it, so folds
         // stay rare.  Precision: the segment's largest p is >= 2^-kHeadroom and its
         // fixed-point error is <= (tokens <= 2^14) * 2^-39 = 2^-25 absolute, i.e.
@@ -1029,6 +1033,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
           has_master = true;
           dirty = false;
         }
+      } else if (i > 0 && !odd) {
+        accumulate(bf ^ 1);   // (b), even warps
       }
       // (c) p of sub-chunk i -> staging buffer bf
 #pragma unroll
@@ -1054,6 +1060,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
         kn = load_code1<SKP>(kcb, Sk, t + 64u, u1);
         vn = load_code1<SVP>(vcb, Sv, t + 64u, u1);
         score(kc, t + 32u < u1, bf ^ 1, sc);
+      }
+      if (!grow && i > 0) {
+        if (odd) accumulate(bf ^ 1);   // (b), odd warps
+        dirty = true;
       }
       __syncthreads();
     }
