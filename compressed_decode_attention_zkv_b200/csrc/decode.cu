@@ -772,12 +772,13 @@ __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t*
 }
 
 // The token loop is software-pipelined with one barrier per sub-chunk.  In interval i every
-// thread (a) reads the partial maxima of sub-chunk i and decides whether the reference grows,
-// (b) adds the staged p of sub-chunk i-1 to the integer histograms, (c) computes and stages
-// the p of sub-chunk i, and (d) gathers the key scores and partial maxima of sub-chunk i+1.
-// Staging buffers and partial maxima alternate between two copies, so no interval reads what
-// the same interval writes.  A growth of the reference with non-empty histograms takes a
-// slow path (barrier, fold, barrier, zero, barrier) after (b), uniformly across the block.
+// thread (b) adds the staged p of sub-chunk i-1 to the integer histograms, (c) computes and
+// stages the p of sub-chunk i, and (d) gathers the key scores of sub-chunk i+1 and checks
+// them against the reference; the interval's barrier ORs those checks.  Staging buffers
+// alternate between two copies, so no interval reads what the same interval writes.  When a
+// score exceeded the reference (rare: the reference is the maximum so far plus a headroom), the
+// next interval first takes the block maxima (a) and, with non-empty histograms, a slow path
+// (barrier, fold, barrier, zero, barrier) after (b), uniformly across the block.
 template <int GP, int SKP, int SVP>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   using C = ScanCfg<GP, SKP, SVP>;
@@ -868,14 +869,28 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       }
     }
   };
-  // key scores of this thread's token of a sub-chunk and the warp's partial maxima -> redk[bf]
-  auto score = [&](const Code<SKP>& kc, bool ok, int bf, float (&sc)[GP]) {
-    key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
+  // block maxima of the scores in sc (tokens with okk): warp maxima -> redk, barrier, every
+  // lane reads the NW x GP partial maxima (entry w * GP + g in lane (w * GP + g) % 32), folds
+  // over w with xor-shuffles and broadcasts each head
+  auto block_max = [&](const float (&sc)[GP], bool okk, float (&mn)[GP]) {
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
-      const uint32_t k = __reduce_max_sync(0xffffffffu, ok ? ord_key(sc[g]) : 0u);
-      if (lane == 0) sts32u(redk_a + 4u * (uint32_t)((bf * C::NW + warp) * GP + g), k);
+      const uint32_t k = __reduce_max_sync(0xffffffffu, okk ? ord_key(sc[g]) : 0u);
+      if (lane == 0) sts32u(redk_a + 4u * (uint32_t)(warp * GP + g), k);
     }
+    __syncthreads();
+    uint32_t k = 0u;
+#pragma unroll
+    for (int e = 0; e < C::NW * GP; e += 32)
+      if (e + lane < C::NW * GP) {
+        uint32_t v;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(redk_a + 4u * (uint32_t)(e + lane)));
+        k = max(k, v);
+      }
+#pragma unroll
+    for (int o = GP; o < 32 && o < C::NW * GP; o <<= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+#pragma unroll
+    for (int g = 0; g < GP; ++g) mn[g] = ord_val(__shfl_sync(0xffffffffu, k, g));
   };
 
   for (int pr = pfirst; pr < npairs && a.pre[pr] < hi; ++pr) {
@@ -970,40 +985,24 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       lacc[g] = 0.f;
     }
     bool dirty = false, has_master = false;   // uniform across the block
-    // prologue: scores of sub-chunk 0
+    // prologue: scores of sub-chunk 0 (the reference starts at -inf, so interval 0 grows it)
     float sc[GP];
-    score(kc, tw < u1, 0, sc);
-    __syncthreads();
+    key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
+    bool over = true;   // uniform: some score of the current sub-chunk exceeds the reference
     for (int i = 0; i < nsub; ++i) {
       const int bf = i & 1;
       const uint32_t t = tw + 32u * (uint32_t)i;
       const bool ok = t < u1;
-      // (a) maxima of sub-chunk i: lanes read the NW x GP partial maxima (entry w * GP + g in
-      // lane (w * GP + g) % 32), fold over w with xor-shuffles, broadcast each head
-      float mn[GP];
-      {
-        uint32_t k = 0u;
-#pragma unroll
-        for (int e = 0; e < C::NW * GP; e += 32)
-          if (e + lane < C::NW * GP) {
-            uint32_t v;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(redk_a + 4u * (uint32_t)(bf * C::NW * GP + e + lane)));
-            k = max(k, v);
-          }
-#pragma unroll
-        for (int o = GP; o < 32 && o < C::NW * GP; o <<= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
-#pragma unroll
-        for (int g = 0; g < GP; ++g) mn[g] = ord_val(__shfl_sync(0xffffffffu, k, g));
-      }
-      bool grow = false;
-#pragma unroll
-      for (int g = 0; g < GP; ++g) grow |= mn[g] > mref[g];
       // Phase order: even warps (b), (c), (d); odd warps (c), (d), (b) -- half of the block
       // issues the reduction-heavy phase while the other half gathers, so the shared-memory
       // pipe sees a mix.  (c) must precede (d) (it reads this sub-chunk's scores and value
-      // codes, which (d) replaces).  A growth takes (b) first on every warp, then the fold.
+      // codes, which (d) replaces).  A growth of the reference (known from the previous
+      // interval's barrier) takes (b) first on every warp, then the fold.
       const bool odd = (warp & 1) != 0;
-      if (grow) {   // uniform: every thread read the same maxima
+      if (over) {
+        // (a) the block maxima of sub-chunk i set the new reference
+        float mn[GP];
+        block_max(sc, ok, mn);
         if (i > 0) {
           accumulate(bf ^ 1);
           dirty = true;
@@ -1036,7 +1035,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       } else if (i > 0 && !odd) {
         accumulate(bf ^ 1);   // (b), even warps
       }
-      // (c) p of sub-chunk i -> staging buffer bf
+      // (c) p of sub-chunk i -> staging buffer bf (every score is <= the reference: p <= 1)
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         uint32_t hv = 0u, lv = 0u;
@@ -1053,19 +1052,25 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       } else {
         sts64u(cst_a + 4u * (uint32_t)(bf * C::CBUFW), vc.w[0], vc.w[1]);
       }
-      // (d) scores of sub-chunk i+1; codes of sub-chunk i+2 in flight
+      // (d) scores of sub-chunk i+1 and whether any exceeds the reference; codes of
+      // sub-chunk i+2 in flight
+      bool ex = false;
       if (i + 1 < nsub) {
         kc = kn;
         vc = vn;
         kn = load_code1<SKP>(kcb, Sk, t + 64u, u1);
         vn = load_code1<SVP>(vcb, Sv, t + 64u, u1);
-        score(kc, t + 32u < u1, bf ^ 1, sc);
+        key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
+        if (t + 32u < u1) {
+#pragma unroll
+          for (int g = 0; g < GP; ++g) ex |= sc[g] > mref[g];
+        }
       }
-      if (!grow && i > 0) {
+      if (!over && i > 0) {
         if (odd) accumulate(bf ^ 1);   // (b), odd warps
         dirty = true;
       }
-      __syncthreads();
+      over = __syncthreads_or(ex) != 0;
     }
     // histograms += p of the last sub-chunk
     accumulate((nsub - 1) & 1);
