@@ -9,9 +9,8 @@
 //
 // Four kernels per call:
 //   1. lut_kernel    q_tilde = H q / sqrt(d) (float32 transform), per stage
-//                    LUT_s[c] = (scale * log2 e) * q_tilde . Ck_s[c] -> workspace; the dense
-//                    window attention of every (sequence, kv head); prefix sums of the
-//                    compressed lengths that partition the token space among scan CTAs.
+//                    LUT_s[c] = (scale * log2 e) * q_tilde . Ck_s[c] -> workspace; prefix sums
+//                    of the compressed lengths that partition the token space among scan CTAs.
 //   2. scan_kernel   one CTA per SM walks a contiguous range of the concatenated compressed
 //                    tokens of all (sequence, kv head) pairs.  Per pair segment it takes
 //                    score_t = sum_s LUT_s[zk_{t,s}] (base-2 logits), keeps a running reference
@@ -22,8 +21,9 @@
 //   3. merge_kernel  grid (codeword quarter, value stage, kv head): merges the segment
 //                    histograms by their maxima and contracts W_s with its Cv_s codewords for
 //                    every sequence (Cv_s is read once per call).
-//   4. finalize_kernel  one block per (sequence, kv head): sums the partials, rotates back, and
-//                    merges with the window by log-sum-exp.
+//   4. finalize_kernel  one block per (sequence, kv head): the dense attention over the fp16
+//                    window (while the merge still runs), then sums the partials, rotates
+//                    back, and merges the two parts by log-sum-exp.
 //
 // Shared-memory design of the scan (shared memory bandwidth, not HBM, bounds this kernel):
 //  * key tables are replicated per lane group so that the 8 (or 16, 32) lanes of a 128-bit
@@ -187,11 +187,11 @@ __device__ __forceinline__ int64_t clamp_win_len(const DecodeArgs& a, int b) {
 }
 
 // ------------------------------------------------------------------------------------------
-// 1. Query rotation + lookup tables; window attention; length prefix sums.
-//    1-D grid: [0, n_lut_blocks) tables, then one block per (sequence, kv head) window.
+// 1. Query rotation + lookup tables; length prefix sums (block 0).  The dense window
+//    attention (window_item) runs in the finalize kernel.
 // ------------------------------------------------------------------------------------------
-constexpr int kLutC = 128;    // codewords per block (2 per thread)
-constexpr int kLutH = 32;     // attached query heads per block (b * G + g)
+constexpr int kLutC = 64;     // codewords per table block (one per thread and head quad)
+constexpr int kLutH = 16;     // attached query heads per table block (b * G + g)
 
 template <int D>
 struct LutSmem {
@@ -372,117 +372,120 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
   }
 }
 
+// ceil(x * m / d) for x, m >= 0 and d > 0, exact (128-bit product).
+__device__ __forceinline__ int64_t ceil_muldiv(int64_t x, int64_t m, int64_t d) {
+  const unsigned __int128 pr = (unsigned __int128)(uint64_t)x * (uint64_t)m;
+  return (int64_t)((pr + (uint64_t)(d - 1)) / (uint64_t)d);
+}
+
+// The partition of the compressed token space among the scan CTAs (one block):
+// pre = prefix sums of the clamped compressed lengths, vs = prefix sums of the virtual lengths
+// len + kSegCost (nonempty pairs).  Scan CTA c covers virtual positions [v_c, v_(c+1)) with
+// v_c = floor(V c / grid); a cut inside a pair's kSegCost gap moves to the pair's first token.
+// Each pair's thread places the cuts that fall in its virtual range directly (the first cut at
+// or after position x is c = ceil(x grid / V)), so no search is needed.
+__device__ void partition_block(const DecodeArgs& a) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // exclusive prefix sums of the clamped compressed lengths (pre) and of the virtual lengths
+  // len + kSegCost * (len > 0) (vs), 256 pairs per round
+  __shared__ int64_t warp_tot[2][8];
+  __shared__ int64_t carry_s[2];
+  const int npairs = a.B * a.Hkv;
+  if (tid == 0) {
+    carry_s[0] = 0;
+    carry_s[1] = 0;
+    a.pre[0] = 0;
+    a.vs[0] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < npairs; base += 256) {
+    const int pr = base + tid;
+    int64_t c = 0;
+    if (pr < npairs) {
+      c = a.comp_len[pr / a.Hkv];
+      if (c < 0 || c > a.Tcap) {
+        set_error(a.err, ZKV_DEVERR_COMP_LEN);
+        c = c < 0 ? 0 : a.Tcap;
+      }
+      c = c < a.max_comp ? c : a.max_comp;
+    }
+    int64_t x = c, y = c > 0 ? c + kSegCost : 0;   // inclusive warp scans
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t ux = __shfl_up_sync(0xffffffffu, x, o);
+      const int64_t uy = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) {
+        x += ux;
+        y += uy;
+      }
+    }
+    if (lane == 31) {
+      warp_tot[0][warp] = x;
+      warp_tot[1][warp] = y;
+    }
+    __syncthreads();
+    int64_t ox = carry_s[0], oy = carry_s[1];
+    for (int w = 0; w < warp; ++w) {
+      ox += warp_tot[0][w];
+      oy += warp_tot[1][w];
+    }
+    if (pr < npairs) {
+      a.pre[pr + 1] = ox + x;
+      a.vs[pr + 1] = oy + y;
+    }
+    __syncthreads();
+    if (tid == 255) {
+      carry_s[0] = ox + x;
+      carry_s[1] = oy + y;
+    }
+    __syncthreads();
+  }
+  const int64_t V = carry_s[1], tot = carry_s[0];
+  const int grid = a.grid;
+  if (V == 0) {   // no compressed token at all
+    for (int c = tid; c <= grid; c += 256) a.bounds[c] = 0;
+    for (int k = tid; k < npairs; k += 256) {
+      a.pfirst[k] = 1;
+      a.plast[k] = 0;
+    }
+    return;
+  }
+  if (tid == 0) {
+    a.bounds[0] = 0;
+    a.bounds[grid] = tot;
+  }
+  for (int k = tid; k < npairs; k += 256) {
+    const int64_t v0 = a.vs[k], v1 = a.vs[k + 1], p0 = a.pre[k], len = a.pre[k + 1] - p0;
+    int f = 1, t = 0;   // first / last scan CTA holding the pair's tokens (f > t: none)
+    if (len > 0) {
+      const int64_t clo = ceil_muldiv(v0, grid, V);       // cuts c in [clo, chi] lie in [v0, v1)
+      const int64_t chi = ceil_muldiv(v1, grid, V) - 1;
+      for (int64_t c = clo > 1 ? clo : 1; c <= chi && c < grid; ++c) {
+        const int64_t off = (int64_t)(((unsigned __int128)(uint64_t)V * (uint64_t)c) / (uint64_t)grid) - v0;
+        a.bounds[c] = off < kSegCost ? p0 : p0 + (off - kSegCost < len ? off - kSegCost : len);
+      }
+      // the CTA holding the first token: the last cut at or before v0 + kSegCost (its bound is
+      // p0); the one holding the last token: the last cut before v1
+      const int64_t cf = ceil_muldiv(v0 + kSegCost + 1, grid, V) - 1;
+      f = (int)(cf < chi ? cf : chi);
+      t = (int)chi;
+    }
+    a.pfirst[k] = f;
+    a.plast[k] = t;
+  }
+}
+
+// Table blocks: block = (64-codeword slice, key stage, group of 16 attached query heads, kv
+// head); thread (codeword cc, head quad hq) forms 4 dot products.  Block n_lut_blocks is the
+// partition block.
 template <int D, int GP>
 __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
   constexpr int E = D / 32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if ((int)blockIdx.x >= a.n_lut_blocks) {
-    const int pair = blockIdx.x - a.n_lut_blocks;
-    window_item<D, GP>(a, pair / a.Hkv, pair % a.Hkv, smem_raw);
+  if ((int)blockIdx.x == a.n_lut_blocks) {
+    partition_block(a);
     return;
-  }
-  if (blockIdx.x == 0) {
-    // exclusive prefix sums of the clamped compressed lengths (pre) and of the virtual lengths
-    // len + kSegCost * (len > 0) (vs), 256 pairs per round
-    __shared__ int64_t warp_tot[2][8];
-    __shared__ int64_t carry_s[2];
-    const int npairs = a.B * a.Hkv;
-    if (tid == 0) {
-      carry_s[0] = 0;
-      carry_s[1] = 0;
-      a.pre[0] = 0;
-      a.vs[0] = 0;
-    }
-    __syncthreads();
-    for (int base = 0; base < npairs; base += 256) {
-      const int pr = base + tid;
-      int64_t c = 0;
-      if (pr < npairs) {
-        c = a.comp_len[pr / a.Hkv];
-        if (c < 0 || c > a.Tcap) {
-          set_error(a.err, ZKV_DEVERR_COMP_LEN);
-          c = c < 0 ? 0 : a.Tcap;
-        }
-        c = c < a.max_comp ? c : a.max_comp;
-      }
-      int64_t x = c, y = c > 0 ? c + kSegCost : 0;   // inclusive warp scans
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int64_t ux = __shfl_up_sync(0xffffffffu, x, o);
-        const int64_t uy = __shfl_up_sync(0xffffffffu, y, o);
-        if (lane >= o) {
-          x += ux;
-          y += uy;
-        }
-      }
-      if (lane == 31) {
-        warp_tot[0][warp] = x;
-        warp_tot[1][warp] = y;
-      }
-      __syncthreads();
-      int64_t ox = carry_s[0], oy = carry_s[1];
-      for (int w = 0; w < warp; ++w) {
-        ox += warp_tot[0][w];
-        oy += warp_tot[1][w];
-      }
-      if (pr < npairs) {
-        a.pre[pr + 1] = ox + x;
-        a.vs[pr + 1] = oy + y;
-      }
-      __syncthreads();
-      if (tid == 255) {
-        carry_s[0] = ox + x;
-        carry_s[1] = oy + y;
-      }
-      __syncthreads();
-    }
-    // scan CTA c covers virtual positions [c V / grid, (c+1) V / grid); a cut inside a pair's
-    // kSegCost gap moves to the pair's first token
-    const int64_t V = carry_s[1], tot = carry_s[0];
-    const int grid = a.grid;
-    for (int c = tid; c <= grid; c += 256) {
-      int64_t x;
-      if (c == 0) {
-        x = 0;
-      } else if (c == grid) {
-        x = tot;
-      } else {
-        const int64_t v = (V / grid) * c + ((V % grid) * c) / grid;
-        int l = 0, r = npairs;   // largest k with vs[k] <= v: vs[l] <= v < vs[r] (vs[npairs] = V > v)
-        while (r - l > 1) {
-          const int m = (l + r) >> 1;
-          if (a.vs[m] <= v) l = m; else r = m;
-        }
-        const int64_t off = v - a.vs[l];
-        const int64_t len = a.pre[l + 1] - a.pre[l];
-        x = off < kSegCost ? a.pre[l] : a.pre[l] + (off - kSegCost < len ? off - kSegCost : len);
-      }
-      a.bounds[c] = x;
-    }
-    __syncthreads();
-    // first and last scan CTA of every pair: the CTAs whose ranges hold its first / last token
-    for (int k = tid; k < npairs; k += 256) {
-      const int64_t p0 = a.pre[k], p1 = a.pre[k + 1];
-      int f = 1, t = 0;
-      if (p1 > p0) {
-        int l = 0, r = grid;   // largest c with bounds[c] <= p0
-        while (r - l > 1) {
-          const int m = (l + r) >> 1;
-          if (a.bounds[m] <= p0) l = m; else r = m;
-        }
-        f = l;
-        l = 0;
-        r = grid;              // largest c with bounds[c] <= p1 - 1
-        while (r - l > 1) {
-          const int m = (l + r) >> 1;
-          if (a.bounds[m] <= p1 - 1) l = m; else r = m;
-        }
-        t = l;
-      }
-      a.pfirst[k] = f;
-      a.plast[k] = t;
-    }
   }
   if ((int)blockIdx.x < a.Hkv * a.Sv && tid == 0) {
     // the merge kernel reads every value codebook; stream them into L2 meanwhile
@@ -501,7 +504,7 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
   const int hg = rest % n_hg;
   const int kvh = rest / n_hg;
   const int c0 = cblk * kLutC;
-  // codebook slice C[kvh][s][c0 .. c0+63][:] -> shared memory, in flight during the rotation
+  // codebook slice C[kvh][s][c0 .. c0 + kLutC)[:] -> shared memory, in flight during the rotation
   {
     const float* C = a.Ck + (((size_t)kvh * a.Sk + s) * kCodebook + c0) * D;
     for (int f = tid; f < kLutC * D / 4; f += 256) {
@@ -538,42 +541,32 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
   }
   cp_async_wait_all();
   __syncthreads();
-  // thread (codewords cc and cc + 64, head group hq): 16 dot products; the codewords are read
-  // as 16-byte pieces (conflict-free thanks to the swizzle), the query columns are broadcasts
-  const int cc = tid & 63, hq = tid >> 6;   // 4 groups of 8 heads
-  const float* row0 = sm.cb + cc * D;
-  const float* row1 = sm.cb + (cc + 64) * D;
-  const int sw = cc & 7;                   // (cc + 64) & 7 == cc & 7
-  float acc[2][8];
-#pragma unroll
-  for (int u = 0; u < 2; ++u)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) acc[u][k] = 0.f;
-#pragma unroll 2
+  // thread (codeword cc, heads 4 hq .. 4 hq + 3): the codeword is read as 16-byte pieces
+  // (conflict-free thanks to the swizzle), the query columns are broadcasts
+  const int cc = tid & (kLutC - 1), hq = tid / kLutC;
+  const float* row = sm.cb + cc * D;
+  const int sw = cc & 7;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
   for (int qq = 0; qq < D / 4; ++qq) {
-    const float4 ca = *reinterpret_cast<const float4*>(row0 + 4 * (qq ^ sw));
-    const float4 cb = *reinterpret_cast<const float4*>(row1 + 4 * (qq ^ sw));
-    const float cv[2][4] = {{ca.x, ca.y, ca.z, ca.w}, {cb.x, cb.y, cb.z, cb.w}};
+    const float4 c4 = *reinterpret_cast<const float4*>(row + 4 * (qq ^ sw));
+    const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int i = 4 * qq + e;
-      const float4 q0 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8]);
-      const float4 q1 = *reinterpret_cast<const float4*>(&sm.qT[i][hq * 8 + 4]);
-      const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[u][k] = fmaf(qv[k], cv[u][e], acc[u][k]);
+      const float4 q4 = *reinterpret_cast<const float4*>(&sm.qT[4 * qq + e][hq * 4]);
+      acc[0] = fmaf(q4.x, cv[e], acc[0]);
+      acc[1] = fmaf(q4.y, cv[e], acc[1]);
+      acc[2] = fmaf(q4.z, cv[e], acc[2]);
+      acc[3] = fmaf(q4.w, cv[e], acc[3]);
     }
   }
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int j = hg * kLutH + hq * 8 + k;
+  for (int k = 0; k < 4; ++k) {
+    const int j = hg * kLutH + hq * 4 + k;
     if (j < a.B * a.G) {
       const int b = j / a.G, g = j % a.G;
-      float* dst = a.lut + ((((int64_t)b * a.Hkv + kvh) * a.Sk + s) * kCodebook + c0 + cc) * GP + g;
-      dst[0] = acc[0][k] * a.scale_log2;
-      dst[64 * GP] = acc[1][k] * a.scale_log2;
+      a.lut[((((int64_t)b * a.Hkv + kvh) * a.Sk + s) * kCodebook + c0 + cc) * GP + g] =
+          acc[k] * a.scale_log2;
     }
   }
 }
@@ -1139,6 +1132,7 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
   const int tid = threadIdx.x;
   const int qtr = blockIdx.x, s = blockIdx.y, kvh = blockIdx.z;
   const int c0 = qtr * kMergeC;
+  pdl_trigger();   // the finalize blocks start their window attention meanwhile
   {
     const float* src = a.Cv + (((size_t)kvh * a.Sv + s) * kCodebook + c0) * D;
     for (int f = tid; f < kMergeC * D / 4; f += 256) cp_async16(Cs + 4 * f, src + 4 * f);
@@ -1249,13 +1243,16 @@ __global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
 template <int D, int GP>
 __global__ void __launch_bounds__(256) finalize_kernel(DecodeArgs a) {
   constexpr int E = D / 32;
+  extern __shared__ __align__(16) unsigned char win_smem[];
   __shared__ __align__(16) float oc[GP * D];
   __shared__ float mstar_s[GP], lstar_s[GP];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pair = blockIdx.x;
   const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
-  // window terms of this warp's first head (written by the table kernel, which completed before
-  // the scan started): loaded before waiting for the merge
+  // The window attention reads only the call's inputs (written before the table kernel, which
+  // this kernel follows on the stream): it runs before waiting for the merge.
+  window_item<D, GP>(a, b, kvh, win_smem);
+  __syncthreads();   // this block's window terms (global) are visible to all its threads
   const int g0 = warp;
   float mw0 = -INFINITY, lw0 = 0.f, ow0[E];
   if (g0 < a.G) {
@@ -1371,13 +1368,11 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
   // 1. tables, window, prefix sums
   trace(ev, 0, st);
   {
-    const size_t lut_smem = sizeof(LutSmem<D>);
-    const size_t win_smem = window_smem_bytes<D, GP>();
-    const size_t smem = lut_smem > win_smem ? lut_smem : win_smem;
+    const size_t smem = sizeof(LutSmem<D>);
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
     a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
-    const int64_t blocks = (int64_t)a.n_lut_blocks + (int64_t)a.B * a.Hkv;
+    const int64_t blocks = (int64_t)a.n_lut_blocks + 1;   // + the partition block
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
     // a normal launch: the caller's preceding work (which may write q) must be complete, since
     // the table blocks do not wait
@@ -1403,7 +1398,9 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     if (ensure_smem_limit(merge_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const dim3 grid((unsigned)kMergeQ, (unsigned)a.Sv, (unsigned)a.Hkv);
     if (launch_pdl(merge_kernel<D, GP>, grid, dim3(256), smem, st, a) != cudaSuccess) return ZKV_ERR_CUDA;
-    if (launch_pdl(finalize_kernel<D, GP>, dim3((unsigned)(a.B * a.Hkv)), dim3(256), 0, st, a) != cudaSuccess)
+    const size_t fsmem = window_smem_bytes<D, GP>();
+    if (ensure_smem_limit(finalize_kernel<D, GP>, fsmem) != cudaSuccess) return ZKV_ERR_CUDA;
+    if (launch_pdl(finalize_kernel<D, GP>, dim3((unsigned)(a.B * a.Hkv)), dim3(256), fsmem, st, a) != cudaSuccess)
       return ZKV_ERR_CUDA;
   }
   trace(ev, 3, st);
