@@ -164,14 +164,14 @@ def replica_bytes(rep):
 
 
 def step_fn(rep, ws, max_comp, events=None):
+    """One serving step through the library's single serving-step call (append of the new
+    tokens, then decode attention over the updated cache)."""
     from compressed_decode_attention_zkv_b200 import zkv
-    zkv.rvq_append(rep["new_k"], rep["new_v"], rep["win_k"], rep["win_v"], rep["win_len"],
-                   rep["win_head"], rep["comp_len"], rep["k_codes"], rep["v_codes"], rep["Ck"],
-                   rep["Cv"], error_flag=rep["err"])
-    zkv.rvq_decode_attn(rep["q"], rep["k_codes"], rep["v_codes"], rep["comp_len"], rep["Ck"],
-                        rep["Cv"], rep["win_k"], rep["win_v"], rep["win_len"], out=rep["out"],
-                        lse=rep["lse"], max_comp_len=max_comp, workspace=ws,
-                        error_flag=rep["err"], trace_events=events)
+    zkv.rvq_serve_step(rep["new_k"], rep["new_v"], rep["q"], rep["win_k"], rep["win_v"],
+                       rep["win_len"], rep["win_head"], rep["comp_len"], rep["k_codes"],
+                       rep["v_codes"], rep["Ck"], rep["Cv"], out=rep["out"], lse=rep["lse"],
+                       max_comp_len=max_comp, workspace=ws, error_flag=rep["err"],
+                       trace_events=events)
 
 
 # --------------------------------------------------------------------------------------------
@@ -376,16 +376,15 @@ def run_ours(args):
     wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
     host_comp = [wl.Tc] * R          # compressed length of every sequence of each replica
 
-    # trace events per replica: before LUT, before scan, before merge, after merge; plus
-    # before append
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(R)]
+    # trace events per replica: start of the step (tables, encode, length update and
+    # partition follow), before the scan, before the merge, after the last kernel
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(R)]
     for e in (e for row in evs for e in row):   # torch only times events it has seen recorded;
         e.record()                               # the library re-records the same handles
     torch.cuda.synchronize()
 
     def one_step(r):
-        evs[r][4].record()
-        step_fn(reps[r], wss[r], max_comp, events=evs[r][:4])
+        step_fn(reps[r], wss[r], max_comp, events=evs[r])
 
     def decode_only(r):
         from compressed_decode_attention_zkv_b200 import zkv as Z
@@ -470,37 +469,36 @@ def run_ours(args):
     def span(r, a, b):
         return evs[r][a].elapsed_time(evs[r][b]) / 1000.0
     try:
-        t_append = statistics.mean(span(r, 4, 0) for r in range(R))
-        t_lut = statistics.mean(span(r, 0, 1) for r in range(R))
+        t_pre = statistics.mean(span(r, 0, 1) for r in range(R))
         t_scan = statistics.mean(span(r, 1, 2) for r in range(R))
         t_merge = statistics.mean(span(r, 2, 3) for r in range(R))
         trace_src = "CUDA events captured in the step graphs (last replay of each replica)"
     except Exception as exc:   # event timing inside graphs unavailable: eager pass instead
         print(f"[bench] graph-captured event timing failed ({exc}); timing kernels eagerly",
               file=sys.stderr)
-        acc = {k: [] for k in ("append", "lut", "scan", "merge")}
+        acc = {k: [] for k in ("pre", "scan", "merge")}
         for i in range(min(args.steps, 64)):
             r = i % R
             one_step(r)
             host_comp[r] += 1
             torch.cuda.synchronize()
-            acc["append"].append(span(r, 4, 0))
-            acc["lut"].append(span(r, 0, 1))
+            acc["pre"].append(span(r, 0, 1))
             acc["scan"].append(span(r, 1, 2))
             acc["merge"].append(span(r, 2, 3))
-        t_append, t_lut, t_scan, t_merge = (statistics.mean(acc[k]) for k in
-                                            ("append", "lut", "scan", "merge"))
+        t_pre, t_scan, t_merge = (statistics.mean(acc[k]) for k in ("pre", "scan", "merge"))
         trace_src = "CUDA events around each kernel, eager steps after the timed region"
-    per = {"append": t_append, "lut": t_lut, "scan": t_scan, "merge": t_merge}
-    dominant = max(per, key=lambda k: per[k] if per[k] == per[k] else -1)
+    per = {"tables+append+partition": t_pre, "scan": t_scan, "merge+finalize": t_merge}
     Tc_avg = tokens / (wl.B * args.steps)
     # algorithmic bytes (counted once per distinct byte).  The scan kernel reads the codes of
     # every compressed token: (Sk + Sv) bytes per (token, kv head).
     scan_bytes = wl.B * wl.Hkv * Tc_avg * (wl.Sk + wl.Sv)
+    # the whole step: codes, window, codebooks (read by the encode and the decode alike), q,
+    # out + lse; the append's new tokens (read, written to the window), evicted rows and codes
     call_bytes = (scan_bytes + wl.B * wl.Hkv * wl.W * wl.d * 2 * 2
                   + wl.Hkv * (wl.Sk + wl.Sv) * 256 * wl.d * 4
-                  + wl.B * wl.Hq * wl.d * 2 + wl.B * wl.Hq * (wl.d + 1) * 4)
-    decode_time = t_lut + t_scan + t_merge
+                  + wl.B * wl.Hq * wl.d * 2 + wl.B * wl.Hq * (wl.d + 1) * 4
+                  + wl.B * wl.Hkv * 2 * (3 * wl.d * 2) + wl.B * wl.Hkv * (wl.Sk + wl.Sv))
+    step_time = t_pre + t_scan + t_merge
     traffic = (SCAN_TRAFFIC["bytes_per_launch"]
                if SCAN_TRAFFIC["scan_src_sha1"] == scan_src_sha1() else None)
     roof = {"bound": "hbm", "kernel": "scan_kernel", "achieved": scan_bytes / t_scan / 1e9,
@@ -512,7 +510,7 @@ def run_ours(args):
     # e2e: public API, inputs copied from pinned host memory, result read back, every step.
     # Per replica the step's inputs (new K, new V, q) are views of one device buffer filled by
     # one copy from one pinned host buffer; out and lse are views of one buffer read back by
-    # one copy.  The calls are the binding's prepared append / decode objects.
+    # one copy.  The call is the binding's prepared serving step (one library call).
     e2e = None
     if True:
         nk = wl.B * wl.Hkv * wl.d
@@ -530,18 +528,16 @@ def run_ours(args):
             q = din[2 * nk:].view(wl.B, wl.Hq, wl.d)
             out = dout[:nq].view(wl.B, wl.Hq, wl.d)
             lse = dout[nq:].view(wl.B, wl.Hq)
-            app = zkv.PreparedAppend(new_k, new_v, rep["win_k"], rep["win_v"], rep["win_len"],
-                                     rep["win_head"], rep["comp_len"], rep["k_codes"],
-                                     rep["v_codes"], rep["Ck"], rep["Cv"], error_flag=rep["err"])
-            dec = zkv.PreparedDecode(q, rep["k_codes"], rep["v_codes"], rep["comp_len"], rep["Ck"],
-                                     rep["Cv"], rep["win_k"], rep["win_v"], rep["win_len"],
-                                     out=out, lse=lse, max_comp_len=max_comp, workspace=wss[r],
-                                     error_flag=rep["err"])
+            call = zkv.PreparedServeStep(new_k, new_v, q, rep["win_k"], rep["win_v"],
+                                         rep["win_len"], rep["win_head"], rep["comp_len"],
+                                         rep["k_codes"], rep["v_codes"], rep["Ck"], rep["Cv"],
+                                         out=out, lse=lse, max_comp_len=max_comp,
+                                         workspace=wss[r], error_flag=rep["err"])
             host_in.append(hin)
             host_out.append(torch.empty(n_out, dtype=torch.float32).pin_memory())
             dev_in.append(din)
             dev_out.append(dout)
-            calls.append((app, dec))
+            calls.append(call)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -551,8 +547,7 @@ def run_ours(args):
         for i in range(n_e2e):
             r = i % R
             dev_in[r].copy_(host_in[r], non_blocking=True)
-            calls[r][0]()
-            calls[r][1]()
+            calls[r]()
             host_out[r].copy_(dev_out[r], non_blocking=True)
             host_comp[r] += 1
             tok2 += wl.B * host_comp[r]
@@ -567,8 +562,9 @@ def run_ours(args):
         d2h = n_out * 4
         e2e = {"value": tok2 * world / t2, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "path": "zkv.PreparedAppend + zkv.PreparedDecode (ctypes C-ABI), eager, per step; "
-                       "one pinned H2D copy of the step's inputs, one D2H copy of out + lse"}
+               "path": "zkv.PreparedServeStep (one ctypes C-ABI call: zkv_rvq_serve_step), eager, "
+                       "per step; one pinned H2D copy of the step's inputs, one D2H copy of "
+                       "out + lse"}
 
     extras = {}
     if not args.no_encode and rank == 0:
@@ -591,12 +587,12 @@ def run_ours(args):
                            l2=f"{R} rotating replicas x {rep_mb:.1f} MB = {R * rep_mb:.0f} MB > 126 MB L2",
                            parallelism=f"replicas x{world}, no collective",
                            graph="one CUDA graph per replica step"),
-            "gpu_launches": 6 * args.steps,   # append (2), lut, scan, merge, finalize
+            "gpu_launches": 6 * args.steps,   # tables, encode, lengths+partition, scan, merge, finalize
             "roofline": roof,
             "kernels_s": per,
-            "decode_call": {"seconds": decode_time, "algorithmic_bytes": call_bytes,
-                            "gbs": call_bytes / decode_time / 1e9,
-                            "frac": call_bytes / decode_time / 1e9 / hbm_peak},
+            "step_call": {"seconds": step_time, "algorithmic_bytes": call_bytes,
+                          "gbs": call_bytes / step_time / 1e9,
+                          "frac": call_bytes / step_time / 1e9 / hbm_peak},
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,

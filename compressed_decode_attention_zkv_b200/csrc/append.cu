@@ -22,6 +22,7 @@
 #include <cooperative_groups.h>
 
 #include "encode_rows.cuh"
+#include "lengths.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -268,6 +269,10 @@ __global__ void __cluster_dims__(kAppendCl, 1, 1) __launch_bounds__(256)
     }
   }
   cluster.sync();   // no CTA leaves while another may still read its shared memory
+  // Launched as a dependent of the table kernel (the serving step), this kernel completes only
+  // after that kernel has: whatever waits for this one then also sees the tables.  Returns at
+  // once after a normal launch.
+  pdl_wait();
   if (rank != 0) return;
   if (tid < kAppendR) {
     const int64_t j = row0 + tid;
@@ -302,23 +307,10 @@ __global__ void append_lengths_kernel(int B, int64_t Tcap, int64_t Wcap, int32_t
   pdl_wait();   // the encode kernel read the pre-step lengths
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;
-  const int64_t wl = win_len[b];
-  if (wl < 0 || wl > Wcap) return;
-  if (wl < Wcap) {
-    win_len[b] = (int32_t)(wl + 1);
-    return;
-  }
-  const int64_t c = comp_len[b], hd = win_head[b];
-  if (c < 0 || c >= Tcap || hd < 0 || hd >= Wcap) return;
-  comp_len[b] = (int32_t)(c + 1);
-  win_head[b] = (int32_t)((hd + 1) % Wcap);
+  advance_lengths(b, Tcap, Wcap, win_len, win_head, comp_len);
 }
 
-}  // namespace zkv
-
-using namespace zkv;
-
-extern "C" int zkv_rvq_append(const zkv_append_params* p, void* stream) {
+int validate_append(const zkv_append_params* p) {
   if (!p) return ZKV_ERR_INVALID_ARG;
   if (p->B < 1 || p->Hkv < 1 || p->Tcap < 0 || p->Wcap < 1) return ZKV_ERR_INVALID_ARG;
   if (!supported_d(p->d)) return ZKV_ERR_UNSUPPORTED;
@@ -330,21 +322,50 @@ extern "C" int zkv_rvq_append(const zkv_append_params* p, void* stream) {
   const uintptr_t al = (uintptr_t)p->win_k | (uintptr_t)p->win_v | (uintptr_t)p->k_codebooks |
                        (uintptr_t)p->v_codebooks;
   if (al & 15) return ZKV_ERR_INVALID_ARG;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const double rot = 1.0 / std::sqrt((double)p->d);
-  const unsigned groups = (unsigned)((p->B + kAppendR - 1) / kAppendR);
-  const dim3 grid(groups * kAppendCl, (unsigned)p->Hkv, 2);
+  return ZKV_OK;
+}
+
+// The encode + window-write kernel; with pdl, as a programmatic dependent of the previous
+// kernel on the stream (it never reads that kernel's results).
+int launch_append_cluster(const zkv_append_params& p, cudaStream_t st, bool pdl) {
+  const double rot = 1.0 / std::sqrt((double)p.d);
+  const unsigned groups = (unsigned)((p.B + kAppendR - 1) / kAppendR);
+  const dim3 grid(groups * kAppendCl, (unsigned)p.Hkv, 2);
   const bool ok =
       ensure_smem_limit(append_cluster_kernel<64>, sizeof(AppendSmem<64>)) == cudaSuccess &&
       ensure_smem_limit(append_cluster_kernel<128>, sizeof(AppendSmem<128>)) == cudaSuccess &&
       ensure_smem_limit(append_cluster_kernel<256>, sizeof(AppendSmem<256>)) == cudaSuccess;
   if (!ok) return ZKV_ERR_CUDA;
-  switch (p->d) {
-    case 64: append_cluster_kernel<64><<<grid, 256, sizeof(AppendSmem<64>), st>>>(*p, rot); break;
-    case 128: append_cluster_kernel<128><<<grid, 256, sizeof(AppendSmem<128>), st>>>(*p, rot); break;
-    default: append_cluster_kernel<256><<<grid, 256, sizeof(AppendSmem<256>), st>>>(*p, rot); break;
+  cudaError_t e = cudaSuccess;
+  switch (p.d) {
+    case 64:
+      if (pdl) e = launch_pdl(append_cluster_kernel<64>, grid, dim3(256), sizeof(AppendSmem<64>), st, p, rot);
+      else append_cluster_kernel<64><<<grid, 256, sizeof(AppendSmem<64>), st>>>(p, rot);
+      break;
+    case 128:
+      if (pdl) e = launch_pdl(append_cluster_kernel<128>, grid, dim3(256), sizeof(AppendSmem<128>), st, p, rot);
+      else append_cluster_kernel<128><<<grid, 256, sizeof(AppendSmem<128>), st>>>(p, rot);
+      break;
+    default:
+      if (pdl) e = launch_pdl(append_cluster_kernel<256>, grid, dim3(256), sizeof(AppendSmem<256>), st, p, rot);
+      else append_cluster_kernel<256><<<grid, 256, sizeof(AppendSmem<256>), st>>>(p, rot);
+      break;
   }
+  if (e != cudaSuccess) return ZKV_ERR_CUDA;
   ZKV_CHECK_LAUNCH();
+  return ZKV_OK;
+}
+
+}  // namespace zkv
+
+using namespace zkv;
+
+extern "C" int zkv_rvq_append(const zkv_append_params* p, void* stream) {
+  const int v = validate_append(p);
+  if (v != ZKV_OK) return v;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int rc = launch_append_cluster(*p, st, false);
+  if (rc != ZKV_OK) return rc;
   if (launch_pdl(append_lengths_kernel, dim3((p->B + 127) / 128), dim3(128), 0, st, p->B, p->Tcap,
                  p->Wcap, p->win_len, p->win_head, p->comp_len) != cudaSuccess)
     return ZKV_ERR_CUDA;

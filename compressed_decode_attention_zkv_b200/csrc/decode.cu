@@ -34,6 +34,7 @@
 //    are mapped to (token slot, stage, head) so one instruction touches 32 distinct banks.
 //    Column sums stay below 2^32 because a segment holds at most 8176 tokens per column.
 #include "zkv_internal.cuh"
+#include "lengths.cuh"
 
 #include <algorithm>
 #include <cfloat>
@@ -147,6 +148,7 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, d, Sk, Sv, Rk, grid, n_lut_blocks;
+  int do_partition;   // the table kernel also runs the partition block
   int64_t Tcap, Wcap, max_comp;
   float scale_log2;   // softmax_scale * log2(e)
   double rot;         // 1 / sqrt(d)
@@ -372,10 +374,16 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
   }
 }
 
-// ceil(x * m / d) for x, m >= 0 and d > 0, exact (128-bit product).
-__device__ __forceinline__ int64_t ceil_muldiv(int64_t x, int64_t m, int64_t d) {
-  const unsigned __int128 pr = (unsigned __int128)(uint64_t)x * (uint64_t)m;
-  return (int64_t)((pr + (uint64_t)(d - 1)) / (uint64_t)d);
+// floor(x * m / d) and ceil(x * m / d) for x, m >= 0 and d > 0, exact.  wide: the product may
+// exceed 2^63 (128-bit arithmetic, slow); otherwise 64-bit.
+__device__ __forceinline__ int64_t floor_muldiv(int64_t x, int64_t m, int64_t d, bool wide) {
+  if (wide) return (int64_t)(((unsigned __int128)(uint64_t)x * (uint64_t)m) / (uint64_t)d);
+  return (int64_t)(((uint64_t)x * (uint64_t)m) / (uint64_t)d);
+}
+__device__ __forceinline__ int64_t ceil_muldiv(int64_t x, int64_t m, int64_t d, bool wide) {
+  if (wide)
+    return (int64_t)(((unsigned __int128)(uint64_t)x * (uint64_t)m + (uint64_t)(d - 1)) / (uint64_t)d);
+  return (int64_t)(((uint64_t)x * (uint64_t)m + (uint64_t)(d - 1)) / (uint64_t)d);
 }
 
 // The partition of the compressed token space among the scan CTAs (one block):
@@ -442,6 +450,9 @@ __device__ void partition_block(const DecodeArgs& a) {
   }
   const int64_t V = carry_s[1], tot = carry_s[0];
   const int grid = a.grid;
+  // V <= pairs * (Tcap + kSegCost) < 2^53 here; products with grid stay below 2^62 unless the
+  // grid is very large
+  const bool wide = (double)(V + kSegCost + 1) * (double)grid >= 4.0e18;
   if (V == 0) {   // no compressed token at all
     for (int c = tid; c <= grid; c += 256) a.bounds[c] = 0;
     for (int k = tid; k < npairs; k += 256) {
@@ -458,15 +469,15 @@ __device__ void partition_block(const DecodeArgs& a) {
     const int64_t v0 = a.vs[k], v1 = a.vs[k + 1], p0 = a.pre[k], len = a.pre[k + 1] - p0;
     int f = 1, t = 0;   // first / last scan CTA holding the pair's tokens (f > t: none)
     if (len > 0) {
-      const int64_t clo = ceil_muldiv(v0, grid, V);       // cuts c in [clo, chi] lie in [v0, v1)
-      const int64_t chi = ceil_muldiv(v1, grid, V) - 1;
+      const int64_t clo = ceil_muldiv(v0, grid, V, wide);   // cuts c in [clo, chi] lie in [v0, v1)
+      const int64_t chi = ceil_muldiv(v1, grid, V, wide) - 1;
       for (int64_t c = clo > 1 ? clo : 1; c <= chi && c < grid; ++c) {
-        const int64_t off = (int64_t)(((unsigned __int128)(uint64_t)V * (uint64_t)c) / (uint64_t)grid) - v0;
+        const int64_t off = floor_muldiv(V, c, grid, wide) - v0;
         a.bounds[c] = off < kSegCost ? p0 : p0 + (off - kSegCost < len ? off - kSegCost : len);
       }
       // the CTA holding the first token: the last cut at or before v0 + kSegCost (its bound is
       // p0); the one holding the last token: the last cut before v1
-      const int64_t cf = ceil_muldiv(v0 + kSegCost + 1, grid, V) - 1;
+      const int64_t cf = ceil_muldiv(v0 + kSegCost + 1, grid, V, wide) - 1;
       f = (int)(cf < chi ? cf : chi);
       t = (int)chi;
     }
@@ -483,6 +494,7 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
   constexpr int E = D / 32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();   // the next kernel waits for this one before reading the tables
   if ((int)blockIdx.x == a.n_lut_blocks) {
     partition_block(a);
     return;
@@ -569,6 +581,19 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
           acc[k] * a.scale_log2;
     }
   }
+}
+
+// Serving step: the length update of the append (one evicted token per full window) followed
+// by the partition, in one block.  Launched after the encode kernel, whose completion implies
+// the table kernel's.
+__global__ void __launch_bounds__(256) lengths_partition_kernel(DecodeArgs a, int32_t* win_len,
+                                                                int32_t* win_head,
+                                                                int32_t* comp_len) {
+  pdl_wait();   // the encode kernel read the pre-step lengths
+  for (int b = threadIdx.x; b < a.B; b += 256)
+    advance_lengths(b, a.Tcap, a.Wcap, win_len, win_head, comp_len);
+  __syncthreads();   // the partition reads the updated lengths
+  partition_block(a);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1363,21 +1388,35 @@ static int launch_scan_kv(const DecodeArgs& a, int SKP, int SVP, size_t smem, cu
   }
 }
 
+int launch_append_cluster(const zkv_append_params& p, cudaStream_t st, bool pdl);   // append.cu
+
+// ap == nullptr: one decode call.  Otherwise the serving step: the tables (which depend only on
+// q and the key codebooks) run while the evicted tokens are encoded; then the length update
+// and the partition, then the decode proper.
 template <int D, int GP>
-static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cudaStream_t st) {
-  // 1. tables, window, prefix sums
+static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cudaStream_t st,
+                         const zkv_append_params* ap) {
+  // 1. tables and partition (with the serving step's encode in between)
   trace(ev, 0, st);
   {
     const size_t smem = sizeof(LutSmem<D>);
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
     a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
-    const int64_t blocks = (int64_t)a.n_lut_blocks + 1;   // + the partition block
+    a.do_partition = ap ? 0 : 1;
+    const int64_t blocks = (int64_t)a.n_lut_blocks + a.do_partition;
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
     // a normal launch: the caller's preceding work (which may write q) must be complete, since
     // the table blocks do not wait
     lut_kernel<D, GP><<<(unsigned)blocks, 256, smem, st>>>(a);
     ZKV_CHECK_LAUNCH();
+    if (ap) {
+      const int rc = launch_append_cluster(*ap, st, true);
+      if (rc != ZKV_OK) return rc;
+      if (launch_pdl(lengths_partition_kernel, dim3(1), dim3(256), 0, st, a, ap->win_len,
+                     ap->win_head, ap->comp_len) != cudaSuccess)
+        return ZKV_ERR_CUDA;
+    }
   }
   // 2. scan
   trace(ev, 1, st);
@@ -1409,12 +1448,12 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
 
 template <int D>
 static int launch_decode_g(const DecodeArgs& a, const DecodePlan& pl, void* const* ev,
-                           cudaStream_t st) {
+                           cudaStream_t st, const zkv_append_params* ap) {
   switch (pl.GP) {
-    case 1: return launch_decode<D, 1>(a, pl, ev, st);
-    case 2: return launch_decode<D, 2>(a, pl, ev, st);
-    case 4: return launch_decode<D, 4>(a, pl, ev, st);
-    default: return launch_decode<D, 8>(a, pl, ev, st);
+    case 1: return launch_decode<D, 1>(a, pl, ev, st, ap);
+    case 2: return launch_decode<D, 2>(a, pl, ev, st, ap);
+    case 4: return launch_decode<D, 4>(a, pl, ev, st, ap);
+    default: return launch_decode<D, 8>(a, pl, ev, st, ap);
   }
 }
 
@@ -1455,8 +1494,12 @@ extern "C" size_t zkv_decode_workspace_size(const zkv_decode_params* p) {
   return make_plan(p).total;
 }
 
-extern "C" int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+namespace zkv {
+int validate_append(const zkv_append_params* p);   // append.cu
+
+// Shared by the decode call and the serving step (ap != nullptr).
+static int decode_common(const zkv_decode_params* p, void* workspace, size_t workspace_bytes,
+                         void* stream, const zkv_append_params* ap) {
   const int v = validate_decode(p);
   if (v != ZKV_OK) return v;
   const DecodePlan pl = make_plan(p);
@@ -1466,7 +1509,7 @@ extern "C" int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace,
   unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
   DecodeArgs a;
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = pl.G; a.d = p->d; a.Sk = p->Sk; a.Sv = p->Sv;
-  a.Rk = pl.Rk; a.grid = pl.grid; a.n_lut_blocks = 0;
+  a.Rk = pl.Rk; a.grid = pl.grid; a.n_lut_blocks = 0; a.do_partition = 1;
   a.Tcap = p->Tcap; a.Wcap = p->Wcap; a.max_comp = p->max_comp_len;
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale : (float)(1.0 / std::sqrt((double)p->d));
   a.scale_log2 = scale * kLog2e;
@@ -1492,10 +1535,35 @@ extern "C" int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace,
   a.so = reinterpret_cast<float*>(ws + pl.off_so);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (p->d) {
-    case 64: return launch_decode_g<64>(a, pl, p->trace_events, st);
-    case 128: return launch_decode_g<128>(a, pl, p->trace_events, st);
-    default: return launch_decode_g<256>(a, pl, p->trace_events, st);
+    case 64: return launch_decode_g<64>(a, pl, p->trace_events, st, ap);
+    case 128: return launch_decode_g<128>(a, pl, p->trace_events, st, ap);
+    default: return launch_decode_g<256>(a, pl, p->trace_events, st, ap);
   }
+}
+
+}  // namespace zkv
+
+extern "C" int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return decode_common(p, workspace, workspace_bytes, stream, nullptr);
+}
+
+extern "C" int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_params* dp,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  const int va = validate_append(ap);
+  if (va != ZKV_OK) return va;
+  const int vd = validate_decode(dp);
+  if (vd != ZKV_OK) return vd;
+  // one cache: the same shapes and the same buffers
+  if (ap->B != dp->B || ap->Hkv != dp->Hkv || ap->d != dp->d || ap->Sk != dp->Sk ||
+      ap->Sv != dp->Sv || ap->Tcap != dp->Tcap || ap->Wcap != dp->Wcap)
+    return ZKV_ERR_INVALID_ARG;
+  if (ap->k_codes != dp->k_codes || ap->v_codes != dp->v_codes ||
+      ap->k_codebooks != dp->k_codebooks || ap->v_codebooks != dp->v_codebooks ||
+      ap->win_k != dp->win_k || ap->win_v != dp->win_v || ap->win_len != dp->win_len ||
+      ap->comp_len != dp->comp_len)
+    return ZKV_ERR_INVALID_ARG;
+  return decode_common(dp, workspace, workspace_bytes, stream, ap);
 }
 
 // ------------------------------------------------------------------------------------------

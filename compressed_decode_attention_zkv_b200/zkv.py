@@ -105,6 +105,9 @@ def lib() -> ctypes.CDLL:
         L.zkv_rvq_decode_attn_noalloc.argtypes = [POINTER(DecodeParams), c_void_p]
         L.zkv_rvq_append.restype = c_int
         L.zkv_rvq_append.argtypes = [POINTER(AppendParams), c_void_p]
+        L.zkv_rvq_serve_step.restype = c_int
+        L.zkv_rvq_serve_step.argtypes = [POINTER(AppendParams), POINTER(DecodeParams), c_void_p,
+                                         c_size_t, c_void_p]
         _lib = L
     return _lib
 
@@ -327,9 +330,8 @@ def rvq_decode_attn_noalloc(q, k_codes, v_codes, comp_len, k_codebooks, v_codebo
     return out, lse
 
 
-def rvq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
-               k_codebooks, v_codebooks, error_flag=None):
-    """One serving step of cache maintenance (see include/zkv.h); state updated in place."""
+def _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
+                   k_codebooks, v_codebooks, error_flag):
     _need(new_k, "new_k", torch.float16)
     _need(new_v, "new_v", torch.float16)
     for n, t in (("win_k", win_k), ("win_v", win_v)):
@@ -343,12 +345,19 @@ def rvq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
     if error_flag is not None:
         _need(error_flag, "error_flag", torch.int32)
     B, Hkv, Tcap, Sk = k_codes.shape
-    p = AppendParams(B=B, Hkv=Hkv, d=new_k.shape[-1], Sk=Sk, Sv=v_codes.shape[3], Tcap=Tcap,
-                     Wcap=win_k.shape[2], new_k=_ptr(new_k), new_v=_ptr(new_v),
-                     win_k=_ptr(win_k), win_v=_ptr(win_v), win_len=_ptr(win_len),
-                     win_head=_ptr(win_head), comp_len=_ptr(comp_len), k_codes=_ptr(k_codes),
-                     v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
-                     v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag))
+    return AppendParams(B=B, Hkv=Hkv, d=new_k.shape[-1], Sk=Sk, Sv=v_codes.shape[3], Tcap=Tcap,
+                        Wcap=win_k.shape[2], new_k=_ptr(new_k), new_v=_ptr(new_v),
+                        win_k=_ptr(win_k), win_v=_ptr(win_v), win_len=_ptr(win_len),
+                        win_head=_ptr(win_head), comp_len=_ptr(comp_len), k_codes=_ptr(k_codes),
+                        v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
+                        v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag))
+
+
+def rvq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
+               k_codebooks, v_codebooks, error_flag=None):
+    """One serving step of cache maintenance (see include/zkv.h); state updated in place."""
+    p = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
+                       v_codes, k_codebooks, v_codebooks, error_flag)
     _check("zkv_rvq_append", lib().zkv_rvq_append(ctypes.byref(p), _stream()))
 
 
@@ -359,28 +368,10 @@ class PreparedAppend:
 
     def __init__(self, new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
                  v_codes, k_codebooks, v_codebooks, error_flag=None):
-        _need(new_k, "new_k", torch.float16)
-        _need(new_v, "new_v", torch.float16)
-        for n, t in (("win_k", win_k), ("win_v", win_v)):
-            _need(t, n, torch.float16)
-        for n, t in (("win_len", win_len), ("win_head", win_head), ("comp_len", comp_len)):
-            _need(t, n, torch.int32)
-        _need(k_codes, "k_codes", torch.uint8)
-        _need(v_codes, "v_codes", torch.uint8)
-        _need(k_codebooks, "k_codebooks", torch.float32)
-        _need(v_codebooks, "v_codebooks", torch.float32)
-        if error_flag is not None:
-            _need(error_flag, "error_flag", torch.int32)
-        B, Hkv, Tcap, Sk = k_codes.shape
         self._keep = (new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
                       k_codebooks, v_codebooks, error_flag)
-        self._p = AppendParams(B=B, Hkv=Hkv, d=new_k.shape[-1], Sk=Sk, Sv=v_codes.shape[3],
-                               Tcap=Tcap, Wcap=win_k.shape[2], new_k=_ptr(new_k),
-                               new_v=_ptr(new_v), win_k=_ptr(win_k), win_v=_ptr(win_v),
-                               win_len=_ptr(win_len), win_head=_ptr(win_head),
-                               comp_len=_ptr(comp_len), k_codes=_ptr(k_codes),
-                               v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
-                               v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag))
+        self._p = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len,
+                                 k_codes, v_codes, k_codebooks, v_codebooks, error_flag)
         self._ref = ctypes.byref(self._p)
         self._fn = lib().zkv_rvq_append
 
@@ -388,6 +379,70 @@ class PreparedAppend:
         st = self._fn(self._ref, torch.cuda.current_stream().cuda_stream)
         if st != ZKV_OK:
             raise ZkvError("zkv_rvq_append", st)
+
+
+class PreparedServeStep:
+    """One serving step (append of the new tokens, then decode attention of q over the updated
+    cache) as a single library call, zkv_rvq_serve_step, with its arguments marshalled once.
+    The tensors must keep their storage; max_comp_len must stay an upper bound of every
+    comp_len after the step.  Calling it runs the step on the current stream and returns
+    (out, lse)."""
+
+    def __init__(self, new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes,
+                 v_codes, k_codebooks, v_codebooks, out=None, lse=None, max_comp_len=None,
+                 softmax_scale=None, workspace: torch.Tensor | None = None, error_flag=None,
+                 trace_events=None):
+        B, Hq, d = q.shape
+        if out is None:
+            out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+        if lse is None:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        self._pa = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len,
+                                  k_codes, v_codes, k_codebooks, v_codebooks, error_flag)
+        self._pd = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
+                                  win_v, win_len, out, lse, max_comp_len, softmax_scale,
+                                  error_flag)
+        self._ev = None
+        if trace_events is not None:   # recorded before the tables, the scan, the merge, and last
+            if len(trace_events) != 4:
+                raise ValueError("trace_events needs 4 events")
+            self._ev = (c_void_p * 4)(*[e.cuda_event for e in trace_events])
+            self._pd.trace_events = ctypes.cast(self._ev, c_void_p)
+        need = lib().zkv_decode_workspace_size(ctypes.byref(self._pd))
+        if need == 0:
+            raise ZkvError("zkv_decode_workspace_size", ZKV_ERR_INVALID_ARG)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8)
+        if workspace.numel() < need:
+            raise ZkvError("zkv_rvq_serve_step", ZKV_ERR_WORKSPACE,
+                           f"workspace holds {workspace.numel()} bytes, {need} needed")
+        self.out, self.lse = out, lse
+        self._keep = (new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes,
+                      v_codes, k_codebooks, v_codebooks, workspace, error_flag)
+        self._refa, self._refd = ctypes.byref(self._pa), ctypes.byref(self._pd)
+        self._ws = ctypes.c_void_p(workspace.data_ptr())
+        self._wsn = ctypes.c_size_t(workspace.numel())
+        self._fn = lib().zkv_rvq_serve_step
+
+    def __call__(self):
+        st = self._fn(self._refa, self._refd, self._ws, self._wsn,
+                      torch.cuda.current_stream().cuda_stream)
+        if st != ZKV_OK:
+            raise ZkvError("zkv_rvq_serve_step", st)
+        return self.out, self.lse
+
+
+def rvq_serve_step(new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
+                   k_codebooks, v_codebooks, out=None, lse=None, max_comp_len=None,
+                   softmax_scale=None, workspace=None, error_flag=None, trace_events=None):
+    """rvq_append(new_k, new_v, ...) then rvq_decode_attn(q, ...) on the updated cache, in one
+    library call (see include/zkv.h).  Returns (out, lse)."""
+    if max_comp_len is None:
+        max_comp_len = k_codes.shape[2]
+    return PreparedServeStep(new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len,
+                             k_codes, v_codes, k_codebooks, v_codebooks, out, lse, max_comp_len,
+                             softmax_scale, workspace, error_flag, trace_events)()
 
 
 class PreparedDecode:

@@ -169,7 +169,8 @@ int zkv_rvq_reconstruct(const zkv_reconstruct_params* p, void* stream);
  * calls into a CUDA graph.
  * Workspace: device buffer of at least zkv_decode_workspace_size(p) bytes, 256-byte aligned,
  *   no initial contents required; it must not be shared by calls that run concurrently.
- * Errors: INVALID_ARG, UNSUPPORTED (d, S, Hq/Hkv > 8), WORKSPACE, CUDA.
+ * Errors: INVALID_ARG, UNSUPPORTED (d, S, Hq/Hkv > 8, or a GQA group of 5..8 with Sv > 4,
+ *         whose value histograms do not fit in one SM's shared memory), WORKSPACE, CUDA.
  */
 typedef struct {
   int B, Hq, Hkv, d, Sk, Sv;
@@ -257,6 +258,26 @@ typedef struct {
 } zkv_append_params;
 
 int zkv_rvq_append(const zkv_append_params* p, void* stream);
+
+/*
+ * zkv_rvq_serve_step -- one whole decode step of a serving loop: zkv_rvq_append(ap) followed
+ * by zkv_rvq_decode_attn(dp) on the updated cache, in one call.
+ * Passages: VeloxQuant "Quick start" (cache.append(k, v), then cache.attend(q)); VQKV section
+ * 2.3 "Local Sliding Window" and "Decoding Stage".
+ * Results are identical to the two calls made in that order.  The library overlaps the
+ * decode's lookup-table construction (which needs only q and the key codebooks) with the encode
+ * of the evicted tokens, and folds the length update into the decode's partition step.
+ * ap and dp describe one cache: B, Hkv, d, Sk, Sv, Tcap and Wcap must be equal, and so must
+ * k_codes, v_codes, k_codebooks, v_codebooks, win_k, win_v, win_len and comp_len (else
+ * ZKV_ERR_INVALID_ARG).  dp->comp_len and dp->win_len are read after the update, so
+ * dp->max_comp_len must allow for the new token.  workspace: as zkv_rvq_decode_attn
+ * (zkv_decode_workspace_size(dp)); dp->trace_events: as zkv_rvq_decode_attn, where the first
+ * interval covers the tables, the encode and the length update.
+ * Errors: those of zkv_rvq_append and zkv_rvq_decode_attn; validation of both happens before
+ * any launch.
+ */
+int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_params* dp,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -115,6 +115,33 @@ def test_append_validation(L):
     assert L.zkv_rvq_append(ctypes.byref(p), None) == zkv.ZKV_ERR_INVALID_ARG  # null pointers
 
 
+def _append_params(**kw):
+    # the same cache as _decode_params (shapes and shared buffers)
+    base = dict(B=2, Hkv=2, d=128, Sk=4, Sv=4, Tcap=64, Wcap=16, new_k=0xb000, new_v=0xc000,
+                win_k=0x7000, win_v=0x8000, win_len=0x9000, win_head=0xd000, comp_len=0x4000,
+                k_codes=0x2000, v_codes=0x3000, k_codebooks=0x5000, v_codebooks=0x6000)
+    base.update(kw)
+    return zkv.AppendParams(**base)
+
+
+@pytest.mark.parametrize("akw,dkw,status", [
+    (dict(k_codes=0x2100), {}, zkv.ZKV_ERR_INVALID_ARG),      # another cache's codes
+    (dict(comp_len=0x4100), {}, zkv.ZKV_ERR_INVALID_ARG),
+    (dict(win_v=0x8100), {}, zkv.ZKV_ERR_INVALID_ARG),
+    (dict(Tcap=128), {}, zkv.ZKV_ERR_INVALID_ARG),            # shapes differ
+    (dict(B=3), {}, zkv.ZKV_ERR_INVALID_ARG),
+    (dict(Sv=3), {}, zkv.ZKV_ERR_INVALID_ARG),
+    (dict(new_k=0), {}, zkv.ZKV_ERR_INVALID_ARG),             # the append itself is invalid
+    (dict(d=96), dict(d=96), zkv.ZKV_ERR_UNSUPPORTED),
+    ({}, dict(Hq=6, Hkv=4), zkv.ZKV_ERR_INVALID_ARG),          # the decode itself is invalid
+    ({}, {}, zkv.ZKV_ERR_WORKSPACE),                           # consistent, but no workspace
+])
+def test_serve_step_validation(L, akw, dkw, status):
+    """zkv_rvq_serve_step refuses inconsistent or invalid arguments before any launch."""
+    ap, dp = _append_params(**akw), _decode_params(**dkw)
+    assert L.zkv_rvq_serve_step(ctypes.byref(ap), ctypes.byref(dp), None, 0, None) == status
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 128, dtype=torch.float16)

@@ -332,3 +332,87 @@ def test_prepared_calls_match_the_plain_entry_points():
         assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {step}"
         for key in ("k_codes", "v_codes", "win_k", "win_v", "comp_len", "win_len", "win_head"):
             assert torch.equal(a[key], b[key]), f"{key} step {step}"
+
+
+@pytest.mark.parametrize("B_,Hq,Hkv,d,S,Sv,Tcap,Wcap,win_len,win_head,comp_len", [
+    (3, 8, 2, 128, 4, 4, 64, 4, [4, 4, 2], [1, 0, 0], [10, 0, 33]),
+    (9, 14, 2, 64, 2, 3, 48, 3, [3, 1, 3, 0, 3, 3, 2, 3, 3], [2, 0, 0, 0, 1, 0, 0, 2, 1],
+     [47, 5, 0, 0, 20, 48, 3, 8, 16]),
+])
+def test_serve_step_matches_append_then_decode(B_, Hq, Hkv, d, S, Sv, Tcap, Wcap, win_len,
+                                               win_head, comp_len):
+    """zkv_rvq_serve_step gives bit-identical outputs and cache state to zkv_rvq_append followed
+    by zkv_rvq_decode_attn, step after step (free slots, evictions, a full prefix)."""
+    st = _state(90 + B_, B_=B_, Hkv=Hkv, d=d, S=S, Sv=Sv, Tcap=Tcap, Wcap=Wcap, win_len=win_len,
+                win_head=win_head, comp_len=comp_len)
+    rng = np.random.default_rng(91 + B_)
+    sides = []
+    for _ in range(2):
+        g = {k: _cuda(v.astype(np.int32) if k in ("comp_len", "win_len", "win_head") else v)
+             for k, v in st.items()}
+        g["err"] = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sides.append(g)
+    a, b = sides
+    for step in range(4):
+        nk = _cuda(rng.standard_normal((B_, Hkv, d)).astype(np.float16))
+        nv = _cuda(rng.standard_normal((B_, Hkv, d)).astype(np.float16))
+        q = _cuda(rng.standard_normal((B_, Hq, d)).astype(np.float16))
+        zkv.rvq_append(nk, nv, a["win_k"], a["win_v"], a["win_len"], a["win_head"],
+                       a["comp_len"], a["k_codes"], a["v_codes"], a["Ck"], a["Cv"],
+                       error_flag=a["err"])
+        o1, l1 = zkv.rvq_decode_attn(q, a["k_codes"], a["v_codes"], a["comp_len"], a["Ck"],
+                                     a["Cv"], a["win_k"], a["win_v"], a["win_len"],
+                                     max_comp_len=Tcap, error_flag=a["err"])
+        o2, l2 = zkv.rvq_serve_step(nk, nv, q, b["win_k"], b["win_v"], b["win_len"],
+                                    b["win_head"], b["comp_len"], b["k_codes"], b["v_codes"],
+                                    b["Ck"], b["Cv"], max_comp_len=Tcap, error_flag=b["err"])
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {step}"
+        for key in ("k_codes", "v_codes", "win_k", "win_v", "comp_len", "win_len", "win_head",
+                    "err"):
+            assert torch.equal(a[key], b[key]), f"{key} step {step}"
+
+
+def test_serve_step_loop_matches_oracle():
+    """Prepared serving steps on a trained-codebook cache vs the oracle's append step followed
+    by its decode (plain definition)."""
+    rng = np.random.default_rng(95)
+    wl = I.workload("llama3_8b_32k", B=2, Hq=8, Hkv=2, T=700, W=16, n_cal=2048, kmeans_iters=4)
+    Ck, Cv = I.train_codebooks(wl, "k"), I.train_codebooks(wl, "v")
+    Tc, Tcap = wl.Tc, (wl.Tc + 32 + 15) // 16 * 16   # capacities are multiples of 16
+    zk = np.zeros((wl.B, wl.Hkv, Tcap, wl.Sk), np.uint8)
+    zv = np.zeros((wl.B, wl.Hkv, Tcap, wl.Sv), np.uint8)
+    wk = np.zeros((wl.B, wl.Hkv, wl.W, wl.d), np.float16)
+    wv = np.zeros((wl.B, wl.Hkv, wl.W, wl.d), np.float16)
+    for b in range(wl.B):
+        xk, xv = I.kv_tokens(wl, "k", b, 0, wl.T), I.kv_tokens(wl, "v", b, 0, wl.T)
+        for h in range(wl.Hkv):
+            zk[b, h, :Tc] = O.rvq_encode(xk[h, :Tc], Ck[h])[0]
+            zv[b, h, :Tc] = O.rvq_encode(xv[h, :Tc], Cv[h])[0]
+        wk[b], wv[b] = xk[:, Tc:], xv[:, Tc:]
+    st = dict(k_codes=zk, v_codes=zv, comp_len=np.full(wl.B, Tc), win_len=np.full(wl.B, wl.W),
+              win_head=np.zeros(wl.B, np.int64), win_k=wk, win_v=wv, Ck=Ck, Cv=Cv)
+    g = {k: _cuda(v.astype(np.int32) if k in ("comp_len", "win_len", "win_head") else v)
+         for k, v in st.items()}
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nk_d = torch.zeros((wl.B, wl.Hkv, wl.d), dtype=torch.float16, device="cuda")
+    nv_d, q_d = torch.zeros_like(nk_d), torch.zeros((wl.B, wl.Hq, wl.d), dtype=torch.float16,
+                                                     device="cuda")
+    step_fn = zkv.PreparedServeStep(nk_d, nv_d, q_d, g["win_k"], g["win_v"], g["win_len"],
+                                    g["win_head"], g["comp_len"], g["k_codes"], g["v_codes"],
+                                    g["Ck"], g["Cv"], max_comp_len=Tcap, error_flag=err)
+    for step in range(3):
+        nk = rng.standard_normal((wl.B, wl.Hkv, wl.d)).astype(np.float16)
+        nv = rng.standard_normal((wl.B, wl.Hkv, wl.d)).astype(np.float16)
+        q = rng.standard_normal((wl.B, wl.Hq, wl.d)).astype(np.float16)
+        nk_d.copy_(_cuda(nk))
+        nv_d.copy_(_cuda(nv))
+        q_d.copy_(_cuda(q))
+        out, lse = step_fn()
+        st = O.append_step(st, nk, nv)
+        case = (q, st["k_codes"], st["v_codes"], st["comp_len"], Ck, Cv, st["win_k"],
+                st["win_v"], st["win_len"])
+        _compare(case, out.cpu().numpy(), lse.cpu().numpy())
+        assert np.array_equal(g["k_codes"].cpu().numpy(), st["k_codes"])
+        assert np.array_equal(g["v_codes"].cpu().numpy(), st["v_codes"])
+    assert int(err.item()) == 0
