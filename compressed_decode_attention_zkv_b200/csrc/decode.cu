@@ -148,7 +148,11 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, d, Sk, Sv, Rk, grid, n_lut_blocks;
-  int do_partition;   // the table kernel also runs the partition block
+  // Serving step: the partition uses the lengths after this step's append (predicted from
+  // the pre-step state with the append's rule), and scan block 0 stores them.  Null otherwise.
+  int32_t* upd_win_len;
+  int32_t* upd_win_head;
+  int32_t* upd_comp_len;
   int64_t Tcap, Wcap, max_comp;
   float scale_log2;   // softmax_scale * log2(e)
   double rot;         // 1 / sqrt(d)
@@ -410,7 +414,12 @@ __device__ void partition_block(const DecodeArgs& a) {
     const int pr = base + tid;
     int64_t c = 0;
     if (pr < npairs) {
-      c = a.comp_len[pr / a.Hkv];
+      const int b = pr / a.Hkv;
+      c = a.comp_len[b];
+      if (a.upd_comp_len) {   // this step's append evicts a token onto the prefix
+        const int64_t wl = a.upd_win_len[b], hd = a.upd_win_head[b];
+        if (wl == a.Wcap && hd >= 0 && hd < a.Wcap && c >= 0 && c < a.Tcap) c += 1;
+      }
       if (c < 0 || c > a.Tcap) {
         set_error(a.err, ZKV_DEVERR_COMP_LEN);
         c = c < 0 ? 0 : a.Tcap;
@@ -581,19 +590,6 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
           acc[k] * a.scale_log2;
     }
   }
-}
-
-// Serving step: the length update of the append (one evicted token per full window) followed
-// by the partition, in one block.  Launched after the encode kernel, whose completion implies
-// the table kernel's.
-__global__ void __launch_bounds__(256) lengths_partition_kernel(DecodeArgs a, int32_t* win_len,
-                                                                int32_t* win_head,
-                                                                int32_t* comp_len) {
-  pdl_wait();   // the encode kernel read the pre-step lengths
-  for (int b = threadIdx.x; b < a.B; b += 256)
-    advance_lengths(b, a.Tcap, a.Wcap, win_len, win_head, comp_len);
-  __syncthreads();   // the partition reads the updated lengths
-  partition_block(a);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -803,6 +799,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) unsigned char smraw[];
   pdl_wait();   // tables, prefix sums and codes
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (a.upd_comp_len && blockIdx.x == 0) {
+    // serving step: the append has read the pre-step lengths; store the new ones (nothing in
+    // this kernel reads them)
+    for (int b = tid; b < a.B; b += kScanThreads)
+      advance_lengths(b, a.Tcap, a.Wcap, a.upd_win_len, a.upd_win_head, a.upd_comp_len);
+  }
   const int Rk = a.Rk, Sk = a.Sk, Sv = a.Sv, G = a.G;
   const int ntab = Sv * kCodebook * GP;           // histogram entries (s, c, g)
   float* lut = reinterpret_cast<float*>(smraw);                                 // [Sk][256][Rk][GP]
@@ -1391,8 +1393,8 @@ static int launch_scan_kv(const DecodeArgs& a, int SKP, int SVP, size_t smem, cu
 int launch_append_cluster(const zkv_append_params& p, cudaStream_t st, bool pdl);   // append.cu
 
 // ap == nullptr: one decode call.  Otherwise the serving step: the tables (which depend only on
-// q and the key codebooks) run while the evicted tokens are encoded; then the length update
-// and the partition, then the decode proper.
+// q and the key codebooks) and the partition (on the lengths this step's append produces) run
+// while the evicted tokens are encoded; scan block 0 stores the new lengths.
 template <int D, int GP>
 static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cudaStream_t st,
                          const zkv_append_params* ap) {
@@ -1403,19 +1405,16 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
     a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
-    a.do_partition = ap ? 0 : 1;
-    const int64_t blocks = (int64_t)a.n_lut_blocks + a.do_partition;
+    const int64_t blocks = (int64_t)a.n_lut_blocks + 1;   // + the partition block
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
     // a normal launch: the caller's preceding work (which may write q) must be complete, since
     // the table blocks do not wait
     lut_kernel<D, GP><<<(unsigned)blocks, 256, smem, st>>>(a);
     ZKV_CHECK_LAUNCH();
     if (ap) {
+      // its completion implies the table kernel's (it waits for it before exiting)
       const int rc = launch_append_cluster(*ap, st, true);
       if (rc != ZKV_OK) return rc;
-      if (launch_pdl(lengths_partition_kernel, dim3(1), dim3(256), 0, st, a, ap->win_len,
-                     ap->win_head, ap->comp_len) != cudaSuccess)
-        return ZKV_ERR_CUDA;
     }
   }
   // 2. scan
@@ -1509,7 +1508,10 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
   DecodeArgs a;
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = pl.G; a.d = p->d; a.Sk = p->Sk; a.Sv = p->Sv;
-  a.Rk = pl.Rk; a.grid = pl.grid; a.n_lut_blocks = 0; a.do_partition = 1;
+  a.Rk = pl.Rk; a.grid = pl.grid; a.n_lut_blocks = 0;
+  a.upd_win_len = ap ? ap->win_len : nullptr;
+  a.upd_win_head = ap ? ap->win_head : nullptr;
+  a.upd_comp_len = ap ? ap->comp_len : nullptr;
   a.Tcap = p->Tcap; a.Wcap = p->Wcap; a.max_comp = p->max_comp_len;
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale : (float)(1.0 / std::sqrt((double)p->d));
   a.scale_log2 = scale * kLog2e;

@@ -265,8 +265,9 @@ int zkv_rvq_append(const zkv_append_params* p, void* stream);
  * Passages: VeloxQuant "Quick start" (cache.append(k, v), then cache.attend(q)); VQKV section
  * 2.3 "Local Sliding Window" and "Decoding Stage".
  * Results are identical to the two calls made in that order.  The library overlaps the
- * decode's lookup-table construction (which needs only q and the key codebooks) with the encode
- * of the evicted tokens, and folds the length update into the decode's partition step.
+ * decode's lookup-table construction (which needs only q and the key codebooks) and its
+ * partition of the token space (computed from the lengths the append will produce) with the
+ * encode of the evicted tokens; the new lengths are stored by the decode's scan kernel.
  * ap and dp describe one cache: B, Hkv, d, Sk, Sv, Tcap and Wcap must be equal, and so must
  * k_codes, v_codes, k_codebooks, v_codebooks, win_k, win_v, win_len and comp_len (else
  * ZKV_ERR_INVALID_ARG).  dp->comp_len and dp->win_len are read after the update, so
