@@ -587,7 +587,7 @@ def run_ours(args):
                            l2=f"{R} rotating replicas x {rep_mb:.1f} MB = {R * rep_mb:.0f} MB > 126 MB L2",
                            parallelism=f"replicas x{world}, no collective",
                            graph="one CUDA graph per replica step"),
-            "gpu_launches": 6 * args.steps,   # tables, encode, lengths+partition, scan, merge, finalize
+            "gpu_launches": 5 * args.steps,   # tables+partition, encode, scan, merge, finalize
             "roofline": roof,
             "kernels_s": per,
             "step_call": {"seconds": step_time, "algorithmic_bytes": call_bytes,
