@@ -1578,7 +1578,7 @@ extern "C" int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_
 // (allocated by the driver when the module loads) instead of a buffer they own.
 //
 // Nothing in the array has to start at zero: every word a call reads is written earlier in
-// the same call (the first kernel clears the completion counters).  There is one array per
+// the same call.  There is one array per
 // device, so calls on one device that overlap in time (two streams, two host threads) race
 // on it; the caller orders them.
 // ------------------------------------------------------------------------------------------
