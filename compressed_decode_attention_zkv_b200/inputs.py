@@ -276,20 +276,35 @@ def _kmeans_zero_pinned(X: np.ndarray, K: int, iters: int,
     return C, assign(C)
 
 
+def key_smooth_factors(wl: Workload, seed_cal: int = SEED_CALIB) -> np.ndarray:
+    """Per-channel key smoothing factors calibrated on the calibration sample, float32
+    [Hkv][d]: the square root of each channel's largest magnitude (1 for an all-zero channel).
+    Like the codebooks, a pre-calibrated input of the quantiser, shared by both sides."""
+    lam = np.ones((wl.Hkv, wl.d), np.float32)
+    for h in range(wl.Hkv):
+        m = np.abs(_calibration_sample(wl, "k", h, wl.n_cal, seed_cal).astype(np.float64)).max(0)
+        lam[h] = np.where(m > 0, np.sqrt(m), 1.0)
+    return lam
+
+
 def train_codebooks(wl: Workload, kind: str, S: int | None = None,
-                    seed_cal: int = SEED_CALIB, seed_km: int = SEED_KMEANS) -> np.ndarray:
+                    seed_cal: int = SEED_CALIB, seed_km: int = SEED_KMEANS,
+                    smooth: np.ndarray | None = None) -> np.ndarray:
     """Residual k-means codebooks in the Walsh-Hadamard domain, float32 [Hkv][S][256][d].
 
     Stage s is trained on the calibration residuals left after stages < s; codeword 0 of every
-    stage is the zero vector.
+    stage is the zero vector.  ``smooth`` ([Hkv][d] key smoothing factors): the calibration
+    vectors are divided by them before the rotation.
     """
     if S is None:
         S = wl.Sk if kind == "k" else wl.Sv
     Hn = scipy.linalg.hadamard(wl.d).astype(np.float64) / np.sqrt(wl.d)
     books = np.zeros((wl.Hkv, S, K_CODEWORDS, wl.d), np.float32)
     for h in range(wl.Hkv):
-        X = _calibration_sample(wl, kind, h, wl.n_cal, seed_cal)
-        R = (X.astype(np.float64) @ Hn.T).astype(np.float32)
+        X = _calibration_sample(wl, kind, h, wl.n_cal, seed_cal).astype(np.float64)
+        if smooth is not None:
+            X = X / np.asarray(smooth[h], np.float64)[None, :]
+        R = (X @ Hn.T).astype(np.float32)
         krng = _rng(seed_km, 200 + (0 if kind == "k" else 1), h)
         for s in range(S):
             C, a = _kmeans_zero_pinned(R, K_CODEWORDS, wl.kmeans_iters, krng)

@@ -16,7 +16,8 @@ blocking, fusion or reordering beyond what each definition states.  Sources (web
 * "zerokv-neo 4.0.0" (pypi), "Architecture": FWHT energy spreading before quantisation; hot
   tier of recent tokens kept in FP16.
 * "VeloxQuant-MLX 0.5.1" (pypi), "VecInfer": Walsh-Hadamard rotation whose inverse is absorbed
-  into the query, q_tilde . K_tilde^T == q . K^T.
+  into the query, q_tilde . K_tilde^T == q . K^T; the optional per-channel smooth scaling of the
+  keys before the rotation, lambda_i = sqrt(max |K_i|), also absorbed into the query.
 * "Differential-KV" (GitHub README), "Decode & Prefill Innovations": flash-style fp32
   log-sum-exp combine of the compressed part with a dense recency window.
 
@@ -28,6 +29,9 @@ Readings where the pages are silent (each is also listed in the design notes):
 * Greedy stage decision: squared L2 distance evaluated in float64, ties to the lowest index.
   The residual update r <- r - C_s[z_s] is an elementwise float32 subtraction.
 * Residual norm n_s = ||r|| after stage s (float64 accumulate, stored float32).
+* Smooth scaling (keys only): the key is multiplied by 1/lambda channel by channel in float64
+  (1/lambda itself a float64 division of the float32 factor) before the rotation; the query is
+  multiplied by lambda.  A channel that is zero on every calibration token gets lambda = 1.
 * Attention: scores = softmax_scale * q . k with softmax_scale defaulting to 1/sqrt(d); the
   first T_c tokens of a sequence are compressed, the window holds the newest ones (order inside
   the window is irrelevant); GQA maps query head h to kv head h // (Hq // Hkv); lse is the
@@ -80,6 +84,25 @@ def rotate_to_f32(x: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------------
+# Smooth scaling  (VeloxQuant "VecInfer": per-channel lambda_i = sqrt(max |K_i|) before the
+# Walsh-Hadamard rotation, inverse absorbed into the query)
+# --------------------------------------------------------------------------------------------
+
+def smooth_factors(K: np.ndarray) -> np.ndarray:
+    """lambda_i = sqrt(max_t |K[t, i]|) over calibration keys K [n][d] of one kv head, as
+    float32; 1 for a channel that is zero on every token."""
+    m = np.abs(np.asarray(K, F64)).max(axis=0)
+    lam = np.sqrt(m)
+    return np.where(m > 0, lam, 1.0).astype(F32)
+
+
+def smooth_keys(x: np.ndarray, lam: np.ndarray) -> np.ndarray:
+    """x / lambda per channel: float64(x) times the float64 reciprocal of the float32 factor."""
+    inv = F64(1.0) / np.asarray(lam, F32).astype(F64)
+    return np.asarray(x, F64) * inv
+
+
+# --------------------------------------------------------------------------------------------
 # Greedy residual vector quantisation  (VQKV section 2.1, "Process" and "Reconstruction")
 # --------------------------------------------------------------------------------------------
 
@@ -94,15 +117,18 @@ def stage_distances(r: np.ndarray, C: np.ndarray, chunk: int = 256) -> np.ndarra
     return D
 
 
-def rvq_encode(x: np.ndarray, codebooks: np.ndarray, rotate: bool = True):
+def rvq_encode(x: np.ndarray, codebooks: np.ndarray, rotate: bool = True, smooth=None):
     """Greedy RVQ of rows of x against stage codebooks [S][K][d] (float32, rotated domain).
 
-    Step 1: y = rotate(x) (or x as float32 when ``rotate`` is False).
+    Step 1: y = rotate(x) (or x as float32 when ``rotate`` is False); with ``smooth`` (the
+    head's lambda [d]) the rows are first divided by lambda channel by channel.
     For each stage s: z_s = argmin_c ||r - C_s[c]||^2 (lowest index on ties),
     r <- r - C_s[z_s] (float32), n_s = ||r||.
     Returns (codes uint8 [n][S], norms float32 [n][S], y float32 [n][d], r_final float32).
     """
     x = np.asarray(x)
+    if smooth is not None:
+        x = smooth_keys(x, smooth)
     y = rotate_to_f32(x) if rotate else np.asarray(x, F32)
     S = codebooks.shape[0]
     n = y.shape[0]
@@ -120,7 +146,7 @@ def rvq_encode(x: np.ndarray, codebooks: np.ndarray, rotate: bool = True):
 
 
 def rvq_match_walk(x: np.ndarray, codebooks: np.ndarray, codes: np.ndarray,
-                   rel_gap: float = 1e-5, rotate: bool = True) -> dict:
+                   rel_gap: float = 1e-5, rotate: bool = True, smooth=None) -> dict:
     """Check candidate codes against the greedy rule, stage by stage.
 
     At each stage the oracle's float64 distances of the current residual are computed.  A
@@ -129,8 +155,11 @@ def rvq_match_walk(x: np.ndarray, codebooks: np.ndarray, codes: np.ndarray,
     Anything else is a mismatch.  The walk continues along the candidate's codes, so one
     near-tie does not cascade into later stages.
     Returns counts and the first few mismatches (row, stage, candidate, oracle, rel gap).
+    ``smooth``: as in rvq_encode.
     """
     x = np.asarray(x)
+    if smooth is not None:
+        x = smooth_keys(x, smooth)
     y = rotate_to_f32(x) if rotate else np.asarray(x, F32)
     S = codebooks.shape[0]
     r = y.copy()
@@ -241,7 +270,7 @@ def _check_decode_shapes(q, k_codes, v_codes, Ck, Cv, win_k, win_v):
 
 
 def decode_attn(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len,
-                scale: float | None = None, pairs=None):
+                scale: float | None = None, pairs=None, k_smooth=None):
     """Decode-step attention over a compressed prefix plus an fp16 window (direct form).
 
     q [B][Hq][d] fp16; k_codes [B][Hkv][Tcap][Sk] / v_codes [B][Hkv][Tcap][Sv] uint8;
@@ -250,7 +279,9 @@ def decode_attn(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len,
 
     For every (b, h): the compressed keys and values are reconstructed and rotated back,
     k_t = (1/sqrt(d)) H sum_s Ck_s[zk_{t,s}] (likewise v), joined with the window tokens, and
-    exact softmax attention of q over that set is taken in float64.
+    exact softmax attention of q over that set is taken in float64.  With ``k_smooth``
+    ([Hkv][d] lambda) the compressed keys were smoothed before encoding, so the reconstructed
+    key is lambda * k_t (the window keys are raw).
     Returns (out float64 [B][Hq][d], lse float64 [B][Hq]); ``pairs`` restricts to a list of
     (b, h) (other entries are NaN).
     """
@@ -269,6 +300,8 @@ def decode_attn(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len,
             tc = int(comp_len[b])
             wl = int(win_len[b])
             kh = reconstruct(k_codes[b, kvh, :tc], Ck[kvh], unrotate=True)
+            if k_smooth is not None:
+                kh = kh * np.asarray(k_smooth[kvh], F32).astype(F64)
             vh = reconstruct(v_codes[b, kvh, :tc], Cv[kvh], unrotate=True)
             Kall = np.concatenate([kh, np.asarray(win_k[b, kvh, :wl], F64)], axis=0)
             Vall = np.concatenate([vh, np.asarray(win_v[b, kvh, :wl], F64)], axis=0)
@@ -281,7 +314,7 @@ def decode_attn(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len,
 
 
 def decode_attn_lut(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len,
-                    scale: float | None = None, pairs=None):
+                    scale: float | None = None, pairs=None, k_smooth=None):
     """The same attention computed the way the method reads codes (second, independent path).
 
     Compressed part, in the rotated domain: q_tilde = (1/sqrt(d)) H q;
@@ -289,7 +322,8 @@ def decode_attn_lut(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len
     o_tilde = sum_t softmax(score)_t sum_s Cv_s[zv_{t,s}], rotated back by (1/sqrt(d)) H.
     Window part: plain attention of q over the fp16 window.  The two parts are joined by the
     log-sum-exp combine.  Equality with ``decode_attn`` pins the rotation absorption
-    (q_tilde . k_tilde = q . k) and the combine.
+    (q_tilde . k_tilde = q . k) and the combine.  With ``k_smooth`` the query of the
+    compressed part is q_tilde = (1/sqrt(d)) H (lambda * q).
     """
     B, Hq, Hkv, d = _check_decode_shapes(q, k_codes, v_codes, Ck, Cv, win_k, win_v)
     G = Hq // Hkv
@@ -303,7 +337,10 @@ def decode_attn_lut(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len
         kvh = h // G
         tc = int(comp_len[b])
         wl = int(win_len[b])
-        qt = fwht(np.asarray(q[b, h], F64), 1.0 / np.sqrt(F64(d)))
+        qs = np.asarray(q[b, h], F64)
+        if k_smooth is not None:
+            qs = qs * np.asarray(k_smooth[kvh], F32).astype(F64)
+        qt = fwht(qs, 1.0 / np.sqrt(F64(d)))
         parts = []
         if tc > 0:
             zk = k_codes[b, kvh, :tc].astype(np.int64)
@@ -340,7 +377,8 @@ def append_step(state: dict, new_k: np.ndarray, new_v: np.ndarray) -> dict:
 
     state: k_codes, v_codes [B][Hkv][Tcap][S] uint8; comp_len [B]; win_k, win_v
     [B][Hkv][Wcap][d] fp16; win_len [B]; win_head [B] (slot of the oldest token once the window
-    is full); Ck, Cv codebooks.  new_k / new_v: [B][Hkv][d] fp16.
+    is full); Ck, Cv codebooks; optional k_smooth [Hkv][d] (evicted keys are smoothed before
+    encoding).  new_k / new_v: [B][Hkv][d] fp16.
     While win_len < Wcap the token goes to slot win_len.  Otherwise slot win_head is evicted
     (its key and value are encoded to position comp_len), overwritten, and win_head advances.
     If an eviction is due while comp_len == Tcap, that sequence is left unchanged and the
@@ -363,7 +401,9 @@ def append_step(state: dict, new_k: np.ndarray, new_v: np.ndarray) -> dict:
                 st["error"] = True
                 continue
             for h in range(Hkv):
-                zk, _, _, _ = rvq_encode(st["win_k"][b, h, slot][None], st["Ck"][h])
+                ks = st.get("k_smooth")
+                zk, _, _, _ = rvq_encode(st["win_k"][b, h, slot][None], st["Ck"][h],
+                                         smooth=None if ks is None else ks[h])
                 zv, _, _, _ = rvq_encode(st["win_v"][b, h, slot][None], st["Cv"][h])
                 st["k_codes"][b, h, pos] = zk[0]
                 st["v_codes"][b, h, pos] = zv[0]

@@ -424,3 +424,75 @@ def test_append_step_at_capacity_leaves_sequence_unchanged():
     assert out["error"]
     for k in ("k_codes", "v_codes", "comp_len", "win_k", "win_v", "win_len", "win_head"):
         np.testing.assert_array_equal(out[k], st[k])
+
+
+# ------------------------------------------------------------------ smooth scaling (VecInfer)
+
+def test_smooth_factors_hand_example():
+    # lambda_i = sqrt(max_t |K[t, i]|); an all-zero channel gets 1
+    K = np.array([[1.0, -4.0, 0.0, 0.25], [-2.0, 3.0, 0.0, -0.0625]])
+    lam = O.smooth_factors(K)
+    assert lam.dtype == np.float32
+    np.testing.assert_array_equal(lam, np.array([math.sqrt(2.0), 2.0, 1.0, 0.5], np.float32))
+
+
+def test_smoothing_flattens_channel_ranges():
+    # after division by lambda every nonzero channel's largest magnitude is sqrt(max |K_i|)
+    rng = np.random.default_rng(40)
+    K = rng.standard_normal((300, 16)) * np.exp(rng.standard_normal(16) * 2)
+    lam = O.smooth_factors(K).astype(np.float64)
+    peak = np.abs(O.smooth_keys(K, lam)).max(axis=0)
+    np.testing.assert_allclose(peak, np.sqrt(np.abs(K).max(axis=0)), rtol=1e-6)
+
+
+def test_smooth_ones_changes_nothing():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((20, 32)).astype(np.float16)
+    C = (rng.standard_normal((3, 16, 32)) * 0.5).astype(np.float32)
+    a = O.rvq_encode(x, C)
+    b = O.rvq_encode(x, C, smooth=np.ones(32, np.float32))
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+    case = _rand_decode_case(rng, comp=[40, 11], win=[8, 2])
+    o1, l1 = O.decode_attn(*case)
+    o2, l2 = O.decode_attn(*case, k_smooth=np.ones((2, 64), np.float32))
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_smoothed_direct_equals_lut_form():
+    # the query absorbs lambda exactly: (lambda q) . (H k~ / sqrt d) == q . (lambda H k~ / sqrt d)
+    rng = np.random.default_rng(42)
+    case = _rand_decode_case(rng, comp=[40, 23], win=[8, 0])
+    lam = np.exp(rng.standard_normal((2, 64)) * 0.7).astype(np.float32)
+    o1, l1 = O.decode_attn(*case, k_smooth=lam)
+    o2, l2 = O.decode_attn_lut(*case, k_smooth=lam)
+    np.testing.assert_allclose(o2, o1, atol=1e-9, rtol=0)
+    np.testing.assert_allclose(l2, l1, atol=1e-9, rtol=0)
+    o0, _ = O.decode_attn(*case)
+    assert np.max(np.abs(o0 - o1)) > 1e-3     # lambda really changes the keys
+
+
+def test_smoothed_encode_decode_recovers_the_original_scores():
+    # Codebooks that hold the smoothed, rotated keys exactly (one stage): the decoded scores
+    # are q . k of the ORIGINAL keys (to float32 rounding), which fixes the direction of lambda
+    rng = np.random.default_rng(43)
+    d, n = 64, 5
+    keys = (rng.standard_normal((n, d)) * np.exp(rng.standard_normal(d))).astype(np.float16)
+    lam = O.smooth_factors(keys)
+    y = O.rotate_to_f32(O.smooth_keys(keys, lam))
+    Ck = np.zeros((1, 1, 16, d), np.float32)
+    Ck[0, 0, 1:1 + n] = y
+    codes, _, _, _ = O.rvq_encode(keys, Ck[0], smooth=lam)
+    np.testing.assert_array_equal(codes[:, 0], np.arange(1, 1 + n))
+    q = rng.standard_normal((1, 1, d)).astype(np.float16)
+    kc = np.zeros((1, 1, 16, 1), np.uint8)
+    kc[0, 0, :n, 0] = codes[:, 0]
+    vc = np.zeros((1, 1, 16, 1), np.uint8)
+    Cv = np.zeros((1, 1, 16, d), np.float32)
+    wk = np.zeros((1, 1, 1, d), np.float16)
+    _, lse = O.decode_attn(q, kc, vc, [n], Ck, Cv, wk, wk, [0], k_smooth=lam[None])
+    sc = keys.astype(np.float64) @ q[0, 0].astype(np.float64) / math.sqrt(d)
+    assert abs(lse[0, 0] - scipy.special.logsumexp(sc)) < 1e-4
+    _, lse_wrong = O.decode_attn(q, kc, vc, [n], Ck, Cv, wk, wk, [0])
+    assert abs(lse_wrong[0, 0] - scipy.special.logsumexp(sc)) > 1e-2
