@@ -96,6 +96,11 @@ __global__ void __cluster_dims__(kAppendCl, 1, 1) __launch_bounds__(256)
     if (row_valid(j)) {
       double v[E];
       load_row_f64<E>(win, ZKV_DTYPE_F16, ((j * p.Hkv + h) * p.Wcap + p.win_head[j]) * D, lane, v);
+      if (kind == 0 && p.k_smooth) {   // keys: x / lambda per channel before the rotation
+        const float* l = p.k_smooth + (int64_t)h * D;
+#pragma unroll
+        for (int q = 0; q < E; ++q) v[q] *= 1.0 / (double)l[q * 32 + lane];
+      }
       fwht_warp_f64<D>(v, lane);
 #pragma unroll
       for (int q = 0; q < E; ++q) {

@@ -161,6 +161,7 @@ struct DecodeArgs {
   const uint8_t* v_codes;
   const int32_t* comp_len;
   const float* Ck;
+  const float* k_smooth;   // [Hkv][d] key smoothing factors (the query is scaled by them) or null
   const float* Cv;
   const __half* win_k;
   const __half* win_v;
@@ -547,6 +548,11 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
         const __half* qr = a.q + ((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D + lane;
 #pragma unroll
         for (int q = 0; q < E; ++q) v[k][q] = __half2float(qr[q * 32]);
+        if (a.k_smooth) {   // the query absorbs the keys' smoothing: lambda * q
+          const float* l = a.k_smooth + (int64_t)kvh * D + lane;
+#pragma unroll
+          for (int q = 0; q < E; ++q) v[k][q] *= l[q * 32];
+        }
       } else {
 #pragma unroll
         for (int q = 0; q < E; ++q) v[k][q] = 0.f;
@@ -1518,7 +1524,7 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   a.rot = 1.0 / std::sqrt((double)p->d);
   a.q = reinterpret_cast<const __half*>(p->q);
   a.k_codes = p->k_codes; a.v_codes = p->v_codes; a.comp_len = p->comp_len;
-  a.Ck = p->k_codebooks; a.Cv = p->v_codebooks;
+  a.Ck = p->k_codebooks; a.Cv = p->v_codebooks; a.k_smooth = p->k_smooth;
   a.win_k = reinterpret_cast<const __half*>(p->win_k);
   a.win_v = reinterpret_cast<const __half*>(p->win_v);
   a.win_len = p->win_len; a.out = p->out; a.lse = p->lse; a.err = p->error_flag;
@@ -1563,7 +1569,7 @@ extern "C" int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_
   if (ap->k_codes != dp->k_codes || ap->v_codes != dp->v_codes ||
       ap->k_codebooks != dp->k_codebooks || ap->v_codebooks != dp->v_codebooks ||
       ap->win_k != dp->win_k || ap->win_v != dp->win_v || ap->win_len != dp->win_len ||
-      ap->comp_len != dp->comp_len)
+      ap->comp_len != dp->comp_len || ap->k_smooth != dp->k_smooth)
     return ZKV_ERR_INVALID_ARG;
   return decode_common(dp, workspace, workspace_bytes, stream, ap);
 }

@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(256, 2) encode_tile_kernel(StridedRows map,
     if (map.valid(j, h)) {
       double v[E];
       load_row_f64<E>(map.src(), map.dtype(), map.x_off(j, h), lane, v);
+      map.apply_smooth<E>(v, h, lane);
       if (map.do_rotate()) {
         fwht_warp_f64<D>(v, lane);
 #pragma unroll
@@ -355,6 +356,7 @@ extern "C" int zkv_rvq_encode(const zkv_encode_params* p, void* stream) {
   m.n_sb = p->n_sb;
   m.n_st = p->n_st;
   m.n_sh = p->n_sh;
+  m.smooth = p->smooth;
   return launch_encode(m, p->n_head, p->d, p->S, p->codebooks, p->error_flag,
                        reinterpret_cast<cudaStream_t>(stream));
 }

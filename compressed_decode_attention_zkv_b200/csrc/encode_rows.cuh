@@ -20,8 +20,17 @@ struct StridedRows {
   int64_t c_sb, c_st, c_sh;
   float* norms;
   int64_t n_sb, n_st, n_sh;
+  const float* smooth;    // [n_head][d] key smoothing factors or null
 
   __device__ bool valid(int64_t j, int) const { return j < n_rows; }
+  // x / lambda per channel (before the rotation): float64 times the float64 reciprocal
+  template <int E>
+  __device__ void apply_smooth(double (&v)[E], int h, int lane) const {
+    if (!smooth) return;
+    const float* l = smooth + (int64_t)h * (E * 32);
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[q] *= 1.0 / (double)l[q * 32 + lane];
+  }
   __device__ const void* src() const { return x; }
   __device__ int dtype() const { return x_dtype; }
   __device__ bool do_rotate() const { return rotate != 0; }
@@ -97,6 +106,7 @@ __device__ __forceinline__ void encode_rows_body(const Map& map, const float* __
     if (map.valid(j, h)) {
       double v[E];
       load_row_f64<E>(map.src(), map.dtype(), map.x_off(j, h), lane, v);
+      map.apply_smooth<E>(v, h, lane);
       if (map.do_rotate()) {
         fwht_warp_f64<D>(v, lane);
 #pragma unroll

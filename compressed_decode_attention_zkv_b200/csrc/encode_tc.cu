@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(StridedRows ma
       ok[u] = map.valid(j, h);
       if (ok[u]) {
         load_row_f64<E>(map.src(), map.dtype(), map.x_off(j, h), lane, v[u]);
+        map.apply_smooth<E>(v[u], h, lane);
       } else {
 #pragma unroll
         for (int q = 0; q < E; ++q) v[u][q] = 0.0;

@@ -46,7 +46,7 @@ class EncodeParams(ctypes.Structure):
                 ("codebooks", c_void_p),
                 ("codes", c_void_p), ("c_sb", c_int64), ("c_st", c_int64), ("c_sh", c_int64),
                 ("norms", c_void_p), ("n_sb", c_int64), ("n_st", c_int64), ("n_sh", c_int64),
-                ("error_flag", c_void_p)]
+                ("error_flag", c_void_p), ("smooth", c_void_p)]
 
 
 class ReconstructParams(ctypes.Structure):
@@ -65,7 +65,7 @@ class DecodeParams(ctypes.Structure):
                 ("comp_len", c_void_p), ("k_codebooks", c_void_p), ("v_codebooks", c_void_p),
                 ("win_k", c_void_p), ("win_v", c_void_p), ("win_len", c_void_p),
                 ("out", c_void_p), ("lse", c_void_p), ("error_flag", c_void_p),
-                ("trace_events", c_void_p)]
+                ("trace_events", c_void_p), ("k_smooth", c_void_p)]
 
 
 class AppendParams(ctypes.Structure):
@@ -74,7 +74,8 @@ class AppendParams(ctypes.Structure):
                 ("new_k", c_void_p), ("new_v", c_void_p), ("win_k", c_void_p),
                 ("win_v", c_void_p), ("win_len", c_void_p), ("win_head", c_void_p),
                 ("comp_len", c_void_p), ("k_codes", c_void_p), ("v_codes", c_void_p),
-                ("k_codebooks", c_void_p), ("v_codebooks", c_void_p), ("error_flag", c_void_p)]
+                ("k_codebooks", c_void_p), ("v_codebooks", c_void_p), ("error_flag", c_void_p),
+                ("k_smooth", c_void_p)]
 
 
 _lib = None
@@ -129,6 +130,16 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
+def _smooth_ptr(lam, heads: int, d: int, name: str) -> int | None:
+    """Pointer of a float32 [heads, d] contiguous CUDA tensor of smoothing factors (or None)."""
+    if lam is None:
+        return None
+    _need(lam, name, torch.float32)
+    if tuple(lam.shape) != (heads, d):
+        raise ValueError(f"{name} must be [{heads}, {d}], got {tuple(lam.shape)}")
+    return _ptr(lam)
+
+
 def _need(t: torch.Tensor, name: str, dtype, contiguous=True):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -171,10 +182,12 @@ def _as4(t: torch.Tensor, name: str) -> torch.Tensor:
 
 def rvq_encode(x: torch.Tensor, codebooks: torch.Tensor, codes: torch.Tensor | None = None,
                norms: torch.Tensor | None = None, rotate: bool = True,
-               with_norms: bool = True, error_flag: torch.Tensor | None = None):
+               with_norms: bool = True, error_flag: torch.Tensor | None = None,
+               smooth: torch.Tensor | None = None):
     """Greedy RVQ of x rows.  x: [B, T, H, d] view (any strides, d contiguous), or [T, H, d],
     or [N, d] (one head).  codebooks: [H, S, 256, d] float32 contiguous.  error_flag: optional
-    int32 device word that receives ZKV_DEVERR_TIMEOUT.
+    int32 device word that receives ZKV_DEVERR_TIMEOUT.  smooth: optional float32 [H, d] key
+    smoothing factors (rows are divided by them before the rotation).
     Returns (codes uint8 [B, T, H, S] view, norms float32 [B, T, H, S] or None)."""
     if x.dtype not in (torch.float16, torch.float32):
         raise TypeError("x must be fp16 or fp32")
@@ -209,6 +222,7 @@ def rvq_encode(x: torch.Tensor, codebooks: torch.Tensor, codes: torch.Tensor | N
     if error_flag is not None:
         _need(error_flag, "error_flag", torch.int32)
         p.error_flag = _ptr(error_flag)
+    p.smooth = _smooth_ptr(smooth, H, d, "smooth")
     _check("zkv_rvq_encode", lib().zkv_rvq_encode(ctypes.byref(p), _stream()))
     return codes, norms
 
@@ -237,7 +251,8 @@ def rvq_reconstruct(codes: torch.Tensor, codebooks: torch.Tensor, unrotate: bool
 
 
 def _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
-                   win_len, out, lse, max_comp_len, softmax_scale, error_flag) -> DecodeParams:
+                   win_len, out, lse, max_comp_len, softmax_scale, error_flag,
+                   k_smooth=None) -> DecodeParams:
     _need(q, "q", torch.float16)
     _need(k_codes, "k_codes", torch.uint8)
     _need(v_codes, "v_codes", torch.uint8)
@@ -264,7 +279,8 @@ def _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_
                         comp_len=_ptr(comp_len), k_codebooks=_ptr(k_codebooks),
                         v_codebooks=_ptr(v_codebooks), win_k=_ptr(win_k), win_v=_ptr(win_v),
                         win_len=_ptr(win_len), out=_ptr(out), lse=_ptr(lse),
-                        error_flag=_ptr(error_flag))
+                        error_flag=_ptr(error_flag),
+                        k_smooth=_smooth_ptr(k_smooth, Hkv, d, "k_smooth"))
 
 
 def decode_workspace_size(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
@@ -279,10 +295,12 @@ def decode_workspace_size(q, k_codes, v_codes, comp_len, k_codebooks, v_codebook
 
 def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
                     win_len, out=None, lse=None, max_comp_len=None, softmax_scale=None,
-                    workspace: torch.Tensor | None = None, error_flag=None, trace_events=None):
+                    workspace: torch.Tensor | None = None, error_flag=None, trace_events=None,
+                    k_smooth=None):
     """Decode attention over the compressed prefix plus the fp16 window (see include/zkv.h).
     ``trace_events``: optional 4 torch.cuda.Event(enable_timing=True) recorded before the
-    table, scan and merge stages and after the last kernel.
+    table, scan and merge stages and after the last kernel.  ``k_smooth``: the [Hkv, d] key
+    smoothing factors the prefix was encoded with.
     Returns (out float32 [B, Hq, d], lse float32 [B, Hq])."""
     B, Hq, d = q.shape
     if out is None:
@@ -290,7 +308,7 @@ def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
-                       win_len, out, lse, max_comp_len, softmax_scale, error_flag)
+                       win_len, out, lse, max_comp_len, softmax_scale, error_flag, k_smooth)
     ev_arr = None
     if trace_events is not None:
         if len(trace_events) != 4:
@@ -309,7 +327,7 @@ def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win
 
 def rvq_decode_attn_noalloc(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
                             win_v, win_len, out=None, lse=None, max_comp_len=None,
-                            softmax_scale=None, error_flag=None):
+                            softmax_scale=None, error_flag=None, k_smooth=None):
     """rvq_decode_attn with the library's fixed device scratch array as workspace
     (zkv_rvq_decode_attn_noalloc).  Calls on one device must not overlap in time.  Raises
     ZkvError(ZKV_ERR_WORKSPACE) when the shapes need more than DECODE_SCRATCH_BYTES."""
@@ -319,7 +337,7 @@ def rvq_decode_attn_noalloc(q, k_codes, v_codes, comp_len, k_codebooks, v_codebo
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
-                       win_len, out, lse, max_comp_len, softmax_scale, error_flag)
+                       win_len, out, lse, max_comp_len, softmax_scale, error_flag, k_smooth)
     status = lib().zkv_rvq_decode_attn_noalloc(ctypes.byref(p), _stream())
     if status == ZKV_ERR_WORKSPACE:
         need = lib().zkv_decode_workspace_size(ctypes.byref(p))
@@ -331,7 +349,7 @@ def rvq_decode_attn_noalloc(q, k_codes, v_codes, comp_len, k_codebooks, v_codebo
 
 
 def _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
-                   k_codebooks, v_codebooks, error_flag):
+                   k_codebooks, v_codebooks, error_flag, k_smooth=None):
     _need(new_k, "new_k", torch.float16)
     _need(new_v, "new_v", torch.float16)
     for n, t in (("win_k", win_k), ("win_v", win_v)):
@@ -350,14 +368,15 @@ def _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_co
                         win_k=_ptr(win_k), win_v=_ptr(win_v), win_len=_ptr(win_len),
                         win_head=_ptr(win_head), comp_len=_ptr(comp_len), k_codes=_ptr(k_codes),
                         v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
-                        v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag))
+                        v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag),
+                        k_smooth=_smooth_ptr(k_smooth, Hkv, new_k.shape[-1], "k_smooth"))
 
 
 def rvq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
-               k_codebooks, v_codebooks, error_flag=None):
+               k_codebooks, v_codebooks, error_flag=None, k_smooth=None):
     """One serving step of cache maintenance (see include/zkv.h); state updated in place."""
     p = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
-                       v_codes, k_codebooks, v_codebooks, error_flag)
+                       v_codes, k_codebooks, v_codebooks, error_flag, k_smooth)
     _check("zkv_rvq_append", lib().zkv_rvq_append(ctypes.byref(p), _stream()))
 
 
@@ -367,11 +386,11 @@ class PreparedAppend:
     step on the current stream with no per-call Python work beyond the library call."""
 
     def __init__(self, new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
-                 v_codes, k_codebooks, v_codebooks, error_flag=None):
+                 v_codes, k_codebooks, v_codebooks, error_flag=None, k_smooth=None):
         self._keep = (new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
-                      k_codebooks, v_codebooks, error_flag)
+                      k_codebooks, v_codebooks, error_flag, k_smooth)
         self._p = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len,
-                                 k_codes, v_codes, k_codebooks, v_codebooks, error_flag)
+                                 k_codes, v_codes, k_codebooks, v_codebooks, error_flag, k_smooth)
         self._ref = ctypes.byref(self._p)
         self._fn = lib().zkv_rvq_append
 
@@ -391,17 +410,18 @@ class PreparedServeStep:
     def __init__(self, new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes,
                  v_codes, k_codebooks, v_codebooks, out=None, lse=None, max_comp_len=None,
                  softmax_scale=None, workspace: torch.Tensor | None = None, error_flag=None,
-                 trace_events=None):
+                 trace_events=None, k_smooth=None):
         B, Hq, d = q.shape
         if out is None:
             out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
         if lse is None:
             lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
         self._pa = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len,
-                                  k_codes, v_codes, k_codebooks, v_codebooks, error_flag)
+                                  k_codes, v_codes, k_codebooks, v_codebooks, error_flag,
+                                  k_smooth)
         self._pd = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
                                   win_v, win_len, out, lse, max_comp_len, softmax_scale,
-                                  error_flag)
+                                  error_flag, k_smooth)
         self._ev = None
         if trace_events is not None:   # recorded before the tables, the scan, the merge, and last
             if len(trace_events) != 4:
@@ -419,7 +439,7 @@ class PreparedServeStep:
                            f"workspace holds {workspace.numel()} bytes, {need} needed")
         self.out, self.lse = out, lse
         self._keep = (new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes,
-                      v_codes, k_codebooks, v_codebooks, workspace, error_flag)
+                      v_codes, k_codebooks, v_codebooks, workspace, error_flag, k_smooth)
         self._refa, self._refd = ctypes.byref(self._pa), ctypes.byref(self._pd)
         self._ws = ctypes.c_void_p(workspace.data_ptr())
         self._wsn = ctypes.c_size_t(workspace.numel())
@@ -435,14 +455,15 @@ class PreparedServeStep:
 
 def rvq_serve_step(new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
                    k_codebooks, v_codebooks, out=None, lse=None, max_comp_len=None,
-                   softmax_scale=None, workspace=None, error_flag=None, trace_events=None):
+                   softmax_scale=None, workspace=None, error_flag=None, trace_events=None,
+                   k_smooth=None):
     """rvq_append(new_k, new_v, ...) then rvq_decode_attn(q, ...) on the updated cache, in one
     library call (see include/zkv.h).  Returns (out, lse)."""
     if max_comp_len is None:
         max_comp_len = k_codes.shape[2]
     return PreparedServeStep(new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len,
                              k_codes, v_codes, k_codebooks, v_codebooks, out, lse, max_comp_len,
-                             softmax_scale, workspace, error_flag, trace_events)()
+                             softmax_scale, workspace, error_flag, trace_events, k_smooth)()
 
 
 class PreparedDecode:
@@ -453,7 +474,7 @@ class PreparedDecode:
 
     def __init__(self, q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
                  win_len, out=None, lse=None, max_comp_len=None, softmax_scale=None,
-                 workspace: torch.Tensor | None = None, error_flag=None):
+                 workspace: torch.Tensor | None = None, error_flag=None, k_smooth=None):
         B, Hq, d = q.shape
         if out is None:
             out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
@@ -461,7 +482,7 @@ class PreparedDecode:
             lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
         self._p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
                                  win_v, win_len, out, lse, max_comp_len, softmax_scale,
-                                 error_flag)
+                                 error_flag, k_smooth)
         need = lib().zkv_decode_workspace_size(ctypes.byref(self._p))
         if need == 0:
             raise ZkvError("zkv_decode_workspace_size", ZKV_ERR_INVALID_ARG)
@@ -473,7 +494,7 @@ class PreparedDecode:
                            f"workspace holds {workspace.numel()} bytes, {need} needed")
         self.out, self.lse = out, lse
         self._keep = (q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
-                      win_len, workspace, error_flag)
+                      win_len, workspace, error_flag, k_smooth)
         self._ref = ctypes.byref(self._p)
         self._ws = ctypes.c_void_p(workspace.data_ptr())
         self._wsn = ctypes.c_size_t(workspace.numel())
@@ -494,13 +515,16 @@ class RVQKVCache:
     """Compressed KV cache of one attention layer: RVQ codes for old tokens, an fp16 window for
     the newest ones.  prefill() encodes a prompt, append() inserts one token per sequence
     (evicting and encoding the oldest window token when the window is full), attend() runs one
-    decode step of attention.  All state lives on the GPU; lengths never leave the device."""
+    decode step of attention.  All state lives on the GPU; lengths never leave the device.
+    k_smooth: optional float32 [Hkv, d] key smoothing factors (the key codebooks must have been
+    trained on smoothed keys)."""
 
     def __init__(self, k_codebooks: torch.Tensor, v_codebooks: torch.Tensor, batch: int,
-                 capacity: int, window: int, device="cuda"):
+                 capacity: int, window: int, device="cuda", k_smooth: torch.Tensor | None = None):
         Hkv, Sk, _, d = k_codebooks.shape
         Sv = v_codebooks.shape[1]
         self.Ck, self.Cv = k_codebooks.contiguous(), v_codebooks.contiguous()
+        self.k_smooth = None if k_smooth is None else k_smooth.contiguous()
         self.B, self.Hkv, self.d, self.Sk, self.Sv = batch, Hkv, d, Sk, Sv
         self.Tcap = (capacity + 15) // 16 * 16
         self.Wcap = window
@@ -526,7 +550,8 @@ class RVQKVCache:
             raise ValueError("prompt longer than capacity + window")
         if Tc > 0:
             rvq_encode(k[:, :, :Tc].permute(0, 2, 1, 3), self.Ck,
-                       codes=self.k_codes[:, :, :Tc].permute(0, 2, 1, 3), with_norms=False)
+                       codes=self.k_codes[:, :, :Tc].permute(0, 2, 1, 3), with_norms=False,
+                       smooth=self.k_smooth)
             rvq_encode(v[:, :, :Tc].permute(0, 2, 1, 3), self.Cv,
                        codes=self.v_codes[:, :, :Tc].permute(0, 2, 1, 3), with_norms=False)
         self.win_k[:, :, :W].copy_(k[:, :, Tc:])
@@ -540,7 +565,7 @@ class RVQKVCache:
         """k_new, v_new: fp16 [B, Hkv, d]."""
         rvq_append(k_new.contiguous(), v_new.contiguous(), self.win_k, self.win_v, self.win_len,
                    self.win_head, self.comp_len, self.k_codes, self.v_codes, self.Ck, self.Cv,
-                   self.error_flag)
+                   self.error_flag, self.k_smooth)
         self.max_comp_len = min(self.max_comp_len + 1, self.Tcap)
 
     def attend(self, q: torch.Tensor, softmax_scale=None, out=None, lse=None):
@@ -552,7 +577,7 @@ class RVQKVCache:
             self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
         return rvq_decode_attn(*args, out=out, lse=lse, max_comp_len=self.max_comp_len,
                                softmax_scale=softmax_scale, workspace=self._ws,
-                               error_flag=self.error_flag)
+                               error_flag=self.error_flag, k_smooth=self.k_smooth)
 
     def memory_bytes(self) -> int:
         """Bytes held by codes and window (codebooks are shared across layers' caches)."""

@@ -100,6 +100,10 @@ int zkv_fwht(const void* in, int in_dtype, float* out, int64_t n_vec, int d, flo
  *   codebooks float32 [n_head][S][256][d]
  * Alignment: x rows 16-byte aligned (x base and strides multiples of 8 fp16 / 4 fp32 elements).
  * error_flag: optional device int32 that receives ZKV_DEVERR_TIMEOUT (see the conventions above).
+ * smooth: optional float32 [n_head][d] per-channel key smoothing factors lambda (VeloxQuant
+ *   "VecInfer": lambda_i = sqrt(max |K_i|) calibrated offline): each row is multiplied by
+ *   1/lambda (float64 reciprocal, float64 product) before the rotation.  NULL: no smoothing.
+ *   Decode must then be given the same factors (zkv_decode_params.k_smooth).
  * Errors: INVALID_ARG, UNSUPPORTED (d, S), CUDA.
  */
 typedef struct {
@@ -115,6 +119,7 @@ typedef struct {
   float* norms;
   int64_t n_sb, n_st, n_sh;
   int32_t* error_flag;
+  const float* smooth;
 } zkv_encode_params;
 
 int zkv_rvq_encode(const zkv_encode_params* p, void* stream);
@@ -193,6 +198,11 @@ typedef struct {
    * the lookup-table kernel, before the scan kernel, before the two merge kernels and after
    * them. */
   void* const* trace_events;
+  /* Optional float32 [Hkv][d]: the per-channel smoothing factors the compressed keys were
+   * encoded with (zkv_encode_params.smooth).  The query is multiplied by them before its
+   * rotation, so q_tilde . k_tilde = q . k (VeloxQuant "VecInfer").  The window keys are raw.
+   * NULL: no smoothing. */
+  const float* k_smooth;
 } zkv_decode_params;
 
 /* Workspace bytes for a call with these shapes (data pointers are not read); 0 if the shapes
@@ -255,6 +265,7 @@ typedef struct {
   const float* k_codebooks;
   const float* v_codebooks;
   int32_t* error_flag;
+  const float* k_smooth;   /* optional [Hkv][d]: evicted keys are smoothed as in zkv_rvq_encode */
 } zkv_append_params;
 
 int zkv_rvq_append(const zkv_append_params* p, void* stream);
@@ -269,7 +280,7 @@ int zkv_rvq_append(const zkv_append_params* p, void* stream);
  * partition of the token space (computed from the lengths the append will produce) with the
  * encode of the evicted tokens; the new lengths are stored by the decode's scan kernel.
  * ap and dp describe one cache: B, Hkv, d, Sk, Sv, Tcap and Wcap must be equal, and so must
- * k_codes, v_codes, k_codebooks, v_codebooks, win_k, win_v, win_len and comp_len (else
+ * k_codes, v_codes, k_codebooks, v_codebooks, win_k, win_v, win_len, comp_len and k_smooth (else
  * ZKV_ERR_INVALID_ARG).  dp->comp_len and dp->win_len are read after the update, so
  * dp->max_comp_len must allow for the new token.  workspace: as zkv_rvq_decode_attn
  * (zkv_decode_workspace_size(dp)); dp->trace_events: as zkv_rvq_decode_attn, where the first

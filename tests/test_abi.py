@@ -132,6 +132,7 @@ def _append_params(**kw):
     (dict(B=3), {}, zkv.ZKV_ERR_INVALID_ARG),
     (dict(Sv=3), {}, zkv.ZKV_ERR_INVALID_ARG),
     (dict(new_k=0), {}, zkv.ZKV_ERR_INVALID_ARG),             # the append itself is invalid
+    (dict(k_smooth=0xe000), {}, zkv.ZKV_ERR_INVALID_ARG),     # different smoothing factors
     (dict(d=96), dict(d=96), zkv.ZKV_ERR_UNSUPPORTED),
     ({}, dict(Hq=6, Hkv=4), zkv.ZKV_ERR_INVALID_ARG),          # the decode itself is invalid
     ({}, {}, zkv.ZKV_ERR_WORKSPACE),                           # consistent, but no workspace
