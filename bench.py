@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--replicas", type=int, default=8)
     ap.add_argument("--soak-s", type=float, default=1.0, help="extra warm-up time (clocks)")
     ap.add_argument("--no-encode", action="store_true", help="skip the bulk-encode extra")
+    ap.add_argument("--no-smooth", action="store_true",
+                    help="skip the serving step with key smoothing (extra)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -117,14 +119,18 @@ class ClockSampler:
 # Workload state on the GPU
 # --------------------------------------------------------------------------------------------
 
-def build_state(wl, R, Tcap_extra, dev):
-    """Encode the workload's prefixes on the GPU (prefill) and make R replicas."""
+def build_state(wl, R, Tcap_extra, dev, smooth=False):
+    """Encode the workload's prefixes on the GPU (prefill) and make R replicas.  smooth: key
+    smoothing factors calibrated on the calibration sample, key codebooks trained on smoothed
+    keys, prefixes encoded with them (each replica carries "k_smooth")."""
     import torch
 
     from compressed_decode_attention_zkv_b200 import inputs as I
     from compressed_decode_attention_zkv_b200 import zkv
 
-    Ck = torch.from_numpy(I.train_codebooks(wl, "k")).to(dev)
+    lam_np = I.key_smooth_factors(wl) if smooth else None
+    lam = None if lam_np is None else torch.from_numpy(lam_np).to(dev)
+    Ck = torch.from_numpy(I.train_codebooks(wl, "k", smooth=lam_np)).to(dev)
     Cv = torch.from_numpy(I.train_codebooks(wl, "v")).to(dev)
     Tc = wl.Tc
     Tcap = (Tc + Tcap_extra + 15) // 16 * 16
@@ -136,7 +142,8 @@ def build_state(wl, R, Tcap_extra, dev):
         for kind, codes, books, win in (("k", kc, Ck, wk), ("v", vc, Cv, wv)):
             x = torch.from_numpy(I.kv_tokens(wl, kind, b, 0, wl.T)).to(dev)   # [Hkv][T][d]
             zkv.rvq_encode(x[:, :Tc].permute(1, 0, 2)[None], books,
-                           codes=codes[b, :, :Tc].permute(1, 0, 2)[None], with_norms=False)
+                           codes=codes[b, :, :Tc].permute(1, 0, 2)[None], with_norms=False,
+                           smooth=lam if kind == "k" else None)
             win[b].copy_(x[:, Tc:])
             del x
     torch.cuda.synchronize()
@@ -153,14 +160,16 @@ def build_state(wl, R, Tcap_extra, dev):
             new_v=torch.from_numpy(I.new_tokens(wl, r, "v", np.full(wl.B, wl.T))).to(dev),
             out=torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32, device=dev),
             lse=torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev),
-            err=torch.zeros(1, dtype=torch.int32, device=dev)))
+            err=torch.zeros(1, dtype=torch.int32, device=dev),
+            k_smooth=None if lam is None else lam.clone()))
     del kc, vc, wk, wv
     return reps, Tcap
 
 
 def replica_bytes(rep):
     return sum(t.numel() * t.element_size() for k, t in rep.items()
-               if k in ("Ck", "Cv", "k_codes", "v_codes", "win_k", "win_v", "q"))
+               if k in ("Ck", "Cv", "k_codes", "v_codes", "win_k", "win_v", "q", "k_smooth")
+               and t is not None)
 
 
 def step_fn(rep, ws, max_comp, events=None):
@@ -171,7 +180,7 @@ def step_fn(rep, ws, max_comp, events=None):
                        rep["win_len"], rep["win_head"], rep["comp_len"], rep["k_codes"],
                        rep["v_codes"], rep["Ck"], rep["Cv"], out=rep["out"], lse=rep["lse"],
                        max_comp_len=max_comp, workspace=ws, error_flag=rep["err"],
-                       trace_events=events)
+                       trace_events=events, k_smooth=rep.get("k_smooth"))
 
 
 # --------------------------------------------------------------------------------------------
@@ -336,6 +345,58 @@ def encode_extra(dev, hbm, bf16):
             "frac": flops / sec / 1e12 / tf32_peak,
             "note": "tcgen05 kind::tf32 distance GEMM (M=128 rows, N=256 codewords) into TMEM; "
                     "exact decision: TF32-margin candidates re-scored in float32, then float64"}
+
+
+def smooth_extra(wl, args, dev, R, base_ms):
+    """The serving step with the VecInfer key smoothing (per-channel factors before the
+    rotation, absorbed into the query) on the same workload: its own replicas, codebooks
+    trained on smoothed keys, CUDA graphs, the same timing rules.  Returns the extra's dict."""
+    import torch
+
+    from compressed_decode_attention_zkv_b200 import zkv
+    steps = min(args.steps, 200)
+    per_rep = (R + 3 + steps + R - 1) // R + 2
+    reps, _ = build_state(wl, R, per_rep, dev, smooth=True)
+    max_comp = wl.Tc + per_rep
+    need = zkv.decode_workspace_size(reps[0]["q"], reps[0]["k_codes"], reps[0]["v_codes"],
+                                     reps[0]["comp_len"], reps[0]["Ck"], reps[0]["Cv"],
+                                     reps[0]["win_k"], reps[0]["win_v"], reps[0]["win_len"],
+                                     max_comp_len=max_comp)
+    wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
+    host_comp = [wl.Tc] * R
+    for r in range(R):   # eager call per replica (kernel attributes before capture)
+        step_fn(reps[r], wss[r], max_comp)
+        host_comp[r] += 1
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step_fn(reps[r], wss[r], max_comp)
+        graphs.append(g)
+    for i in range(3):
+        graphs[i % R].replay()
+        host_comp[i % R] += 1
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tokens = 0
+    s.record()
+    for i in range(steps):
+        r = (3 + i) % R
+        graphs[r].replay()
+        host_comp[r] += 1
+        tokens += wl.B * host_comp[r]
+    e.record()
+    torch.cuda.synchronize()
+    sec = s.elapsed_time(e) / 1000.0
+    assert sum(int(rep["err"].item()) for rep in reps) == 0
+    del graphs
+    return {"workload": f"{wl.name} with VecInfer key smoothing (lambda_i = sqrt(max|K_i|), "
+                        f"codebooks trained on smoothed keys)",
+            "value": tokens / sec, "unit": UNIT, "ms_per_step": 1000.0 * sec / steps,
+            "steps": steps, "vs_unsmoothed_step": base_ms / (1000.0 * sec / steps),
+            "note": "one zkv_rvq_serve_step per step with k_smooth; graphs over "
+                    f"{R} rotating replicas (inputs larger than L2)"}
 
 
 def run_ours(args):
@@ -570,6 +631,11 @@ def run_ours(args):
     if not args.no_encode and rank == 0:
         del graphs, soak_graphs
         extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
+    if not args.no_smooth and rank == 0:
+        reps.clear()
+        wss.clear()
+        torch.cuda.empty_cache()
+        extras["smooth"] = smooth_extra(wl, args, dev, R, 1000.0 * elapsed / args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
