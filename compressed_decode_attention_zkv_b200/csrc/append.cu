@@ -282,8 +282,18 @@ __global__ void __cluster_dims__(kAppendCl, 1, 1) __launch_bounds__(256)
   if (tid < kAppendR) {
     const int64_t j = row0 + tid;
     if (row_valid(j)) {
-      uint8_t* c = codes + ((j * p.Hkv + h) * p.Tcap + p.comp_len[j]) * S;
-      for (int s = 0; s < S; ++s) c[s] = sm.code[tid][s];
+      const int64_t t = p.comp_len[j];
+      uint8_t* c = nullptr;
+      if (!p.block_table) {
+        c = codes + ((j * p.Hkv + h) * p.Tcap + t) * S;
+      } else {   // paged: row (h, t % P) of page block_table[j][t / P]
+        const int64_t P = p.page_tokens;
+        const int64_t pg = p.block_table[j * p.max_pages + t / P];
+        if (pg >= 0 && pg < p.n_pages) c = codes + ((pg * p.Hkv + h) * P + t % P) * S;
+        else set_error(p.error_flag, ZKV_DEVERR_PAGE);
+      }
+      if (c)
+        for (int s = 0; s < S; ++s) c[s] = sm.code[tid][s];
     }
   }
   // every CTA read the evicted slots before its first cluster barrier
@@ -327,7 +337,7 @@ int validate_append(const zkv_append_params* p) {
   const uintptr_t al = (uintptr_t)p->win_k | (uintptr_t)p->win_v | (uintptr_t)p->k_codebooks |
                        (uintptr_t)p->v_codebooks;
   if (al & 15) return ZKV_ERR_INVALID_ARG;
-  return ZKV_OK;
+  return validate_paged(p->block_table, p->page_tokens, p->max_pages, p->n_pages, p->Tcap);
 }
 
 // The encode + window-write kernel; with pdl, as a programmatic dependent of the previous

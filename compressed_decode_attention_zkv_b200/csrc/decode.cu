@@ -157,8 +157,11 @@ struct DecodeArgs {
   float scale_log2;   // softmax_scale * log2(e)
   double rot;         // 1 / sqrt(d)
   const __half* q;
-  const uint8_t* k_codes;
+  const uint8_t* k_codes;   // [B][Hkv][Tcap][Sk], or a page pool [n_pages][Hkv][P][Sk]
   const uint8_t* v_codes;
+  const int32_t* bt;        // paged layout: block table [B][max_pages], else null
+  int64_t max_pages, n_pages;
+  int pshift;               // log2 P (tokens per page)
   const int32_t* comp_len;
   const float* Ck;
   const float* k_smooth;   // [Hkv][d] key smoothing factors (the query is scaled by them) or null
@@ -650,17 +653,39 @@ struct Code {
   }
 };
 
-// Codes of token t (0 when t >= tend).  When S equals its padded size SP a single naturally
-// aligned 2-, 4- or 8-byte load reads them; otherwise byte loads.
+// The code rows of one (sequence, kv head): contiguous (base = the pair's row 0) or, with a
+// block table, token t in page bt_row[t / P] at row kvh_off + t % P of that page (base = the
+// page pool).  Both layouts give a row address aligned to the row size.
+struct PairRows {
+  const uint8_t* base;
+  const int32_t* bt_row;   // null: contiguous
+  int64_t kvh_off;         // kvh * P
+};
+__device__ __forceinline__ const uint8_t* pair_row(const DecodeArgs& a, const PairRows& pr,
+                                                   uint32_t t, int S) {
+  if (!pr.bt_row) return pr.base + (int64_t)t * S;
+  const int64_t pg = __ldg(pr.bt_row + (t >> a.pshift));
+  if (pg < 0 || pg >= a.n_pages) {
+    set_error(a.err, ZKV_DEVERR_PAGE);
+    return nullptr;
+  }
+  return pr.base + ((pg * a.Hkv << a.pshift) + pr.kvh_off + (t & ((1u << a.pshift) - 1u))) * S;
+}
+
+// Codes of token t (0 when t >= tend or its page is invalid).  When S equals its padded size SP
+// a single naturally aligned 2-, 4- or 8-byte load reads them; otherwise byte loads.
 template <int SP>
-__device__ __forceinline__ Code<SP> load_code1(const uint8_t* base, int S, uint32_t t, uint32_t tend) {
+__device__ __forceinline__ Code<SP> load_code1(const DecodeArgs& a, const PairRows& pr, int S,
+                                               uint32_t t, uint32_t tend) {
   // t is a pair-local token index (Tcap * S < 2^32 bytes per pair)
   Code<SP> r;
 #pragma unroll
   for (int q = 0; q < (SP <= 4 ? 1 : 2); ++q) r.w[q] = 0u;
   if (t >= tend) return r;
+  const uint8_t* row = pair_row(a, pr, t, S);
+  if (!row) return r;
   if (S == SP) {
-    const uint8_t* p = base + t * SP;
+    const uint8_t* p = row;
     if constexpr (SP == 2) {
       r.w[0] = __ldg(reinterpret_cast<const unsigned short*>(p));
     } else if constexpr (SP == 4) {
@@ -671,7 +696,7 @@ __device__ __forceinline__ Code<SP> load_code1(const uint8_t* base, int S, uint3
       r.w[1] = v.y;
     }
   } else {
-    const uint8_t* p = base + t * S;
+    const uint8_t* p = row;
 #pragma unroll
     for (int s = 0; s < SP; ++s)
       if (s < S) r.w[s >> 2] |= (uint32_t)__ldg(p + s) << (8 * (s & 3));
@@ -925,15 +950,39 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     if (seg0 >= seg1) continue;
     const int64_t s0 = seg0 - a.pre[pr], s1 = seg1 - a.pre[pr];   // pair-local token range
     const int64_t slot = (int64_t)pr + blockIdx.x;
-    const uint8_t* kcb = a.k_codes + (int64_t)pr * a.Tcap * Sk;
-    const uint8_t* vcb = a.v_codes + (int64_t)pr * a.Tcap * Sv;
-
-    if (tid == 0) {
-      // the segment's codes stream into L2 while the tables are filled; the per-thread loads
-      // below then find them there
-      const int64_t pbytes_k = (int64_t)a.Tcap * Sk, pbytes_v = (int64_t)a.Tcap * Sv;
-      prefetch_l2(kcb, kcb + pbytes_k, kcb + (s0 & ~int64_t(15)) * Sk, (s1 - (s0 & ~int64_t(15))) * Sk);
-      prefetch_l2(vcb, vcb + pbytes_v, vcb + (s0 & ~int64_t(15)) * Sv, (s1 - (s0 & ~int64_t(15))) * Sv);
+    PairRows kcb, vcb;
+    if (a.bt) {
+      const int b = pr / a.Hkv, kvh = pr - b * a.Hkv;
+      kcb = PairRows{a.k_codes, a.bt + (int64_t)b * a.max_pages, (int64_t)kvh << a.pshift};
+      vcb = PairRows{a.v_codes, kcb.bt_row, kcb.kvh_off};
+    } else {
+      kcb = PairRows{a.k_codes + (int64_t)pr * a.Tcap * Sk, nullptr, 0};
+      vcb = PairRows{a.v_codes + (int64_t)pr * a.Tcap * Sv, nullptr, 0};
+    }
+    // the segment's codes stream into L2 while the tables are filled; the per-thread loads
+    // below then find them there
+    if (!a.bt) {
+      if (tid == 0) {
+        const int64_t pbytes_k = (int64_t)a.Tcap * Sk, pbytes_v = (int64_t)a.Tcap * Sv;
+        const int64_t a0 = s0 & ~int64_t(15);
+        prefetch_l2(kcb.base, kcb.base + pbytes_k, kcb.base + a0 * Sk, (s1 - a0) * Sk);
+        prefetch_l2(vcb.base, vcb.base + pbytes_v, vcb.base + a0 * Sv, (s1 - a0) * Sv);
+      }
+    } else {
+      // one thread per page the segment touches (a page's rows of one head are contiguous)
+      const int64_t P = int64_t(1) << a.pshift;
+      const int64_t p0 = s0 >> a.pshift, np = ((s1 - 1) >> a.pshift) - p0 + 1;
+      for (int64_t k = tid; k < np; k += kScanThreads) {
+        const int64_t r0 = (p0 + k) * P > s0 ? (p0 + k) * P : s0;
+        const int64_t r1 = (p0 + k + 1) * P < s1 ? (p0 + k + 1) * P : s1;
+        // page blocks of P * S bytes start 16-byte aligned (P >= 32 is a power of two); the
+        // prefetch is rounded outward to 16-byte granules inside the block
+        const uint8_t* bk = pair_row(a, kcb, (uint32_t)((p0 + k) * P), Sk);
+        const uint8_t* bv = pair_row(a, vcb, (uint32_t)((p0 + k) * P), Sv);
+        const int64_t o = r0 - (p0 + k) * P;
+        if (bk) prefetch_l2(bk, bk + P * Sk, bk + o * Sk, (r1 - r0) * Sk);
+        if (bv) prefetch_l2(bv, bv + P * Sv, bv + o * Sv, (r1 - r0) * Sv);
+      }
     }
     const uint32_t u0 = (uint32_t)s0, u1 = (uint32_t)s1;
     const int nsub = (int)((u1 - u0 + kScanSub - 1) / kScanSub);   // same on every thread
@@ -944,10 +993,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     // later growth of the reference (a fold) is rare.  The histograms do not depend on order.
     const uint32_t tw = u0 + (uint32_t)(warp * nsub) * 32u + (uint32_t)lane;   // token of sub-chunk 0
     // codes of sub-chunks 0 and 1 in flight during the table fill
-    Code<SKP> kc = load_code1<SKP>(kcb, Sk, tw, u1);
-    Code<SVP> vc = load_code1<SVP>(vcb, Sv, tw, u1);
-    Code<SKP> kn = load_code1<SKP>(kcb, Sk, tw + 32u, u1);
-    Code<SVP> vn = load_code1<SVP>(vcb, Sv, tw + 32u, u1);
+    Code<SKP> kc = load_code1<SKP>(a, kcb, Sk, tw, u1);
+    Code<SVP> vc = load_code1<SVP>(a, vcb, Sv, tw, u1);
+    Code<SKP> kn = load_code1<SKP>(a, kcb, Sk, tw + 32u, u1);
+    Code<SVP> vn = load_code1<SVP>(a, vcb, Sv, tw + 32u, u1);
     __syncthreads();   // previous segment's shared memory is free
     {
       // zero the histograms, then copy the pair's table entries (s, c) -> every lane-group
@@ -1084,8 +1133,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       if (i + 1 < nsub) {
         kc = kn;
         vc = vn;
-        kn = load_code1<SKP>(kcb, Sk, t + 64u, u1);
-        vn = load_code1<SVP>(vcb, Sv, t + 64u, u1);
+        kn = load_code1<SKP>(a, kcb, Sk, t + 64u, u1);
+        vn = load_code1<SVP>(a, vcb, Sv, t + 64u, u1);
         key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
         if (t + 32u < u1) {
 #pragma unroll
@@ -1474,7 +1523,7 @@ static int validate_decode_shapes(const zkv_decode_params* p) {
     return ZKV_ERR_INVALID_ARG;
   if (p->Tcap % 16) return ZKV_ERR_INVALID_ARG;
   if (p->Tcap > (int64_t(1) << 28)) return ZKV_ERR_UNSUPPORTED;   // 32-bit in-pair offsets
-  return ZKV_OK;
+  return validate_paged(p->block_table, p->page_tokens, p->max_pages, p->n_pages, p->Tcap);
 }
 
 static int validate_decode(const zkv_decode_params* p) {
@@ -1524,6 +1573,8 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   a.rot = 1.0 / std::sqrt((double)p->d);
   a.q = reinterpret_cast<const __half*>(p->q);
   a.k_codes = p->k_codes; a.v_codes = p->v_codes; a.comp_len = p->comp_len;
+  a.bt = p->block_table; a.max_pages = p->max_pages; a.n_pages = p->n_pages;
+  a.pshift = p->block_table ? log2_pow2(p->page_tokens) : 0;
   a.Ck = p->k_codebooks; a.Cv = p->v_codebooks; a.k_smooth = p->k_smooth;
   a.win_k = reinterpret_cast<const __half*>(p->win_k);
   a.win_v = reinterpret_cast<const __half*>(p->win_v);
@@ -1570,6 +1621,10 @@ extern "C" int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_
       ap->k_codebooks != dp->k_codebooks || ap->v_codebooks != dp->v_codebooks ||
       ap->win_k != dp->win_k || ap->win_v != dp->win_v || ap->win_len != dp->win_len ||
       ap->comp_len != dp->comp_len || ap->k_smooth != dp->k_smooth)
+    return ZKV_ERR_INVALID_ARG;
+  if (ap->block_table != dp->block_table ||
+      (ap->block_table && (ap->page_tokens != dp->page_tokens || ap->max_pages != dp->max_pages ||
+                           ap->n_pages != dp->n_pages)))
     return ZKV_ERR_INVALID_ARG;
   return decode_common(dp, workspace, workspace_bytes, stream, ap);
 }

@@ -18,6 +18,18 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 inline bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
 
+// Paged code layout (block table): P a power of two in [32, 65536], Tcap = max_pages * P,
+// page indices fit int32.  No block table: the contiguous layout, nothing to check.
+inline int validate_paged(const int32_t* bt, int64_t P, int64_t max_pages, int64_t n_pages,
+                          int64_t Tcap) {
+  if (!bt) return ZKV_OK;
+  if (P < 32 || P > 65536 || (P & (P - 1))) return ZKV_ERR_INVALID_ARG;
+  if (max_pages < 1 || n_pages < 1 || n_pages > 0x7fffffffLL) return ZKV_ERR_INVALID_ARG;
+  if (max_pages > (int64_t(1) << 28) / P || max_pages * P != Tcap) return ZKV_ERR_INVALID_ARG;
+  return ZKV_OK;
+}
+inline int log2_pow2(int64_t x) { int s = 0; while ((int64_t(1) << s) < x) ++s; return s; }
+
 #define ZKV_CHECK_LAUNCH()                                   \
   do {                                                       \
     if (cudaGetLastError() != cudaSuccess) return ZKV_ERR_CUDA; \

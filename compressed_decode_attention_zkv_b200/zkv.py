@@ -27,6 +27,7 @@ ZKV_OK, ZKV_ERR_INVALID_ARG, ZKV_ERR_UNSUPPORTED, ZKV_ERR_WORKSPACE, ZKV_ERR_CUD
 ZKV_DEVERR_COMP_LEN = 1
 ZKV_DEVERR_WIN_LEN = 2
 ZKV_DEVERR_TIMEOUT = 4
+ZKV_DEVERR_PAGE = 8
 ZKV_DTYPE_F16, ZKV_DTYPE_F32 = 0, 1
 CODEBOOK_SIZE = 256
 DECODE_SCRATCH_BYTES = 8 << 20   # ZKV_DECODE_SCRATCH_BYTES: the no-allocation decode's array
@@ -65,7 +66,9 @@ class DecodeParams(ctypes.Structure):
                 ("comp_len", c_void_p), ("k_codebooks", c_void_p), ("v_codebooks", c_void_p),
                 ("win_k", c_void_p), ("win_v", c_void_p), ("win_len", c_void_p),
                 ("out", c_void_p), ("lse", c_void_p), ("error_flag", c_void_p),
-                ("trace_events", c_void_p), ("k_smooth", c_void_p)]
+                ("trace_events", c_void_p), ("k_smooth", c_void_p),
+                ("block_table", c_void_p), ("page_tokens", c_int64), ("max_pages", c_int64),
+                ("n_pages", c_int64)]
 
 
 class AppendParams(ctypes.Structure):
@@ -75,7 +78,8 @@ class AppendParams(ctypes.Structure):
                 ("win_v", c_void_p), ("win_len", c_void_p), ("win_head", c_void_p),
                 ("comp_len", c_void_p), ("k_codes", c_void_p), ("v_codes", c_void_p),
                 ("k_codebooks", c_void_p), ("v_codebooks", c_void_p), ("error_flag", c_void_p),
-                ("k_smooth", c_void_p)]
+                ("k_smooth", c_void_p), ("block_table", c_void_p), ("page_tokens", c_int64),
+                ("max_pages", c_int64), ("n_pages", c_int64)]
 
 
 _lib = None
@@ -128,6 +132,19 @@ def _stream() -> int:
 
 def _ptr(t):
     return None if t is None else t.data_ptr()
+
+
+def _code_layout(k_codes, block_table):
+    """(Hkv, Tcap, Sk, paged fields) of a contiguous [B, Hkv, Tcap, Sk] code array, or of a page
+    pool [n_pages, Hkv, P, Sk] with an int32 [B, max_pages] block table."""
+    if block_table is None:
+        _, Hkv, Tcap, Sk = k_codes.shape
+        return Hkv, Tcap, Sk, dict(block_table=None, page_tokens=0, max_pages=0, n_pages=0)
+    _need(block_table, "block_table", torch.int32)
+    n_pages, Hkv, P, Sk = k_codes.shape
+    max_pages = block_table.shape[1]
+    return Hkv, max_pages * P, Sk, dict(block_table=_ptr(block_table), page_tokens=P,
+                                        max_pages=max_pages, n_pages=n_pages)
 
 
 def _smooth_ptr(lam, heads: int, d: int, name: str) -> int | None:
@@ -252,7 +269,7 @@ def rvq_reconstruct(codes: torch.Tensor, codebooks: torch.Tensor, unrotate: bool
 
 def _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
                    win_len, out, lse, max_comp_len, softmax_scale, error_flag,
-                   k_smooth=None) -> DecodeParams:
+                   k_smooth=None, block_table=None) -> DecodeParams:
     _need(q, "q", torch.float16)
     _need(k_codes, "k_codes", torch.uint8)
     _need(v_codes, "v_codes", torch.uint8)
@@ -263,7 +280,7 @@ def _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_
     _need(win_k, "win_k", torch.float16)
     _need(win_v, "win_v", torch.float16)
     B, Hq, d = q.shape
-    _, Hkv, Tcap, Sk = k_codes.shape
+    Hkv, Tcap, Sk, paged = _code_layout(k_codes, block_table)
     Sv = v_codes.shape[3]
     Wcap = win_k.shape[2]
     if out is not None:
@@ -280,7 +297,7 @@ def _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_
                         v_codebooks=_ptr(v_codebooks), win_k=_ptr(win_k), win_v=_ptr(win_v),
                         win_len=_ptr(win_len), out=_ptr(out), lse=_ptr(lse),
                         error_flag=_ptr(error_flag),
-                        k_smooth=_smooth_ptr(k_smooth, Hkv, d, "k_smooth"))
+                        k_smooth=_smooth_ptr(k_smooth, Hkv, d, "k_smooth"), **paged)
 
 
 def decode_workspace_size(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
@@ -296,11 +313,12 @@ def decode_workspace_size(q, k_codes, v_codes, comp_len, k_codebooks, v_codebook
 def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
                     win_len, out=None, lse=None, max_comp_len=None, softmax_scale=None,
                     workspace: torch.Tensor | None = None, error_flag=None, trace_events=None,
-                    k_smooth=None):
+                    k_smooth=None, block_table=None):
     """Decode attention over the compressed prefix plus the fp16 window (see include/zkv.h).
     ``trace_events``: optional 4 torch.cuda.Event(enable_timing=True) recorded before the
     table, scan and merge stages and after the last kernel.  ``k_smooth``: the [Hkv, d] key
-    smoothing factors the prefix was encoded with.
+    smoothing factors the prefix was encoded with.  ``block_table``: int32 [B, max_pages] for
+    the paged layout (k_codes / v_codes are then page pools [n_pages, Hkv, P, S]).
     Returns (out float32 [B, Hq, d], lse float32 [B, Hq])."""
     B, Hq, d = q.shape
     if out is None:
@@ -308,7 +326,8 @@ def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
-                       win_len, out, lse, max_comp_len, softmax_scale, error_flag, k_smooth)
+                       win_len, out, lse, max_comp_len, softmax_scale, error_flag, k_smooth,
+                       block_table)
     ev_arr = None
     if trace_events is not None:
         if len(trace_events) != 4:
@@ -349,7 +368,7 @@ def rvq_decode_attn_noalloc(q, k_codes, v_codes, comp_len, k_codebooks, v_codebo
 
 
 def _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
-                   k_codebooks, v_codebooks, error_flag, k_smooth=None):
+                   k_codebooks, v_codebooks, error_flag, k_smooth=None, block_table=None):
     _need(new_k, "new_k", torch.float16)
     _need(new_v, "new_v", torch.float16)
     for n, t in (("win_k", win_k), ("win_v", win_v)):
@@ -362,21 +381,23 @@ def _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_co
     _need(v_codebooks, "v_codebooks", torch.float32)
     if error_flag is not None:
         _need(error_flag, "error_flag", torch.int32)
-    B, Hkv, Tcap, Sk = k_codes.shape
+    B = new_k.shape[0]
+    Hkv, Tcap, Sk, paged = _code_layout(k_codes, block_table)
     return AppendParams(B=B, Hkv=Hkv, d=new_k.shape[-1], Sk=Sk, Sv=v_codes.shape[3], Tcap=Tcap,
                         Wcap=win_k.shape[2], new_k=_ptr(new_k), new_v=_ptr(new_v),
                         win_k=_ptr(win_k), win_v=_ptr(win_v), win_len=_ptr(win_len),
                         win_head=_ptr(win_head), comp_len=_ptr(comp_len), k_codes=_ptr(k_codes),
                         v_codes=_ptr(v_codes), k_codebooks=_ptr(k_codebooks),
                         v_codebooks=_ptr(v_codebooks), error_flag=_ptr(error_flag),
-                        k_smooth=_smooth_ptr(k_smooth, Hkv, new_k.shape[-1], "k_smooth"))
+                        k_smooth=_smooth_ptr(k_smooth, Hkv, new_k.shape[-1], "k_smooth"),
+                        **paged)
 
 
 def rvq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
-               k_codebooks, v_codebooks, error_flag=None, k_smooth=None):
+               k_codebooks, v_codebooks, error_flag=None, k_smooth=None, block_table=None):
     """One serving step of cache maintenance (see include/zkv.h); state updated in place."""
     p = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes,
-                       v_codes, k_codebooks, v_codebooks, error_flag, k_smooth)
+                       v_codes, k_codebooks, v_codebooks, error_flag, k_smooth, block_table)
     _check("zkv_rvq_append", lib().zkv_rvq_append(ctypes.byref(p), _stream()))
 
 
@@ -410,7 +431,7 @@ class PreparedServeStep:
     def __init__(self, new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes,
                  v_codes, k_codebooks, v_codebooks, out=None, lse=None, max_comp_len=None,
                  softmax_scale=None, workspace: torch.Tensor | None = None, error_flag=None,
-                 trace_events=None, k_smooth=None):
+                 trace_events=None, k_smooth=None, block_table=None):
         B, Hq, d = q.shape
         if out is None:
             out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
@@ -418,10 +439,10 @@ class PreparedServeStep:
             lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
         self._pa = _append_params(new_k, new_v, win_k, win_v, win_len, win_head, comp_len,
                                   k_codes, v_codes, k_codebooks, v_codebooks, error_flag,
-                                  k_smooth)
+                                  k_smooth, block_table)
         self._pd = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
                                   win_v, win_len, out, lse, max_comp_len, softmax_scale,
-                                  error_flag, k_smooth)
+                                  error_flag, k_smooth, block_table)
         self._ev = None
         if trace_events is not None:   # recorded before the tables, the scan, the merge, and last
             if len(trace_events) != 4:
@@ -439,7 +460,8 @@ class PreparedServeStep:
                            f"workspace holds {workspace.numel()} bytes, {need} needed")
         self.out, self.lse = out, lse
         self._keep = (new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes,
-                      v_codes, k_codebooks, v_codebooks, workspace, error_flag, k_smooth)
+                      v_codes, k_codebooks, v_codebooks, workspace, error_flag, k_smooth,
+                      block_table)
         self._refa, self._refd = ctypes.byref(self._pa), ctypes.byref(self._pd)
         self._ws = ctypes.c_void_p(workspace.data_ptr())
         self._wsn = ctypes.c_size_t(workspace.numel())
@@ -456,14 +478,15 @@ class PreparedServeStep:
 def rvq_serve_step(new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
                    k_codebooks, v_codebooks, out=None, lse=None, max_comp_len=None,
                    softmax_scale=None, workspace=None, error_flag=None, trace_events=None,
-                   k_smooth=None):
+                   k_smooth=None, block_table=None):
     """rvq_append(new_k, new_v, ...) then rvq_decode_attn(q, ...) on the updated cache, in one
     library call (see include/zkv.h).  Returns (out, lse)."""
     if max_comp_len is None:
-        max_comp_len = k_codes.shape[2]
+        max_comp_len = _code_layout(k_codes, block_table)[1]
     return PreparedServeStep(new_k, new_v, q, win_k, win_v, win_len, win_head, comp_len,
                              k_codes, v_codes, k_codebooks, v_codebooks, out, lse, max_comp_len,
-                             softmax_scale, workspace, error_flag, trace_events, k_smooth)()
+                             softmax_scale, workspace, error_flag, trace_events, k_smooth,
+                             block_table)()
 
 
 class PreparedDecode:

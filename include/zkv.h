@@ -55,6 +55,8 @@ typedef enum {
 #define ZKV_DEVERR_COMP_LEN 1   /* comp_len[b] > Tcap (clamped) or append at Tcap (skipped) */
 #define ZKV_DEVERR_WIN_LEN 2    /* win_len[b] > Wcap (clamped)                              */
 #define ZKV_DEVERR_TIMEOUT 4    /* a bounded on-chip wait ran out (results of that tile absent) */
+#define ZKV_DEVERR_PAGE 8       /* a block-table entry outside [0, n_pages): its tokens read as code
+                                   0 (decode) / the append writes nothing for that sequence      */
 
 #define ZKV_DTYPE_F16 0
 #define ZKV_DTYPE_F32 1
@@ -203,6 +205,14 @@ typedef struct {
    * rotation, so q_tilde . k_tilde = q . k (VeloxQuant "VecInfer").  The window keys are raw.
    * NULL: no smoothing. */
   const float* k_smooth;
+  /* Optional paged code layout (serving with fixed token blocks): block_table int32
+   * [B][max_pages] maps a sequence's page p (its tokens [p P, (p+1) P)) to a page of the pools;
+   * k_codes / v_codes are then pools [n_pages][Hkv][P][Sk | Sv] (page index outermost, every
+   * kv head's P rows contiguous inside a page), P = page_tokens a power of two in [32, 65536],
+   * and Tcap must equal max_pages * P (the per-sequence capacity).  Pages need not be distinct
+   * across sequences that never write them.  NULL: the contiguous layout above. */
+  const int32_t* block_table;
+  int64_t page_tokens, max_pages, n_pages;
 } zkv_decode_params;
 
 /* Workspace bytes for a call with these shapes (data pointers are not read); 0 if the shapes
@@ -266,6 +276,10 @@ typedef struct {
   const float* v_codebooks;
   int32_t* error_flag;
   const float* k_smooth;   /* optional [Hkv][d]: evicted keys are smoothed as in zkv_rvq_encode */
+  /* optional paged layout, as in zkv_decode_params (the evicted token's codes go to page
+   * block_table[b][comp_len[b] / P]) */
+  const int32_t* block_table;
+  int64_t page_tokens, max_pages, n_pages;
 } zkv_append_params;
 
 int zkv_rvq_append(const zkv_append_params* p, void* stream);
@@ -280,7 +294,8 @@ int zkv_rvq_append(const zkv_append_params* p, void* stream);
  * partition of the token space (computed from the lengths the append will produce) with the
  * encode of the evicted tokens; the new lengths are stored by the decode's scan kernel.
  * ap and dp describe one cache: B, Hkv, d, Sk, Sv, Tcap and Wcap must be equal, and so must
- * k_codes, v_codes, k_codebooks, v_codebooks, win_k, win_v, win_len, comp_len and k_smooth (else
+ * k_codes, v_codes, k_codebooks, v_codebooks, win_k, win_v, win_len, comp_len, k_smooth and the
+ * paged layout (block_table, page_tokens, max_pages, n_pages) (else
  * ZKV_ERR_INVALID_ARG).  dp->comp_len and dp->win_len are read after the update, so
  * dp->max_comp_len must allow for the new token.  workspace: as zkv_rvq_decode_attn
  * (zkv_decode_workspace_size(dp)); dp->trace_events: as zkv_rvq_decode_attn, where the first

@@ -115,6 +115,20 @@ def test_append_validation(L):
     assert L.zkv_rvq_append(ctypes.byref(p), None) == zkv.ZKV_ERR_INVALID_ARG  # null pointers
 
 
+@pytest.mark.parametrize("kw", [
+    dict(page_tokens=48, max_pages=4, n_pages=8, Tcap=192, max_comp_len=64),   # not a power of two
+    dict(page_tokens=16, max_pages=4, n_pages=8),                             # below 32
+    dict(page_tokens=32, max_pages=4, n_pages=8),                             # 4 * 32 != Tcap (64)
+    dict(page_tokens=32, max_pages=2, n_pages=0),                             # empty pool
+])
+def test_paged_layout_validation(L, kw):
+    p = _decode_params(block_table=0xf000, **kw)
+    assert L.zkv_rvq_decode_attn(ctypes.byref(p), None, 0, None) == zkv.ZKV_ERR_INVALID_ARG
+    assert L.zkv_decode_workspace_size(ctypes.byref(p)) == 0
+    ok = _decode_params(block_table=0xf000, page_tokens=32, max_pages=2, n_pages=8)
+    assert L.zkv_decode_workspace_size(ctypes.byref(ok)) > 0
+
+
 def _append_params(**kw):
     # the same cache as _decode_params (shapes and shared buffers)
     base = dict(B=2, Hkv=2, d=128, Sk=4, Sv=4, Tcap=64, Wcap=16, new_k=0xb000, new_v=0xc000,
@@ -133,6 +147,8 @@ def _append_params(**kw):
     (dict(Sv=3), {}, zkv.ZKV_ERR_INVALID_ARG),
     (dict(new_k=0), {}, zkv.ZKV_ERR_INVALID_ARG),             # the append itself is invalid
     (dict(k_smooth=0xe000), {}, zkv.ZKV_ERR_INVALID_ARG),     # different smoothing factors
+    (dict(block_table=0xf000, page_tokens=32, max_pages=2, n_pages=8), {},
+     zkv.ZKV_ERR_INVALID_ARG),                                 # paged append, contiguous decode
     (dict(d=96), dict(d=96), zkv.ZKV_ERR_UNSUPPORTED),
     ({}, dict(Hq=6, Hkv=4), zkv.ZKV_ERR_INVALID_ARG),          # the decode itself is invalid
     ({}, {}, zkv.ZKV_ERR_WORKSPACE),                           # consistent, but no workspace
