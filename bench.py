@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-encode", action="store_true", help="skip the bulk-encode extra")
     ap.add_argument("--no-smooth", action="store_true",
                     help="skip the serving step with key smoothing (extra)")
+    ap.add_argument("--no-paged", action="store_true",
+                    help="skip the serving step with the paged code layout (extra)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -119,7 +121,7 @@ class ClockSampler:
 # Workload state on the GPU
 # --------------------------------------------------------------------------------------------
 
-def build_state(wl, R, Tcap_extra, dev, smooth=False):
+def build_state(wl, R, Tcap_extra, dev, smooth=False, tcap_multiple=16):
     """Encode the workload's prefixes on the GPU (prefill) and make R replicas.  smooth: key
     smoothing factors calibrated on the calibration sample, key codebooks trained on smoothed
     keys, prefixes encoded with them (each replica carries "k_smooth")."""
@@ -133,7 +135,7 @@ def build_state(wl, R, Tcap_extra, dev, smooth=False):
     Ck = torch.from_numpy(I.train_codebooks(wl, "k", smooth=lam_np)).to(dev)
     Cv = torch.from_numpy(I.train_codebooks(wl, "v")).to(dev)
     Tc = wl.Tc
-    Tcap = (Tc + Tcap_extra + 15) // 16 * 16
+    Tcap = (Tc + Tcap_extra + tcap_multiple - 1) // tcap_multiple * tcap_multiple
     kc = torch.zeros((wl.B, wl.Hkv, Tcap, wl.Sk), dtype=torch.uint8, device=dev)
     vc = torch.zeros((wl.B, wl.Hkv, Tcap, wl.Sv), dtype=torch.uint8, device=dev)
     wk = torch.empty((wl.B, wl.Hkv, wl.W, wl.d), dtype=torch.float16, device=dev)
@@ -180,7 +182,8 @@ def step_fn(rep, ws, max_comp, events=None):
                        rep["win_len"], rep["win_head"], rep["comp_len"], rep["k_codes"],
                        rep["v_codes"], rep["Ck"], rep["Cv"], out=rep["out"], lse=rep["lse"],
                        max_comp_len=max_comp, workspace=ws, error_flag=rep["err"],
-                       trace_events=events, k_smooth=rep.get("k_smooth"))
+                       trace_events=events, k_smooth=rep.get("k_smooth"),
+                       block_table=rep.get("bt"))
 
 
 # --------------------------------------------------------------------------------------------
@@ -347,21 +350,45 @@ def encode_extra(dev, hbm, bf16):
                     "exact decision: TF32-margin candidates re-scored in float32, then float64"}
 
 
-def smooth_extra(wl, args, dev, R, base_ms):
-    """The serving step with the VecInfer key smoothing (per-channel factors before the
-    rotation, absorbed into the query) on the same workload: its own replicas, codebooks
-    trained on smoothed keys, CUDA graphs, the same timing rules.  Returns the extra's dict."""
+def paginate_replica(rep, P, seed):
+    """Move a replica's codes into page pools [n_pages, Hkv, P, S] (pages shuffled through a
+    pool with spare pages) and give it the block table."""
+    import torch
+    Bn, Hkv, Tcap, _ = rep["k_codes"].shape
+    mp = Tcap // P
+    n_pages = Bn * mp + 16
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(n_pages, generator=g)[:Bn * mp].to(rep["k_codes"].device)
+    for key in ("k_codes", "v_codes"):
+        c = rep[key]
+        S = c.shape[3]
+        pages = c.view(Bn, Hkv, mp, P, S).permute(0, 2, 1, 3, 4).reshape(Bn * mp, Hkv, P, S)
+        pool = torch.zeros((n_pages, Hkv, P, S), dtype=torch.uint8, device=c.device)
+        pool[perm] = pages
+        rep[key] = pool
+    rep["bt"] = perm.view(Bn, mp).to(torch.int32).contiguous()
+
+
+def variant_extra(wl, args, dev, R, base_ms, smooth=False, page_tokens=0):
+    """The serving step of the main line in a variant on the same workload: with the VecInfer
+    key smoothing (per-channel factors before the rotation, absorbed into the query; codebooks
+    trained on smoothed keys) or with the paged code layout (pages of page_tokens tokens behind
+    a block table).  Own replicas, CUDA graphs, the same timing rules.  Returns a dict."""
     import torch
 
     from compressed_decode_attention_zkv_b200 import zkv
     steps = min(args.steps, 200)
     per_rep = (R + 3 + steps + R - 1) // R + 2
-    reps, _ = build_state(wl, R, per_rep, dev, smooth=True)
+    reps, Tcap = build_state(wl, R, per_rep, dev, smooth=smooth,
+                             tcap_multiple=page_tokens if page_tokens else 16)
+    if page_tokens:
+        for r, rep in enumerate(reps):
+            paginate_replica(rep, page_tokens, 1000 + r)
     max_comp = wl.Tc + per_rep
     need = zkv.decode_workspace_size(reps[0]["q"], reps[0]["k_codes"], reps[0]["v_codes"],
                                      reps[0]["comp_len"], reps[0]["Ck"], reps[0]["Cv"],
                                      reps[0]["win_k"], reps[0]["win_v"], reps[0]["win_len"],
-                                     max_comp_len=max_comp)
+                                     max_comp_len=max_comp, block_table=reps[0].get("bt"))
     wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
     host_comp = [wl.Tc] * R
     for r in range(R):   # eager call per replica (kernel attributes before capture)
@@ -391,11 +418,13 @@ def smooth_extra(wl, args, dev, R, base_ms):
     sec = s.elapsed_time(e) / 1000.0
     assert sum(int(rep["err"].item()) for rep in reps) == 0
     del graphs
-    return {"workload": f"{wl.name} with VecInfer key smoothing (lambda_i = sqrt(max|K_i|), "
-                        f"codebooks trained on smoothed keys)",
+    what = ("VecInfer key smoothing (lambda_i = sqrt(max|K_i|), codebooks trained on smoothed "
+            "keys)" if smooth else f"paged codes ({page_tokens}-token pages shuffled through a "
+            f"pool, block table [B][{Tcap // page_tokens}])")
+    return {"workload": f"{wl.name} with {what}",
             "value": tokens / sec, "unit": UNIT, "ms_per_step": 1000.0 * sec / steps,
-            "steps": steps, "vs_unsmoothed_step": base_ms / (1000.0 * sec / steps),
-            "note": "one zkv_rvq_serve_step per step with k_smooth; graphs over "
+            "steps": steps, "main_step_over_this_step": base_ms / (1000.0 * sec / steps),
+            "note": "one zkv_rvq_serve_step per step; graphs over "
                     f"{R} rotating replicas (inputs larger than L2)"}
 
 
@@ -631,11 +660,18 @@ def run_ours(args):
     if not args.no_encode and rank == 0:
         del graphs, soak_graphs
         extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
-    if not args.no_smooth and rank == 0:
+    base_ms = 1000.0 * elapsed / args.steps
+    for name, kw, skip in (("smooth", dict(smooth=True), args.no_smooth),
+                           ("paged", dict(page_tokens=256), args.no_paged)):
+        if skip or rank != 0:
+            continue
         reps.clear()
         wss.clear()
         torch.cuda.empty_cache()
-        extras["smooth"] = smooth_extra(wl, args, dev, R, 1000.0 * elapsed / args.steps)
+        try:
+            extras[name] = variant_extra(wl, args, dev, R, base_ms, **kw)
+        except Exception as exc:   # an extra never takes the main line down
+            extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -301,9 +301,9 @@ def _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_
 
 
 def decode_workspace_size(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k,
-                          win_v, win_len, max_comp_len=None) -> int:
+                          win_v, win_len, max_comp_len=None, block_table=None) -> int:
     p = _decode_params(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win_k, win_v,
-                       win_len, None, None, max_comp_len, None, None)
+                       win_len, None, None, max_comp_len, None, None, None, block_table)
     n = lib().zkv_decode_workspace_size(ctypes.byref(p))
     if n == 0:
         raise ZkvError("zkv_decode_workspace_size", ZKV_ERR_INVALID_ARG)
