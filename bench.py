@@ -39,8 +39,8 @@ WORKLOAD = "llama3_8b_32k"
 # the scan kernel source is unchanged (hash of decode.cu at capture time).
 # DRAM bytes (read + write) of one scan_kernel launch on this workload, from one ncu capture
 # (profiles/scan_kernel_llama3_8b_32k.md), valid while the scan's source is unchanged.
-SCAN_TRAFFIC = {"scan_src_sha1": "72a8c114efe07b5fd333dcbbc0d847e535b0d60c",
-                "bytes_per_launch": 17807445}
+SCAN_TRAFFIC = {"scan_src_sha1": "1ecd1b7d8d96ab3f59999e8ee579ed14f7a50b1d",
+                "bytes_per_launch": 17806251}
 
 
 def parse():

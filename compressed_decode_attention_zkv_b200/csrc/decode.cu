@@ -661,9 +661,10 @@ struct PairRows {
   const int32_t* bt_row;   // null: contiguous
   int64_t kvh_off;         // kvh * P
 };
+template <bool PAGED>
 __device__ __forceinline__ const uint8_t* pair_row(const DecodeArgs& a, const PairRows& pr,
                                                    uint32_t t, int S) {
-  if (!pr.bt_row) return pr.base + (int64_t)t * S;
+  if constexpr (!PAGED) return pr.base + (int64_t)t * S;
   const int64_t pg = __ldg(pr.bt_row + (t >> a.pshift));
   if (pg < 0 || pg >= a.n_pages) {
     set_error(a.err, ZKV_DEVERR_PAGE);
@@ -674,7 +675,7 @@ __device__ __forceinline__ const uint8_t* pair_row(const DecodeArgs& a, const Pa
 
 // Codes of token t (0 when t >= tend or its page is invalid).  When S equals its padded size SP
 // a single naturally aligned 2-, 4- or 8-byte load reads them; otherwise byte loads.
-template <int SP>
+template <int SP, bool PAGED>
 __device__ __forceinline__ Code<SP> load_code1(const DecodeArgs& a, const PairRows& pr, int S,
                                                uint32_t t, uint32_t tend) {
   // t is a pair-local token index (Tcap * S < 2^32 bytes per pair)
@@ -682,7 +683,7 @@ __device__ __forceinline__ Code<SP> load_code1(const DecodeArgs& a, const PairRo
 #pragma unroll
   for (int q = 0; q < (SP <= 4 ? 1 : 2); ++q) r.w[q] = 0u;
   if (t >= tend) return r;
-  const uint8_t* row = pair_row(a, pr, t, S);
+  const uint8_t* row = pair_row<PAGED>(a, pr, t, S);
   if (!row) return r;
   if (S == SP) {
     const uint8_t* p = row;
@@ -824,7 +825,7 @@ __device__ __forceinline__ void fold_tables(const uint32_t* vhi, const uint32_t*
 // score exceeded the reference (rare: the reference is the maximum so far plus a headroom), the
 // next interval first takes the block maxima (a) and, with non-empty histograms, a slow path
 // (barrier, fold, barrier, zero, barrier) after (b), uniformly across the block.
-template <int GP, int SKP, int SVP>
+template <int GP, int SKP, int SVP, bool PAGED>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   using C = ScanCfg<GP, SKP, SVP>;
   extern __shared__ __align__(16) unsigned char smraw[];
@@ -951,7 +952,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     const int64_t s0 = seg0 - a.pre[pr], s1 = seg1 - a.pre[pr];   // pair-local token range
     const int64_t slot = (int64_t)pr + blockIdx.x;
     PairRows kcb, vcb;
-    if (a.bt) {
+    if constexpr (PAGED) {
       const int b = pr / a.Hkv, kvh = pr - b * a.Hkv;
       kcb = PairRows{a.k_codes, a.bt + (int64_t)b * a.max_pages, (int64_t)kvh << a.pshift};
       vcb = PairRows{a.v_codes, kcb.bt_row, kcb.kvh_off};
@@ -961,7 +962,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     }
     // the segment's codes stream into L2 while the tables are filled; the per-thread loads
     // below then find them there
-    if (!a.bt) {
+    if constexpr (!PAGED) {
       if (tid == 0) {
         const int64_t pbytes_k = (int64_t)a.Tcap * Sk, pbytes_v = (int64_t)a.Tcap * Sv;
         const int64_t a0 = s0 & ~int64_t(15);
@@ -977,8 +978,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
         const int64_t r1 = (p0 + k + 1) * P < s1 ? (p0 + k + 1) * P : s1;
         // page blocks of P * S bytes start 16-byte aligned (P >= 32 is a power of two); the
         // prefetch is rounded outward to 16-byte granules inside the block
-        const uint8_t* bk = pair_row(a, kcb, (uint32_t)((p0 + k) * P), Sk);
-        const uint8_t* bv = pair_row(a, vcb, (uint32_t)((p0 + k) * P), Sv);
+        const uint8_t* bk = pair_row<true>(a, kcb, (uint32_t)((p0 + k) * P), Sk);
+        const uint8_t* bv = pair_row<true>(a, vcb, (uint32_t)((p0 + k) * P), Sv);
         const int64_t o = r0 - (p0 + k) * P;
         if (bk) prefetch_l2(bk, bk + P * Sk, bk + o * Sk, (r1 - r0) * Sk);
         if (bv) prefetch_l2(bv, bv + P * Sv, bv + o * Sv, (r1 - r0) * Sv);
@@ -993,10 +994,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
     // later growth of the reference (a fold) is rare.  The histograms do not depend on order.
     const uint32_t tw = u0 + (uint32_t)(warp * nsub) * 32u + (uint32_t)lane;   // token of sub-chunk 0
     // codes of sub-chunks 0 and 1 in flight during the table fill
-    Code<SKP> kc = load_code1<SKP>(a, kcb, Sk, tw, u1);
-    Code<SVP> vc = load_code1<SVP>(a, vcb, Sv, tw, u1);
-    Code<SKP> kn = load_code1<SKP>(a, kcb, Sk, tw + 32u, u1);
-    Code<SVP> vn = load_code1<SVP>(a, vcb, Sv, tw + 32u, u1);
+    Code<SKP> kc = load_code1<SKP, PAGED>(a, kcb, Sk, tw, u1);
+    Code<SVP> vc = load_code1<SVP, PAGED>(a, vcb, Sv, tw, u1);
+    Code<SKP> kn = load_code1<SKP, PAGED>(a, kcb, Sk, tw + 32u, u1);
+    Code<SVP> vn = load_code1<SVP, PAGED>(a, vcb, Sv, tw + 32u, u1);
     __syncthreads();   // previous segment's shared memory is free
     {
       // zero the histograms, then copy the pair's table entries (s, c) -> every lane-group
@@ -1133,8 +1134,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
       if (i + 1 < nsub) {
         kc = kn;
         vc = vn;
-        kn = load_code1<SKP>(a, kcb, Sk, t + 64u, u1);
-        vn = load_code1<SVP>(a, vcb, Sv, t + 64u, u1);
+        kn = load_code1<SKP, PAGED>(a, kcb, Sk, t + 64u, u1);
+        vn = load_code1<SVP, PAGED>(a, vcb, Sv, t + 64u, u1);
         key_score<GP, SKP>(sbase, Sk, csh, lane, kc, sc);
         if (t + 32u < u1) {
 #pragma unroll
@@ -1421,8 +1422,10 @@ static inline void trace(void* const* ev, int i, cudaStream_t st) {
 
 template <int GP, int SKP, int SVP>
 static int launch_scan(const DecodeArgs& a, size_t smem, cudaStream_t st) {
-  if (ensure_smem_limit(scan_kernel<GP, SKP, SVP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
-  if (launch_pdl(scan_kernel<GP, SKP, SVP>, dim3(a.grid), dim3(kScanThreads), smem, st, a) != cudaSuccess)
+  // the code layout is a template parameter: the contiguous loop carries no paging logic
+  auto* k = a.bt ? scan_kernel<GP, SKP, SVP, true> : scan_kernel<GP, SKP, SVP, false>;
+  if (ensure_smem_limit(k, smem) != cudaSuccess) return ZKV_ERR_CUDA;
+  if (launch_pdl(k, dim3(a.grid), dim3(kScanThreads), smem, st, a) != cudaSuccess)
     return ZKV_ERR_CUDA;
   return ZKV_OK;
 }
