@@ -313,6 +313,23 @@ def train_codebooks(wl: Workload, kind: str, S: int | None = None,
     return books
 
 
+def train_pq_codebook(wl: Workload, kind: str, m: int, seed_cal: int = SEED_CALIB,
+                      seed_km: int = SEED_KMEANS, smooth: np.ndarray | None = None) -> np.ndarray:
+    """Product-VQ codebooks, float32 [Hkv][256][m]: seeded k-means over every m-dim sub-vector
+    of the rotated calibration vectors of a head (the sub-vectors share one codebook);
+    ``smooth`` as in train_codebooks."""
+    Hn = scipy.linalg.hadamard(wl.d).astype(np.float64) / np.sqrt(wl.d)
+    books = np.zeros((wl.Hkv, K_CODEWORDS, m), np.float32)
+    for h in range(wl.Hkv):
+        X = _calibration_sample(wl, kind, h, wl.n_cal, seed_cal).astype(np.float64)
+        if smooth is not None:
+            X = X / np.asarray(smooth[h], np.float64)[None, :]
+        R = (X @ Hn.T).astype(np.float32).reshape(-1, m)
+        krng = _rng(seed_km, 300 + (0 if kind == "k" else 1), h, m)
+        books[h], _ = _kmeans_zero_pinned(R, K_CODEWORDS, wl.kmeans_iters, krng)
+    return books
+
+
 # --------------------------------------------------------------------------------------------
 # Synthetic code streams for decode-only cases
 # --------------------------------------------------------------------------------------------

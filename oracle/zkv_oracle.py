@@ -29,6 +29,10 @@ Readings where the pages are silent (each is also listed in the design notes):
 * Greedy stage decision: squared L2 distance evaluated in float64, ties to the lowest index.
   The residual update r <- r - C_s[z_s] is an elementwise float32 subtraction.
 * Residual norm n_s = ||r|| after stage s (float64 accumulate, stored float32).
+* Product VQ (VecInfer): the rotated (keys: smoothed, then rotated) float32 vector is cut into
+  d/m consecutive sub-vectors of m dims; one 256-entry codebook [256][m] per kv head and K or V
+  is shared by every sub-vector; each sub-vector takes the nearest codeword (float64 distance,
+  lowest index on ties).  Values are rotated, not smoothed.
 * Smooth scaling (keys only): the key is multiplied by 1/lambda channel by channel in float64
   (1/lambda itself a float64 division of the float32 factor) before the rotation; the query is
   multiplied by lambda.  A channel that is zero on every calibration token gets lambda = 1.
@@ -364,6 +368,123 @@ def decode_attn_lut(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len
         o, l = lse_merge(parts)
         out[b, h] = o
         lse[b, h] = l
+    return out, lse
+
+
+# --------------------------------------------------------------------------------------------
+# Product vector quantisation  (VeloxQuant "VecInfer": smooth scaling + Walsh-Hadamard dual
+# transform, then a K-means codebook over sub-vectors; key_sub_dim = 4 gives 2 bits/elem,
+# 8 gives 1 bit/elem with 8-bit codes)
+# --------------------------------------------------------------------------------------------
+
+def pq_encode(x: np.ndarray, codebook: np.ndarray, smooth=None, rotate: bool = True):
+    """Product VQ of rows of x [n][d] against one codebook [K][m] shared by the d/m sub-vectors.
+
+    y = rotate(x / lambda) (or rotate(x); or x as float32 when ``rotate`` is False), cut into
+    y_j = y[j m : (j+1) m]; z_j = argmin_c ||y_j - C[c]||^2 (float64, lowest index on ties).
+    Returns (codes uint8 [n][d/m], y float32 [n][d]).
+    """
+    x = np.asarray(x)
+    if smooth is not None:
+        x = smooth_keys(x, smooth)
+    y = rotate_to_f32(x) if rotate else np.asarray(x, F32)
+    C = np.asarray(codebook, F32)
+    m = C.shape[1]
+    n, d = y.shape
+    assert d % m == 0
+    sub = y.reshape(n * (d // m), m)
+    z = np.argmin(stage_distances(sub, C), axis=1)
+    return z.reshape(n, d // m).astype(np.uint8), y
+
+
+def pq_reconstruct(codes: np.ndarray, codebook: np.ndarray, unrotate: bool = False) -> np.ndarray:
+    """y_hat = concatenation of C[z_j] over the sub-vectors (float64), or (1/sqrt(d)) H y_hat."""
+    C = np.asarray(codebook, F64)
+    codes = np.asarray(codes).astype(np.int64)
+    y = C[codes].reshape(codes.shape[:-1] + (codes.shape[-1] * C.shape[1],))
+    if unrotate:
+        y = fwht(y, 1.0 / np.sqrt(F64(y.shape[-1])))
+    return y
+
+
+def pq_decode_attn(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len,
+                   scale: float | None = None, pairs=None, k_smooth=None):
+    """decode_attn for product-VQ codes (direct form): k_codes / v_codes [B][Hkv][Tcap][d/m]
+    uint8, Ck / Cv [Hkv][K][m].  Keys are reconstructed, rotated back and multiplied by lambda
+    (with ``k_smooth``), values reconstructed and rotated back, then exact softmax attention
+    over them and the fp16 window in float64."""
+    B, Hq, d = q.shape
+    Hkv = k_codes.shape[1]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.full((B, Hq, d), np.nan, F64)
+    lse = np.full((B, Hq), np.nan, F64)
+    if pairs is None:
+        pairs = [(b, h) for b in range(B) for h in range(Hq)]
+    cache = {}
+    for b, h in pairs:
+        kvh = h // G
+        if (b, kvh) not in cache:
+            tc, wl = int(comp_len[b]), int(win_len[b])
+            kh = pq_reconstruct(k_codes[b, kvh, :tc], Ck[kvh], unrotate=True)
+            if k_smooth is not None:
+                kh = kh * np.asarray(k_smooth[kvh], F32).astype(F64)
+            vh = pq_reconstruct(v_codes[b, kvh, :tc], Cv[kvh], unrotate=True)
+            cache[(b, kvh)] = (np.concatenate([kh, np.asarray(win_k[b, kvh, :wl], F64)]),
+                               np.concatenate([vh, np.asarray(win_v[b, kvh, :wl], F64)]))
+        Kall, Vall = cache[(b, kvh)]
+        out[b, h], lse[b, h] = softmax_attention(np.asarray(q[b, h], F64), Kall, Vall, scale)
+    return out, lse
+
+
+def pq_decode_attn_lut(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_len,
+                       scale: float | None = None, pairs=None, k_smooth=None):
+    """The same attention the way the method reads product-VQ codes: q_tilde = (1/sqrt(d))
+    H (lambda q); per sub-vector j a table LUT_j[c] = scale * q_tilde_j . Ck[c]; score_t =
+    sum_j LUT_j[zk_{t,j}]; the values as per-sub-vector codeword weights W_j[c] (sum of p over
+    tokens with zv_{t,j} = c), o_tilde_j = sum_c W_j[c] Cv[c] / sum p, rotated back; joined with
+    the window by the log-sum-exp combine."""
+    B, Hq, d = q.shape
+    Hkv = k_codes.shape[1]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.full((B, Hq, d), np.nan, F64)
+    lse = np.full((B, Hq), np.nan, F64)
+    if pairs is None:
+        pairs = [(b, h) for b in range(B) for h in range(Hq)]
+    for b, h in pairs:
+        kvh = h // G
+        tc, wl = int(comp_len[b]), int(win_len[b])
+        CK = np.asarray(Ck[kvh], F64)
+        CV = np.asarray(Cv[kvh], F64)
+        m = CK.shape[1]
+        qs = np.asarray(q[b, h], F64)
+        if k_smooth is not None:
+            qs = qs * np.asarray(k_smooth[kvh], F32).astype(F64)
+        qt = fwht(qs, 1.0 / np.sqrt(F64(d)))
+        parts = []
+        if tc > 0:
+            zk = k_codes[b, kvh, :tc].astype(np.int64)
+            zv = v_codes[b, kvh, :tc].astype(np.int64)
+            score = np.zeros(tc, F64)
+            for j in range(d // m):
+                lut = F64(scale) * (CK @ qt[j * m:(j + 1) * m])
+                score += lut[zk[:, j]]
+            mx = score.max()
+            p = np.exp(score - mx)
+            ot = np.zeros(d, F64)
+            for j in range(d // m):
+                W = np.bincount(zv[:, j], weights=p, minlength=CV.shape[0])
+                ot[j * m:(j + 1) * m] = W @ CV
+            ot /= p.sum()
+            parts.append((fwht(ot, 1.0 / np.sqrt(F64(d))), mx + np.log(p.sum())))
+        else:
+            parts.append((np.zeros(d, F64), -np.inf))
+        parts.append(softmax_attention(np.asarray(q[b, h], F64), np.asarray(win_k[b, kvh, :wl], F64),
+                                       np.asarray(win_v[b, kvh, :wl], F64), scale))
+        out[b, h], lse[b, h] = lse_merge(parts)
     return out, lse
 
 

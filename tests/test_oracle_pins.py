@@ -496,3 +496,93 @@ def test_smoothed_encode_decode_recovers_the_original_scores():
     assert abs(lse[0, 0] - scipy.special.logsumexp(sc)) < 1e-4
     _, lse_wrong = O.decode_attn(q, kc, vc, [n], Ck, Cv, wk, wk, [0])
     assert abs(lse_wrong[0, 0] - scipy.special.logsumexp(sc)) > 1e-2
+
+
+# ------------------------------------------------------------------ product VQ (VecInfer)
+
+def test_pq_one_subvector_is_single_stage_vq():
+    # m = d: one sub-vector, so product VQ is the first RVQ stage with the same codebook
+    rng = np.random.default_rng(50)
+    x = rng.standard_normal((40, 16)).astype(np.float16)
+    C = (rng.standard_normal((32, 16)) * 0.6).astype(np.float32)
+    z, y = O.pq_encode(x, C)
+    zr, _, yr, _ = O.rvq_encode(x, C[None])
+    np.testing.assert_array_equal(z[:, 0], zr[:, 0])
+    np.testing.assert_array_equal(y, yr)
+
+
+def test_pq_matches_brute_force_per_subvector():
+    rng = np.random.default_rng(51)
+    d, m, K = 8, 2, 5
+    x = rng.standard_normal((12, d)).astype(np.float16)
+    C = rng.standard_normal((K, m)).astype(np.float32)
+    z, y = O.pq_encode(x, C)
+    for n in range(x.shape[0]):
+        for j in range(d // m):
+            dist = [sum((float(y[n, j * m + i]) - float(C[c, i])) ** 2 for i in range(m))
+                    for c in range(K)]
+            assert z[n, j] == min(range(K), key=lambda c: (dist[c], c))
+
+
+def test_pq_exact_codewords_round_trip():
+    # codewords cut from the rotated vectors themselves: every sub-vector finds its own piece
+    # and the reconstruction rotated back is the input (to float32 rounding)
+    rng = np.random.default_rng(52)
+    d, m = 32, 4
+    x = rng.standard_normal((3, d)).astype(np.float16)
+    y = O.rotate_to_f32(x)
+    pieces = y.reshape(-1, m)
+    C = np.concatenate([np.zeros((1, m), np.float32), pieces])
+    z, _ = O.pq_encode(x, C)
+    np.testing.assert_array_equal(z.reshape(-1), np.arange(1, 1 + pieces.shape[0]))
+    xr = O.pq_reconstruct(z, C, unrotate=True)
+    np.testing.assert_allclose(xr, x.astype(np.float64), atol=1e-5)
+
+
+def test_pq_duplicate_codewords_pick_lowest_index():
+    C = np.array([[1.0, 0.0], [0.0, 1.0], [0.0, 1.0]], np.float32)
+    y = np.array([[0.1, 0.9, 0.0, 1.2]], np.float32)
+    z, _ = O.pq_encode(y, C, rotate=False)
+    np.testing.assert_array_equal(z, [[1, 1]])
+
+
+def test_pq_distortion_is_the_sum_over_subvectors():
+    rng = np.random.default_rng(53)
+    d, m = 64, 8
+    x = rng.standard_normal((25, d)).astype(np.float16)
+    C = (rng.standard_normal((64, m)) * 0.4).astype(np.float32)
+    z, y = O.pq_encode(x, C)
+    err = ((y.astype(np.float64) - O.pq_reconstruct(z, C)) ** 2).sum(axis=1)
+    per = np.zeros(x.shape[0])
+    for j in range(d // m):
+        sub = y[:, j * m:(j + 1) * m].astype(np.float64)
+        per += (((sub[:, None, :] - C[None].astype(np.float64)) ** 2).sum(-1)).min(axis=1)
+    np.testing.assert_allclose(err, per, rtol=1e-12)
+
+
+@pytest.mark.parametrize("smooth", [False, True])
+def test_pq_direct_equals_lut_form(smooth):
+    rng = np.random.default_rng(54)
+    B, Hq, Hkv, d, m, Tcap, Wcap = 2, 4, 2, 64, 4, 30, 6
+    q = rng.standard_normal((B, Hq, d)).astype(np.float16)
+    kc = rng.integers(0, 32, (B, Hkv, Tcap, d // m)).astype(np.uint8)
+    vc = rng.integers(0, 32, (B, Hkv, Tcap, d // m)).astype(np.uint8)
+    Ck = (rng.standard_normal((Hkv, 32, m)) * 0.7).astype(np.float32)
+    Cv = rng.standard_normal((Hkv, 32, m)).astype(np.float32)
+    wk = rng.standard_normal((B, Hkv, Wcap, d)).astype(np.float16)
+    wv = rng.standard_normal((B, Hkv, Wcap, d)).astype(np.float16)
+    lam = np.exp(rng.standard_normal((Hkv, d)) * 0.5).astype(np.float32) if smooth else None
+    for comp, win in (([30, 11], [6, 2]), ([0, 30], [6, 0]), ([5, 0], [0, 6])):
+        case = (q, kc, vc, np.array(comp), Ck, Cv, wk, wv, np.array(win))
+        o1, l1 = O.pq_decode_attn(*case, k_smooth=lam)
+        o2, l2 = O.pq_decode_attn_lut(*case, k_smooth=lam)
+        np.testing.assert_allclose(o2, o1, atol=1e-9, rtol=0)
+        np.testing.assert_allclose(l2, l1, atol=1e-9, rtol=0)
+
+
+def test_pq_code_bytes_give_the_stated_bit_rates():
+    # 8-bit codes over sub-vectors of 4 (8) dims: 2 (1) bits per element
+    x = np.zeros((1, 128), np.float16)
+    for m, bits in ((4, 2), (8, 1)):
+        z, _ = O.pq_encode(x, np.zeros((256, m), np.float32))
+        assert z.dtype == np.uint8 and z.shape[1] * 8 / 128 == bits
