@@ -302,6 +302,25 @@ def scan_src_sha1():
     return hashlib.sha1(scan.encode()).hexdigest()
 
 
+def max_over_ranks(seconds: float, world: int, dev) -> float:
+    """The slowest rank's time (every rank calls this at the same point; a no-op for one
+    rank).  dev: the rank's device (a CUDA device under NCCL, the CPU under gloo)."""
+    if world <= 1:
+        return seconds
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([seconds], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, seconds: float) -> float:
+    """Whole-job throughput of the replicated step: every rank processes its own copy of the
+    workload, so the job attends world times the tokens of one rank in the slowest rank's
+    time."""
+    return tokens_per_rank * world / seconds
+
+
 def sha1_of(path):
     with open(path, "rb") as f:
         return hashlib.sha1(f.read()).hexdigest()
@@ -538,11 +557,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    elapsed = start.elapsed_time(stop) / 1000.0
-    if world > 1:
-        t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(start.elapsed_time(stop) / 1000.0, world, dev)
     # tokens attended in the timed steps: step i uses replica i % R whose prefix grew by one
     tokens = 0
     comp_now = list(comp_before)
@@ -550,8 +565,7 @@ def run_ours(args):
         r = i % R
         comp_now[r] += 1                 # the append inside the step grows the prefix first
         tokens += wl.B * comp_now[r]
-    tokens_all = tokens * world
-    value = tokens_all / elapsed
+    value = weak_scaling_value(tokens, world, elapsed)
     errs = sum(int(rep["err"].item()) for rep in reps)
     assert errs == 0, f"device error flag set: {errs}"
 
@@ -643,11 +657,7 @@ def run_ours(args):
             tok2 += wl.B * host_comp[r]
         e2.record()
         torch.cuda.synchronize()
-        t2 = s2.elapsed_time(e2) / 1000.0
-        if world > 1:
-            t = torch.tensor([t2], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t2 = float(t.item())
+        t2 = max_over_ranks(s2.elapsed_time(e2) / 1000.0, world, dev)
         h2d = n_in * 2
         d2h = n_out * 4
         e2e = {"value": tok2 * world / t2, "unit": UNIT, "h2d_bytes_per_step": h2d,

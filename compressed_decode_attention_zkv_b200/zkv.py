@@ -82,6 +82,13 @@ class AppendParams(ctypes.Structure):
                 ("max_pages", c_int64), ("n_pages", c_int64)]
 
 
+class MergeParams(ctypes.Structure):
+    _fields_ = [("n_parts", c_int64), ("rows", c_int64), ("d", c_int),
+                ("part_out", c_void_p), ("out_part_stride", c_int64), ("out_row_stride", c_int64),
+                ("part_lse", c_void_p), ("lse_part_stride", c_int64), ("lse_row_stride", c_int64),
+                ("out", c_void_p), ("lse", c_void_p)]
+
+
 _lib = None
 
 
@@ -110,6 +117,8 @@ def lib() -> ctypes.CDLL:
         L.zkv_rvq_decode_attn_noalloc.argtypes = [POINTER(DecodeParams), c_void_p]
         L.zkv_rvq_append.restype = c_int
         L.zkv_rvq_append.argtypes = [POINTER(AppendParams), c_void_p]
+        L.zkv_lse_merge.restype = c_int
+        L.zkv_lse_merge.argtypes = [POINTER(MergeParams), c_void_p]
         L.zkv_rvq_serve_step.restype = c_int
         L.zkv_rvq_serve_step.argtypes = [POINTER(AppendParams), POINTER(DecodeParams), c_void_p,
                                          c_size_t, c_void_p]
@@ -533,6 +542,35 @@ class PreparedDecode:
 # --------------------------------------------------------------------------------------------
 # A layer's compressed cache
 # --------------------------------------------------------------------------------------------
+
+def lse_merge(part_out: torch.Tensor, part_lse: torch.Tensor, out=None, lse=None):
+    """Log-sum-exp combine of N partial attentions over disjoint key sets (see include/zkv.h).
+    part_out float32 [N, ..., d] and part_lse float32 [N, ...] may be views (any part and row
+    strides, d contiguous; e.g. the two halves of a gathered [N, ..., d + 1] buffer of packed
+    rows).  Returns (out float32 [..., d], lse float32 [...])."""
+    _need(part_out, "part_out", torch.float32, contiguous=False)
+    _need(part_lse, "part_lse", torch.float32, contiguous=False)
+    N, d = part_out.shape[0], part_out.shape[-1]
+    lead = tuple(part_out.shape[1:-1])
+    if tuple(part_lse.shape) != (N,) + lead:
+        raise ValueError("part_lse must be [N, ...] matching part_out [N, ..., d]")
+    po = part_out.reshape(N, -1, d) if part_out.dim() != 3 else part_out
+    pl = part_lse.reshape(N, -1) if part_lse.dim() != 2 else part_lse
+    if po.stride(-1) != 1:
+        raise ValueError("part_out rows must be contiguous")
+    rows = po.shape[1]
+    if out is None:
+        out = torch.empty(lead + (d,), dtype=torch.float32, device=part_out.device)
+    if lse is None:
+        lse = torch.empty(lead, dtype=torch.float32, device=part_out.device)
+    _need(out, "out", torch.float32)
+    _need(lse, "lse", torch.float32)
+    p = MergeParams(n_parts=N, rows=rows, d=d, part_out=_ptr(po), out_part_stride=po.stride(0),
+                    out_row_stride=po.stride(1), part_lse=_ptr(pl), lse_part_stride=pl.stride(0),
+                    lse_row_stride=pl.stride(1), out=_ptr(out), lse=_ptr(lse))
+    _check("zkv_lse_merge", lib().zkv_lse_merge(ctypes.byref(p), _stream()))
+    return out, lse
+
 
 class RVQKVCache:
     """Compressed KV cache of one attention layer: RVQ codes for old tokens, an fp16 window for

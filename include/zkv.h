@@ -306,6 +306,34 @@ int zkv_rvq_append(const zkv_append_params* p, void* stream);
 int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_params* dp,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * zkv_lse_merge -- log-sum-exp combine of partial attention results over disjoint key sets
+ * (context-parallel decode: every rank attends over its shard of each compressed prefix, the
+ * shards' (out, lse) are gathered and combined).
+ * Passage: Differential-KV "Decode & Prefill Innovations" (fp32 log-sum-exp combine).
+ * For each row r:  M = max_i lse[i][r];  w_i = exp(lse[i][r] - M);  L = sum_i w_i;
+ *   out[r] = sum_i w_i part_out[i][r] / L;  lse_out[r] = M + log L   (float32)
+ * A part with lse = -inf (no keys) has weight 0; a row whose parts are all empty gets out = 0,
+ * lse = -inf.  Layouts (strides in floats): part_out element (i, r, e) at
+ * part_out[i * out_part_stride + r * out_row_stride + e]; part_lse element (i, r) at
+ * part_lse[i * lse_part_stride + r * lse_row_stride] (natural log, as zkv_rvq_decode_attn
+ * writes it) -- so a gathered [n_parts][rows][d + 1] buffer of packed (out, lse) rows is read in
+ * place; out float32 [rows][d] contiguous, lse [rows] (may be NULL).
+ * Errors: INVALID_ARG (n_parts < 1, d not in 1..4096, null pointers with rows > 0), CUDA.
+ */
+typedef struct {
+  int64_t n_parts, rows;
+  int d;
+  const float* part_out;
+  int64_t out_part_stride, out_row_stride;
+  const float* part_lse;
+  int64_t lse_part_stride, lse_row_stride;
+  float* out;
+  float* lse;
+} zkv_lse_merge_params;
+
+int zkv_lse_merge(const zkv_lse_merge_params* p, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

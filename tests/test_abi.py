@@ -159,6 +159,19 @@ def test_serve_step_validation(L, akw, dkw, status):
     assert L.zkv_rvq_serve_step(ctypes.byref(ap), ctypes.byref(dp), None, 0, None) == status
 
 
+def test_lse_merge_validation(L):
+    def mk(**kw):
+        base = dict(n_parts=2, rows=4, d=8, part_out=0x1000, out_part_stride=36, out_row_stride=9,
+                    part_lse=0x1020, lse_part_stride=36, lse_row_stride=9, out=0x3000, lse=0x4000)
+        base.update(kw)
+        return zkv.MergeParams(**base)
+    for kw in (dict(n_parts=0), dict(d=0), dict(d=5000), dict(rows=-1), dict(part_out=0),
+               dict(part_lse=0), dict(out=0)):
+        assert L.zkv_lse_merge(ctypes.byref(mk(**kw)), None) == zkv.ZKV_ERR_INVALID_ARG, kw
+    assert L.zkv_lse_merge(ctypes.byref(mk(rows=0)), None) == zkv.ZKV_OK   # nothing to do
+    assert L.zkv_lse_merge(None, None) == zkv.ZKV_ERR_INVALID_ARG
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 128, dtype=torch.float16)
@@ -175,7 +188,8 @@ def test_ctypes_structs_match_the_header_layout(tmp_path):
     if cc is None:
         pytest.skip("no C compiler")
     pairs = [("zkv_encode_params", zkv.EncodeParams), ("zkv_reconstruct_params", zkv.ReconstructParams),
-             ("zkv_decode_params", zkv.DecodeParams), ("zkv_append_params", zkv.AppendParams)]
+             ("zkv_decode_params", zkv.DecodeParams), ("zkv_append_params", zkv.AppendParams),
+             ("zkv_lse_merge_params", zkv.MergeParams)]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zkv.h"', "int main(void) {"]
     for cname, cls in pairs:
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
