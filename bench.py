@@ -369,6 +369,38 @@ def encode_extra(dev, hbm, bf16):
                     "exact decision: TF32-margin candidates re-scored in float32, then float64"}
 
 
+def pq_encode_extra(dev):
+    """Product-VQ (VecInfer) encode of the prefill_encode_64k keys (65536 tokens x 8 kv heads,
+    d = 128, sub-vectors of 4 with the smoothing factors): vectors/s."""
+    import torch
+
+    from compressed_decode_attention_zkv_b200 import inputs as I
+    from compressed_decode_attention_zkv_b200 import zkv
+    wl = I.workload("prefill_encode_64k")
+    m = 4
+    lam_np = I.key_smooth_factors(wl)
+    lam = torch.from_numpy(lam_np).to(dev)
+    book = torch.from_numpy(I.train_pq_codebook(wl, "k", m, smooth=lam_np)).to(dev)
+    x = torch.from_numpy(I.kv_tokens(wl, "k", 0, 0, wl.T)).to(dev).permute(1, 0, 2)   # [T, H, d]
+    codes = torch.empty((wl.T, wl.Hkv, wl.d // m), dtype=torch.uint8, device=dev)
+    zkv.pq_encode(x, book, codes=codes, smooth=lam)
+    torch.cuda.synchronize()
+    n_iter = 5
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(n_iter):
+        zkv.pq_encode(x, book, codes=codes, smooth=lam)
+    e.record()
+    torch.cuda.synchronize()
+    sec = s.elapsed_time(e) / 1000.0 / n_iter
+    rows = wl.T * wl.Hkv
+    return {"workload": "prefill_encode_64k keys (65536 tok x 8 kv heads, d=128), product VQ "
+                        "with 4-dim sub-vectors (2 bits/elem) and key smoothing",
+            "vectors_per_s": rows / sec, "ms_per_call": sec * 1000.0,
+            "fp64_gflops": 2.0 * rows * (wl.d // m) * 256 * m / sec / 1e9,
+            "note": "one warp per row; float64 distances to all 256 codewords of every sub-vector"}
+
+
 def paginate_replica(rep, P, seed):
     """Move a replica's codes into page pools [n_pages, Hkv, P, S] (pages shuffled through a
     pool with spare pages) and give it the block table."""
@@ -670,6 +702,11 @@ def run_ours(args):
     if not args.no_encode and rank == 0:
         del graphs, soak_graphs
         extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
+    if not args.no_encode and rank == 0:
+        try:
+            extras["pq_encode"] = pq_encode_extra(dev)
+        except Exception as exc:   # an extra never takes the main line down
+            extras["pq_encode"] = {"error": f"{type(exc).__name__}: {exc}"}
     base_ms = 1000.0 * elapsed / args.steps
     for name, kw, skip in (("smooth", dict(smooth=True), args.no_smooth),
                            ("paged", dict(page_tokens=256), args.no_paged)):

@@ -82,6 +82,15 @@ class AppendParams(ctypes.Structure):
                 ("max_pages", c_int64), ("n_pages", c_int64)]
 
 
+class PQEncodeParams(ctypes.Structure):
+    _fields_ = [("n_batch", c_int64), ("n_tok", c_int64), ("n_head", c_int64),
+                ("d", c_int), ("m", c_int), ("rotate", c_int), ("x_dtype", c_int),
+                ("x", c_void_p), ("x_sb", c_int64), ("x_st", c_int64), ("x_sh", c_int64),
+                ("codebook", c_void_p),
+                ("codes", c_void_p), ("c_sb", c_int64), ("c_st", c_int64), ("c_sh", c_int64),
+                ("smooth", c_void_p)]
+
+
 class MergeParams(ctypes.Structure):
     _fields_ = [("n_parts", c_int64), ("rows", c_int64), ("d", c_int),
                 ("part_out", c_void_p), ("out_part_stride", c_int64), ("out_row_stride", c_int64),
@@ -117,6 +126,8 @@ def lib() -> ctypes.CDLL:
         L.zkv_rvq_decode_attn_noalloc.argtypes = [POINTER(DecodeParams), c_void_p]
         L.zkv_rvq_append.restype = c_int
         L.zkv_rvq_append.argtypes = [POINTER(AppendParams), c_void_p]
+        L.zkv_pq_encode.restype = c_int
+        L.zkv_pq_encode.argtypes = [POINTER(PQEncodeParams), c_void_p]
         L.zkv_lse_merge.restype = c_int
         L.zkv_lse_merge.argtypes = [POINTER(MergeParams), c_void_p]
         L.zkv_rvq_serve_step.restype = c_int
@@ -542,6 +553,41 @@ class PreparedDecode:
 # --------------------------------------------------------------------------------------------
 # A layer's compressed cache
 # --------------------------------------------------------------------------------------------
+
+def pq_encode(x: torch.Tensor, codebook: torch.Tensor, codes: torch.Tensor | None = None,
+              rotate: bool = True, smooth: torch.Tensor | None = None) -> torch.Tensor:
+    """Product VQ (VecInfer) of x rows.  x: [B, T, H, d] view (any strides, d contiguous), or
+    [T, H, d], or [N, d] (one head).  codebook: [H, 256, m] float32 contiguous (shared by the d/m
+    sub-vectors of a head).  smooth: optional [H, d] key smoothing factors.
+    Returns codes uint8 [B, T, H, d/m] (a view when ``codes`` is given)."""
+    if x.dtype not in (torch.float16, torch.float32):
+        raise TypeError("x must be fp16 or fp32")
+    _need(x, "x", x.dtype, contiguous=False)
+    _need(codebook, "codebook", torch.float32)
+    x4 = _as4(x, "x")
+    if x4.stride(-1) != 1:
+        raise ValueError("x rows must be contiguous")
+    Bn, T, H, d = x4.shape
+    if codebook.dim() != 3 or codebook.shape[0] != H or codebook.shape[1] != CODEBOOK_SIZE:
+        raise ValueError(f"codebook must be [H={H}, 256, m], got {tuple(codebook.shape)}")
+    m = codebook.shape[2]
+    if d % m:
+        raise ValueError("d must be a multiple of the sub-vector size")
+    if codes is None:
+        codes = torch.empty((Bn, T, H, d // m), dtype=torch.uint8, device=x.device)
+    _need(codes, "codes", torch.uint8, contiguous=False)
+    c4 = _as4(codes, "codes")
+    if c4.shape != (Bn, T, H, d // m) or c4.stride(-1) != 1:
+        raise ValueError("codes must be a [B, T, H, d/m] view with contiguous sub-vector codes")
+    p = PQEncodeParams(n_batch=Bn, n_tok=T, n_head=H, d=d, m=m, rotate=int(bool(rotate)),
+                       x_dtype=ZKV_DTYPE_F16 if x.dtype == torch.float16 else ZKV_DTYPE_F32,
+                       x=_ptr(x4), x_sb=x4.stride(0), x_st=x4.stride(1), x_sh=x4.stride(2),
+                       codebook=_ptr(codebook), codes=_ptr(c4), c_sb=c4.stride(0),
+                       c_st=c4.stride(1), c_sh=c4.stride(2),
+                       smooth=_smooth_ptr(smooth, H, d, "smooth"))
+    _check("zkv_pq_encode", lib().zkv_pq_encode(ctypes.byref(p), _stream()))
+    return codes
+
 
 def lse_merge(part_out: torch.Tensor, part_lse: torch.Tensor, out=None, lse=None):
     """Log-sum-exp combine of N partial attentions over disjoint key sets (see include/zkv.h).

@@ -307,6 +307,34 @@ int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_params* dp,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * zkv_pq_encode -- product vector quantisation of KV head vectors (VecInfer).
+ * Passage: VeloxQuant "VecInfer" (smooth scaling + Walsh-Hadamard dual transform, then a
+ * pre-trained K-means codebook over sub-vectors; key_sub_dim 4 or 8 with 8-bit codes).
+ * Rows are addressed as in zkv_rvq_encode.  For each row:
+ *   y = rotate ? float32(H_d (x / lambda) / sqrt(d)) : x / lambda   (lambda = smooth, or 1)
+ *   z_j = argmin_c ||y[j m : (j+1) m] - C[h][c]||^2 for j < d / m  (float64, ties -> lowest c)
+ * Layouts: x as in zkv_rvq_encode; codebook float32 [n_head][256][m] (one codebook per head,
+ * shared by the sub-vectors); codes uint8, code j of (b,t,h) at
+ * codes[b*c_sb + t*c_st + h*c_sh + j] (d / m contiguous bytes); smooth float32 [n_head][d] or
+ * NULL.  d in {64, 128, 256}, m in {2, 4, 8, 16}.
+ * Errors: INVALID_ARG, UNSUPPORTED (d, m), CUDA.
+ */
+typedef struct {
+  int64_t n_batch, n_tok, n_head;
+  int d, m;
+  int rotate;
+  int x_dtype;
+  const void* x;
+  int64_t x_sb, x_st, x_sh;
+  const float* codebook;
+  uint8_t* codes;
+  int64_t c_sb, c_st, c_sh;
+  const float* smooth;
+} zkv_pq_encode_params;
+
+int zkv_pq_encode(const zkv_pq_encode_params* p, void* stream);
+
+/*
  * zkv_lse_merge -- log-sum-exp combine of partial attention results over disjoint key sets
  * (context-parallel decode: every rank attends over its shard of each compressed prefix, the
  * shards' (out, lse) are gathered and combined).

@@ -397,6 +397,28 @@ def pq_encode(x: np.ndarray, codebook: np.ndarray, smooth=None, rotate: bool = T
     return z.reshape(n, d // m).astype(np.uint8), y
 
 
+def pq_match_walk(x: np.ndarray, codebook: np.ndarray, codes: np.ndarray, rel_gap: float = 1e-5,
+                  smooth=None, rotate: bool = True) -> dict:
+    """Check candidate product-VQ codes sub-vector by sub-vector: equal to the float64 argmin,
+    or a counted near-tie (distance within ``rel_gap`` relative of the minimum), else a
+    mismatch.  Returns counts and the first few mismatches (row, sub-vector, code, oracle)."""
+    z, y = pq_encode(x, codebook, smooth=smooth, rotate=rotate)
+    C = np.asarray(codebook, F32)
+    m = C.shape[1]
+    sub = y.reshape(-1, m)
+    D = stage_distances(sub, C)
+    cand = np.asarray(codes).reshape(-1).astype(np.int64)
+    rows = np.arange(sub.shape[0])
+    dz, db = D[rows, cand], D[rows, z.reshape(-1).astype(np.int64)]
+    same = cand == z.reshape(-1)
+    near = (~same) & ((dz - db) <= rel_gap * db)
+    wrong = (~same) & (~near)
+    bad = [(int(i) // (y.shape[1] // m), int(i) % (y.shape[1] // m), int(cand[i]),
+            int(z.reshape(-1)[i])) for i in np.nonzero(wrong)[0][:8]]
+    return {"exact": int(same.sum()), "exceptions": int(near.sum()),
+            "mismatches": int(wrong.sum()), "bad": bad}
+
+
 def pq_reconstruct(codes: np.ndarray, codebook: np.ndarray, unrotate: bool = False) -> np.ndarray:
     """y_hat = concatenation of C[z_j] over the sub-vectors (float64), or (1/sqrt(d)) H y_hat."""
     C = np.asarray(codebook, F64)

@@ -159,6 +159,21 @@ def test_serve_step_validation(L, akw, dkw, status):
     assert L.zkv_rvq_serve_step(ctypes.byref(ap), ctypes.byref(dp), None, 0, None) == status
 
 
+def test_pq_encode_validation(L):
+    def mk(**kw):
+        base = dict(n_batch=1, n_tok=4, n_head=1, d=128, m=4, rotate=1, x_dtype=0, x=0x1000,
+                    codebook=0x2000, codes=0x3000)
+        base.update(kw)
+        return zkv.PQEncodeParams(**base)
+    for kw, st in ((dict(m=3), zkv.ZKV_ERR_UNSUPPORTED), (dict(m=32), zkv.ZKV_ERR_UNSUPPORTED),
+                   (dict(d=96), zkv.ZKV_ERR_UNSUPPORTED), (dict(x_dtype=7), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(x=0), zkv.ZKV_ERR_INVALID_ARG), (dict(codes=0), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(x=0x1002), zkv.ZKV_ERR_INVALID_ARG), (dict(n_tok=-1), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(n_tok=0), zkv.ZKV_OK)):
+        assert L.zkv_pq_encode(ctypes.byref(mk(**kw)), None) == st, kw
+    assert L.zkv_pq_encode(None, None) == zkv.ZKV_ERR_INVALID_ARG
+
+
 def test_lse_merge_validation(L):
     def mk(**kw):
         base = dict(n_parts=2, rows=4, d=8, part_out=0x1000, out_part_stride=36, out_row_stride=9,
@@ -189,7 +204,7 @@ def test_ctypes_structs_match_the_header_layout(tmp_path):
         pytest.skip("no C compiler")
     pairs = [("zkv_encode_params", zkv.EncodeParams), ("zkv_reconstruct_params", zkv.ReconstructParams),
              ("zkv_decode_params", zkv.DecodeParams), ("zkv_append_params", zkv.AppendParams),
-             ("zkv_lse_merge_params", zkv.MergeParams)]
+             ("zkv_lse_merge_params", zkv.MergeParams), ("zkv_pq_encode_params", zkv.PQEncodeParams)]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zkv.h"', "int main(void) {"]
     for cname, cls in pairs:
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
