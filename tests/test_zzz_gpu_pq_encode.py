@@ -1,6 +1,8 @@
 """GPU parity of the product-VQ (VecInfer) encode against the oracle: codes equal to the
 float64 argmin of every sub-vector except counted near-ties (distance gap below 1e-5
-relative), with and without key smoothing, every head dimension and several sub-vector sizes."""
+relative), with and without key smoothing, every head dimension and several sub-vector sizes.
+The file name keeps it after every other GPU test in collection order, so that under
+``pytest -x`` a failure here cannot hide the results of the established paths."""
 import numpy as np
 import pytest
 import torch
