@@ -401,6 +401,52 @@ def pq_encode_extra(dev):
             "note": "one warp per row; float64 distances to all 256 codewords of every sub-vector"}
 
 
+def pq_decode_extra(dev, hbm_peak):
+    """Product-VQ decode (4-dim sub-vectors, 2 bits/elem on K and V) on the llama3_8b_32k shape:
+    seeded codes and codebooks, 2 rotating replicas (268 MB > L2), CUDA-event timed calls."""
+    import torch
+
+    from compressed_decode_attention_zkv_b200 import inputs as I
+    from compressed_decode_attention_zkv_b200 import zkv
+    wl = I.workload(WORKLOAD)
+    m, R = 4, 2
+    Tc, nsub = wl.Tc, wl.d // m
+    g = torch.Generator(device=dev).manual_seed(11)
+    reps = []
+    for r in range(R):
+        kc = torch.randint(0, 256, (wl.B, wl.Hkv, Tc, nsub), dtype=torch.uint8, device=dev, generator=g)
+        vc = torch.randint(0, 256, (wl.B, wl.Hkv, Tc, nsub), dtype=torch.uint8, device=dev, generator=g)
+        Ck = torch.randn((wl.Hkv, 256, m), device=dev, generator=g) * 0.25
+        Cv = torch.randn((wl.Hkv, 256, m), device=dev, generator=g)
+        q = torch.randn((wl.B, wl.Hq, wl.d), device=dev, generator=g).half()
+        wk = torch.randn((wl.B, wl.Hkv, wl.W, wl.d), device=dev, generator=g).half()
+        wv = torch.randn((wl.B, wl.Hkv, wl.W, wl.d), device=dev, generator=g).half()
+        comp = torch.full((wl.B,), Tc, dtype=torch.int32, device=dev)
+        win = torch.full((wl.B,), wl.W, dtype=torch.int32, device=dev)
+        reps.append((q, kc, vc, comp, Ck, Cv, wk, wv, win))
+    ws = torch.empty(zkv.pq_decode_workspace_size(reps[0][0], reps[0][1], reps[0][4], reps[0][6]),
+                     dtype=torch.uint8, device=dev)
+    outs = [zkv.pq_decode_attn(*rp, workspace=ws) for rp in reps]   # warm-up, kernel attributes
+    torch.cuda.synchronize()
+    steps = 100
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        rp = reps[i % R]
+        zkv.pq_decode_attn(*rp, out=outs[i % R][0], lse=outs[i % R][1], workspace=ws)
+    e.record()
+    torch.cuda.synchronize()
+    sec = s.elapsed_time(e) / 1000.0 / steps
+    code_bytes = 2 * wl.B * wl.Hkv * Tc * nsub
+    byts = code_bytes + 2 * wl.B * wl.Hkv * wl.W * wl.d * 2 + wl.B * wl.Hq * wl.d * (2 + 4)
+    return {"workload": f"{wl.name} shape, product VQ with 4-dim sub-vectors on K and V "
+                        "(2 bits/elem, 64 code bytes per token and kv head)",
+            "value": wl.B * Tc / sec, "unit": UNIT, "us_per_call": sec * 1e6,
+            "hbm_gbs": byts / sec / 1e9, "hbm_frac": byts / sec / 1e9 / hbm_peak,
+            "note": "zkv_pq_decode_attn (lane = sub-vector scan + finalize), eager calls over "
+                    f"{R} rotating replicas"}
+
+
 def paginate_replica(rep, P, seed):
     """Move a replica's codes into page pools [n_pages, Hkv, P, S] (pages shuffled through a
     pool with spare pages) and give it the block table."""
@@ -707,6 +753,11 @@ def run_ours(args):
             extras["pq_encode"] = pq_encode_extra(dev)
         except Exception as exc:   # an extra never takes the main line down
             extras["pq_encode"] = {"error": f"{type(exc).__name__}: {exc}"}
+    if not args.no_encode and rank == 0:
+        try:
+            extras["pq_decode"] = pq_decode_extra(dev, hbm_peak)
+        except Exception as exc:   # an extra never takes the main line down
+            extras["pq_decode"] = {"error": f"{type(exc).__name__}: {exc}"}
     base_ms = 1000.0 * elapsed / args.steps
     for name, kw, skip in (("smooth", dict(smooth=True), args.no_smooth),
                            ("paged", dict(page_tokens=256), args.no_paged)):

@@ -1414,6 +1414,259 @@ __global__ void __launch_bounds__(256) finalize_kernel(DecodeArgs a) {
 }
 
 // ------------------------------------------------------------------------------------------
+// 4. Product-VQ decode (VeloxQuant "VecInfer": keys and values quantised by sub-vectors
+//    against one shared 256-entry codebook per kv head).  With d / m = 32 sub-vectors a warp's
+//    lane j owns sub-vector j of every token: it gathers Ck[zk_j] and Cv[zv_j] from shared
+//    memory, forms its partial scores for the GP heads, and the partial scores of TB = 32 / GP
+//    tokens are reduced together by one transpose-sum (after it lane L holds the score of
+//    token L / GP, head L % GP).  Per head the warp keeps a running maximum; each lane
+//    accumulates p * Cv[zv_j] into its m output dims in registers.  No histograms.
+//    pq_scan_kernel:     grid (chunks of kPqChunk tokens, pairs); chunk partials -> workspace.
+//    pq_finalize_kernel: per pair, the window attention (beside nothing: it is the last kernel),
+//                        the log-sum-exp combine of the chunks, rotation back, merge with the
+//                        window.
+// ------------------------------------------------------------------------------------------
+constexpr int kPqChunk = 2048;   // tokens per scan CTA
+
+struct PqArgs {
+  int B, Hq, Hkv, G, d, m, n_chunks;
+  int64_t Tcap, max_comp;
+  float scale_log2;
+  double rot;
+  const __half* q;
+  const uint8_t* k_codes;   // [B][Hkv][Tcap][d/m]
+  const uint8_t* v_codes;
+  const int32_t* comp_len;
+  const float* Ck;          // [Hkv][256][m]
+  const float* Cv;
+  const float* k_smooth;    // [Hkv][d] or null
+  int32_t* err;
+  float* cm;                // [pairs][n_chunks][GP] chunk maxima (log2 units)
+  float* cl;                // [pairs][n_chunks][GP] chunk sums of p
+  float* co;                // [pairs][n_chunks][GP][d] chunk sums of p * v (rotated domain)
+};
+
+template <int D, int M, int GP>
+__global__ void __launch_bounds__(256) pq_scan_kernel(PqArgs a) {
+  constexpr int NSUB = D / M;
+  static_assert(NSUB == 32, "one sub-vector per lane");
+  constexpr int TB = 32 / GP;        // tokens per transpose-sum batch
+  constexpr int E = D / 32;
+  __shared__ __align__(16) float ck[kCodebook * M];
+  __shared__ __align__(16) float cv[kCodebook * M];
+  __shared__ __align__(16) float qs[GP][D];
+  __shared__ float wm[8][GP], wl[8][GP];
+  __shared__ __align__(16) float wo[8][GP][D];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int chunk = blockIdx.x;
+  const int64_t pair = blockIdx.y;
+  const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
+  for (int f = tid; f < kCodebook * M; f += 256) {
+    ck[f] = a.Ck[(size_t)kvh * kCodebook * M + f];
+    cv[f] = a.Cv[(size_t)kvh * kCodebook * M + f];
+  }
+  if (warp < GP) {   // q_tilde of head g = warp: H (lambda * q) / sqrt(d), float32
+    float v[E];
+    const int g = warp;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float x = 0.f;
+      if (g < a.G) {
+        x = __half2float(a.q[((int64_t)b * a.Hq + (int64_t)kvh * a.G + g) * D + e * 32 + lane]);
+        if (a.k_smooth) x *= a.k_smooth[(int64_t)kvh * D + e * 32 + lane];
+      }
+      v[e] = x;
+    }
+    fwht_warp_f32<D>(v, lane);
+    const float rs = (float)a.rot;
+#pragma unroll
+    for (int e = 0; e < E; ++e) qs[g][e * 32 + lane] = v[e] * rs;
+  }
+  __syncthreads();
+  int64_t c = a.comp_len[b];
+  if (c < 0 || c > a.Tcap) c = c < 0 ? 0 : a.Tcap;   // (the finalize reports it)
+  c = c < a.max_comp ? c : a.max_comp;
+  const int64_t t0 = (int64_t)chunk * kPqChunk;
+  const int64_t t1 = t0 + kPqChunk < c ? t0 + kPqChunk : c;
+  const int64_t n = t1 > t0 ? t1 - t0 : 0;
+  // warp w takes the contiguous run [w0, w1) of the chunk
+  const int64_t per = (n + 7) / 8;
+  const int64_t w0 = t0 + warp * per < t1 ? t0 + warp * per : t1;
+  const int64_t w1 = w0 + per < t1 ? w0 + per : t1;
+  float qr[GP][M];
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int i = 0; i < M; ++i) qr[g][i] = qs[g][lane * M + i];
+  const uint8_t* kz = a.k_codes + (pair * a.Tcap) * NSUB + lane;
+  const uint8_t* vz = a.v_codes + (pair * a.Tcap) * NSUB + lane;
+  float mrun[GP], acc[GP][M];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    mrun[g] = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < M; ++i) acc[g][i] = 0.f;
+  }
+  float lp = 0.f;   // this lane's share of the sum of p of head lane % GP
+  const int gl = lane % GP;
+  for (int64_t base = w0; base < w1; base += TB) {
+    const int nv = (int)(w1 - base < TB ? w1 - base : TB);
+    float x[32];
+#pragma unroll
+    for (int u = 0; u < TB; ++u) {
+      float kv[M];
+      if (u < nv) {
+        const int z = kz[(base + u) * NSUB];
+#pragma unroll
+        for (int i = 0; i < M; ++i) kv[i] = ck[z * M + i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < M; ++i) kv[i] = 0.f;
+      }
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < M; ++i) s = fmaf(qr[g][i], kv[i], s);
+        x[u * GP + g] = s;
+      }
+    }
+    int hidx = 0;
+    float sc = TransposeSum<32, 32, 16>::run(x, lane, hidx) * a.scale_log2;   // hidx == lane
+    const bool ok = lane / GP < nv;
+    if (!ok) sc = -INFINITY;
+    float bm = sc;   // batch maximum of head lane % GP
+#pragma unroll
+    for (int o = GP; o < 32; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+    float alpha_l = 1.f, mnew_l = 0.f;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float mb = __shfl_sync(0xffffffffu, bm, g);
+      const float mn = fmaxf(mrun[g], mb);
+      const float alpha = mrun[g] == -INFINITY ? 0.f : ex2_approx(mrun[g] - mn);
+#pragma unroll
+      for (int i = 0; i < M; ++i) acc[g][i] *= alpha;
+      if (g == gl) {
+        alpha_l = alpha;
+        mnew_l = mn;
+      }
+      mrun[g] = mn;
+    }
+    const float p = ok ? ex2_approx(sc - mnew_l) : 0.f;
+    lp = lp * alpha_l + p;
+#pragma unroll
+    for (int u = 0; u < TB; ++u) {
+      if (u < nv) {
+        const int z = vz[(base + u) * NSUB];
+        float vv[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) vv[i] = cv[z * M + i];
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float pg = __shfl_sync(0xffffffffu, p, u * GP + g);
+#pragma unroll
+          for (int i = 0; i < M; ++i) acc[g][i] = fmaf(pg, vv[i], acc[g][i]);
+        }
+      }
+    }
+  }
+  // warp partials: per head the sum of p over the lanes of that head
+#pragma unroll
+  for (int o = GP; o < 32; o <<= 1) lp += __shfl_xor_sync(0xffffffffu, lp, o);
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float l = __shfl_sync(0xffffffffu, lp, g);
+    if (lane == 0) {
+      wm[warp][g] = mrun[g];
+      wl[warp][g] = l;
+    }
+#pragma unroll
+    for (int i = 0; i < M; ++i) wo[warp][g][lane * M + i] = acc[g][i];
+  }
+  __syncthreads();
+  // combine the 8 warps: weight 2^(m_w - M*) (0 for a warp without tokens)
+  const int64_t slot = pair * a.n_chunks + chunk;
+  for (int f = tid; f < GP * D; f += 256) {
+    const int g = f / D, e = f % D;
+    float ms = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) ms = fmaxf(ms, wm[w][g]);
+    float o = 0.f, l = 0.f;
+    if (ms != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const float wt = wm[w][g] == -INFINITY ? 0.f : ex2_approx(wm[w][g] - ms);
+        o = fmaf(wt, wo[w][g][e], o);
+        l = fmaf(wt, wl[w][g], l);
+      }
+    }
+    a.co[(slot * GP + g) * D + e] = o;
+    if (e == 0) {
+      a.cm[slot * GP + g] = ms;
+      a.cl[slot * GP + g] = l;
+    }
+  }
+}
+
+template <int D, int GP>
+__global__ void __launch_bounds__(256) pq_finalize_kernel(PqArgs a, DecodeArgs w) {
+  constexpr int E = D / 32;
+  extern __shared__ __align__(16) unsigned char win_smem[];
+  __shared__ __align__(16) float oc[GP * D];
+  __shared__ float ms_s[GP], ls_s[GP];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t pair = blockIdx.x;
+  const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
+  window_item<D, GP>(w, b, kvh, win_smem);
+  if (tid == 0) {
+    const int64_t c = a.comp_len[b];
+    if (c < 0 || c > a.Tcap) set_error(a.err, ZKV_DEVERR_COMP_LEN);
+  }
+  const int64_t s0 = pair * a.n_chunks;
+  for (int f = tid; f < GP * D; f += 256) {
+    const int g = f / D, e = f % D;
+    float m = -INFINITY;
+    for (int k = 0; k < a.n_chunks; ++k) m = fmaxf(m, a.cm[(s0 + k) * GP + g]);
+    float o = 0.f, l = 0.f;
+    if (m != -INFINITY) {
+      for (int k = 0; k < a.n_chunks; ++k) {
+        const float cmk = a.cm[(s0 + k) * GP + g];
+        const float wt = cmk == -INFINITY ? 0.f : ex2_approx(cmk - m);
+        o = fmaf(wt, a.co[((s0 + k) * GP + g) * D + e], o);
+        l = fmaf(wt, a.cl[(s0 + k) * GP + g], l);
+      }
+    }
+    oc[f] = o;
+    if (e == 0) {
+      ms_s[g] = m;
+      ls_s[g] = l;
+    }
+  }
+  __syncthreads();   // chunk combine and this block's window terms are visible
+  for (int g = warp; g < a.G; g += 8) {
+    const float mc = ms_s[g], lc = ls_s[g];
+    double v[E];   // the compressed part's sum of p * v, rotated back
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[q] = (double)oc[g * D + q * 32 + lane];
+    fwht_warp_f64<D>(v, lane);
+    const float mw = w.wm[pair * GP + g], lw = w.wl[pair * GP + g];
+    const float M = fmaxf(mc, mw);
+    const float wc = (mc == -INFINITY) ? 0.f : ex2_approx(mc - M);
+    const float ww = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+    const float L = wc * lc + ww * lw;
+    const int64_t h = (int64_t)kvh * a.G + g;
+    float* o = w.out + ((int64_t)b * a.Hq + h) * D;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+      const int i = q * 32 + lane;
+      o[i] = (wc * (float)(v[q] * a.rot) + ww * w.wo[(pair * GP + g) * D + i]) * inv;
+    }
+    if (lane == 0 && w.lse) w.lse[(int64_t)b * a.Hq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 // Launch
 // ------------------------------------------------------------------------------------------
 static inline void trace(void* const* ev, int i, cudaStream_t st) {
@@ -1630,6 +1883,125 @@ extern "C" int zkv_rvq_serve_step(const zkv_append_params* ap, const zkv_decode_
                            ap->n_pages != dp->n_pages)))
     return ZKV_ERR_INVALID_ARG;
   return decode_common(dp, workspace, workspace_bytes, stream, ap);
+}
+
+namespace zkv {
+// ------------------------------------------------------------------------------------------
+// Product-VQ decode: validation, workspace, launch.
+// ------------------------------------------------------------------------------------------
+struct PqPlan {
+  int G, GP, n_chunks;
+  size_t off_cm, off_cl, off_co, off_wm, off_wl, off_wo, total;
+};
+
+static bool pq_shape_supported(int d, int m, int GP) {
+  if (d == 64) return m == 2;
+  if (d == 128) return m == 4;
+  if (d == 256) return m == 8 && GP <= 2;   // shared memory of the scan's warp partials
+  return false;
+}
+
+static int validate_pq_shapes(const zkv_pq_decode_params* p) {
+  if (!p) return ZKV_ERR_INVALID_ARG;
+  if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->Hq % p->Hkv) return ZKV_ERR_INVALID_ARG;
+  if (p->Hq / p->Hkv > 8) return ZKV_ERR_UNSUPPORTED;
+  if (!pq_shape_supported(p->d, p->m, pad_heads(p->Hq / p->Hkv))) return ZKV_ERR_UNSUPPORTED;
+  if (p->B > 65535 || p->Hkv > 65535 || (int64_t)p->B * p->Hkv > 65535) return ZKV_ERR_UNSUPPORTED;
+  if (p->Tcap < 0 || p->Wcap < 0 || p->max_comp_len < 0 || p->max_comp_len > p->Tcap)
+    return ZKV_ERR_INVALID_ARG;
+  if (p->Tcap > (int64_t(1) << 28)) return ZKV_ERR_UNSUPPORTED;
+  return ZKV_OK;
+}
+
+static PqPlan make_pq_plan(const zkv_pq_decode_params* p) {
+  PqPlan pl{};
+  pl.G = p->Hq / p->Hkv;
+  pl.GP = pad_heads(pl.G);
+  pl.n_chunks = (int)std::max<int64_t>(1, (p->max_comp_len + kPqChunk - 1) / kPqChunk);
+  const size_t pairs = (size_t)p->B * p->Hkv, f = sizeof(float);
+  size_t o = 0;
+  pl.off_cm = o; o = align256(o + pairs * pl.n_chunks * pl.GP * f);
+  pl.off_cl = o; o = align256(o + pairs * pl.n_chunks * pl.GP * f);
+  pl.off_co = o; o = align256(o + pairs * pl.n_chunks * pl.GP * p->d * f);
+  pl.off_wm = o; o = align256(o + pairs * pl.GP * f);
+  pl.off_wl = o; o = align256(o + pairs * pl.GP * f);
+  pl.off_wo = o; o = align256(o + pairs * pl.GP * p->d * f);
+  pl.total = o;
+  return pl;
+}
+
+template <int D, int M, int GP>
+static int launch_pq(const PqArgs& a, const DecodeArgs& w, cudaStream_t st) {
+  const int pairs = a.B * a.Hkv;
+  pq_scan_kernel<D, M, GP><<<dim3((unsigned)a.n_chunks, (unsigned)pairs), 256, 0, st>>>(a);
+  ZKV_CHECK_LAUNCH();
+  const size_t fsmem = window_smem_bytes<D, GP>();
+  if (ensure_smem_limit(pq_finalize_kernel<D, GP>, fsmem) != cudaSuccess) return ZKV_ERR_CUDA;
+  pq_finalize_kernel<D, GP><<<(unsigned)pairs, 256, fsmem, st>>>(a, w);
+  ZKV_CHECK_LAUNCH();
+  return ZKV_OK;
+}
+
+template <int D, int M>
+static int launch_pq_g(int GP, const PqArgs& a, const DecodeArgs& w, cudaStream_t st) {
+  switch (GP) {
+    case 1: return launch_pq<D, M, 1>(a, w, st);
+    case 2: return launch_pq<D, M, 2>(a, w, st);
+    case 4: if constexpr (D <= 128) return launch_pq<D, M, 4>(a, w, st); else return ZKV_ERR_UNSUPPORTED;
+    default: if constexpr (D <= 128) return launch_pq<D, M, 8>(a, w, st); else return ZKV_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace zkv
+
+extern "C" size_t zkv_pq_decode_workspace_size(const zkv_pq_decode_params* p) {
+  if (validate_pq_shapes(p) != ZKV_OK) return 0;
+  return make_pq_plan(p).total;
+}
+
+extern "C" int zkv_pq_decode_attn(const zkv_pq_decode_params* p, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  const int v = validate_pq_shapes(p);
+  if (v != ZKV_OK) return v;
+  if (!p->q || !p->comp_len || !p->win_len || !p->out || !p->k_codes || !p->v_codes ||
+      !p->k_codebook || !p->v_codebook)
+    return ZKV_ERR_INVALID_ARG;
+  if (p->Wcap > 0 && (!p->win_k || !p->win_v)) return ZKV_ERR_INVALID_ARG;
+  if (((uintptr_t)p->q | (uintptr_t)p->win_k | (uintptr_t)p->win_v) & 15) return ZKV_ERR_INVALID_ARG;
+  const PqPlan pl = make_pq_plan(p);
+  if (!workspace || workspace_bytes < pl.total || ((uintptr_t)workspace & 255))
+    return ZKV_ERR_WORKSPACE;
+  unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : (float)(1.0 / std::sqrt((double)p->d));
+  PqArgs a{};
+  a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = pl.G; a.d = p->d; a.m = p->m;
+  a.n_chunks = pl.n_chunks; a.Tcap = p->Tcap; a.max_comp = p->max_comp_len;
+  a.scale_log2 = scale * kLog2e;
+  a.rot = 1.0 / std::sqrt((double)p->d);
+  a.q = reinterpret_cast<const __half*>(p->q);
+  a.k_codes = p->k_codes; a.v_codes = p->v_codes; a.comp_len = p->comp_len;
+  a.Ck = p->k_codebook; a.Cv = p->v_codebook; a.k_smooth = p->k_smooth; a.err = p->error_flag;
+  a.cm = reinterpret_cast<float*>(ws + pl.off_cm);
+  a.cl = reinterpret_cast<float*>(ws + pl.off_cl);
+  a.co = reinterpret_cast<float*>(ws + pl.off_co);
+  // the window attention and the output go through the decode's own argument block
+  DecodeArgs w{};
+  w.B = p->B; w.Hq = p->Hq; w.Hkv = p->Hkv; w.G = pl.G; w.d = p->d;
+  w.Wcap = p->Wcap; w.Tcap = p->Tcap;
+  w.scale_log2 = a.scale_log2; w.rot = a.rot;
+  w.q = a.q;
+  w.win_k = reinterpret_cast<const __half*>(p->win_k);
+  w.win_v = reinterpret_cast<const __half*>(p->win_v);
+  w.win_len = p->win_len; w.out = p->out; w.lse = p->lse; w.err = p->error_flag;
+  w.wm = reinterpret_cast<float*>(ws + pl.off_wm);
+  w.wl = reinterpret_cast<float*>(ws + pl.off_wl);
+  w.wo = reinterpret_cast<float*>(ws + pl.off_wo);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  switch (p->d) {
+    case 64: return launch_pq_g<64, 2>(pl.GP, a, w, st);
+    case 128: return launch_pq_g<128, 4>(pl.GP, a, w, st);
+    default: return launch_pq_g<256, 8>(pl.GP, a, w, st);
+  }
 }
 
 // ------------------------------------------------------------------------------------------

@@ -91,6 +91,17 @@ class PQEncodeParams(ctypes.Structure):
                 ("smooth", c_void_p)]
 
 
+class PQDecodeParams(ctypes.Structure):
+    _fields_ = [("B", c_int), ("Hq", c_int), ("Hkv", c_int), ("d", c_int), ("m", c_int),
+                ("Tcap", c_int64), ("Wcap", c_int64), ("max_comp_len", c_int64),
+                ("softmax_scale", c_float),
+                ("q", c_void_p), ("k_codes", c_void_p), ("v_codes", c_void_p),
+                ("comp_len", c_void_p), ("k_codebook", c_void_p), ("v_codebook", c_void_p),
+                ("win_k", c_void_p), ("win_v", c_void_p), ("win_len", c_void_p),
+                ("out", c_void_p), ("lse", c_void_p), ("error_flag", c_void_p),
+                ("k_smooth", c_void_p)]
+
+
 class MergeParams(ctypes.Structure):
     _fields_ = [("n_parts", c_int64), ("rows", c_int64), ("d", c_int),
                 ("part_out", c_void_p), ("out_part_stride", c_int64), ("out_row_stride", c_int64),
@@ -128,6 +139,10 @@ def lib() -> ctypes.CDLL:
         L.zkv_rvq_append.argtypes = [POINTER(AppendParams), c_void_p]
         L.zkv_pq_encode.restype = c_int
         L.zkv_pq_encode.argtypes = [POINTER(PQEncodeParams), c_void_p]
+        L.zkv_pq_decode_workspace_size.restype = c_size_t
+        L.zkv_pq_decode_workspace_size.argtypes = [POINTER(PQDecodeParams)]
+        L.zkv_pq_decode_attn.restype = c_int
+        L.zkv_pq_decode_attn.argtypes = [POINTER(PQDecodeParams), c_void_p, c_size_t, c_void_p]
         L.zkv_lse_merge.restype = c_int
         L.zkv_lse_merge.argtypes = [POINTER(MergeParams), c_void_p]
         L.zkv_rvq_serve_step.restype = c_int
@@ -587,6 +602,69 @@ def pq_encode(x: torch.Tensor, codebook: torch.Tensor, codes: torch.Tensor | Non
                        smooth=_smooth_ptr(smooth, H, d, "smooth"))
     _check("zkv_pq_encode", lib().zkv_pq_encode(ctypes.byref(p), _stream()))
     return codes
+
+
+def pq_decode_workspace_size(q, k_codes, k_codebook, win_k, max_comp_len=None) -> int:
+    """Bytes of device workspace zkv_pq_decode_attn needs for these shapes (see include/zkv.h);
+    pass a buffer of this size as ``workspace`` to keep allocation out of a timed loop."""
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, _ = k_codes.shape
+    p = PQDecodeParams(B=B, Hq=Hq, Hkv=Hkv, d=d, m=k_codebook.shape[-1], Tcap=Tcap,
+                       Wcap=win_k.shape[2],
+                       max_comp_len=Tcap if max_comp_len is None else int(max_comp_len))
+    need = lib().zkv_pq_decode_workspace_size(ctypes.byref(p))
+    if need == 0:
+        raise ZkvError("zkv_pq_decode_workspace_size", ZKV_ERR_UNSUPPORTED)
+    return int(need)
+
+
+def pq_decode_attn(q, k_codes, v_codes, comp_len, k_codebook, v_codebook, win_k, win_v, win_len,
+                   out=None, lse=None, max_comp_len=None, softmax_scale=None,
+                   workspace: torch.Tensor | None = None, error_flag=None, k_smooth=None):
+    """Decode attention over product-VQ codes (see include/zkv.h).  k_codes / v_codes uint8
+    [B, Hkv, Tcap, d/m]; k_codebook / v_codebook float32 [Hkv, 256, m].
+    Returns (out float32 [B, Hq, d], lse float32 [B, Hq])."""
+    _need(q, "q", torch.float16)
+    for n, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, n, torch.uint8)
+    for n, t in (("comp_len", comp_len), ("win_len", win_len)):
+        _need(t, n, torch.int32)
+    for n, t in (("k_codebook", k_codebook), ("v_codebook", v_codebook)):
+        _need(t, n, torch.float32)
+    _need(win_k, "win_k", torch.float16)
+    _need(win_v, "win_v", torch.float16)
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, nsub = k_codes.shape
+    m = k_codebook.shape[-1]
+    if nsub * m != d or tuple(v_codes.shape) != tuple(k_codes.shape):
+        raise ValueError("codes must be [B, Hkv, Tcap, d/m] for K and V")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32)
+    _need(lse, "lse", torch.float32)
+    if error_flag is not None:
+        _need(error_flag, "error_flag", torch.int32)
+    p = PQDecodeParams(B=B, Hq=Hq, Hkv=Hkv, d=d, m=m, Tcap=Tcap, Wcap=win_k.shape[2],
+                       max_comp_len=Tcap if max_comp_len is None else int(max_comp_len),
+                       softmax_scale=0.0 if softmax_scale is None else float(softmax_scale),
+                       q=_ptr(q), k_codes=_ptr(k_codes), v_codes=_ptr(v_codes),
+                       comp_len=_ptr(comp_len), k_codebook=_ptr(k_codebook),
+                       v_codebook=_ptr(v_codebook), win_k=_ptr(win_k), win_v=_ptr(win_v),
+                       win_len=_ptr(win_len), out=_ptr(out), lse=_ptr(lse),
+                       error_flag=_ptr(error_flag),
+                       k_smooth=_smooth_ptr(k_smooth, Hkv, d, "k_smooth"))
+    need = lib().zkv_pq_decode_workspace_size(ctypes.byref(p))
+    if need == 0:
+        raise ZkvError("zkv_pq_decode_workspace_size", ZKV_ERR_UNSUPPORTED)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8)
+    _check("zkv_pq_decode_attn",
+           lib().zkv_pq_decode_attn(ctypes.byref(p), _ptr(workspace), workspace.numel(),
+                                    _stream()))
+    return out, lse
 
 
 def lse_merge(part_out: torch.Tensor, part_lse: torch.Tensor, out=None, lse=None):

@@ -335,6 +335,47 @@ typedef struct {
 int zkv_pq_encode(const zkv_pq_encode_params* p, void* stream);
 
 /*
+ * zkv_pq_decode_attn -- decode attention over a product-VQ compressed prefix (zkv_pq_encode's
+ * codes, keys and values) plus the fp16 recency window.
+ * Passages: VeloxQuant "VecInfer" (product VQ with the dual transform absorbed into the query);
+ * VQKV section 2.3 "Decoding Stage" and "Local Sliding Window"; Differential-KV "Flash-Style
+ * LSE Combine".
+ * Computes what zkv_rvq_decode_attn computes with the keys / values reconstructed as
+ *   k_t = lambda * H concat_j Ck[kvh][zk_{t,j}] / sqrt(d),  v_t = H concat_j Cv[kvh][zv_{t,j}] / sqrt(d)
+ * (lambda = k_smooth, or 1).  Internally a warp's lane j owns sub-vector j of every token (the
+ * scores of 32 / GP tokens are reduced together), per head a running maximum, the values
+ * accumulated per lane: no histograms.
+ * Shapes: d / m must be 32 -- (d, m) in {(64, 2), (128, 4), (256, 8)}; Hq / Hkv <= 8 (<= 2 at
+ * d = 256).  Layouts: k_codes / v_codes uint8 [B][Hkv][Tcap][d / m]; k_codebook / v_codebook
+ * float32 [Hkv][256][m]; the rest as zkv_rvq_decode_attn.  Workspace:
+ * zkv_pq_decode_workspace_size(p) bytes, 256-byte aligned.  Two kernels are launched.
+ * Errors: INVALID_ARG, UNSUPPORTED (shapes), WORKSPACE, CUDA; device-side length errors as in
+ * zkv_rvq_decode_attn.
+ */
+typedef struct {
+  int B, Hq, Hkv, d, m;
+  int64_t Tcap, Wcap, max_comp_len;
+  float softmax_scale;
+  const uint16_t* q;
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const int32_t* comp_len;
+  const float* k_codebook;
+  const float* v_codebook;
+  const uint16_t* win_k;
+  const uint16_t* win_v;
+  const int32_t* win_len;
+  float* out;
+  float* lse;
+  int32_t* error_flag;
+  const float* k_smooth;
+} zkv_pq_decode_params;
+
+size_t zkv_pq_decode_workspace_size(const zkv_pq_decode_params* p);
+int zkv_pq_decode_attn(const zkv_pq_decode_params* p, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
  * zkv_lse_merge -- log-sum-exp combine of partial attention results over disjoint key sets
  * (context-parallel decode: every rank attends over its shard of each compressed prefix, the
  * shards' (out, lse) are gathered and combined).

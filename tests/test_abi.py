@@ -174,6 +174,44 @@ def test_pq_encode_validation(L):
     assert L.zkv_pq_encode(None, None) == zkv.ZKV_ERR_INVALID_ARG
 
 
+def test_pq_decode_validation(L):
+    def mk(**kw):
+        base = dict(B=2, Hq=8, Hkv=2, d=128, m=4, Tcap=64, Wcap=16, max_comp_len=64,
+                    softmax_scale=0.0, q=0x1000, k_codes=0x2000, v_codes=0x3000, comp_len=0x4000,
+                    k_codebook=0x5000, v_codebook=0x6000, win_k=0x7000, win_v=0x8000,
+                    win_len=0x9000, out=0xa000)
+        base.update(kw)
+        return zkv.PQDecodeParams(**base)
+    for kw, st in ((dict(m=8), zkv.ZKV_ERR_UNSUPPORTED),               # d / m must be 32
+                   (dict(d=256, m=8, Hq=8, Hkv=2), zkv.ZKV_ERR_UNSUPPORTED),   # GQA 4 at d 256
+                   (dict(Hq=6, Hkv=4), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(max_comp_len=65), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(q=0), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(q=0x1008), zkv.ZKV_ERR_INVALID_ARG)):
+        assert L.zkv_pq_decode_attn(ctypes.byref(mk(**kw)), None, 0, None) == st, kw
+    ok = mk()
+    assert L.zkv_pq_decode_workspace_size(ctypes.byref(ok)) > 0
+    assert L.zkv_pq_decode_attn(ctypes.byref(ok), None, 0, None) == zkv.ZKV_ERR_WORKSPACE
+    assert L.zkv_pq_decode_workspace_size(ctypes.byref(mk(m=8))) == 0
+
+
+def test_pq_decode_workspace_size_binding(L):
+    """The binding's size query reads shapes only; the layout is six 256-byte-aligned float32
+    arrays: chunk maxima, sums and outputs, then the window's maxima, sums and outputs."""
+    import torch
+    B, Hq, Hkv, d, m, W = 2, 8, 2, 128, 4, 16
+    q = torch.empty((B, Hq, d), device="meta", dtype=torch.float16)
+    wk = torch.empty((B, Hkv, W, d), device="meta", dtype=torch.float16)
+    Ck = torch.empty((Hkv, 256, m), device="meta")
+    for Tcap, chunks in ((64, 1), (2048, 1), (2049, 2), (5000, 3)):
+        kc = torch.empty((B, Hkv, Tcap, d // m), device="meta", dtype=torch.uint8)
+        pairs, GP = B * Hkv, Hq // Hkv
+        a256 = lambda n: (n + 255) // 256 * 256   # noqa: E731
+        want = (2 * a256(pairs * chunks * GP * 4) + a256(pairs * chunks * GP * d * 4)
+                + 2 * a256(pairs * GP * 4) + a256(pairs * GP * d * 4))
+        assert zkv.pq_decode_workspace_size(q, kc, Ck, wk) == want, Tcap
+
+
 def test_lse_merge_validation(L):
     def mk(**kw):
         base = dict(n_parts=2, rows=4, d=8, part_out=0x1000, out_part_stride=36, out_row_stride=9,
@@ -204,7 +242,8 @@ def test_ctypes_structs_match_the_header_layout(tmp_path):
         pytest.skip("no C compiler")
     pairs = [("zkv_encode_params", zkv.EncodeParams), ("zkv_reconstruct_params", zkv.ReconstructParams),
              ("zkv_decode_params", zkv.DecodeParams), ("zkv_append_params", zkv.AppendParams),
-             ("zkv_lse_merge_params", zkv.MergeParams), ("zkv_pq_encode_params", zkv.PQEncodeParams)]
+             ("zkv_lse_merge_params", zkv.MergeParams), ("zkv_pq_encode_params", zkv.PQEncodeParams),
+             ("zkv_pq_decode_params", zkv.PQDecodeParams)]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zkv.h"', "int main(void) {"]
     for cname, cls in pairs:
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
