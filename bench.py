@@ -748,16 +748,6 @@ def run_ours(args):
     if not args.no_encode and rank == 0:
         del graphs, soak_graphs
         extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
-    if not args.no_encode and rank == 0:
-        try:
-            extras["pq_encode"] = pq_encode_extra(dev)
-        except Exception as exc:   # an extra never takes the main line down
-            extras["pq_encode"] = {"error": f"{type(exc).__name__}: {exc}"}
-    if not args.no_encode and rank == 0:
-        try:
-            extras["pq_decode"] = pq_decode_extra(dev, hbm_peak)
-        except Exception as exc:   # an extra never takes the main line down
-            extras["pq_decode"] = {"error": f"{type(exc).__name__}: {exc}"}
     base_ms = 1000.0 * elapsed / args.steps
     for name, kw, skip in (("smooth", dict(smooth=True), args.no_smooth),
                            ("paged", dict(page_tokens=256), args.no_paged)):
@@ -768,6 +758,15 @@ def run_ours(args):
         torch.cuda.empty_cache()
         try:
             extras[name] = variant_extra(wl, args, dev, R, base_ms, **kw)
+        except Exception as exc:   # an extra never takes the main line down
+            extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
+    # the product-VQ extras come last: nothing measured above depends on them
+    for name, fn in (("pq_encode", lambda: pq_encode_extra(dev)),
+                     ("pq_decode", lambda: pq_decode_extra(dev, hbm_peak))):
+        if args.no_encode or rank != 0:
+            continue
+        try:
+            extras[name] = fn()
         except Exception as exc:   # an extra never takes the main line down
             extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
 
