@@ -56,6 +56,8 @@ def parse():
                     help="skip the serving step with key smoothing (extra)")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the serving step with the paged code layout (extra)")
+    ap.add_argument("--no-ragged", action="store_true",
+                    help="skip the serving step on the ragged 64-sequence batch (extra)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -367,6 +369,91 @@ def encode_extra(dev, hbm, bf16):
             "frac": flops / sec / 1e12 / tf32_peak,
             "note": "tcgen05 kind::tf32 distance GEMM (M=128 rows, N=256 codewords) into TMEM; "
                     "exact decision: TF32-margin candidates re-scored in float32, then float64"}
+
+
+def ragged_extra(dev, hbm_peak, R=4, steps=100):
+    """The serving step on the ragged batch: 64 sequences with seeded lengths U{1024..16384}
+    (Hq 32, Hkv 8, d 128, Sk = Sv = 4, full 128-token windows), one appended token per sequence
+    per step.  Codes drawn from the input generator's skewed code distribution (encoding half a
+    million prefix tokens on the host would dominate the run), R rotating replicas larger than
+    L2, one CUDA graph per replica step, CUDA-event timed."""
+    import torch
+
+    from compressed_decode_attention_zkv_b200 import inputs as I
+    from compressed_decode_attention_zkv_b200 import zkv
+    wl = I.workload("ragged_serving_64")
+    lens = I.ragged_lengths(wl)
+    comp = (lens - wl.W).astype(np.int64)
+    grow = (3 + steps + R - 1) // R + 2
+    Tcap = int((comp.max() + grow + 15) // 16 * 16)
+    kc = torch.from_numpy(I.random_codes(wl, "k", Tcap)).to(dev)
+    vc = torch.from_numpy(I.random_codes(wl, "v", Tcap, seed=1)).to(dev)
+    Ck = torch.from_numpy(I.train_codebooks(wl, "k")).to(dev)
+    Cv = torch.from_numpy(I.train_codebooks(wl, "v")).to(dev)
+    wk = torch.from_numpy(I.window_tokens(wl, "k", lens)).to(dev)
+    wv = torch.from_numpy(I.window_tokens(wl, "v", lens)).to(dev)
+    reps = []
+    for r in range(R):
+        reps.append(dict(
+            Ck=Ck.clone(), Cv=Cv.clone(), k_codes=kc.clone(), v_codes=vc.clone(),
+            win_k=wk.clone(), win_v=wv.clone(),
+            comp_len=torch.from_numpy(comp.astype(np.int32)).to(dev),
+            win_len=torch.full((wl.B,), wl.W, dtype=torch.int32, device=dev),
+            win_head=torch.zeros((wl.B,), dtype=torch.int32, device=dev),
+            q=torch.from_numpy(I.queries(wl, step=r)).to(dev),
+            new_k=torch.from_numpy(I.new_tokens(wl, r, "k", lens)).to(dev),
+            new_v=torch.from_numpy(I.new_tokens(wl, r, "v", lens)).to(dev),
+            out=torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32, device=dev),
+            lse=torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev),
+            err=torch.zeros(1, dtype=torch.int32, device=dev)))
+    del kc, vc, wk, wv
+    max_comp = int(comp.max()) + grow
+    need = zkv.decode_workspace_size(reps[0]["q"], reps[0]["k_codes"], reps[0]["v_codes"],
+                                     reps[0]["comp_len"], reps[0]["Ck"], reps[0]["Cv"],
+                                     reps[0]["win_k"], reps[0]["win_v"], reps[0]["win_len"],
+                                     max_comp_len=max_comp)
+    wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
+    host_comp = [int(comp.sum())] * R   # compressed tokens of all sequences, per replica
+    for r in range(R):   # eager call per replica (kernel attributes before capture)
+        step_fn(reps[r], wss[r], max_comp)
+        host_comp[r] += wl.B
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step_fn(reps[r], wss[r], max_comp)
+        graphs.append(g)
+    for i in range(3):
+        graphs[i % R].replay()
+        host_comp[i % R] += wl.B
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tokens = 0
+    s.record()
+    for i in range(steps):
+        r = (3 + i) % R
+        graphs[r].replay()
+        host_comp[r] += wl.B            # the step's append grows every prefix first
+        tokens += host_comp[r]
+    e.record()
+    torch.cuda.synchronize()
+    sec = s.elapsed_time(e) / 1000.0
+    assert sum(int(rep["err"].item()) for rep in reps) == 0
+    del graphs
+    step_s = sec / steps
+    tc_avg = tokens / steps
+    byts = (tc_avg * wl.Hkv * (wl.Sk + wl.Sv) + wl.B * wl.Hkv * wl.W * wl.d * 2 * 2
+            + wl.Hkv * (wl.Sk + wl.Sv) * 256 * wl.d * 4 + wl.B * wl.Hq * wl.d * (2 + 4))
+    rep_mb = replica_bytes(reps[0]) / 1e6
+    return {"workload": "ragged_serving_64 (64 seqs, lengths U{1024..16384} seed 3, Hq 32, "
+                        "Hkv 8, d 128, Sk = Sv = 4, W 128)",
+            "value": tokens / sec, "unit": UNIT, "ms_per_step": 1000.0 * step_s,
+            "seq_tokens_per_s": wl.B / step_s, "compressed_tokens_per_step": tc_avg,
+            "step_gbs": byts / step_s / 1e9, "step_frac": byts / step_s / 1e9 / hbm_peak,
+            "steps": steps,
+            "note": f"one zkv_rvq_serve_step per step; graphs over {R} rotating replicas x "
+                    f"{rep_mb:.0f} MB (> L2); codes from the skewed code distribution"}
 
 
 def pq_encode_extra(dev):
@@ -760,6 +847,12 @@ def run_ours(args):
             extras[name] = variant_extra(wl, args, dev, R, base_ms, **kw)
         except Exception as exc:   # an extra never takes the main line down
             extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
+    if rank == 0 and not args.no_ragged:
+        try:
+            extras["ragged_serving"] = ragged_extra(dev, hbm_peak)
+        except Exception as exc:   # an extra never takes the main line down
+            extras["ragged_serving"] = {"error": f"{type(exc).__name__}: {exc}"}
+        torch.cuda.empty_cache()
     # the product-VQ extras come last: nothing measured above depends on them
     for name, fn in (("pq_encode", lambda: pq_encode_extra(dev)),
                      ("pq_decode", lambda: pq_decode_extra(dev, hbm_peak))):
