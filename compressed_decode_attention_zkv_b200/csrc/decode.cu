@@ -1449,8 +1449,10 @@ struct PqArgs {
 template <int D, int M, int GP>
 __global__ void __launch_bounds__(256) pq_scan_kernel(PqArgs a) {
   constexpr int NSUB = D / M;
-  static_assert(NSUB == 32, "one sub-vector per lane");
-  constexpr int TB = 32 / GP;        // tokens per transpose-sum batch
+  static_assert(NSUB == 32 || NSUB == 16, "one sub-vector per lane of a 32- or 16-lane group");
+  constexpr int NH = 32 / NSUB;      // lane groups: each takes its own tokens
+  constexpr int TBH = NSUB / GP;     // tokens per group per transpose-sum batch
+  constexpr int TB = NH * TBH;       // tokens per batch (32 / GP)
   constexpr int E = D / 32;
   __shared__ __align__(16) float ck[kCodebook * M];
   __shared__ __align__(16) float cv[kCodebook * M];
@@ -1493,13 +1495,15 @@ __global__ void __launch_bounds__(256) pq_scan_kernel(PqArgs a) {
   const int64_t per = (n + 7) / 8;
   const int64_t w0 = t0 + warp * per < t1 ? t0 + warp * per : t1;
   const int64_t w1 = w0 + per < t1 ? w0 + per : t1;
+  // lane = (group hh, sub-vector j); group hh takes tokens hh * TBH .. hh * TBH + TBH - 1 of a batch
+  const int j = lane % NSUB, hh = lane / NSUB;
   float qr[GP][M];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
 #pragma unroll
-    for (int i = 0; i < M; ++i) qr[g][i] = qs[g][lane * M + i];
-  const uint8_t* kz = a.k_codes + (pair * a.Tcap) * NSUB + lane;
-  const uint8_t* vz = a.v_codes + (pair * a.Tcap) * NSUB + lane;
+    for (int i = 0; i < M; ++i) qr[g][i] = qs[g][j * M + i];
+  const uint8_t* kz = a.k_codes + (pair * a.Tcap) * NSUB + j;
+  const uint8_t* vz = a.v_codes + (pair * a.Tcap) * NSUB + j;
   float mrun[GP], acc[GP][M];
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
@@ -1511,12 +1515,13 @@ __global__ void __launch_bounds__(256) pq_scan_kernel(PqArgs a) {
   const int gl = lane % GP;
   for (int64_t base = w0; base < w1; base += TB) {
     const int nv = (int)(w1 - base < TB ? w1 - base : TB);
-    float x[32];
+    const int64_t gbase = base + hh * TBH;   // this lane group's first token of the batch
+    float x[NSUB];
 #pragma unroll
-    for (int u = 0; u < TB; ++u) {
+    for (int u = 0; u < TBH; ++u) {
       float kv[M];
-      if (u < nv) {
-        const int z = kz[(base + u) * NSUB];
+      if (hh * TBH + u < nv) {
+        const int z = kz[(gbase + u) * NSUB];
 #pragma unroll
         for (int i = 0; i < M; ++i) kv[i] = ck[z * M + i];
       } else {
@@ -1531,9 +1536,10 @@ __global__ void __launch_bounds__(256) pq_scan_kernel(PqArgs a) {
         x[u * GP + g] = s;
       }
     }
+    // lane L ends with the score of its group's token (L % NSUB) / GP, head L % GP
     int hidx = 0;
-    float sc = TransposeSum<32, 32, 16>::run(x, lane, hidx) * a.scale_log2;   // hidx == lane
-    const bool ok = lane / GP < nv;
+    float sc = TransposeSum<NSUB, NSUB, NSUB / 2>::run(x, lane, hidx) * a.scale_log2;   // hidx == j
+    const bool ok = hh * TBH + j / GP < nv;
     if (!ok) sc = -INFINITY;
     float bm = sc;   // batch maximum of head lane % GP
 #pragma unroll
@@ -1555,20 +1561,30 @@ __global__ void __launch_bounds__(256) pq_scan_kernel(PqArgs a) {
     const float p = ok ? ex2_approx(sc - mnew_l) : 0.f;
     lp = lp * alpha_l + p;
 #pragma unroll
-    for (int u = 0; u < TB; ++u) {
-      if (u < nv) {
-        const int z = vz[(base + u) * NSUB];
-        float vv[M];
+    for (int u = 0; u < TBH; ++u) {
+      // the shuffles run on every lane; a token past the end has p = 0 and reads no codes
+      float vv[M];
+      if (hh * TBH + u < nv) {
+        const int z = vz[(gbase + u) * NSUB];
 #pragma unroll
         for (int i = 0; i < M; ++i) vv[i] = cv[z * M + i];
+      } else {
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const float pg = __shfl_sync(0xffffffffu, p, u * GP + g);
+        for (int i = 0; i < M; ++i) vv[i] = 0.f;
+      }
 #pragma unroll
-          for (int i = 0; i < M; ++i) acc[g][i] = fmaf(pg, vv[i], acc[g][i]);
-        }
+      for (int g = 0; g < GP; ++g) {
+        const float pg = __shfl_sync(0xffffffffu, p, hh * NSUB + u * GP + g);
+#pragma unroll
+        for (int i = 0; i < M; ++i) acc[g][i] = fmaf(pg, vv[i], acc[g][i]);
       }
     }
+  }
+  if constexpr (NH == 2) {   // the two groups hold the same dims for different tokens
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+#pragma unroll
+      for (int i = 0; i < M; ++i) acc[g][i] += __shfl_xor_sync(0xffffffffu, acc[g][i], 16);
   }
   // warp partials: per head the sum of p over the lanes of that head
 #pragma unroll
@@ -1580,8 +1596,10 @@ __global__ void __launch_bounds__(256) pq_scan_kernel(PqArgs a) {
       wm[warp][g] = mrun[g];
       wl[warp][g] = l;
     }
+    if (lane < NSUB) {
 #pragma unroll
-    for (int i = 0; i < M; ++i) wo[warp][g][lane * M + i] = acc[g][i];
+      for (int i = 0; i < M; ++i) wo[warp][g][j * M + i] = acc[g][i];
+    }
   }
   __syncthreads();
   // combine the 8 warps: weight 2^(m_w - M*) (0 for a warp without tokens)
@@ -1894,11 +1912,16 @@ struct PqPlan {
   size_t off_cm, off_cl, off_co, off_wm, off_wl, off_wo, total;
 };
 
+// Largest padded GQA group of a (d, m) instantiation: the scan holds G*m query values and
+// G*m accumulators per lane (registers), and its warp partials take 8*G*d floats of shared
+// memory next to the two 256*m codebooks.
+constexpr int pq_max_gp(int d, int m) { return d == 256 ? 2 : (m == 8 ? 4 : 8); }
+
+// d / m = 32 (one token per warp step) or 16 (two tokens, one per 16-lane group)
 static bool pq_shape_supported(int d, int m, int GP) {
-  if (d == 64) return m == 2;
-  if (d == 128) return m == 4;
-  if (d == 256) return m == 8 && GP <= 2;   // shared memory of the scan's warp partials
-  return false;
+  const bool dm = (d == 64 && (m == 2 || m == 4)) || (d == 128 && (m == 4 || m == 8)) ||
+                  (d == 256 && m == 8);
+  return dm && GP <= pq_max_gp(d, m);
 }
 
 static int validate_pq_shapes(const zkv_pq_decode_params* p) {
@@ -1944,11 +1967,12 @@ static int launch_pq(const PqArgs& a, const DecodeArgs& w, cudaStream_t st) {
 
 template <int D, int M>
 static int launch_pq_g(int GP, const PqArgs& a, const DecodeArgs& w, cudaStream_t st) {
+  constexpr int kMax = pq_max_gp(D, M);
   switch (GP) {
     case 1: return launch_pq<D, M, 1>(a, w, st);
     case 2: return launch_pq<D, M, 2>(a, w, st);
-    case 4: if constexpr (D <= 128) return launch_pq<D, M, 4>(a, w, st); else return ZKV_ERR_UNSUPPORTED;
-    default: if constexpr (D <= 128) return launch_pq<D, M, 8>(a, w, st); else return ZKV_ERR_UNSUPPORTED;
+    case 4: if constexpr (kMax >= 4) return launch_pq<D, M, 4>(a, w, st); else return ZKV_ERR_UNSUPPORTED;
+    default: if constexpr (kMax >= 8) return launch_pq<D, M, 8>(a, w, st); else return ZKV_ERR_UNSUPPORTED;
   }
 }
 
@@ -1997,9 +2021,11 @@ extern "C" int zkv_pq_decode_attn(const zkv_pq_decode_params* p, void* workspace
   w.wl = reinterpret_cast<float*>(ws + pl.off_wl);
   w.wo = reinterpret_cast<float*>(ws + pl.off_wo);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  switch (p->d) {
-    case 64: return launch_pq_g<64, 2>(pl.GP, a, w, st);
-    case 128: return launch_pq_g<128, 4>(pl.GP, a, w, st);
+  switch (p->d * 100 + p->m) {   // the shapes validate_pq_shapes admits
+    case 6402: return launch_pq_g<64, 2>(pl.GP, a, w, st);
+    case 6404: return launch_pq_g<64, 4>(pl.GP, a, w, st);
+    case 12804: return launch_pq_g<128, 4>(pl.GP, a, w, st);
+    case 12808: return launch_pq_g<128, 8>(pl.GP, a, w, st);
     default: return launch_pq_g<256, 8>(pl.GP, a, w, st);
   }
 }

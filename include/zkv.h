@@ -342,11 +342,11 @@ int zkv_pq_encode(const zkv_pq_encode_params* p, void* stream);
  * LSE Combine".
  * Computes what zkv_rvq_decode_attn computes with the keys / values reconstructed as
  *   k_t = lambda * H concat_j Ck[kvh][zk_{t,j}] / sqrt(d),  v_t = H concat_j Cv[kvh][zv_{t,j}] / sqrt(d)
- * (lambda = k_smooth, or 1).  Internally a warp's lane j owns sub-vector j of every token (the
- * scores of 32 / GP tokens are reduced together), per head a running maximum, the values
- * accumulated per lane: no histograms.
- * Shapes: d / m must be 32 -- (d, m) in {(64, 2), (128, 4), (256, 8)}; Hq / Hkv <= 8 (<= 2 at
- * d = 256).  Layouts: k_codes / v_codes uint8 [B][Hkv][Tcap][d / m]; k_codebook / v_codebook
+ * (lambda = k_smooth, or 1).  Internally lane j of a warp (of each 16-lane half when d / m = 16)
+ * owns sub-vector j of its tokens (the scores of 32 / GP tokens are reduced together), per head
+ * a running maximum, the values accumulated per lane: no histograms.
+ * Shapes: d / m = 32 or 16 -- (d, m) in {(64, 2), (64, 4), (128, 4), (128, 8), (256, 8)}, i.e.
+ * 2 or 1 code bits per element at d = 128; Hq / Hkv <= 8, <= 4 at (128, 8), <= 2 at d = 256.  Layouts: k_codes / v_codes uint8 [B][Hkv][Tcap][d / m]; k_codebook / v_codebook
  * float32 [Hkv][256][m]; the rest as zkv_rvq_decode_attn.  Workspace:
  * zkv_pq_decode_workspace_size(p) bytes, 256-byte aligned.  Two kernels are launched.
  * Errors: INVALID_ARG, UNSUPPORTED (shapes), WORKSPACE, CUDA; device-side length errors as in

@@ -182,7 +182,8 @@ def test_pq_decode_validation(L):
                     win_len=0x9000, out=0xa000)
         base.update(kw)
         return zkv.PQDecodeParams(**base)
-    for kw, st in ((dict(m=8), zkv.ZKV_ERR_UNSUPPORTED),               # d / m must be 32
+    for kw, st in ((dict(m=16), zkv.ZKV_ERR_UNSUPPORTED),              # d / m must be 32 or 16
+                   (dict(m=8, Hq=16), zkv.ZKV_ERR_UNSUPPORTED),        # GQA 8 at (128, 8)
                    (dict(d=256, m=8, Hq=8, Hkv=2), zkv.ZKV_ERR_UNSUPPORTED),   # GQA 4 at d 256
                    (dict(Hq=6, Hkv=4), zkv.ZKV_ERR_INVALID_ARG),
                    (dict(max_comp_len=65), zkv.ZKV_ERR_INVALID_ARG),
@@ -192,7 +193,9 @@ def test_pq_decode_validation(L):
     ok = mk()
     assert L.zkv_pq_decode_workspace_size(ctypes.byref(ok)) > 0
     assert L.zkv_pq_decode_attn(ctypes.byref(ok), None, 0, None) == zkv.ZKV_ERR_WORKSPACE
-    assert L.zkv_pq_decode_workspace_size(ctypes.byref(mk(m=8))) == 0
+    assert L.zkv_pq_decode_workspace_size(ctypes.byref(mk(m=16))) == 0
+    for kw in (dict(m=8), dict(d=64, m=4, Hq=16), dict(d=64, m=2)):   # supported shapes
+        assert L.zkv_pq_decode_workspace_size(ctypes.byref(mk(**kw))) > 0, kw
 
 
 def test_pq_decode_workspace_size_binding(L):

@@ -2,8 +2,8 @@
 float64 argmin of every sub-vector except counted near-ties (distance gap below 1e-5
 relative), with and without key smoothing, every head dimension and several sub-vector sizes.
 Decode: outputs and lse within 2e-3 of the oracle's direct form (reconstruct, rotate back,
-softmax attention with the window), across chunk boundaries, GQA 1 / 2 / 4 / 7, smoothing and
-empty parts.
+softmax attention with the window), across chunk boundaries, 32 and 16 sub-vectors per token,
+GQA 1 / 2 / 4 / 6 / 7, smoothing and empty parts.
 The file name keeps it after every other GPU test in collection order, so that under
 ``pytest -x`` a failure here cannot hide the results of the established paths."""
 import numpy as np
@@ -83,6 +83,10 @@ def _pq_case(seed, Bn, Hq, Hkv, d, m, Tcap, comp, Wcap, win, smooth):
     dict(Bn=1, Hq=4, Hkv=2, d=256, m=8, Tcap=720, comp=[700], Wcap=4, win=[4], smooth=True),
     dict(Bn=2, Hq=2, Hkv=2, d=128, m=4, Tcap=64, comp=[0, 17], Wcap=4, win=[0, 0],
          smooth=False),
+    # 16 sub-vectors per token (two tokens per warp step): 1 bit per element at d = 128
+    dict(Bn=2, Hq=8, Hkv=2, d=128, m=8, Tcap=2576, comp=[2570, 9], Wcap=8, win=[3, 8],
+         smooth=True),
+    dict(Bn=1, Hq=6, Hkv=1, d=64, m=4, Tcap=2064, comp=[2051], Wcap=4, win=[2], smooth=False),
 ])
 def test_pq_decode_matches_oracle(cfg):
     q, kc, vc, comp, Ck, Cv, wk, wv, win, lam = _pq_case(200 + cfg["d"], **cfg)
