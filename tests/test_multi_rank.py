@@ -1,4 +1,4 @@
-"""Multi-process paths on CPU (world size 2, gloo): the context-parallel decode's sharding and
+"""Multi-process paths on CPU (world sizes 2 and 3, gloo): the context-parallel decode's sharding and
 exchange, and the benchmark's max-over-ranks timing.  No GPU: the context-parallel test runs
 the exchange with oracle-backed stand-ins for the library's decode and combine (the GPU test
 of those is tests/test_gpu_context_parallel.py)."""
@@ -80,8 +80,8 @@ def _cp_rank(rank, world, port, result):
         dist.destroy_process_group()
 
 
-def test_context_parallel_exchange_equals_unsharded_decode():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_exchange_equals_unsharded_decode(world):
     result = mp.Manager().dict()
     mp.spawn(_cp_rank, args=(world, _free_port(), result), nprocs=world, join=True)
     from oracle import zkv_oracle as O
@@ -97,8 +97,9 @@ def test_context_parallel_exchange_equals_unsharded_decode():
         assert window_tokens == (int(win.sum()) if r == world - 1 else 0)
         np.testing.assert_array_equal(cl, end - start)
     np.testing.assert_array_equal(result[0][3], 0)
-    np.testing.assert_array_equal(result[0][4], result[1][3])
-    np.testing.assert_array_equal(result[1][4], comp)
+    for r in range(world - 1):
+        np.testing.assert_array_equal(result[r][4], result[r + 1][3])
+    np.testing.assert_array_equal(result[world - 1][4], comp)
 
 
 def _timing_rank(rank, world, port, result):
