@@ -586,3 +586,38 @@ def test_pq_code_bytes_give_the_stated_bit_rates():
     for m, bits in ((4, 2), (8, 1)):
         z, _ = O.pq_encode(x, np.zeros((256, m), np.float32))
         assert z.dtype == np.uint8 and z.shape[1] * 8 / 128 == bits
+
+
+# ------------------------------------------------------------------ product VQ, worked examples
+
+def test_pq_encode_hand_example():
+    from oracle import c_oracle as C
+    g = _read_fixture("pq_encode_hand_d4.txt")
+    x = g["x"].astype(np.float16)[None]
+    book = g["codebook"].astype(np.float32)
+    lam = g["lambda"].astype(np.float32)
+    z, y = O.pq_encode(x, book, smooth=lam)
+    np.testing.assert_array_equal(y[0], g["y_smoothed"])
+    np.testing.assert_array_equal(z[0], g["codes_smoothed"])
+    z, y = O.pq_encode(x, book)
+    np.testing.assert_array_equal(y[0], g["y_plain"])
+    np.testing.assert_array_equal(z[0], g["codes_plain"])
+    np.testing.assert_array_equal(C.pq_encode(x, book, smooth=lam)[0], g["codes_smoothed"])
+    np.testing.assert_array_equal(C.pq_encode(x, book)[0], g["codes_plain"])
+
+
+def test_pq_decode_hand_example():
+    from oracle import c_oracle as C
+    g = _read_fixture("pq_decode_hand_d4.txt")
+    d = 4
+    q = g["q"].astype(np.float16).reshape(1, 1, d)
+    book = g["codebook"].astype(np.float32).reshape(1, 4, 2)
+    kc = g["k_codes"].astype(np.uint8).reshape(1, 1, 2, 2)
+    vc = g["v_codes"].astype(np.uint8).reshape(1, 1, 2, 2)
+    w = np.zeros((1, 1, 1, d), np.float16)
+    e2 = math.exp(2.0)
+    want = np.array([2 * e2 + 1, 1, 1 - 2 * e2, 1]) / (e2 + 1)
+    for fn in (O.pq_decode_attn, O.pq_decode_attn_lut, C.pq_decode_attn):
+        out, lse = fn(q, kc, vc, [2], book, book, w, w, [0])
+        np.testing.assert_allclose(out[0, 0], want, atol=1e-14)
+        assert abs(lse[0, 0] - math.log(e2 + 1)) < 1e-14
