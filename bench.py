@@ -123,6 +123,19 @@ class ClockSampler:
 # Workload state on the GPU
 # --------------------------------------------------------------------------------------------
 
+_BOOKS = {}
+
+
+def codebooks(wl, kind, smooth=None):
+    """The workload's seeded k-means codebooks (float32 numpy), memoised: the main line and
+    several extras train the same ones."""
+    from compressed_decode_attention_zkv_b200 import inputs as I
+    key = (wl, kind, None if smooth is None else np.asarray(smooth).tobytes())
+    if key not in _BOOKS:
+        _BOOKS[key] = I.train_codebooks(wl, kind, smooth=smooth)
+    return _BOOKS[key]
+
+
 def build_state(wl, R, Tcap_extra, dev, smooth=False, tcap_multiple=16):
     """Encode the workload's prefixes on the GPU (prefill) and make R replicas.  smooth: key
     smoothing factors calibrated on the calibration sample, key codebooks trained on smoothed
@@ -134,8 +147,8 @@ def build_state(wl, R, Tcap_extra, dev, smooth=False, tcap_multiple=16):
 
     lam_np = I.key_smooth_factors(wl) if smooth else None
     lam = None if lam_np is None else torch.from_numpy(lam_np).to(dev)
-    Ck = torch.from_numpy(I.train_codebooks(wl, "k", smooth=lam_np)).to(dev)
-    Cv = torch.from_numpy(I.train_codebooks(wl, "v")).to(dev)
+    Ck = torch.from_numpy(codebooks(wl, "k", smooth=lam_np)).to(dev)
+    Cv = torch.from_numpy(codebooks(wl, "v")).to(dev)
     Tc = wl.Tc
     Tcap = (Tc + Tcap_extra + tcap_multiple - 1) // tcap_multiple * tcap_multiple
     kc = torch.zeros((wl.B, wl.Hkv, Tcap, wl.Sk), dtype=torch.uint8, device=dev)
@@ -335,7 +348,7 @@ def encode_extra(dev, hbm, bf16):
     from compressed_decode_attention_zkv_b200 import inputs as I
     from compressed_decode_attention_zkv_b200 import zkv
     wl = I.workload("prefill_encode_64k")
-    books = {k: torch.from_numpy(I.train_codebooks(wl, k)).to(dev) for k in ("k", "v")}
+    books = {k: torch.from_numpy(codebooks(wl, k)).to(dev) for k in ("k", "v")}
     xs = {k: torch.from_numpy(I.kv_tokens(wl, k, 0, 0, wl.T)).to(dev).permute(1, 0, 2)
           for k in ("k", "v")}                                          # [T, H, d] views
     codes = {k: torch.empty((wl.T, wl.Hkv, wl.Sk), dtype=torch.uint8, device=dev) for k in xs}
@@ -388,8 +401,8 @@ def ragged_extra(dev, hbm_peak, R=4, steps=100):
     Tcap = int((comp.max() + grow + 15) // 16 * 16)
     kc = torch.from_numpy(I.random_codes(wl, "k", Tcap)).to(dev)
     vc = torch.from_numpy(I.random_codes(wl, "v", Tcap, seed=1)).to(dev)
-    Ck = torch.from_numpy(I.train_codebooks(wl, "k")).to(dev)
-    Cv = torch.from_numpy(I.train_codebooks(wl, "v")).to(dev)
+    Ck = torch.from_numpy(codebooks(wl, "k")).to(dev)
+    Cv = torch.from_numpy(codebooks(wl, "v")).to(dev)
     wk = torch.from_numpy(I.window_tokens(wl, "k", lens)).to(dev)
     wv = torch.from_numpy(I.window_tokens(wl, "v", lens)).to(dev)
     reps = []
@@ -463,7 +476,9 @@ def pq_encode_extra(dev):
 
     from compressed_decode_attention_zkv_b200 import inputs as I
     from compressed_decode_attention_zkv_b200 import zkv
-    wl = I.workload("prefill_encode_64k")
+    # a smaller calibration for the codebook: the encode scans all 256 codewords of every
+    # sub-vector whatever they are, and full k-means here would take ~45 s of host time
+    wl = I.workload("prefill_encode_64k", n_cal=2048, kmeans_iters=4)
     m = 4
     lam_np = I.key_smooth_factors(wl)
     lam = torch.from_numpy(lam_np).to(dev)
@@ -485,7 +500,8 @@ def pq_encode_extra(dev):
                         "with 4-dim sub-vectors (2 bits/elem) and key smoothing",
             "vectors_per_s": rows / sec, "ms_per_call": sec * 1000.0,
             "fp64_gflops": 2.0 * rows * (wl.d // m) * 256 * m / sec / 1e9,
-            "note": "one warp per row; float64 distances to all 256 codewords of every sub-vector"}
+            "note": "one warp per row; float64 distances to all 256 codewords of every "
+                    "sub-vector; codebook from 2048 calibration vectors x 4 k-means iterations"}
 
 
 def pq_decode_extra(dev, hbm_peak):
