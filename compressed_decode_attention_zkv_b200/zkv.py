@@ -700,7 +700,7 @@ class RVQKVCache:
     """Compressed KV cache of one attention layer: RVQ codes for old tokens, an fp16 window for
     the newest ones.  prefill() encodes a prompt, append() inserts one token per sequence
     (evicting and encoding the oldest window token when the window is full), attend() runs one
-    decode step of attention.  All state lives on the GPU; lengths never leave the device.
+    decode step of attention, step() does both in one library call.  All state lives on the GPU; lengths never leave the device.
     k_smooth: optional float32 [Hkv, d] key smoothing factors (the key codebooks must have been
     trained on smoothed keys)."""
 
@@ -763,6 +763,24 @@ class RVQKVCache:
         return rvq_decode_attn(*args, out=out, lse=lse, max_comp_len=self.max_comp_len,
                                softmax_scale=softmax_scale, workspace=self._ws,
                                error_flag=self.error_flag, k_smooth=self.k_smooth)
+
+    def step(self, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+             softmax_scale=None, out=None, lse=None):
+        """append(k_new, v_new) then attend(q) as one library call (zkv_rvq_serve_step: the
+        lookup tables are built beside the encode of the evicted token); the same results as
+        the two calls.  k_new, v_new fp16 [B, Hkv, d]; q fp16 [B, Hq, d]."""
+        self.max_comp_len = min(self.max_comp_len + 1, self.Tcap)
+        args = (q, self.k_codes, self.v_codes, self.comp_len, self.Ck, self.Cv, self.win_k,
+                self.win_v, self.win_len)
+        need = decode_workspace_size(*args, max_comp_len=self.max_comp_len)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        return rvq_serve_step(k_new.contiguous(), v_new.contiguous(), q, self.win_k, self.win_v,
+                              self.win_len, self.win_head, self.comp_len, self.k_codes,
+                              self.v_codes, self.Ck, self.Cv, out=out, lse=lse,
+                              max_comp_len=self.max_comp_len, softmax_scale=softmax_scale,
+                              workspace=self._ws, error_flag=self.error_flag,
+                              k_smooth=self.k_smooth)
 
     def memory_bytes(self) -> int:
         """Bytes held by codes and window (codebooks are shared across layers' caches)."""

@@ -291,6 +291,33 @@ def test_serving_loop_matches_oracle():
     assert int(cache.error_flag.item()) == 0
 
 
+def test_cache_step_equals_append_then_attend():
+    """RVQKVCache.step (one serving-step call) is bit-identical to append + attend."""
+    rng = np.random.default_rng(31)
+    Bn, Hq, Hkv, d, S, W = 2, 8, 2, 128, 4, 4
+    Ck = (rng.standard_normal((Hkv, S, 256, d)) * 0.15).astype(np.float32)
+    Cv = (rng.standard_normal((Hkv, S, 256, d)) * 0.3).astype(np.float32)
+    Ck[:, :, 0] = 0
+    Cv[:, :, 0] = 0
+    k = rng.standard_normal((Bn, Hkv, 100, d)).astype(np.float16)
+    v = rng.standard_normal((Bn, Hkv, 100, d)).astype(np.float16)
+    caches = [zkv.RVQKVCache(_cuda(Ck), _cuda(Cv), batch=Bn, capacity=112, window=W)
+              for _ in range(2)]
+    for c in caches:
+        c.prefill(_cuda(k), _cuda(v))
+    for step in range(5):
+        nk = _cuda(rng.standard_normal((Bn, Hkv, d)).astype(np.float16))
+        nv = _cuda(rng.standard_normal((Bn, Hkv, d)).astype(np.float16))
+        q = _cuda(rng.standard_normal((Bn, Hq, d)).astype(np.float16))
+        caches[0].append(nk, nv)
+        o0, l0 = caches[0].attend(q)
+        o1, l1 = caches[1].step(nk, nv, q)
+        assert torch.equal(o0, o1) and torch.equal(l0, l1), step
+    for name in ("k_codes", "v_codes", "win_k", "win_v", "comp_len", "win_len", "win_head"):
+        assert torch.equal(getattr(caches[0], name), getattr(caches[1], name)), name
+    assert int(caches[0].error_flag.item()) == 0 and int(caches[1].error_flag.item()) == 0
+
+
 def test_prepared_calls_match_the_plain_entry_points():
     """PreparedAppend / PreparedDecode (arguments marshalled once) give bit-identical results
     to rvq_append / rvq_decode_attn over several serving steps."""
