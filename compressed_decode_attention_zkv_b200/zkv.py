@@ -102,6 +102,16 @@ class PQDecodeParams(ctypes.Structure):
                 ("k_smooth", c_void_p)]
 
 
+class PQAppendParams(ctypes.Structure):
+    _fields_ = [("B", c_int), ("Hkv", c_int), ("d", c_int), ("m", c_int),
+                ("Tcap", c_int64), ("Wcap", c_int64),
+                ("new_k", c_void_p), ("new_v", c_void_p), ("win_k", c_void_p),
+                ("win_v", c_void_p), ("win_len", c_void_p), ("win_head", c_void_p),
+                ("comp_len", c_void_p), ("k_codes", c_void_p), ("v_codes", c_void_p),
+                ("k_codebook", c_void_p), ("v_codebook", c_void_p), ("error_flag", c_void_p),
+                ("k_smooth", c_void_p)]
+
+
 class MergeParams(ctypes.Structure):
     _fields_ = [("n_parts", c_int64), ("rows", c_int64), ("d", c_int),
                 ("part_out", c_void_p), ("out_part_stride", c_int64), ("out_row_stride", c_int64),
@@ -139,6 +149,8 @@ def lib() -> ctypes.CDLL:
         L.zkv_rvq_append.argtypes = [POINTER(AppendParams), c_void_p]
         L.zkv_pq_encode.restype = c_int
         L.zkv_pq_encode.argtypes = [POINTER(PQEncodeParams), c_void_p]
+        L.zkv_pq_append.restype = c_int
+        L.zkv_pq_append.argtypes = [POINTER(PQAppendParams), c_void_p]
         L.zkv_pq_decode_workspace_size.restype = c_size_t
         L.zkv_pq_decode_workspace_size.argtypes = [POINTER(PQDecodeParams)]
         L.zkv_pq_decode_attn.restype = c_int
@@ -604,6 +616,41 @@ def pq_encode(x: torch.Tensor, codebook: torch.Tensor, codes: torch.Tensor | Non
     return codes
 
 
+def pq_append(new_k, new_v, win_k, win_v, win_len, win_head, comp_len, k_codes, v_codes,
+              k_codebook, v_codebook, error_flag=None, k_smooth=None):
+    """One serving step of cache maintenance for a product-VQ cache (see include/zkv.h):
+    the new token enters the window, a full window's oldest token is product-VQ encoded onto
+    the prefix.  State updated in place.  codes uint8 [B, Hkv, Tcap, d/m]; codebooks float32
+    [Hkv, 256, m]."""
+    _need(new_k, "new_k", torch.float16)
+    _need(new_v, "new_v", torch.float16)
+    for n, t in (("win_k", win_k), ("win_v", win_v)):
+        _need(t, n, torch.float16)
+    for n, t in (("win_len", win_len), ("win_head", win_head), ("comp_len", comp_len)):
+        _need(t, n, torch.int32)
+    for n, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, n, torch.uint8)
+    for n, t in (("k_codebook", k_codebook), ("v_codebook", v_codebook)):
+        _need(t, n, torch.float32)
+    if error_flag is not None:
+        _need(error_flag, "error_flag", torch.int32)
+    B, Hkv, d = new_k.shape
+    _, _, Tcap, nsub = k_codes.shape
+    m = k_codebook.shape[-1]
+    if nsub * m != d or tuple(v_codes.shape) != tuple(k_codes.shape):
+        raise ValueError("codes must be [B, Hkv, Tcap, d/m] for K and V")
+    if tuple(new_v.shape) != (B, Hkv, d) or win_k.shape[:2] != (B, Hkv):
+        raise ValueError("new tokens [B, Hkv, d] and window [B, Hkv, Wcap, d] must agree")
+    p = PQAppendParams(B=B, Hkv=Hkv, d=d, m=m, Tcap=Tcap, Wcap=win_k.shape[2],
+                       new_k=_ptr(new_k), new_v=_ptr(new_v), win_k=_ptr(win_k),
+                       win_v=_ptr(win_v), win_len=_ptr(win_len), win_head=_ptr(win_head),
+                       comp_len=_ptr(comp_len), k_codes=_ptr(k_codes), v_codes=_ptr(v_codes),
+                       k_codebook=_ptr(k_codebook), v_codebook=_ptr(v_codebook),
+                       error_flag=_ptr(error_flag),
+                       k_smooth=_smooth_ptr(k_smooth, Hkv, d, "k_smooth"))
+    _check("zkv_pq_append", lib().zkv_pq_append(ctypes.byref(p), _stream()))
+
+
 def pq_decode_workspace_size(q, k_codes, k_codebook, win_k, max_comp_len=None) -> int:
     """Bytes of device workspace zkv_pq_decode_attn needs for these shapes (see include/zkv.h);
     pass a buffer of this size as ``workspace`` to keep allocation out of a timed loop."""
@@ -781,6 +828,88 @@ class RVQKVCache:
                               max_comp_len=self.max_comp_len, softmax_scale=softmax_scale,
                               workspace=self._ws, error_flag=self.error_flag,
                               k_smooth=self.k_smooth)
+
+    def memory_bytes(self) -> int:
+        """Bytes held by codes and window (codebooks are shared across layers' caches)."""
+        return sum(t.numel() * t.element_size() for t in
+                   (self.k_codes, self.v_codes, self.win_k, self.win_v))
+
+
+class PQKVCache:
+    """Product-VQ (VecInfer-style) compressed KV cache of one attention layer: d/m code bytes
+    per token for K and for V (one 256-entry codebook of m-dim sub-vectors per kv head and K or
+    V), an fp16 window for the newest tokens.  The same interface as RVQKVCache: prefill(),
+    append(), attend(), step(), memory_bytes().  k_smooth: optional float32 [Hkv, d] key
+    smoothing factors (the key codebooks must have been trained on smoothed keys)."""
+
+    def __init__(self, k_codebook: torch.Tensor, v_codebook: torch.Tensor, batch: int,
+                 capacity: int, window: int, head_dim: int, device="cuda",
+                 k_smooth: torch.Tensor | None = None):
+        Hkv, _, m = k_codebook.shape
+        if head_dim % m:
+            raise ValueError("head_dim must be a multiple of the sub-vector size")
+        self.Ck, self.Cv = k_codebook.contiguous(), v_codebook.contiguous()
+        self.k_smooth = None if k_smooth is None else k_smooth.contiguous()
+        self.B, self.Hkv, self.d, self.m = batch, Hkv, head_dim, m
+        self.Tcap = (capacity + 15) // 16 * 16
+        self.Wcap = window
+        dev = torch.device(device)
+        nsub = head_dim // m
+        self.k_codes = torch.zeros((batch, Hkv, self.Tcap, nsub), dtype=torch.uint8, device=dev)
+        self.v_codes = torch.zeros((batch, Hkv, self.Tcap, nsub), dtype=torch.uint8, device=dev)
+        self.win_k = torch.zeros((batch, Hkv, window, head_dim), dtype=torch.float16, device=dev)
+        self.win_v = torch.zeros((batch, Hkv, window, head_dim), dtype=torch.float16, device=dev)
+        self.comp_len = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.win_len = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.win_head = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.error_flag = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.max_comp_len = 0
+        self._ws = None
+
+    def prefill(self, k: torch.Tensor, v: torch.Tensor):
+        """k, v: fp16 [B, Hkv, T, d].  The last min(T, window) tokens go to the window, the
+        rest are encoded."""
+        T = k.shape[2]
+        W = min(T, self.Wcap)
+        Tc = T - W
+        if Tc > self.Tcap:
+            raise ValueError("prompt longer than capacity + window")
+        if Tc > 0:
+            pq_encode(k[:, :, :Tc].permute(0, 2, 1, 3), self.Ck,
+                      codes=self.k_codes[:, :, :Tc].permute(0, 2, 1, 3), smooth=self.k_smooth)
+            pq_encode(v[:, :, :Tc].permute(0, 2, 1, 3), self.Cv,
+                      codes=self.v_codes[:, :, :Tc].permute(0, 2, 1, 3))
+        self.win_k[:, :, :W].copy_(k[:, :, Tc:])
+        self.win_v[:, :, :W].copy_(v[:, :, Tc:])
+        self.comp_len.fill_(Tc)
+        self.win_len.fill_(W)
+        self.win_head.zero_()
+        self.max_comp_len = Tc
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor):
+        """k_new, v_new: fp16 [B, Hkv, d]."""
+        pq_append(k_new.contiguous(), v_new.contiguous(), self.win_k, self.win_v, self.win_len,
+                  self.win_head, self.comp_len, self.k_codes, self.v_codes, self.Ck, self.Cv,
+                  self.error_flag, self.k_smooth)
+        self.max_comp_len = min(self.max_comp_len + 1, self.Tcap)
+
+    def attend(self, q: torch.Tensor, softmax_scale=None, out=None, lse=None):
+        """q: fp16 [B, Hq, d] -> (out float32 [B, Hq, d], lse float32 [B, Hq])."""
+        need = pq_decode_workspace_size(q, self.k_codes, self.Ck, self.win_k,
+                                        max_comp_len=self.max_comp_len)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        return pq_decode_attn(q, self.k_codes, self.v_codes, self.comp_len, self.Ck, self.Cv,
+                              self.win_k, self.win_v, self.win_len, out=out, lse=lse,
+                              max_comp_len=self.max_comp_len, softmax_scale=softmax_scale,
+                              workspace=self._ws, error_flag=self.error_flag,
+                              k_smooth=self.k_smooth)
+
+    def step(self, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+             softmax_scale=None, out=None, lse=None):
+        """append(k_new, v_new) then attend(q)."""
+        self.append(k_new, v_new)
+        return self.attend(q, softmax_scale=softmax_scale, out=out, lse=lse)
 
     def memory_bytes(self) -> int:
         """Bytes held by codes and window (codebooks are shared across layers' caches)."""

@@ -335,6 +335,46 @@ typedef struct {
 int zkv_pq_encode(const zkv_pq_encode_params* p, void* stream);
 
 /*
+ * zkv_pq_append -- one serving step of cache maintenance for a product-VQ cache: each
+ * sequence's new token enters the fp16 window; when the window is full its oldest token is
+ * evicted, product-VQ encoded (as zkv_pq_encode with rotate = 1; keys smoothed by k_smooth
+ * when given) and appended to the compressed prefix.
+ * Passages: VeloxQuant "VecInfer" (product VQ of the smoothed, rotated vectors) and "Quick
+ * start" (cache.append then cache.attend); VQKV section 2.3 "Local Sliding Window".
+ * Per sequence b, the window rule of zkv_rvq_append:
+ *   if win_len[b] < Wcap:  slot = win_len[b]; win_len[b] += 1
+ *   else: slot = win_head[b]; encode win_k/win_v[b][:][slot] into k_codes/v_codes at position
+ *         comp_len[b]; comp_len[b] += 1; win_head[b] = (slot + 1) % Wcap
+ *   win_k[b][:][slot] = new_k[b]; win_v[b][:][slot] = new_v[b]
+ * If comp_len[b] == Tcap when an eviction is due, sequence b is left unchanged and
+ * ZKV_DEVERR_COMP_LEN is set (ZKV_DEVERR_WIN_LEN for a window length outside 0..Wcap).
+ * Layouts: codes uint8 [B][Hkv][Tcap][d / m]; codebooks float32 [Hkv][256][m]; window fp16
+ * [B][Hkv][Wcap][d]; new_k / new_v fp16 [B][Hkv][d]; lengths int32 [B]; k_smooth float32
+ * [Hkv][d] or NULL.  d in {64, 128, 256}, m in {2, 4, 8, 16}, Wcap >= 1.  Two kernels are
+ * launched (encode + window write, then the length update).  No workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED (d, m), CUDA.
+ */
+typedef struct {
+  int B, Hkv, d, m;
+  int64_t Tcap, Wcap;
+  const uint16_t* new_k;
+  const uint16_t* new_v;
+  uint16_t* win_k;
+  uint16_t* win_v;
+  int32_t* win_len;
+  int32_t* win_head;
+  int32_t* comp_len;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  const float* k_codebook;
+  const float* v_codebook;
+  int32_t* error_flag;
+  const float* k_smooth;
+} zkv_pq_append_params;
+
+int zkv_pq_append(const zkv_pq_append_params* p, void* stream);
+
+/*
  * zkv_pq_decode_attn -- decode attention over a product-VQ compressed prefix (zkv_pq_encode's
  * codes, keys and values) plus the fp16 recency window.
  * Passages: VeloxQuant "VecInfer" (product VQ with the dual transform absorbed into the query);

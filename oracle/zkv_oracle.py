@@ -514,9 +514,10 @@ def pq_decode_attn_lut(q, k_codes, v_codes, comp_len, Ck, Cv, win_k, win_v, win_
 # Serving step  (VQKV section 2.3 "Local Sliding Window"; VeloxQuant append / attend)
 # --------------------------------------------------------------------------------------------
 
-def append_step(state: dict, new_k: np.ndarray, new_v: np.ndarray) -> dict:
+def append_step(state: dict, new_k: np.ndarray, new_v: np.ndarray, pq: bool = False) -> dict:
     """One token per sequence enters the window; when the window is full its oldest token
-    leaves it and is RVQ-encoded onto the end of the compressed prefix.
+    leaves it and is RVQ-encoded (product-VQ encoded with ``pq``: codes [d/m] per token,
+    codebooks [Hkv][K][m]) onto the end of the compressed prefix.
 
     state: k_codes, v_codes [B][Hkv][Tcap][S] uint8; comp_len [B]; win_k, win_v
     [B][Hkv][Wcap][d] fp16; win_len [B]; win_head [B] (slot of the oldest token once the window
@@ -545,9 +546,14 @@ def append_step(state: dict, new_k: np.ndarray, new_v: np.ndarray) -> dict:
                 continue
             for h in range(Hkv):
                 ks = st.get("k_smooth")
-                zk, _, _, _ = rvq_encode(st["win_k"][b, h, slot][None], st["Ck"][h],
-                                         smooth=None if ks is None else ks[h])
-                zv, _, _, _ = rvq_encode(st["win_v"][b, h, slot][None], st["Cv"][h])
+                lam = None if ks is None else ks[h]
+                if pq:
+                    zk, _ = pq_encode(st["win_k"][b, h, slot][None], st["Ck"][h], smooth=lam)
+                    zv, _ = pq_encode(st["win_v"][b, h, slot][None], st["Cv"][h])
+                else:
+                    zk, _, _, _ = rvq_encode(st["win_k"][b, h, slot][None], st["Ck"][h],
+                                             smooth=lam)
+                    zv, _, _, _ = rvq_encode(st["win_v"][b, h, slot][None], st["Cv"][h])
                 st["k_codes"][b, h, pos] = zk[0]
                 st["v_codes"][b, h, pos] = zv[0]
             st["comp_len"][b] = pos + 1

@@ -198,6 +198,23 @@ def test_pq_decode_validation(L):
         assert L.zkv_pq_decode_workspace_size(ctypes.byref(mk(**kw))) > 0, kw
 
 
+def test_pq_append_validation(L):
+    def mk(**kw):
+        base = dict(B=2, Hkv=2, d=128, m=4, Tcap=64, Wcap=8, new_k=0x1000, new_v=0x2000,
+                    win_k=0x3000, win_v=0x4000, win_len=0x5000, win_head=0x6000,
+                    comp_len=0x7000, k_codes=0x8000, v_codes=0x9000, k_codebook=0xa000,
+                    v_codebook=0xb000)
+        base.update(kw)
+        return zkv.PQAppendParams(**base)
+    for kw, st in ((dict(d=96), zkv.ZKV_ERR_UNSUPPORTED), (dict(m=3), zkv.ZKV_ERR_UNSUPPORTED),
+                   (dict(Wcap=0), zkv.ZKV_ERR_INVALID_ARG), (dict(B=-1), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(Hkv=0), zkv.ZKV_ERR_INVALID_ARG), (dict(win_head=0), zkv.ZKV_ERR_INVALID_ARG),
+                   (dict(v_codebook=0), zkv.ZKV_ERR_INVALID_ARG)):
+        assert L.zkv_pq_append(ctypes.byref(mk(**kw)), None) == st, kw
+    assert L.zkv_pq_append(ctypes.byref(mk(B=0)), None) == zkv.ZKV_OK   # nothing to do
+    assert L.zkv_pq_append(None, None) == zkv.ZKV_ERR_INVALID_ARG
+
+
 def test_pq_decode_workspace_size_binding(L):
     """The binding's size query reads shapes only; the layout is six 256-byte-aligned float32
     arrays: chunk maxima, sums and outputs, then the window's maxima, sums and outputs."""
@@ -246,7 +263,8 @@ def test_ctypes_structs_match_the_header_layout(tmp_path):
     pairs = [("zkv_encode_params", zkv.EncodeParams), ("zkv_reconstruct_params", zkv.ReconstructParams),
              ("zkv_decode_params", zkv.DecodeParams), ("zkv_append_params", zkv.AppendParams),
              ("zkv_lse_merge_params", zkv.MergeParams), ("zkv_pq_encode_params", zkv.PQEncodeParams),
-             ("zkv_pq_decode_params", zkv.PQDecodeParams)]
+             ("zkv_pq_decode_params", zkv.PQDecodeParams),
+             ("zkv_pq_append_params", zkv.PQAppendParams)]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zkv.h"', "int main(void) {"]
     for cname, cls in pairs:
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')

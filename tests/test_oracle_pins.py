@@ -411,6 +411,36 @@ def test_append_step_window_then_eviction():
     assert st["comp_len"][1] == 5
 
 
+def test_append_step_product_vq_encodes_the_evicted_token():
+    """With pq=True the evicted token is product-VQ encoded (keys smoothed, values not) to
+    position comp_len; the window rule is the RVQ one."""
+    rng = np.random.default_rng(32)
+    B, Hkv, Wcap, d, m, Tcap = 2, 2, 2, 16, 4, 6
+    Ck = rng.standard_normal((Hkv, 256, m)).astype(np.float32)
+    Cv = rng.standard_normal((Hkv, 256, m)).astype(np.float32)
+    lam = np.exp(rng.standard_normal((Hkv, d)) * 0.3).astype(np.float32)
+    st = dict(k_codes=np.zeros((B, Hkv, Tcap, d // m), np.uint8),
+              v_codes=np.zeros((B, Hkv, Tcap, d // m), np.uint8), comp_len=np.array([3, 0]),
+              win_k=rng.standard_normal((B, Hkv, Wcap, d)).astype(np.float16),
+              win_v=rng.standard_normal((B, Hkv, Wcap, d)).astype(np.float16),
+              win_len=np.array([2, 1]), win_head=np.array([1, 0]), Ck=Ck, Cv=Cv, k_smooth=lam)
+    nk = rng.standard_normal((B, Hkv, d)).astype(np.float16)
+    nv = rng.standard_normal((B, Hkv, d)).astype(np.float16)
+    out = O.append_step(st, nk, nv, pq=True)
+    assert out["comp_len"].tolist() == [4, 0] and out["win_len"].tolist() == [2, 2]
+    assert out["win_head"].tolist() == [0, 0]
+    for h in range(Hkv):
+        zk, _ = O.pq_encode(st["win_k"][0, h, 1][None], Ck[h], smooth=lam[h])
+        zv, _ = O.pq_encode(st["win_v"][0, h, 1][None], Cv[h])
+        np.testing.assert_array_equal(out["k_codes"][0, h, 3], zk[0])
+        np.testing.assert_array_equal(out["v_codes"][0, h, 3], zv[0])
+        zk_plain, _ = O.pq_encode(st["win_k"][0, h, 1][None], Ck[h])
+        assert not np.array_equal(zk_plain[0], zk[0])   # the smoothing was applied
+    np.testing.assert_array_equal(out["win_k"][0, :, 1], nk[0])
+    np.testing.assert_array_equal(out["win_v"][1, :, 1], nv[1])
+    assert not out["error"]
+
+
 def test_append_step_at_capacity_leaves_sequence_unchanged():
     rng = np.random.default_rng(31)
     B, Hkv, Wcap, d, Tcap, S, K = 1, 1, 2, 64, 4, 1, 8

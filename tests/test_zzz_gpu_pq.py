@@ -102,3 +102,101 @@ def test_pq_decode_matches_oracle(cfg):
     assert np.max(np.abs(lse[fin] - want_l[fin]), initial=0.0) <= 2e-3
     assert np.all(out[~fin] == 0)
     assert int(err.item()) == 0
+
+
+def _pq_state(seed, Bn, Hkv, d, m, Tcap, Wcap, win_len, win_head, comp_len):
+    rng = np.random.default_rng(seed)
+    nsub = d // m
+    return dict(k_codes=rng.integers(0, 256, (Bn, Hkv, Tcap, nsub)).astype(np.uint8),
+                v_codes=rng.integers(0, 256, (Bn, Hkv, Tcap, nsub)).astype(np.uint8),
+                comp_len=np.array(comp_len), win_len=np.array(win_len),
+                win_head=np.array(win_head),
+                win_k=rng.standard_normal((Bn, Hkv, Wcap, d)).astype(np.float16),
+                win_v=rng.standard_normal((Bn, Hkv, Wcap, d)).astype(np.float16),
+                Ck=(rng.standard_normal((Hkv, 256, m)) * 0.5).astype(np.float32),
+                Cv=rng.standard_normal((Hkv, 256, m)).astype(np.float32),
+                k_smooth=np.exp(rng.standard_normal((Hkv, d)) * 0.3).astype(np.float32))
+
+
+@pytest.mark.parametrize("d,m", [(128, 4), (64, 2), (256, 16)])
+def test_pq_append_steps_match_oracle(d, m):
+    """zkv_pq_append against the oracle's append step (product VQ): free slots, evictions with
+    smoothed keys, a full prefix (left unchanged and flagged), over several steps."""
+    st = _pq_state(300 + d, Bn=5, Hkv=2, d=d, m=m, Tcap=16, Wcap=3, win_len=[0, 2, 3, 3, 3],
+                   win_head=[0, 0, 1, 2, 0], comp_len=[0, 4, 7, 15, 16])
+    rng = np.random.default_rng(301)
+    g = {k: _cuda(v.astype(np.int32) if k in ("comp_len", "win_len", "win_head") else v)
+         for k, v in st.items()}
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for step in range(4):
+        nk = rng.standard_normal((5, 2, d)).astype(np.float16)
+        nv = rng.standard_normal((5, 2, d)).astype(np.float16)
+        zkv.pq_append(_cuda(nk), _cuda(nv), g["win_k"], g["win_v"], g["win_len"], g["win_head"],
+                      g["comp_len"], g["k_codes"], g["v_codes"], g["Ck"], g["Cv"],
+                      error_flag=err, k_smooth=g["k_smooth"])
+        st = O.append_step(st, nk, nv, pq=True)
+        for key in ("k_codes", "v_codes", "win_k", "win_v", "comp_len", "win_len", "win_head"):
+            np.testing.assert_array_equal(g[key].cpu().numpy(), st[key], err_msg=f"{key} {step}")
+    assert st["error"] and int(err.item()) == 1   # the full prefix (ZKV_DEVERR_COMP_LEN)
+
+
+def test_pq_cache_serving_loop_matches_oracle():
+    """PQKVCache: prefill, then step (append + attend) x 5 against the oracle's append step and
+    its decode (direct form), with key smoothing; append + attend equals step."""
+    rng = np.random.default_rng(310)
+    Bn, Hq, Hkv, d, m, W, T0 = 2, 8, 2, 128, 4, 8, 200
+    wl = I.workload("llama3_8b_32k", B=Bn, Hq=Hq, Hkv=Hkv, T=T0, W=W, n_cal=1024,
+                    kmeans_iters=3)
+    lam = I.key_smooth_factors(wl)
+    Ck = I.train_pq_codebook(wl, "k", m, smooth=lam)
+    Cv = I.train_pq_codebook(wl, "v", m)
+    k = np.stack([I.kv_tokens(wl, "k", b, 0, T0) for b in range(Bn)])
+    v = np.stack([I.kv_tokens(wl, "v", b, 0, T0) for b in range(Bn)])
+    caches = [zkv.PQKVCache(_cuda(Ck), _cuda(Cv), batch=Bn, capacity=T0, window=W, head_dim=d,
+                            k_smooth=_cuda(lam)) for _ in range(2)]
+    for c in caches:
+        c.prefill(_cuda(k), _cuda(v))
+    Tc = T0 - W
+    Tcap = caches[0].Tcap
+
+    def walk_ok(rows, book, codes, smooth=None):   # float64 argmin up to counted near-ties
+        w = O.pq_match_walk(rows, book, codes, smooth=smooth)
+        return w["mismatches"] == 0 and w["exceptions"] <= 2
+
+    zk = caches[0].k_codes.cpu().numpy()
+    zv = caches[0].v_codes.cpu().numpy()
+    for b in range(Bn):
+        for h in range(Hkv):
+            assert walk_ok(k[b, h, :Tc], Ck[h], zk[b, h, :Tc], smooth=lam[h])
+            assert walk_ok(v[b, h, :Tc], Cv[h], zv[b, h, :Tc])
+    # the oracle continues from the GPU's (verified) codes
+    st = dict(k_codes=zk, v_codes=zv, comp_len=np.full(Bn, Tc), win_len=np.full(Bn, W),
+              win_head=np.zeros(Bn, np.int64), win_k=k[:, :, Tc:].copy(),
+              win_v=v[:, :, Tc:].copy(), Ck=Ck, Cv=Cv, k_smooth=lam)
+    for step in range(5):
+        nk = rng.standard_normal((Bn, Hkv, d)).astype(np.float16)
+        nv = rng.standard_normal((Bn, Hkv, d)).astype(np.float16)
+        q = rng.standard_normal((Bn, Hq, d)).astype(np.float16)
+        o1, l1 = caches[0].step(_cuda(nk), _cuda(nv), _cuda(q))
+        caches[1].append(_cuda(nk), _cuda(nv))
+        o2, l2 = caches[1].attend(_cuda(q))
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        before = st
+        st = O.append_step(st, nk, nv, pq=True)
+        gk, gv = caches[0].k_codes.cpu().numpy(), caches[0].v_codes.cpu().numpy()
+        for b in range(Bn):   # the evicted token of every sequence, encoded at comp_len
+            pos, slot = int(before["comp_len"][b]), int(before["win_head"][b])
+            for h in range(Hkv):
+                assert walk_ok(before["win_k"][b, h, slot][None], Ck[h], gk[b, h, pos][None],
+                               smooth=lam[h])
+                assert walk_ok(before["win_v"][b, h, slot][None], Cv[h], gv[b, h, pos][None])
+        st["k_codes"], st["v_codes"] = gk, gv
+        for key in ("win_k", "win_v", "comp_len", "win_len", "win_head"):
+            np.testing.assert_array_equal(getattr(caches[0], key).cpu().numpy(), st[key])
+        want_o, want_l = O.pq_decode_attn(q, st["k_codes"], st["v_codes"], st["comp_len"], Ck,
+                                          Cv, st["win_k"], st["win_v"], st["win_len"],
+                                          k_smooth=lam)
+        assert np.max(np.abs(o1.cpu().numpy() - want_o)) <= 2e-3
+        assert np.max(np.abs(l1.cpu().numpy() - want_l)) <= 2e-3
+    assert int(caches[0].error_flag.item()) == 0
+    assert caches[0].memory_bytes() == 2 * Bn * Hkv * (Tcap * d // m + W * d * 2)
