@@ -850,7 +850,10 @@ def run_ours(args):
     extras = {}
     if not args.no_encode and rank == 0:
         del graphs, soak_graphs
-        extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
+        try:
+            extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
+        except Exception as exc:   # an extra never takes the main line down
+            extras["encode"] = {"error": f"{type(exc).__name__}: {exc}"}
     base_ms = 1000.0 * elapsed / args.steps
     for name, kw, skip in (("smooth", dict(smooth=True), args.no_smooth),
                            ("paged", dict(page_tokens=256), args.no_paged)):
