@@ -119,6 +119,13 @@ class MergeParams(ctypes.Structure):
                 ("out", c_void_p), ("lse", c_void_p)]
 
 
+class MergePeersParams(ctypes.Structure):
+    _fields_ = [("n_ranks", c_int), ("rank", c_int), ("rows", c_int64), ("d", c_int),
+                ("part_out", c_void_p), ("part_lse", c_void_p), ("flags", c_void_p),
+                ("epoch", ctypes.c_uint32), ("timeout_ns", c_int64),
+                ("out", c_void_p), ("lse", c_void_p), ("error_flag", c_void_p)]
+
+
 _lib = None
 
 
@@ -155,6 +162,8 @@ def lib() -> ctypes.CDLL:
         L.zkv_pq_decode_workspace_size.argtypes = [POINTER(PQDecodeParams)]
         L.zkv_pq_decode_attn.restype = c_int
         L.zkv_pq_decode_attn.argtypes = [POINTER(PQDecodeParams), c_void_p, c_size_t, c_void_p]
+        L.zkv_lse_merge_peers.restype = c_int
+        L.zkv_lse_merge_peers.argtypes = [POINTER(MergePeersParams), c_void_p]
         L.zkv_lse_merge.restype = c_int
         L.zkv_lse_merge.argtypes = [POINTER(MergeParams), c_void_p]
         L.zkv_rvq_serve_step.restype = c_int
@@ -740,6 +749,37 @@ def lse_merge(part_out: torch.Tensor, part_lse: torch.Tensor, out=None, lse=None
                     out_row_stride=po.stride(1), part_lse=_ptr(pl), lse_part_stride=pl.stride(0),
                     lse_row_stride=pl.stride(1), out=_ptr(out), lse=_ptr(lse))
     _check("zkv_lse_merge", lib().zkv_lse_merge(ctypes.byref(p), _stream()))
+    return out, lse
+
+
+def lse_merge_peers(part_out_ptrs: torch.Tensor, part_lse_ptrs: torch.Tensor,
+                    flag_ptrs: torch.Tensor, rank: int, epoch: int, rows: int, d: int,
+                    out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                    error_flag: torch.Tensor | None = None, timeout_s: float = 2.0):
+    """The context-parallel exchange and combine in one kernel over peer memory (see
+    include/zkv.h).  part_out_ptrs / part_lse_ptrs / flag_ptrs: int64 CUDA tensors [n_ranks]
+    holding every rank's out-rows / lse-rows / flag-array device addresses as mapped in this
+    process.  Returns (out float32 [rows, d], lse float32 [rows])."""
+    for n, t in (("part_out_ptrs", part_out_ptrs), ("part_lse_ptrs", part_lse_ptrs),
+                 ("flag_ptrs", flag_ptrs)):
+        _need(t, n, torch.int64)
+    n = part_out_ptrs.numel()
+    if part_lse_ptrs.numel() != n or flag_ptrs.numel() != n:
+        raise ValueError("one out, lse and flag address per rank")
+    dev = part_out_ptrs.device
+    if out is None:
+        out = torch.empty((rows, d), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((rows,), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32)
+    _need(lse, "lse", torch.float32)
+    if error_flag is not None:
+        _need(error_flag, "error_flag", torch.int32)
+    p = MergePeersParams(n_ranks=n, rank=rank, rows=rows, d=d, part_out=_ptr(part_out_ptrs),
+                         part_lse=_ptr(part_lse_ptrs), flags=_ptr(flag_ptrs),
+                         epoch=epoch & 0xFFFFFFFF, timeout_ns=int(timeout_s * 1e9),
+                         out=_ptr(out), lse=_ptr(lse), error_flag=_ptr(error_flag))
+    _check("zkv_lse_merge_peers", lib().zkv_lse_merge_peers(ctypes.byref(p), _stream()))
     return out, lse
 
 

@@ -443,6 +443,47 @@ typedef struct {
 
 int zkv_lse_merge(const zkv_lse_merge_params* p, void* stream);
 
+/*
+ * zkv_lse_merge_peers -- the context-parallel exchange and the log-sum-exp combine as ONE
+ * kernel over peer memory (in place of an all-gather followed by zkv_lse_merge).
+ * Passage: Differential-KV "Decode & Prefill Innovations" (fp32 log-sum-exp combine of
+ * partial attentions over disjoint key sets).
+ * Every rank's decode has written its partial (out [rows][d], lse [rows]) into buffers that
+ * every rank can address (symmetric / IPC-mapped device memory).  The kernel, on rank `rank`
+ * of n_ranks:
+ *   1. signals: stores `epoch` into word `rank` of every rank's flag array (release, system
+ *      scope; every block stores the same value, so no block waits for another to run);
+ *   2. waits until every word of its own flag array has reached `epoch` (acquire, system
+ *      scope), for at most timeout_ns nanoseconds of the device's global timer;
+ *   3. reads every rank's rows straight from that rank's memory (cache-bypassing loads over
+ *      NVLink) and combines them exactly as zkv_lse_merge.
+ * If the wait runs out, ZKV_DEVERR_TIMEOUT is OR-ed into error_flag and the blocks that timed
+ * out leave their rows of out / lse unwritten; nothing hangs.
+ * Arguments: part_out / part_lse / flags are DEVICE arrays of n_ranks device pointers
+ * (rank i's out rows, lse rows and flag array of n_ranks uint32 words, as mapped in this
+ * process); epoch >= 1, one more than the previous call's on the same flags (flags start at
+ * 0; compared modulo 2^32).  A rank's out / lse buffers must not be rewritten until every
+ * rank has passed the next call's wait: alternating two buffer sets by epoch parity gives
+ * exactly that.  out float32 [rows][d], lse [rows] (may be NULL).  d in 1..4096,
+ * 1 <= n_ranks <= 64, 0 <= rank < n_ranks.
+ * Errors: INVALID_ARG, CUDA.
+ */
+typedef struct {
+  int n_ranks, rank;
+  int64_t rows;
+  int d;
+  const float* const* part_out;
+  const float* const* part_lse;
+  uint32_t* const* flags;
+  uint32_t epoch;
+  int64_t timeout_ns;
+  float* out;
+  float* lse;
+  int32_t* error_flag;
+} zkv_lse_merge_peers_params;
+
+int zkv_lse_merge_peers(const zkv_lse_merge_peers_params* p, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -245,6 +245,19 @@ def test_lse_merge_validation(L):
     assert L.zkv_lse_merge(None, None) == zkv.ZKV_ERR_INVALID_ARG
 
 
+def test_lse_merge_peers_validation(L):
+    def mk(**kw):
+        base = dict(n_ranks=2, rank=1, rows=4, d=8, part_out=0x1000, part_lse=0x2000,
+                    flags=0x3000, epoch=1, timeout_ns=1000000, out=0x4000, lse=0x5000)
+        base.update(kw)
+        return zkv.MergePeersParams(**base)
+    for kw in (dict(n_ranks=0), dict(n_ranks=65), dict(rank=2), dict(rank=-1), dict(d=0),
+               dict(d=5000), dict(rows=-1), dict(epoch=0), dict(timeout_ns=0),
+               dict(part_out=0), dict(part_lse=0), dict(flags=0), dict(out=0)):
+        assert L.zkv_lse_merge_peers(ctypes.byref(mk(**kw)), None) == zkv.ZKV_ERR_INVALID_ARG, kw
+    assert L.zkv_lse_merge_peers(None, None) == zkv.ZKV_ERR_INVALID_ARG
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 128, dtype=torch.float16)
@@ -264,7 +277,8 @@ def test_ctypes_structs_match_the_header_layout(tmp_path):
              ("zkv_decode_params", zkv.DecodeParams), ("zkv_append_params", zkv.AppendParams),
              ("zkv_lse_merge_params", zkv.MergeParams), ("zkv_pq_encode_params", zkv.PQEncodeParams),
              ("zkv_pq_decode_params", zkv.PQDecodeParams),
-             ("zkv_pq_append_params", zkv.PQAppendParams)]
+             ("zkv_pq_append_params", zkv.PQAppendParams),
+             ("zkv_lse_merge_peers_params", zkv.MergePeersParams)]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zkv.h"', "int main(void) {"]
     for cname, cls in pairs:
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')

@@ -102,6 +102,96 @@ def test_context_parallel_exchange_equals_unsharded_decode(world):
     np.testing.assert_array_equal(result[world - 1][4], comp)
 
 
+class _FakeSymmMem:
+    """Stands in for torch symmetric memory on CPU: plain tensors, and a rendezvous that
+    exchanges every rank's data address (meaningless across processes, but enough to check
+    the pointer tables the exchange builds)."""
+
+    def empty(self, shape, dtype, device):
+        return torch.zeros(shape, dtype=dtype, device=device)
+
+    def rendezvous(self, t, group):
+        mine = torch.tensor([t.data_ptr()], dtype=torch.int64)
+        every = [torch.zeros(1, dtype=torch.int64) for _ in range(dist.get_world_size(group))]
+        dist.all_gather(every, mine, group=group)
+
+        class Handle:
+            buffer_ptrs = [int(x) for x in every]
+        return Handle()
+
+
+def _fused_rank(rank, world, port, result):
+    """cp_decode_attn with a PeerExchange: the decode writes into this step's slot set and the
+    combine (emulated on CPU: gather the slots, oracle combine) receives the right pointer
+    tables, epoch and parity, step after step."""
+    from compressed_decode_attention_zkv_b200 import context_parallel as CP
+    from oracle import zkv_oracle as O
+    _init(rank, world, port)
+    try:
+        q, kc, vc, comp, Ck, Cv, wk, wv, win = (torch.from_numpy(a) for a in _case())
+        kl, vl, cl = CP.take_shard(kc, vc, comp, rank, world)
+        B, Hq, d = q.shape
+        calls = []
+
+        def decode_into(*args, out=None, lse=None, **kw):
+            o, l = _oracle_decode(*args)
+            out.copy_(o.to(torch.float32))
+            lse.copy_(l.to(torch.float32))
+            return out, lse
+
+        def merge(out_ptrs, lse_ptrs, flag_ptrs, r, epoch, rows, dd, out=None, lse=None,
+                  error_flag=None, timeout_s=None):
+            s = epoch & 1
+            calls.append((epoch, int(out_ptrs[r]), int(lse_ptrs[r]), int(flag_ptrs[r]),
+                          ex.out_buf[s].data_ptr(), ex.lse_buf[s].data_ptr(),
+                          ex.flag_buf.data_ptr(), r, rows, dd))
+            outs = [torch.zeros(rows, dd) for _ in range(world)]
+            lses = [torch.zeros(rows) for _ in range(world)]
+            dist.all_gather(outs, ex.out_buf[s].clone())
+            dist.all_gather(lses, ex.lse_buf[s].clone())
+            o = torch.empty(rows, dd, dtype=torch.float64)
+            lo = torch.empty(rows, dtype=torch.float64)
+            for i in range(rows):
+                oi, li = O.lse_merge([(outs[j][i].numpy(), float(lses[j][i]))
+                                      for j in range(world)])
+                o[i] = torch.from_numpy(np.asarray(oi))
+                lo[i] = li
+            return o, lo
+
+        ex = CP.PeerExchange(B * Hq, d, device=torch.device("cpu"), symm_mem=_FakeSymmMem(),
+                             merge_fn=merge)
+        outs = []
+        for _ in range(3):
+            out, lse = CP.cp_decode_attn(q, kl, vl, cl, Ck, Cv, wk, wv, win, decode_fn=decode_into,
+                                         exchange=ex)
+            outs.append((out.numpy(), lse.numpy()))
+        result[rank] = (outs, calls)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_fused_exchange_bookkeeping():
+    world = 2
+    result = mp.Manager().dict()
+    mp.spawn(_fused_rank, args=(world, _free_port(), result), nprocs=world, join=True)
+    from oracle import zkv_oracle as O
+    q, kc, vc, comp, Ck, Cv, wk, wv, win = _case()
+    want_o, want_l = O.decode_attn(q, kc, vc, comp, Ck, Cv, wk, wv, win)
+    fin = np.isfinite(want_l)
+    for r in range(world):
+        outs, calls = result[r]
+        for out, lse in outs:   # every step equals the unsharded decode (float32 partials)
+            np.testing.assert_allclose(out, want_o, atol=1e-5, rtol=0)
+            assert np.array_equal(fin, np.isfinite(lse))
+            np.testing.assert_allclose(lse[fin], want_l[fin], atol=1e-5, rtol=0)
+        assert [c[0] for c in calls] == [1, 2, 3]   # one epoch per step
+        for epoch, o_ptr, l_ptr, f_ptr, o_slot, l_slot, f_buf, rr, rows, dd in calls:
+            # this rank's entry of each table is the slot set of the step's parity
+            assert (o_ptr, l_ptr, f_ptr) == (o_slot, l_slot, f_buf)
+            assert rr == r and (rows, dd) == (q.shape[0] * q.shape[1], q.shape[2])
+        assert calls[0][4] != calls[1][4] and calls[0][4] == calls[2][4]   # sets alternate
+
+
 def _timing_rank(rank, world, port, result):
     import bench
     _init(rank, world, port)
