@@ -74,6 +74,9 @@ class PeerExchange:
             device = torch.device("cuda", torch.cuda.current_device())
         self.rows, self.d, self.timeout_s = rows, d, timeout_s
         self.merge_fn = zkv.lse_merge_peers if merge_fn is None else merge_fn
+        enable = getattr(symm_mem, "enable_symm_mem_for_group", None)
+        if enable is not None:   # required before a rendezvous by some torch versions
+            enable(self.group.group_name)
         self.out_buf = symm_mem.empty((2, rows, d), dtype=torch.float32, device=device)
         self.lse_buf = symm_mem.empty((2, rows), dtype=torch.float32, device=device)
         self.flag_buf = symm_mem.empty((self.world,), dtype=torch.int32, device=device)

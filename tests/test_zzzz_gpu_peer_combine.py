@@ -84,3 +84,51 @@ def test_peer_combine_wait_is_bounded_and_reported():
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     torch.testing.assert_close(out, want_o, rtol=0, atol=1e-6)
+
+
+def test_peer_exchange_one_rank_end_to_end(tmp_path):
+    """PeerExchange on a one-rank NCCL group: torch symmetric memory, the rendezvous, the
+    pointer tables and cp_decode_attn's fused path, three steps (both buffer sets).  With one
+    rank the combine of a single part returns it unchanged, so the result equals the plain
+    decode bit for bit."""
+    import datetime
+
+    import numpy as np
+    import torch.distributed as dist
+
+    from compressed_decode_attention_zkv_b200 import context_parallel as CP
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised in this process")
+    store = dist.FileStore(str(tmp_path / "store"), 1)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        rng = np.random.default_rng(400)
+        Bn, Hq, Hkv, d, S, Tcap, W = 2, 8, 2, 128, 4, 512, 8
+        cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()   # noqa: E731
+        kc = cu(rng.integers(0, 256, (Bn, Hkv, Tcap, S)).astype(np.uint8))
+        vc = cu(rng.integers(0, 256, (Bn, Hkv, Tcap, S)).astype(np.uint8))
+        Ck = (rng.standard_normal((Hkv, S, 256, d)) * 0.1).astype(np.float32)
+        Cv = (rng.standard_normal((Hkv, S, 256, d)) * 0.3).astype(np.float32)
+        Ck[:, :, 0] = 0
+        Cv[:, :, 0] = 0
+        Ck, Cv = cu(Ck), cu(Cv)
+        wk = cu(rng.standard_normal((Bn, Hkv, W, d)).astype(np.float16))
+        wv = cu(rng.standard_normal((Bn, Hkv, W, d)).astype(np.float16))
+        comp = cu(np.array([500, 37], np.int32))
+        win = cu(np.array([W, 3], np.int32))
+        try:
+            ex = CP.PeerExchange(Bn * Hq, d)
+        except (RuntimeError, NotImplementedError, AttributeError) as exc:
+            pytest.skip(f"torch symmetric memory unavailable here: {exc}")
+        for step in range(3):
+            q = cu(rng.standard_normal((Bn, Hq, d)).astype(np.float16))
+            out, lse = CP.cp_decode_attn(q, kc, vc, comp, Ck, Cv, wk, wv, win, exchange=ex)
+            want_o, want_l = zkv.rvq_decode_attn(q, kc, vc, comp, Ck, Cv, wk, wv, win)
+            torch.cuda.synchronize()
+            assert torch.equal(out, want_o) and torch.equal(lse, want_l), step
+        assert ex.epoch == 3
+        del ex
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
