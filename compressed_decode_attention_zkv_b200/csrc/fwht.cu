@@ -37,7 +37,7 @@ extern "C" const char* zkv_status_string(int status) {
   }
 }
 
-extern "C" int zkv_version(void) { return 100; }
+extern "C" int zkv_version(void) { return ZKV_VERSION; }
 
 extern "C" int zkv_fwht(const void* in, int in_dtype, float* out, int64_t n_vec, int d,
                         float scale, void* stream) {

@@ -66,7 +66,9 @@ typedef enum {
 /* Human-readable name of a status code (static string). */
 const char* zkv_status_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 1.01 adds the serving step, the paged layout,
+ * key smoothing, product VQ and the context-parallel combines to 1.00's encode / decode. */
+#define ZKV_VERSION 101
 int zkv_version(void);
 
 /*

@@ -42,7 +42,8 @@ def test_status_strings_and_version(L):
     assert zkv.status_string(0) == "ZKV_OK"
     assert zkv.status_string(3) == "ZKV_ERR_WORKSPACE"
     assert zkv.status_string(99) == "ZKV_ERR_UNKNOWN"
-    assert L.zkv_version() >= 100
+    text = open(os.path.join(ROOT, "include", "zkv.h")).read()
+    assert L.zkv_version() == int(re.search(r"#define ZKV_VERSION (\d+)", text).group(1))
 
 
 def test_fwht_validation(L):
