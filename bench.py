@@ -504,15 +504,16 @@ def pq_encode_extra(dev):
                     "sub-vector; codebook from 2048 calibration vectors x 4 k-means iterations"}
 
 
-def pq_decode_extra(dev, hbm_peak):
-    """Product-VQ decode (4-dim sub-vectors, 2 bits/elem on K and V) on the llama3_8b_32k shape:
-    seeded codes and codebooks, 2 rotating replicas (268 MB > L2), CUDA-event timed calls."""
+def pq_decode_extra(dev, hbm_peak, m=4):
+    """Product-VQ decode (m-dim sub-vectors: 2 bits/elem at m = 4, 1 at m = 8, on K and V) on
+    the llama3_8b_32k shape: seeded codes and codebooks, 2 rotating replicas (268 MB > L2 at
+    m = 4, 134 MB at m = 8), CUDA-event timed calls."""
     import torch
 
     from compressed_decode_attention_zkv_b200 import inputs as I
     from compressed_decode_attention_zkv_b200 import zkv
     wl = I.workload(WORKLOAD)
-    m, R = 4, 2
+    R = 2
     Tc, nsub = wl.Tc, wl.d // m
     g = torch.Generator(device=dev).manual_seed(11)
     reps = []
@@ -542,8 +543,8 @@ def pq_decode_extra(dev, hbm_peak):
     sec = s.elapsed_time(e) / 1000.0 / steps
     code_bytes = 2 * wl.B * wl.Hkv * Tc * nsub
     byts = code_bytes + 2 * wl.B * wl.Hkv * wl.W * wl.d * 2 + wl.B * wl.Hq * wl.d * (2 + 4)
-    return {"workload": f"{wl.name} shape, product VQ with 4-dim sub-vectors on K and V "
-                        "(2 bits/elem, 64 code bytes per token and kv head)",
+    return {"workload": f"{wl.name} shape, product VQ with {m}-dim sub-vectors on K and V "
+                        f"({8 // m} bits/elem, {2 * nsub} code bytes per token and kv head)",
             "value": wl.B * Tc / sec, "unit": UNIT, "us_per_call": sec * 1e6,
             "hbm_gbs": byts / sec / 1e9, "hbm_frac": byts / sec / 1e9 / hbm_peak,
             "note": "zkv_pq_decode_attn (lane = sub-vector scan + finalize), eager calls over "
@@ -874,7 +875,8 @@ def run_ours(args):
         torch.cuda.empty_cache()
     # the product-VQ extras come last: nothing measured above depends on them
     for name, fn in (("pq_encode", lambda: pq_encode_extra(dev)),
-                     ("pq_decode", lambda: pq_decode_extra(dev, hbm_peak))):
+                     ("pq_decode", lambda: pq_decode_extra(dev, hbm_peak)),
+                     ("pq_decode_m8", lambda: pq_decode_extra(dev, hbm_peak, m=8))):
         if args.no_encode or rank != 0:
             continue
         try:
