@@ -469,6 +469,78 @@ def ragged_extra(dev, hbm_peak, R=4, steps=100):
                     f"{rep_mb:.0f} MB (> L2); codes from the skewed code distribution"}
 
 
+def long_context_extra(dev, hbm_peak, R=24, calls=240):
+    """Decode attention on the qwen25_7b_128k workload (B 1, Hq 28 over Hkv 4, GQA 7, context
+    131072 with a 256-token window, Sk = 2 / Sv = 4): one zkv_rvq_decode_attn per call,
+    replayed from CUDA graphs over R rotating replicas of all inputs (R x 6.8 MB > L2).  Codes
+    from the input generator's code distribution; codebooks trained as for the main line."""
+    import torch
+
+    from compressed_decode_attention_zkv_b200 import inputs as I
+    from compressed_decode_attention_zkv_b200 import zkv
+    wl = I.workload("qwen25_7b_128k")
+    Tc = wl.Tc
+    Tcap = (Tc + 15) // 16 * 16
+    kc = torch.from_numpy(I.random_codes(wl, "k", Tcap)).to(dev)
+    vc = torch.from_numpy(I.random_codes(wl, "v", Tcap, seed=1)).to(dev)
+    Ck = torch.from_numpy(codebooks(wl, "k")).to(dev)
+    Cv = torch.from_numpy(codebooks(wl, "v")).to(dev)
+    lens = np.full(wl.B, wl.T)
+    wk = torch.from_numpy(I.window_tokens(wl, "k", lens)).to(dev)
+    wv = torch.from_numpy(I.window_tokens(wl, "v", lens)).to(dev)
+    reps = []
+    for r in range(R):
+        reps.append(dict(q=torch.from_numpy(I.queries(wl, step=r)).to(dev), k_codes=kc.clone(),
+                         v_codes=vc.clone(), Ck=Ck.clone(), Cv=Cv.clone(), win_k=wk.clone(),
+                         win_v=wv.clone(),
+                         comp_len=torch.full((wl.B,), Tc, dtype=torch.int32, device=dev),
+                         win_len=torch.full((wl.B,), wl.W, dtype=torch.int32, device=dev),
+                         out=torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32, device=dev),
+                         lse=torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev),
+                         err=torch.zeros(1, dtype=torch.int32, device=dev)))
+    del kc, vc, wk, wv
+    keys = ("q", "k_codes", "v_codes", "comp_len", "Ck", "Cv", "win_k", "win_v", "win_len")
+    need = zkv.decode_workspace_size(*(reps[0][k] for k in keys), max_comp_len=Tc)
+    wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
+
+    def call(r):
+        rep = reps[r]
+        zkv.rvq_decode_attn(*(rep[k] for k in keys), out=rep["out"], lse=rep["lse"],
+                            max_comp_len=Tc, workspace=wss[r], error_flag=rep["err"])
+    for r in range(R):   # eager call per replica (kernel attributes before capture)
+        call(r)
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(r)
+        graphs.append(g)
+    for i in range(2 * R):
+        graphs[i % R].replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(calls):
+        graphs[i % R].replay()
+    e.record()
+    torch.cuda.synchronize()
+    sec = s.elapsed_time(e) / 1000.0 / calls
+    assert sum(int(rep["err"].item()) for rep in reps) == 0
+    del graphs
+    rep_mb = replica_bytes(reps[0]) / 1e6
+    byts = (wl.B * wl.Hkv * Tc * (wl.Sk + wl.Sv) + wl.B * wl.Hkv * wl.W * wl.d * 2 * 2
+            + wl.Hkv * (wl.Sk + wl.Sv) * 256 * wl.d * 4 + wl.B * wl.Hq * wl.d * 2
+            + wl.B * wl.Hq * (wl.d + 1) * 4)
+    return {"workload": "qwen25_7b_128k decode (B 1, Hq 28 / Hkv 4, context 131072, W 256, "
+                        "Sk 2, Sv 4)",
+            "value": wl.B * Tc / sec, "unit": UNIT, "us_per_call": sec * 1e6,
+            "call_gbs": byts / sec / 1e9, "call_frac": byts / sec / 1e9 / hbm_peak,
+            "calls": calls,
+            "note": f"zkv_rvq_decode_attn (4 kernels) from CUDA graphs over {R} rotating "
+                    f"replicas x {rep_mb:.1f} MB (> L2); latency-bound at this size"}
+
+
 def pq_encode_extra(dev):
     """Product-VQ (VecInfer) encode of the prefill_encode_64k keys (65536 tokens x 8 kv heads,
     d = 128, sub-vectors of 4 with the smoothing factors): vectors/s."""
@@ -868,6 +940,10 @@ def run_ours(args):
         except Exception as exc:   # an extra never takes the main line down
             extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0 and not args.no_ragged:
+        try:
+            extras["long_context"] = long_context_extra(dev, hbm_peak)
+        except Exception as exc:   # an extra never takes the main line down
+            extras["long_context"] = {"error": f"{type(exc).__name__}: {exc}"}
         try:
             extras["ragged_serving"] = ragged_extra(dev, hbm_peak)
         except Exception as exc:   # an extra never takes the main line down
