@@ -41,3 +41,15 @@ def test_random_codes_and_lengths():
     small = I.workload("llama3_8b_32k", B=2, Hkv=2, Hq=4)
     codes = I.random_codes(small, "k", 100)
     assert codes.shape == (2, 2, 100, 4) and codes.dtype == np.uint8
+
+
+def test_key_smooth_factors_follow_the_oracle_definition():
+    """The harness's calibrated lambda (an input of both sides) is the oracle's
+    smooth_factors of the same calibration sample, bit for bit."""
+    from oracle import zkv_oracle as O
+    wl = I.workload("llama3_8b_32k", Hkv=2, n_cal=512)
+    lam = I.key_smooth_factors(wl)
+    assert lam.shape == (2, wl.d) and lam.dtype == np.float32
+    for h in range(2):
+        K = I._calibration_sample(wl, "k", h, wl.n_cal, I.SEED_CALIB)
+        np.testing.assert_array_equal(lam[h], O.smooth_factors(K))
