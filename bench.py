@@ -469,16 +469,16 @@ def ragged_extra(dev, hbm_peak, R=4, steps=100):
                     f"{rep_mb:.0f} MB (> L2); codes from the skewed code distribution"}
 
 
-def long_context_extra(dev, hbm_peak, R=24, calls=240):
-    """Decode attention on the qwen25_7b_128k workload (B 1, Hq 28 over Hkv 4, GQA 7, context
-    131072 with a 256-token window, Sk = 2 / Sv = 4): one zkv_rvq_decode_attn per call,
-    replayed from CUDA graphs over R rotating replicas of all inputs (R x 6.8 MB > L2).  Codes
-    from the input generator's code distribution; codebooks trained as for the main line."""
+def decode_only_extra(dev, hbm_peak, name, R, calls, label):
+    """Decode attention alone on a named workload: one zkv_rvq_decode_attn per call, replayed
+    from CUDA graphs over R rotating replicas of all inputs (R chosen so that they exceed L2).
+    Codes from the input generator's code distribution; codebooks trained as for the main
+    line."""
     import torch
 
     from compressed_decode_attention_zkv_b200 import inputs as I
     from compressed_decode_attention_zkv_b200 import zkv
-    wl = I.workload("qwen25_7b_128k")
+    wl = I.workload(name)
     Tc = wl.Tc
     Tcap = (Tc + 15) // 16 * 16
     kc = torch.from_numpy(I.random_codes(wl, "k", Tcap)).to(dev)
@@ -532,13 +532,12 @@ def long_context_extra(dev, hbm_peak, R=24, calls=240):
     byts = (wl.B * wl.Hkv * Tc * (wl.Sk + wl.Sv) + wl.B * wl.Hkv * wl.W * wl.d * 2 * 2
             + wl.Hkv * (wl.Sk + wl.Sv) * 256 * wl.d * 4 + wl.B * wl.Hq * wl.d * 2
             + wl.B * wl.Hq * (wl.d + 1) * 4)
-    return {"workload": "qwen25_7b_128k decode (B 1, Hq 28 / Hkv 4, context 131072, W 256, "
-                        "Sk 2, Sv 4)",
+    return {"workload": label,
             "value": wl.B * Tc / sec, "unit": UNIT, "us_per_call": sec * 1e6,
             "call_gbs": byts / sec / 1e9, "call_frac": byts / sec / 1e9 / hbm_peak,
             "calls": calls,
             "note": f"zkv_rvq_decode_attn (4 kernels) from CUDA graphs over {R} rotating "
-                    f"replicas x {rep_mb:.1f} MB (> L2); latency-bound at this size"}
+                    f"replicas x {rep_mb:.2f} MB (> L2); latency-bound at this size"}
 
 
 def pq_encode_extra(dev):
@@ -940,10 +939,18 @@ def run_ours(args):
         except Exception as exc:   # an extra never takes the main line down
             extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0 and not args.no_ragged:
-        try:
-            extras["long_context"] = long_context_extra(dev, hbm_peak)
-        except Exception as exc:   # an extra never takes the main line down
-            extras["long_context"] = {"error": f"{type(exc).__name__}: {exc}"}
+        for key, kw in (("long_context", dict(
+                            name="qwen25_7b_128k", R=24, calls=240,
+                            label="qwen25_7b_128k decode (B 1, Hq 28 / Hkv 4, context 131072, "
+                                  "W 256, Sk 2, Sv 4)")),
+                        ("tiny", dict(
+                            name="tiny", R=256, calls=1000,
+                            label="tiny decode (1 kv head, d 128, 960 compressed + 64 window "
+                                  "tokens, Sk = Sv = 2)"))):
+            try:
+                extras[key] = decode_only_extra(dev, hbm_peak, **kw)
+            except Exception as exc:   # an extra never takes the main line down
+                extras[key] = {"error": f"{type(exc).__name__}: {exc}"}
         try:
             extras["ragged_serving"] = ragged_extra(dev, hbm_peak)
         except Exception as exc:   # an extra never takes the main line down
