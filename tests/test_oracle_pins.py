@@ -610,6 +610,42 @@ def test_pq_direct_equals_lut_form(smooth):
         np.testing.assert_allclose(l2, l1, atol=1e-9, rtol=0)
 
 
+def test_pq_match_walk_counts_exact_near_tie_and_mismatch():
+    """Product-VQ match walk on a hand-built case (d = 8, m = 2: four sub-vectors per row).
+
+    Codewords C[c] = (2c, -3c) for c < 14 are far apart; every sub-vector is its codeword plus
+    delta = (0.25, 0.125), so its nearest codeword is known by construction.  Two extra
+    codewords sit just on the +x side of C[5] and C[3]; the sub-vectors built on C[5] (row 0,
+    sub-vector 1) and C[3] (row 4, sub-vector 0) are then nearer to the extra codewords:
+      C[14] = C[5] + (1 ulp of 10, 0): D(5) - D(14) ~ 0.5 ulp = 4.8e-7, relative 6.1e-6 < 1e-5;
+      C[15] = C[3] + (7.8e-6, 0):       D(3) - D(15) ~ 3.9e-6,         relative 5.0e-5 > 1e-5.
+    Planted candidates: 5 at (0, 1) is a near tie (one exception), 3 at (4, 0) is a mismatch,
+    13 for 12 at (2, 3) is a plain mismatch.  A near-tie rule applied to the wrong distance, a
+    swapped comparison, or a sub-vector index off by one changes the counts or the tuples."""
+    C = np.array([(2.0 * c, -3.0 * c) for c in range(16)], np.float32)
+    C[14] = (np.nextafter(np.float32(10.0), np.float32(11.0)), -15.0)
+    C[15] = (np.float32(6.0) + np.float32(7.8e-6), -9.0)
+    z = np.array([[1, 5, 2, 6], [4, 6, 7, 8], [9, 10, 11, 12], [13, 0, 1, 2], [3, 4, 6, 7]])
+    x = (C[z] + np.float32([0.25, 0.125])).reshape(5, 8).astype(np.float32)
+    oracle = z.copy()
+    oracle[0, 1] = 14
+    oracle[4, 0] = 15
+    zo, _ = O.pq_encode(x, C, rotate=False)
+    np.testing.assert_array_equal(zo, oracle)        # the construction's nearest codewords
+    res = O.pq_match_walk(x, C, oracle, rotate=False)
+    assert (res["exact"], res["exceptions"], res["mismatches"], res["bad"]) == (20, 0, 0, [])
+    cand = oracle.copy()
+    cand[0, 1] = 5          # near tie
+    cand[4, 0] = 3          # gap above 1e-5 relative
+    cand[2, 3] = 13         # far
+    res = O.pq_match_walk(x, C, cand, rotate=False)
+    assert res["exact"] == 17 and res["exceptions"] == 1 and res["mismatches"] == 2
+    assert res["bad"] == [(2, 3, 13, 12), (4, 0, 3, 15)]
+    # a looser gap turns the second case into an exception too
+    res = O.pq_match_walk(x, C, cand, rotate=False, rel_gap=1e-4)
+    assert (res["exceptions"], res["mismatches"], res["bad"]) == (2, 1, [(2, 3, 13, 12)])
+
+
 def test_pq_code_bytes_give_the_stated_bit_rates():
     # 8-bit codes over sub-vectors of 4 (8) dims: 2 (1) bits per element
     x = np.zeros((1, 128), np.float16)
