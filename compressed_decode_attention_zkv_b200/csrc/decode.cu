@@ -37,6 +37,8 @@
 #include "lengths.cuh"
 
 #include <algorithm>
+#include <utility>
+#include <type_traits>
 #include <cfloat>
 #include <cmath>
 
@@ -55,6 +57,18 @@ constexpr int kMergeQ = 4;          // codeword quarters (64 codewords each) per
 constexpr int kMergeC = kCodebook / kMergeQ;
 constexpr int kMergeRows = 32;      // (sequence, head) rows per merge pass
 constexpr size_t kSmemMax = 227 * 1024;
+
+// Token-per-thread scan (scan_rvq.cuh).
+constexpr int kS2Threads = 512;
+constexpr int kS2Fix = 20;                        // value weights as integers of p * 2^20
+constexpr float kS2Headroom = 1.f;                // log2 units added to a new reference
+constexpr uint32_t kS2KeyRegion = 1u << 16;       // absolute shared address of the key tables
+constexpr uint32_t kS2ValRegion = 2u << 16;       // ... of the value histograms
+constexpr size_t kS2Smem = size_t(3) << 16;       // dynamic shared memory requested
+// Set-up cost of one scan segment (table fill, final fold and write: about 1.5K cycles) in
+// tokens of the loop (about 1.3 cycles per token and SM).
+constexpr int64_t kS2SegCost = 1200;
+
 
 static int sm_count() {
   static int n = 0;
@@ -88,6 +102,8 @@ static VMap vmap(int SVP, int GP) {
 
 struct DecodePlan {
   int G, GP, SKP, SVP, Rk, grid;
+  bool scan2;   // the token-per-thread scan (scan_rvq.cuh) serves this shape
+  int64_t seg_cost;
   int64_t cap, slots;
   size_t scan_smem;
   size_t off_lut, off_pre, off_bounds, off_vs, off_pfirst, off_plast, off_pm, off_pl, off_pw,
@@ -115,17 +131,29 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   int Rk = pl.GP == 1 ? 32 : pl.GP == 2 ? 16 : pl.GP == 4 ? 8 : 4;
   while (Rk > 1 && scan_smem_bytes(Rk, p->Sk, p->Sv, pl.GP, v) > kSmemMax) Rk >>= 1;
   pl.Rk = Rk;
-  pl.scan_smem = scan_smem_bytes(Rk, p->Sk, p->Sv, pl.GP, v);
   const int64_t pairs = (int64_t)p->B * p->Hkv;
-  pl.cap = (int64_t)kColCap * v.J;
   const int64_t bound = pairs * p->max_comp_len;
   const int sms = sm_count();
-  // every CTA's virtual share (tokens + kSegCost per pair) stays below the column capacity
-  int64_t g1 = (bound + kSegCost * pairs + pl.cap - 1) / pl.cap;
-  int64_t g2 = std::min<int64_t>(sms, (bound + 1023) / 1024);
-  int64_t grid = std::max<int64_t>(1, std::max(g1, g2));
-  if (grid > sms) grid = (grid + sms - 1) / sms * sms;
-  pl.grid = (int)grid;
+  auto pow124 = [](int s) { return s == 1 || s == 2 || s == 4; };
+  pl.scan2 = pow124(p->Sk) && pow124(p->Sv);
+  if (pl.scan2) {
+    // no column capacity to respect (the integer words are folded on a schedule)
+    pl.scan_smem = kS2Smem;
+    pl.seg_cost = kS2SegCost;
+    pl.cap = 0;
+    pl.grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms, (bound + 1023) / 1024));
+  } else {
+    pl.scan_smem = scan_smem_bytes(Rk, p->Sk, p->Sv, pl.GP, v);
+    pl.seg_cost = kSegCost;
+    pl.cap = (int64_t)kColCap * v.J;
+    // every CTA's virtual share (tokens + kSegCost per pair) stays below the column capacity
+    int64_t g1 = (bound + kSegCost * pairs + pl.cap - 1) / pl.cap;
+    int64_t g2 = std::min<int64_t>(sms, (bound + 1023) / 1024);
+    int64_t grid = std::max<int64_t>(1, std::max(g1, g2));
+    if (grid > sms) grid = (grid + sms - 1) / sms * sms;
+    pl.grid = (int)grid;
+  }
+  const int64_t grid = pl.grid;
   pl.slots = pairs + grid;
   const size_t f = sizeof(float);
   size_t o = 0;
@@ -147,7 +175,8 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
 }
 
 struct DecodeArgs {
-  int B, Hq, Hkv, G, d, Sk, Sv, Rk, grid, n_lut_blocks;
+  int B, Hq, Hkv, G, GP, d, Sk, Sv, Rk, grid, n_lut_blocks;
+  int64_t seg_cost;   // set-up cost of one scan segment, in tokens (partition weight)
   // Serving step: the partition uses the lengths after this step's append (predicted from
   // the pre-step state with the append's rule), and scan block 0 stores them.  Null otherwise.
   int32_t* upd_win_len;
@@ -403,7 +432,7 @@ __device__ __forceinline__ int64_t ceil_muldiv(int64_t x, int64_t m, int64_t d, 
 __device__ void partition_block(const DecodeArgs& a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // exclusive prefix sums of the clamped compressed lengths (pre) and of the virtual lengths
-  // len + kSegCost * (len > 0) (vs), 256 pairs per round
+  // len + a.seg_cost * (len > 0) (vs), 256 pairs per round
   __shared__ int64_t warp_tot[2][8];
   __shared__ int64_t carry_s[2];
   const int npairs = a.B * a.Hkv;
@@ -430,7 +459,7 @@ __device__ void partition_block(const DecodeArgs& a) {
       }
       c = c < a.max_comp ? c : a.max_comp;
     }
-    int64_t x = c, y = c > 0 ? c + kSegCost : 0;   // inclusive warp scans
+    int64_t x = c, y = c > 0 ? c + a.seg_cost : 0;   // inclusive warp scans
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int64_t ux = __shfl_up_sync(0xffffffffu, x, o);
@@ -463,9 +492,9 @@ __device__ void partition_block(const DecodeArgs& a) {
   }
   const int64_t V = carry_s[1], tot = carry_s[0];
   const int grid = a.grid;
-  // V <= pairs * (Tcap + kSegCost) < 2^53 here; products with grid stay below 2^62 unless the
+  // V <= pairs * (Tcap + a.seg_cost) < 2^53 here; products with grid stay below 2^62 unless the
   // grid is very large
-  const bool wide = (double)(V + kSegCost + 1) * (double)grid >= 4.0e18;
+  const bool wide = (double)(V + a.seg_cost + 1) * (double)grid >= 4.0e18;
   if (V == 0) {   // no compressed token at all
     for (int c = tid; c <= grid; c += 256) a.bounds[c] = 0;
     for (int k = tid; k < npairs; k += 256) {
@@ -486,11 +515,11 @@ __device__ void partition_block(const DecodeArgs& a) {
       const int64_t chi = ceil_muldiv(v1, grid, V, wide) - 1;
       for (int64_t c = clo > 1 ? clo : 1; c <= chi && c < grid; ++c) {
         const int64_t off = floor_muldiv(V, c, grid, wide) - v0;
-        a.bounds[c] = off < kSegCost ? p0 : p0 + (off - kSegCost < len ? off - kSegCost : len);
+        a.bounds[c] = off < a.seg_cost ? p0 : p0 + (off - a.seg_cost < len ? off - a.seg_cost : len);
       }
-      // the CTA holding the first token: the last cut at or before v0 + kSegCost (its bound is
+      // the CTA holding the first token: the last cut at or before v0 + a.seg_cost (its bound is
       // p0); the one holding the last token: the last cut before v1
-      const int64_t cf = ceil_muldiv(v0 + kSegCost + 1, grid, V, wide) - 1;
+      const int64_t cf = ceil_muldiv(v0 + a.seg_cost + 1, grid, V, wide) - 1;
       f = (int)(cf < chi ? cf : chi);
       t = (int)chi;
     }
@@ -1179,6 +1208,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
   }
 }
 
+#include "scan_rvq.cuh"
+
 // ------------------------------------------------------------------------------------------
 // 3. Merge: segment histograms -> W_s, contraction with Cv_s, then (finalize) stage sum,
 //    rotation back, log-sum-exp merge with the window.
@@ -1691,6 +1722,33 @@ static inline void trace(void* const* ev, int i, cudaStream_t st) {
   if (ev && ev[i]) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), st);
 }
 
+template <int GPH, int SKP, int SVP>
+static int launch_scan2(const DecodeArgs& a, cudaStream_t st) {
+  auto* k = a.bt ? scan2_kernel<GPH, SKP, SVP, true> : scan2_kernel<GPH, SKP, SVP, false>;
+  if (ensure_smem_limit(k, kS2Smem) != cudaSuccess) return ZKV_ERR_CUDA;
+  if (launch_pdl(k, dim3(a.grid), dim3(kS2Threads), kS2Smem, st, a) != cudaSuccess)
+    return ZKV_ERR_CUDA;
+  return ZKV_OK;
+}
+
+template <int GPH, int SKP>
+static int launch_scan2_v(const DecodeArgs& a, cudaStream_t st) {
+  switch (a.Sv) {
+    case 1: return launch_scan2<GPH, SKP, 1>(a, st);
+    case 2: return launch_scan2<GPH, SKP, 2>(a, st);
+    default: return launch_scan2<GPH, SKP, 4>(a, st);
+  }
+}
+
+template <int GPH>
+static int launch_scan2_kv(const DecodeArgs& a, cudaStream_t st) {
+  switch (a.Sk) {
+    case 1: return launch_scan2_v<GPH, 1>(a, st);
+    case 2: return launch_scan2_v<GPH, 2>(a, st);
+    default: return launch_scan2_v<GPH, 4>(a, st);
+  }
+}
+
 template <int GP, int SKP, int SVP>
 static int launch_scan(const DecodeArgs& a, size_t smem, cudaStream_t st) {
   // the code layout is a template parameter: the contiguous loop carries no paging logic
@@ -1748,7 +1806,12 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
   }
   // 2. scan
   trace(ev, 1, st);
-  {
+  if (pl.scan2) {
+    // heads in passes of at most four
+    const int rc = GP == 1 ? launch_scan2_kv<1>(a, st) : GP == 2 ? launch_scan2_kv<2>(a, st)
+                                                                 : launch_scan2_kv<4>(a, st);
+    if (rc != ZKV_OK) return rc;
+  } else {
     int rc;
     switch (GP) {
       case 1: rc = launch_scan_kv<1>(a, pl.SKP, pl.SVP, pl.scan_smem, st); break;
@@ -1838,6 +1901,7 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   DecodeArgs a;
   a.B = p->B; a.Hq = p->Hq; a.Hkv = p->Hkv; a.G = pl.G; a.d = p->d; a.Sk = p->Sk; a.Sv = p->Sv;
   a.Rk = pl.Rk; a.grid = pl.grid; a.n_lut_blocks = 0;
+  a.GP = pl.GP; a.seg_cost = pl.seg_cost;
   a.upd_win_len = ap ? ap->win_len : nullptr;
   a.upd_win_head = ap ? ap->win_head : nullptr;
   a.upd_comp_len = ap ? ap->comp_len : nullptr;

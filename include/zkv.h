@@ -57,6 +57,8 @@ typedef enum {
 #define ZKV_DEVERR_TIMEOUT 4    /* a bounded on-chip wait ran out (results of that tile absent) */
 #define ZKV_DEVERR_PAGE 8       /* a block-table entry outside [0, n_pages): its tokens read as code
                                    0 (decode) / the append writes nothing for that sequence      */
+#define ZKV_DEVERR_SMEM 16      /* the decode scan's shared-memory layout did not fit the CTA's
+                                   shared window (its partial results are absent)               */
 
 #define ZKV_DTYPE_F16 0
 #define ZKV_DTYPE_F32 1

@@ -117,6 +117,35 @@ def test_decode_uniform_codes_peaky_scores():
     _compare(case, out, lse)
 
 
+@pytest.mark.parametrize("Hq,Sk,Sv", [(4, 4, 4), (1, 2, 2), (7, 2, 4)])
+def test_decode_rising_scores_raise_the_reference(Hq, Sk, Sv):
+    """Key scores that rise along the prefix (stage-0 codeword c scores c / 255 * 30 nats for the
+    first query head, codes rising with the token index) plus one spike near the end: the scan
+    keeps meeting scores above its reference, lists those tokens, raises the reference and adds
+    them afterwards.  The result must still be the oracle's attention."""
+    rng = np.random.default_rng(40 + Hq)
+    B_, Hkv, d, Tcap, W = 1, 1, 128, 30000, 8
+    q = rng.standard_normal((B_, Hq, d)).astype(np.float16)
+    qt = O.fwht(q[0, 0].astype(np.float64), 1.0 / np.sqrt(d))   # rotated query of head 0
+    scale = 1.0 / np.sqrt(d)
+    Ck = (rng.standard_normal((Hkv, Sk, 256, d)) * 0.02).astype(np.float32)
+    sigma = np.arange(256) / 255.0 * 30.0
+    Ck[0, 0] = (sigma[:, None] / scale * qt[None, :] / np.dot(qt, qt)).astype(np.float32)
+    Ck[:, :, 0] = 0
+    Cv = (rng.standard_normal((Hkv, Sv, 256, d)) * 0.3).astype(np.float32)
+    Cv[:, :, 0] = 0
+    kc = rng.integers(0, 256, (B_, Hkv, Tcap, Sk)).astype(np.uint8)
+    kc[0, 0, :, 0] = (np.arange(Tcap) * 250 // Tcap).astype(np.uint8)
+    kc[0, 0, 29000, 0] = 255                       # a spike near the end
+    vc = rng.integers(0, 256, (B_, Hkv, Tcap, Sv)).astype(np.uint8)
+    wk = rng.standard_normal((B_, Hkv, W, d)).astype(np.float16)
+    wv = rng.standard_normal((B_, Hkv, W, d)).astype(np.float16)
+    case = (q, kc, vc, np.array([Tcap]), Ck, Cv, wk, wv, np.array([W]))
+    out, lse = _run_gpu(case)
+    worst = _compare(case, out, lse)
+    print(f"rising scores Hq {Hq} Sk {Sk} Sv {Sv}: worst max-abs {worst:.2e}")
+
+
 def test_decode_max_comp_len_bounds_the_read():
     case = _random_case(12, B_=2, Hq=4, Hkv=1, d=128, Sk=4, Sv=4, Tcap=4096, comp=[1000, 2000],
                         Wcap=8, win=[8, 8])
