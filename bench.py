@@ -35,12 +35,10 @@ METRIC = "decode-attn compressed tokens/s/GPU & HBM GB/s (% roofline); encode ve
 UNIT = "compressed tokens/s"
 WORKLOAD = "llama3_8b_32k"
 
-# DRAM traffic of one scan-kernel launch from an ncu capture (see profiles/), valid only while
-# the scan kernel source is unchanged (hash of decode.cu at capture time).
-# DRAM bytes (read + write) of one scan_kernel launch on this workload, from one ncu capture
-# (profiles/scan_kernel_llama3_8b_32k.md), valid while the scan's source is unchanged.
-SCAN_TRAFFIC = {"scan_src_sha1": "1ecd1b7d8d96ab3f59999e8ee579ed14f7a50b1d",
-                "bytes_per_launch": 17806251}
+# DRAM bytes (read + write) of one scan2_kernel launch on this workload, from one ncu capture
+# (profiles/), valid while the scan's source (csrc/scan_rvq.cuh) is unchanged; None until a
+# capture of the current source is recorded.
+SCAN_TRAFFIC = {"scan_src_sha1": None, "bytes_per_launch": None}
 
 
 def parse():
@@ -205,49 +203,180 @@ def step_fn(rep, ws, max_comp, events=None):
 # CPU oracle baseline (bounded sample)
 # --------------------------------------------------------------------------------------------
 
+def oracle_sample(wl, n_max: int):
+    """The oracle's bounded sample of the serving step: the (b=0, kv head 0) group with its G
+    query heads, n_max compressed tokens of codes from the input generator, the window, and the
+    seeded codebooks (numpy, float32 / uint8 / fp16)."""
+    from compressed_decode_attention_zkv_b200 import inputs as I
+    one = I.workload(wl.name, B=1, Hkv=1, Hq=wl.G, n_cal=1024, kmeans_iters=2)
+    return dict(q=I.queries(one), kc=I.random_codes(one, "k", max(n_max, 16)),
+                vc=I.random_codes(one, "v", max(n_max, 16)), Ck=I.train_codebooks(one, "k"),
+                Cv=I.train_codebooks(one, "v"), wk=I.window_tokens(one, "k", np.array([wl.T])),
+                wv=I.window_tokens(one, "v", np.array([wl.T])), W=wl.W)
+
+
+def oracle_step(smp, n):
+    """One oracle serving step on the sample: the encode of the evicted window token (K and V)
+    and the decode attention over n compressed tokens plus the window.  Returns seconds."""
+    from oracle import zkv_oracle as O
+    t0 = time.perf_counter()
+    O.rvq_encode(smp["wk"][0, 0, :1], smp["Ck"][0])
+    O.rvq_encode(smp["wv"][0, 0, :1], smp["Cv"][0])
+    O.decode_attn(smp["q"], smp["kc"][:, :, :max(n, 16)], smp["vc"][:, :, :max(n, 16)], [n],
+                  smp["Ck"], smp["Cv"], smp["wk"], smp["wv"], [smp["W"]])
+    return time.perf_counter() - t0
+
+
 def oracle_rate(wl, seconds: float, n_tok_cap: int | None = None):
-    """Time the oracle's serving step on a sample: the (b=0, kv head 0) group with its G query
-    heads, compressed prefix of n tokens (codes from the input generator) plus the window, and
-    the encode of the evicted window token.  Returns (tokens/s in the metric's unit, detail)."""
+    """Time the oracle's serving step on one host core (BLAS limited to one thread) on the
+    bounded sample, its compressed length doubled from 2048 until one step takes a quarter of
+    the budget.  Returns (tokens/s in the metric's unit, detail with the sample and n)."""
     from threadpoolctl import threadpool_limits
 
-    from compressed_decode_attention_zkv_b200 import inputs as I
-    from oracle import zkv_oracle as O
-
-    one = I.workload(wl.name, B=1, Hkv=1, Hq=wl.G, n_cal=1024, kmeans_iters=2)
-    Ck = I.train_codebooks(one, "k")
-    Cv = I.train_codebooks(one, "v")
-    q = I.queries(one)
-    wk = I.window_tokens(one, "k", np.array([wl.T]))
-    wv = I.window_tokens(one, "v", np.array([wl.T]))
-
-    def run(n):
-        kc = I.random_codes(one, "k", max(n, 16))
-        vc = I.random_codes(one, "v", max(n, 16))
-        t0 = time.perf_counter()
-        O.rvq_encode(wk[0, 0, :1], Ck[0])
-        O.rvq_encode(wv[0, 0, :1], Cv[0])
-        O.decode_attn(q, kc, vc, [n], Ck, Cv, wk, wv, [wl.W])
-        return time.perf_counter() - t0
-
+    smp = oracle_sample(wl, wl.Tc)
     with threadpool_limits(1):
         n = min(2048, wl.Tc)
-        t = run(n)
+        t = oracle_step(smp, n)
         while t < seconds / 4 and n < wl.Tc:
             n = min(wl.Tc, n * 2)
-            t = run(n)
+            t = oracle_step(smp, n)
         if n_tok_cap:
             n = min(n, n_tok_cap)
         reps, total = 0, 0.0
         while total < seconds and reps < 64:
-            total += run(n)
+            total += oracle_step(smp, n)
             reps += 1
     tokens = reps * n / wl.Hkv          # one kv-head group = 1/Hkv of a sequence's heads
     return tokens / total, {"sample": f"oracle serving step on 1 of {wl.B * wl.Hkv} (seq, kv-head) "
                                       f"groups (all {wl.G} query heads), {n} compressed + {wl.W} "
                                       f"window tokens, 2 evicted-token encodes; {reps} reps, "
                                       f"{total:.1f} s; scaled by 1/Hkv to sequence-tokens",
-                            "cores": 1}
+                            "cores": 1, "n": n, "smp": smp}
+
+
+def _oracle_worker(smp, n, seconds, barrier, queue):
+    """One host core's share of the all-core oracle timing (a spawned process): after the start
+    barrier, serving steps on the sample until `seconds` have passed."""
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):
+            oracle_step(smp, min(n, 64))            # imports and first-call costs
+            barrier.wait(timeout=300)
+            t0 = time.perf_counter()
+            reps = 0
+            while True:
+                oracle_step(smp, n)
+                reps += 1
+                el = time.perf_counter() - t0
+                if el >= seconds:
+                    break
+        queue.put((reps, el))
+    except Exception as exc:   # reported to the parent, which then gives no all-core number
+        queue.put(("error", f"{type(exc).__name__}: {exc}"))
+
+
+def host_cores() -> int:
+    """The host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_rate_all_cores(wl, smp, n, seconds: float):
+    """The oracle's serving step on every host core at once: one spawned process per core, each
+    running the single-core sample (BLAS one thread) from a common start for `seconds`.
+    Throughput = all processes' tokens / the longest process time.  Returns (tokens/s, cores)."""
+    import multiprocessing as mp
+    cores = host_cores()
+    ctx = mp.get_context("spawn")   # the parent holds a CUDA context: never fork
+    barrier = ctx.Barrier(cores)
+    queue = ctx.Queue()
+    saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS",
+                                            "MKL_NUM_THREADS")}
+    for k in saved:
+        os.environ[k] = "1"
+    procs = []
+    try:
+        for _ in range(cores):
+            pr = ctx.Process(target=_oracle_worker, args=(smp, n, seconds, barrier, queue))
+            pr.start()
+            procs.append(pr)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    results = []
+    try:
+        for _ in procs:
+            results.append(queue.get(timeout=300 + 4 * seconds))
+    finally:
+        for pr in procs:
+            pr.join(timeout=10)
+            if pr.is_alive():
+                pr.kill()
+                pr.join()
+    errs = [r[1] for r in results if r[0] == "error"]
+    if errs:
+        raise RuntimeError(errs[0])
+    tokens = sum(r[0] for r in results) * n / wl.Hkv
+    return tokens / max(r[1] for r in results), cores
+
+
+def encode_match(dev, sample4=None):
+    """The oracle's RVQ encode beside the GPU's codes: the tiny workload's keys and values in
+    full, and (sample4, from encode_extra) every 64th token of the 64K-token prefill encode on
+    all 8 heads.  Codes are walked stage by stage against the oracle's float64 greedy rule:
+    exact, near-tie exceptions (distance gap within 1e-5 relative), mismatches.  Also the
+    oracle's single-core encode rate on those rows."""
+    import torch
+    from threadpoolctl import threadpool_limits
+
+    from compressed_decode_attention_zkv_b200 import inputs as I
+    from compressed_decode_attention_zkv_b200 import zkv
+    from oracle import zkv_oracle as O
+
+    def walk(x, books, codes):   # x [H][n][d], books [H][S][256][d], codes [n][H][S]
+        tot = {"rows": 0, "exact": 0, "exceptions": 0, "mismatches": 0}
+        t = 0.0
+        with threadpool_limits(1):
+            for h in range(x.shape[0]):
+                w = O.rvq_match_walk(x[h], books[h], codes[:, h])
+                for k in ("exact", "exceptions", "mismatches"):
+                    tot[k] += w[k]
+                tot["rows"] += x.shape[1]
+                t0 = time.perf_counter()
+                O.rvq_encode(x[h], books[h])
+                t += time.perf_counter() - t0
+        tot["oracle_encode_vectors_per_s_1core"] = tot["rows"] / t
+        tot["code_decisions"] = tot["exact"] + tot["exceptions"] + tot["mismatches"]
+        return tot
+
+    out = {}
+    wl = I.workload("tiny")
+    parts = []
+    for kind in ("k", "v"):
+        books = codebooks(wl, kind)
+        x = I.kv_tokens(wl, kind, 0, 0, wl.T)            # [Hkv][T][d]
+        codes, _ = zkv.rvq_encode(torch.from_numpy(x).to(dev).permute(1, 0, 2),
+                                  torch.from_numpy(books).to(dev), with_norms=False)
+        parts.append(walk(x, books, codes[0].cpu().numpy()))
+    out["tiny_full"] = {k: sum(p[k] for p in parts) for k in ("rows", "exact", "exceptions",
+                                                               "mismatches", "code_decisions")}
+    out["tiny_full"]["what"] = "tiny K and V, all 1024 tokens, 1 head, S = 2"
+    if sample4 is not None:
+        parts = [walk(sample4[k]["x"], sample4[k]["books"], sample4[k]["codes"]) for k in ("k", "v")]
+        out["prefill_encode_64k_sample"] = {
+            k: sum(p[k] for p in parts) for k in ("rows", "exact", "exceptions", "mismatches",
+                                                  "code_decisions")}
+        out["prefill_encode_64k_sample"]["what"] = (
+            "every 64th of 65536 tokens x 8 heads x {K, V}, S = 8, codes from the timed encode")
+        out["prefill_encode_64k_sample"]["oracle_encode_vectors_per_s_1core"] = (
+            sum(p["rows"] for p in parts) / sum(p["rows"] / p["oracle_encode_vectors_per_s_1core"]
+                                               for p in parts))
+    return out
 
 
 def workload_config(wl):
@@ -270,22 +399,10 @@ def run_reference(args):
     n_cap = int(max(64, min(wl.Tc, rate * wl.Hkv * per_step)))
     times = []
     from threadpoolctl import threadpool_limits
-    from oracle import zkv_oracle as O
-    one = I.workload(wl.name, B=1, Hkv=1, Hq=wl.G, n_cal=1024, kmeans_iters=2)
-    Ck = I.train_codebooks(one, "k")
-    Cv = I.train_codebooks(one, "v")
-    q = I.queries(one)
-    wk = I.window_tokens(one, "k", np.array([wl.T]))
-    wv = I.window_tokens(one, "v", np.array([wl.T]))
-    kc = I.random_codes(one, "k", max(n_cap, 16))
-    vc = I.random_codes(one, "v", max(n_cap, 16))
+    smp = info["smp"]
     with threadpool_limits(1):
         for i in range(args.warmup + args.steps):
-            t0 = time.perf_counter()
-            O.rvq_encode(wk[0, 0, :1], Ck[0])
-            O.rvq_encode(wv[0, 0, :1], Cv[0])
-            O.decode_attn(q, kc, vc, [n_cap], Ck, Cv, wk, wv, [wl.W])
-            dt = time.perf_counter() - t0
+            dt = oracle_step(smp, n_cap)
             if i >= args.warmup:
                 times.append(dt)
     total = sum(times)
@@ -309,12 +426,10 @@ def run_reference(args):
 # --------------------------------------------------------------------------------------------
 
 def scan_src_sha1():
-    """sha1 of the scan kernel's section of decode.cu (the traffic figure stays valid while the
-    kernel's code is unchanged)."""
-    text = open(os.path.join(ROOT, "compressed_decode_attention_zkv_b200", "csrc",
-                             "decode.cu")).read()
-    scan = text.split("// 2. Scan of the compressed tokens.")[1].split("// 3. Merge:")[0]
-    return hashlib.sha1(scan.encode()).hexdigest()
+    """sha1 of the scan kernel's source file (the traffic figure stays valid while it is
+    unchanged)."""
+    return sha1_of(os.path.join(ROOT, "compressed_decode_attention_zkv_b200", "csrc",
+                                "scan_rvq.cuh"))
 
 
 def max_over_ranks(seconds: float, world: int, dev) -> float:
@@ -368,6 +483,10 @@ def encode_extra(dev, hbm, bf16):
     e.record()
     torch.cuda.synchronize()
     sec = s.elapsed_time(e) / 1000.0 / n_iter
+    # every 64th token of each head, for the oracle's code check in the CPU-baseline leg
+    sample = {k: {"x": xs[k][::64].permute(1, 0, 2).contiguous().cpu().numpy(),
+                  "books": codebooks(wl, k), "codes": codes[k][::64].cpu().numpy()}
+              for k in ("k", "v")}
     rows = 2 * wl.T * wl.Hkv
     flops = 2.0 * rows * wl.Sk * 256 * wl.d
     byts = rows * wl.d * 2 + rows * wl.Sk * (1 + 4) + 2 * wl.Hkv * wl.Sk * 256 * wl.d * 4
@@ -381,7 +500,8 @@ def encode_extra(dev, hbm, bf16):
             "peak_kind": "measured bf16 GEMM (burst) x nominal tf32/bf16 ratio",
             "frac": flops / sec / 1e12 / tf32_peak,
             "note": "tcgen05 kind::tf32 distance GEMM (M=128 rows, N=256 codewords) into TMEM; "
-                    "exact decision: TF32-margin candidates re-scored in float32, then float64"}
+                    "exact decision: TF32-margin candidates re-scored in float32, then float64",
+            "_sample": sample}
 
 
 def ragged_extra(dev, hbm_peak, R=4, steps=100):
@@ -503,10 +623,15 @@ def decode_only_extra(dev, hbm_peak, name, R, calls, label):
     need = zkv.decode_workspace_size(*(reps[0][k] for k in keys), max_comp_len=Tc)
     wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
 
-    def call(r):
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(R)]
+    for ev in (ev for row in evs for ev in row):   # torch times only events it saw recorded
+        ev.record()
+
+    def call(r, traced=False):
         rep = reps[r]
         zkv.rvq_decode_attn(*(rep[k] for k in keys), out=rep["out"], lse=rep["lse"],
-                            max_comp_len=Tc, workspace=wss[r], error_flag=rep["err"])
+                            max_comp_len=Tc, workspace=wss[r], error_flag=rep["err"],
+                            trace_events=evs[r] if traced else None)
     for r in range(R):   # eager call per replica (kernel attributes before capture)
         call(r)
     torch.cuda.synchronize()
@@ -528,6 +653,29 @@ def decode_only_extra(dev, hbm_peak, name, R, calls, label):
     sec = s.elapsed_time(e) / 1000.0 / calls
     assert sum(int(rep["err"].item()) for rep in reps) == 0
     del graphs
+    # per-kernel times: graphs with event nodes between the kernels, 4 rounds over the replicas
+    spans = None
+    try:
+        tg = []
+        for r in range(R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                call(r, traced=True)
+            tg.append(g)
+        acc = [[], [], []]
+        for _ in range(4):
+            for r in range(R):
+                tg[r].replay()
+            torch.cuda.synchronize()
+            for r in range(R):
+                for i in range(3):
+                    acc[i].append(evs[r][i].elapsed_time(evs[r][i + 1]) * 1e3)
+        del tg
+        spans = {"tables+window+partition": statistics.mean(acc[0]),
+                 "scan": statistics.mean(acc[1]), "combine": statistics.mean(acc[2]),
+                 "unit": "us", "timing": "event nodes between the kernels (no overlap there)"}
+    except Exception as exc:
+        spans = {"error": f"{type(exc).__name__}: {exc}"}
     rep_mb = replica_bytes(reps[0]) / 1e6
     byts = (wl.B * wl.Hkv * Tc * (wl.Sk + wl.Sv) + wl.B * wl.Hkv * wl.W * wl.d * 2 * 2
             + wl.Hkv * (wl.Sk + wl.Sv) * 256 * wl.d * 4 + wl.B * wl.Hq * wl.d * 2
@@ -536,8 +684,10 @@ def decode_only_extra(dev, hbm_peak, name, R, calls, label):
             "value": wl.B * Tc / sec, "unit": UNIT, "us_per_call": sec * 1e6,
             "call_gbs": byts / sec / 1e9, "call_frac": byts / sec / 1e9 / hbm_peak,
             "calls": calls,
-            "note": f"zkv_rvq_decode_attn (4 kernels) from CUDA graphs over {R} rotating "
-                    f"replicas x {rep_mb:.2f} MB (> L2); latency-bound at this size"}
+            "algorithmic_bytes": byts, "kernels_us": spans,
+            "note": f"zkv_rvq_decode_attn (3 kernels: tables + window + partition, scan, "
+                    f"combine) from CUDA graphs over {R} rotating replicas x {rep_mb:.2f} MB "
+                    f"(> L2)"}
 
 
 def pq_encode_extra(dev):
@@ -726,8 +876,10 @@ def run_ours(args):
     wl = I.workload(WORKLOAD)
     R = args.replicas
     n_e2e = min(args.steps, 400)
-    # every step (eager warm-up, graph warm-up, timed, e2e) grows one replica's prefixes by 1
-    per_rep = (R + args.warmup + args.steps + n_e2e + 64 + R - 1) // R + 2
+    n_trace_rounds = 8
+    # every step (eager warm-up, graph warm-up, timed, traced, e2e, eager fallback) grows one
+    # replica's prefixes by 1
+    per_rep = (R + args.warmup + args.steps + n_e2e + 2 * n_trace_rounds * R + R - 1) // R + 2
     reps, Tcap = build_state(wl, R, per_rep, dev)
     rep_mb = replica_bytes(reps[0]) / 1e6
     max_comp = wl.Tc + per_rep        # host bound on every prefix length during the run
@@ -738,15 +890,15 @@ def run_ours(args):
     wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
     host_comp = [wl.Tc] * R          # compressed length of every sequence of each replica
 
-    # trace events per replica: start of the step (tables, encode, length update and
-    # partition follow), before the scan, before the merge, after the last kernel
+    # trace events per replica: start of the step (tables, partition, encode and length update
+    # follow), before the scan, before the combine, after the last kernel
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(R)]
     for e in (e for row in evs for e in row):   # torch only times events it has seen recorded;
         e.record()                               # the library re-records the same handles
     torch.cuda.synchronize()
 
-    def one_step(r):
-        step_fn(reps[r], wss[r], max_comp, events=evs[r])
+    def one_step(r, traced=False):
+        step_fn(reps[r], wss[r], max_comp, events=evs[r] if traced else None)
 
     def decode_only(r):
         from compressed_decode_attention_zkv_b200 import zkv as Z
@@ -765,7 +917,9 @@ def run_ours(args):
             host_comp[r] += 1
     torch.cuda.current_stream().wait_stream(stream)
     torch.cuda.synchronize()
-    graphs, soak_graphs = [], []
+    # the timed graphs carry no events; a second set with event nodes between the kernels
+    # (which end the programmatic overlap at those points) gives the per-kernel times
+    graphs, soak_graphs, traced_graphs = [], [], []
     for r in range(R):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -775,6 +929,16 @@ def run_ours(args):
         with torch.cuda.graph(g2):
             decode_only(r)
         soak_graphs.append(g2)
+    trace_err = None
+    try:
+        for r in range(R):
+            g3 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g3):
+                one_step(r, traced=True)
+            traced_graphs.append(g3)
+    except Exception as exc:   # no per-kernel times from graphs: the eager pass below
+        trace_err = f"{type(exc).__name__}: {exc}"
+        traced_graphs = []
     # capture does not execute: the state is unchanged
 
     step_counter = [0]
@@ -822,29 +986,42 @@ def run_ours(args):
     errs = sum(int(rep["err"].item()) for rep in reps)
     assert errs == 0, f"device error flag set: {errs}"
 
-    # per-kernel durations of the last replay of each replica graph (live, timed region)
+    # per-kernel durations: the traced graphs replayed back to back in the timed rotation, right
+    # after the timed region; the spans of each replica's replay are read after each round
     def span(r, a, b):
         return evs[r][a].elapsed_time(evs[r][b]) / 1000.0
-    try:
-        t_pre = statistics.mean(span(r, 0, 1) for r in range(R))
-        t_scan = statistics.mean(span(r, 1, 2) for r in range(R))
-        t_merge = statistics.mean(span(r, 2, 3) for r in range(R))
-        trace_src = "CUDA events captured in the step graphs (last replay of each replica)"
-    except Exception as exc:   # event timing inside graphs unavailable: eager pass instead
-        print(f"[bench] graph-captured event timing failed ({exc}); timing kernels eagerly",
+    acc = {k: [] for k in ("pre", "scan", "comb")}
+    if traced_graphs:
+        try:
+            for _ in range(n_trace_rounds):
+                for r in range(R):
+                    traced_graphs[r].replay()
+                    host_comp[r] += 1
+                torch.cuda.synchronize()
+                for r in range(R):
+                    acc["pre"].append(span(r, 0, 1))
+                    acc["scan"].append(span(r, 1, 2))
+                    acc["comb"].append(span(r, 2, 3))
+            trace_src = (f"CUDA event nodes in the step graphs: {n_trace_rounds} rounds of the {R} "
+                         f"replicas replayed back to back after the timed region")
+        except Exception as exc:
+            trace_err = f"{type(exc).__name__}: {exc}"
+            acc = {k: [] for k in acc}
+    if not acc["scan"]:   # event timing inside graphs unavailable: eager steps instead
+        print(f"[bench] graph-captured event timing failed ({trace_err}); timing kernels eagerly",
               file=sys.stderr)
-        acc = {k: [] for k in ("pre", "scan", "merge")}
-        for i in range(min(args.steps, 64)):
+        for i in range(n_trace_rounds * R):
             r = i % R
-            one_step(r)
+            one_step(r, traced=True)
             host_comp[r] += 1
             torch.cuda.synchronize()
             acc["pre"].append(span(r, 0, 1))
             acc["scan"].append(span(r, 1, 2))
-            acc["merge"].append(span(r, 2, 3))
-        t_pre, t_scan, t_merge = (statistics.mean(acc[k]) for k in ("pre", "scan", "merge"))
-        trace_src = "CUDA events around each kernel, eager steps after the timed region"
-    per = {"tables+append+partition": t_pre, "scan": t_scan, "merge+finalize": t_merge}
+            acc["comb"].append(span(r, 2, 3))
+        trace_src = f"CUDA events around each kernel, eager steps ({trace_err})"
+    t_pre, t_scan, t_merge = (statistics.mean(acc[k]) for k in ("pre", "scan", "comb"))
+    del traced_graphs
+    per = {"tables+window+partition+append": t_pre, "scan": t_scan, "combine": t_merge}
     Tc_avg = tokens / (wl.B * args.steps)
     # algorithmic bytes (counted once per distinct byte).  The scan kernel reads the codes of
     # every compressed token: (Sk + Sv) bytes per (token, kv head).
@@ -858,7 +1035,7 @@ def run_ours(args):
     step_time = t_pre + t_scan + t_merge
     traffic = (SCAN_TRAFFIC["bytes_per_launch"]
                if SCAN_TRAFFIC["scan_src_sha1"] == scan_src_sha1() else None)
-    roof = {"bound": "hbm", "kernel": "scan_kernel", "achieved": scan_bytes / t_scan / 1e9,
+    roof = {"bound": "hbm", "kernel": "scan2_kernel", "achieved": scan_bytes / t_scan / 1e9,
             "peak": hbm_peak, "unit": "GB/s", "frac": scan_bytes / t_scan / 1e9 / hbm_peak,
             "traffic": traffic, "peak_kind": f"{peak_kind} (hbm_gbs copy, burst)",
             "algorithmic_bytes_per_launch": scan_bytes, "avg_launch_s": t_scan,
@@ -920,10 +1097,13 @@ def run_ours(args):
                        "out + lse"}
 
     extras = {}
-    if not args.no_encode and rank == 0:
+    sample4 = None
+    if rank == 0:
         del graphs, soak_graphs
+    if not args.no_encode and rank == 0:
         try:
             extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
+            sample4 = extras["encode"].pop("_sample")
         except Exception as exc:   # an extra never takes the main line down
             extras["encode"] = {"error": f"{type(exc).__name__}: {exc}"}
     base_ms = 1000.0 * elapsed / args.steps
@@ -939,7 +1119,11 @@ def run_ours(args):
         except Exception as exc:   # an extra never takes the main line down
             extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0 and not args.no_ragged:
-        for key, kw in (("long_context", dict(
+        for key, kw in (("decode_only", dict(
+                            name="llama3_8b_32k", R=12, calls=600,
+                            label="llama3_8b_32k decode only (B 8, Hq 32 / Hkv 8, context 32768, "
+                                  "W 128, Sk = Sv = 4)")),
+                        ("long_context", dict(
                             name="qwen25_7b_128k", R=24, calls=240,
                             label="qwen25_7b_128k decode (B 1, Hq 28 / Hkv 4, context 131072, "
                                   "W 256, Sk 2, Sv 4)")),
@@ -969,9 +1153,25 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, info = oracle_rate(wl, seconds=args.cpu_seconds)
-        cpu = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
-               "sample": info["sample"]}
+        # the oracle as it stands, on one core and on every host core (one process per core
+        # running the same sample); the encode check reports its matching counts
+        v1, info = oracle_rate(wl, seconds=args.cpu_seconds)
+        try:
+            vall, cores = oracle_rate_all_cores(wl, info["smp"], info["n"], args.cpu_seconds / 2)
+            cpu = {"value": vall, "unit": UNIT, "cores": cores, "kind": "oracle",
+                   "sample": f"{cores} processes (one per host core, BLAS one thread), each: "
+                             + info["sample"].split(";")[0]
+                             + f"; for {args.cpu_seconds / 2:.1f} s from a common start",
+                   "host_cores": host_cores(), "single_core": {"value": v1, "cores": 1,
+                                                               "sample": info["sample"]}}
+        except Exception as exc:   # the single-core figure stands alone
+            cpu = {"value": v1, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample": info["sample"], "host_cores": host_cores(),
+                   "all_cores_error": f"{type(exc).__name__}: {exc}"}
+        try:
+            cpu["encode_match"] = encode_match(dev, sample4)
+        except Exception as exc:
+            cpu["encode_match"] = {"error": f"{type(exc).__name__}: {exc}"}
 
     if rank == 0:
         line = {
@@ -983,7 +1183,7 @@ def run_ours(args):
                            l2=f"{R} rotating replicas x {rep_mb:.1f} MB = {R * rep_mb:.0f} MB > 126 MB L2",
                            parallelism=f"replicas x{world}, no collective",
                            graph="one CUDA graph per replica step"),
-            "gpu_launches": 5 * args.steps,   # tables+partition, encode, scan, merge, finalize
+            "gpu_launches": 4 * args.steps,   # tables+window+partition, encode, scan, combine
             "roofline": roof,
             "kernels_s": per,
             "step_call": {"seconds": step_time, "algorithmic_bytes": call_bytes,

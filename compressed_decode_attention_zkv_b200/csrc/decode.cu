@@ -7,32 +7,33 @@
 // q . k).  Differential-KV README, "Decode & Prefill Innovations": flash-style fp32
 // log-sum-exp combine of the compressed part with the dense recency window.
 //
-// Four kernels per call:
+// Three kernels per call (programmatic dependent launches):
 //   1. lut_kernel    q_tilde = H q / sqrt(d) (float32 transform), per stage
-//                    LUT_s[c] = (scale * log2 e) * q_tilde . Ck_s[c] -> workspace; prefix sums
-//                    of the compressed lengths that partition the token space among scan CTAs.
-//   2. scan_kernel   one CTA per SM walks a contiguous range of the concatenated compressed
+//                    LUT_s[c] = (scale * log2 e) * q_tilde . Ck_s[c] -> workspace; one block
+//                    computes the prefix sums of the compressed lengths that partition the token
+//                    space among scan CTAs; one block per (sequence, kv head) takes the dense
+//                    attention over its fp16 window (partial maximum, sum and output).
+//   2. scan          one CTA per SM walks a contiguous range of the concatenated compressed
 //                    tokens of all (sequence, kv head) pairs.  Per pair segment it takes
-//                    score_t = sum_s LUT_s[zk_{t,s}] (base-2 logits), keeps a running reference
-//                    maximum m, and accumulates p_t = 2^(score_t - m) into per-stage codeword
-//                    weight histograms W_s[c] = sum over tokens with zv_{t,s} = c of p_t.
-//                    sum_t p_t sum_s Cv_s[zv_{t,s}] = sum_s sum_c W_s[c] Cv_s[c]: the value
-//                    reconstruction regrouped by codeword.
-//   3. merge_kernel  grid (codeword quarter, value stage, kv head): merges the segment
-//                    histograms by their maxima and contracts W_s with its Cv_s codewords for
-//                    every sequence (Cv_s is read once per call).
-//   4. finalize_kernel  one block per (sequence, kv head): the dense attention over the fp16
-//                    window (while the merge still runs), then sums the partials, rotates
-//                    back, and merges the two parts by log-sum-exp.
+//                    score_t = sum_s LUT_s[zk_{t,s}] (base-2 logits) against a reference maximum
+//                    m, and accumulates p_t = 2^(score_t - m) into per-stage codeword weight
+//                    histograms W_s[c] = sum over tokens with zv_{t,s} = c of p_t:
+//                    sum_t p_t sum_s Cv_s[zv_{t,s}] = sum_s sum_c W_s[c] Cv_s[c], the value
+//                    reconstruction regrouped by codeword.  scan2_kernel (scan_rvq.cuh) serves
+//                    1, 2 or 4 stages; scan_kernel below the other stage counts.
+//   3. combine_kernel (combine.cuh)  per (pair, value stage, codeword chunk): merges the segment
+//                    histograms by their maxima and contracts W_s with its Cv_s codewords; the
+//                    block that completes a pair sums the stage outputs, rotates back, and merges
+//                    with the window partial by log-sum-exp.
 //
-// Shared-memory design of the scan (shared memory bandwidth, not HBM, bounds this kernel):
+// Shared-memory design of scan_kernel (shared memory bandwidth, not HBM, bounds this kernel):
 //  * key tables are replicated per lane group so that the 8 (or 16, 32) lanes of a 128-bit
 //    (64-, 32-bit) gather always hit distinct banks;
 //  * value histograms use the native shared-memory integer reduction: p is converted to
-//    38-bit fixed point (exact to 2^-39 absolute per token, p <= 1 because the segment maximum
-//    is known after pass 1) split into two 19-bit halves added with red.shared.add.u32; lanes
-//    are mapped to (token slot, stage, head) so one instruction touches 32 distinct banks.
-//    Column sums stay below 2^32 because a segment holds at most 8176 tokens per column.
+//    38-bit fixed point (exact to 2^-39 absolute per token, p <= 1 relative to the segment's
+//    reference) split into two 19-bit halves added with red.shared.add.u32; lanes are mapped to
+//    (token slot, stage, head) so one instruction touches 32 distinct banks.  Column sums stay
+//    below 2^32 because a segment holds at most 8176 tokens per column.
 #include "zkv_internal.cuh"
 #include "lengths.cuh"
 
@@ -53,9 +54,6 @@ constexpr float kHeadroom = 10.f;   // log2 units added to the running maximum o
 // in tokens of the scan loop (about 5.7 cycles per token): the token space is partitioned so
 // that tokens + kSegCost x segments is equal across scan CTAs.
 constexpr int64_t kSegCost = 1900;
-constexpr int kMergeQ = 4;          // codeword quarters (64 codewords each) per value stage
-constexpr int kMergeC = kCodebook / kMergeQ;
-constexpr int kMergeRows = 32;      // (sequence, head) rows per merge pass
 constexpr size_t kSmemMax = 227 * 1024;
 
 // Token-per-thread scan (scan_rvq.cuh).
@@ -107,7 +105,8 @@ struct DecodePlan {
   int64_t cap, slots;
   size_t scan_smem;
   size_t off_lut, off_pre, off_bounds, off_vs, off_pfirst, off_plast, off_pm, off_pl, off_pw,
-      off_wm, off_wl, off_wo, off_so, total;
+      off_wm, off_wl, off_wo, off_so, off_cnt, total;
+  int qc;
 };
 
 static size_t scan_smem_bytes(int Rk, int Sk, int Sv, int GP, const VMap& v) {
@@ -169,7 +168,16 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   pl.off_wm = o;    o = align256(o + (size_t)pairs * pl.GP * f);
   pl.off_wl = o;    o = align256(o + (size_t)pairs * pl.GP * f);
   pl.off_wo = o;    o = align256(o + (size_t)pairs * pl.GP * p->d * f);
-  pl.off_so = o;    o = align256(o + (size_t)pairs * p->Sv * kMergeQ * pl.GP * p->d * f);
+  // combine blocks: (pair, value stage, chunk of 256 / qc codewords); a chunk's codewords take
+  // at most 32 KB of shared memory, and small problems take more chunks (up to 16 or the
+  // 32 KB minimum) so that the grid covers the SMs
+  {
+    int qc = std::max(2, p->d / 32);
+    while (qc < 16 && pairs * p->Sv * qc < sms) qc *= 2;
+    pl.qc = qc;
+  }
+  pl.off_so = o;    o = align256(o + (size_t)pairs * p->Sv * pl.qc * pl.GP * p->d * f);
+  pl.off_cnt = o;   o = align256(o + (size_t)pairs * sizeof(int32_t));
   pl.total = o;
   return pl;
 }
@@ -177,6 +185,8 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
 struct DecodeArgs {
   int B, Hq, Hkv, G, GP, d, Sk, Sv, Rk, grid, n_lut_blocks;
   int64_t seg_cost;   // set-up cost of one scan segment, in tokens (partition weight)
+  int qc;             // codeword chunks per value stage in the combine kernel
+  int n_win_blocks;   // window blocks of the table kernel (one per (sequence, kv head))
   // Serving step: the partition uses the lengths after this step's append (predicted from
   // the pre-step state with the append's rule), and scan block 0 stores them.  Null otherwise.
   int32_t* upd_win_len;
@@ -213,7 +223,8 @@ struct DecodeArgs {
   float* wm;         // [B*Hkv][GP]
   float* wl;         // [B*Hkv][GP]
   float* wo;         // [B*Hkv][GP][d]
-  float* so;         // [B*Hkv][Sv][kMergeQ][GP][d] partial stage outputs
+  float* so;         // [B*Hkv][Sv][qc][GP][d] partial stage outputs
+  int32_t* cnt;      // [B*Hkv] finished combine blocks of each pair (zeroed by the table kernel)
 };
 
 __device__ __forceinline__ int64_t clamp_win_len(const DecodeArgs& a, int b) {
@@ -226,8 +237,9 @@ __device__ __forceinline__ int64_t clamp_win_len(const DecodeArgs& a, int b) {
 }
 
 // ------------------------------------------------------------------------------------------
-// 1. Query rotation + lookup tables; length prefix sums (block 0).  The dense window
-//    attention (window_item) runs in the finalize kernel.
+// 1. Query rotation + lookup tables; length prefix sums (the partition block).  The dense
+//    window attention (window_item) runs here in a decode call and in the combine kernel in
+//    the serving step.
 // ------------------------------------------------------------------------------------------
 constexpr int kLutC = 64;     // codewords per table block (one per thread and head quad)
 constexpr int kLutH = 16;     // attached query heads per table block (b * G + g)
@@ -538,7 +550,15 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_trigger();   // the next kernel waits for this one before reading the tables
   if ((int)blockIdx.x == a.n_lut_blocks) {
+    for (int k = threadIdx.x; k < a.B * a.Hkv; k += blockDim.x) a.cnt[k] = 0;   // combine counters
     partition_block(a);
+    return;
+  }
+  if ((int)blockIdx.x > a.n_lut_blocks) {
+    // dense attention over the fp16 window of one (sequence, kv head); it reads only the call's
+    // inputs, so it runs here, beside the tables and the scan's start
+    const int pair = (int)blockIdx.x - a.n_lut_blocks - 1;
+    window_item<D, GP>(a, pair / a.Hkv, pair % a.Hkv, smem_raw);
     return;
   }
   if ((int)blockIdx.x < a.Hkv * a.Sv && tid == 0) {
@@ -1209,240 +1229,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(DecodeArgs a) {
 }
 
 #include "scan_rvq.cuh"
+#include "combine.cuh"
 
-// ------------------------------------------------------------------------------------------
-// 3. Merge: segment histograms -> W_s, contraction with Cv_s, then (finalize) stage sum,
-//    rotation back, log-sum-exp merge with the window.
-// ------------------------------------------------------------------------------------------
-
-// Scan segments (slots) of a pair: scan CTA c covers the pair's tokens iff first <= c <= last;
-// its partial is in slot pair + c.
-__device__ __forceinline__ void pair_slots(const DecodeArgs& a, int64_t pair, int64_t& first,
-                                           int64_t& last) {
-  first = a.pfirst[pair];
-  last = a.plast[pair];
-}
-
-// grid (codeword quarter, value stage, kv head), 256 threads.  The block copies its 64
-// codewords of Cv_s once and, 32 (sequence, head) rows at a time, merges the segment
-// histograms of those codewords by their maxima (W_s[c] = sum over slots of
-// 2^(m_slot - m*) W_slot[c]) and contracts them: so[pair][s][quarter][g][:] =
-// sum_c W_s[c][g] Cv_s[c][:].  Each row's slot range, maximum m* and first kMergeW slot
-// weights are tabulated once, so the weight sums are runs of independent loads.
-constexpr int kMergeW = 32;   // slot weights tabulated per row
-
-template <int D, int GP>
-__global__ void __launch_bounds__(256) merge_kernel(DecodeArgs a) {
-  constexpr int TG = 256 / D;               // thread groups (one column e per thread)
-  constexpr int RPT = kMergeRows / TG;      // rows per thread
-  extern __shared__ __align__(16) float sm[];
-  float* Cs = sm;                           // [64][D]
-  float* Ws = Cs + kMergeC * D;             // [64][32] (codeword, row)
-  __shared__ float mst[kMergeRows];
-  __shared__ int64_t rfirst[kMergeRows];
-  __shared__ int rcount[kMergeRows];
-  __shared__ float rw[kMergeW][kMergeRows];
-  __shared__ int nmax_s;
-  const int tid = threadIdx.x;
-  const int qtr = blockIdx.x, s = blockIdx.y, kvh = blockIdx.z;
-  const int c0 = qtr * kMergeC;
-  pdl_trigger();   // the finalize blocks start their window attention meanwhile
-  {
-    const float* src = a.Cv + (((size_t)kvh * a.Sv + s) * kCodebook + c0) * D;
-    for (int f = tid; f < kMergeC * D / 4; f += 256) cp_async16(Cs + 4 * f, src + 4 * f);
-    cp_async_commit();
-  }
-  pdl_wait();   // segment partials of the scan
-  const int nrows = a.B * GP;
-  const int e = tid % D, grp = tid / D;
-  for (int r0 = 0; r0 < nrows; r0 += kMergeRows) {
-    if (tid < kMergeRows) {   // warp 0: one row per lane
-      const int r = r0 + tid, b = r / GP, g = r % GP;
-      float m = -INFINITY;
-      int64_t first = 0;
-      int n = 0;
-      if (b < a.B) {
-        const int64_t pair = (int64_t)b * a.Hkv + kvh;
-        int64_t last;
-        pair_slots(a, pair, first, last);
-        n = last >= first ? (int)(last - first + 1) : 0;
-        first += pair;   // absolute slot index
-      }
-      // groups of 8 predicated loads: one round trip for up to 8 slots
-      for (int k0 = 0; k0 < n; k0 += 8) {
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = k0 + i < n ? a.pm[(first + k0 + i) * GP + g] : -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, v[i]);
-      }
-      for (int k0 = 0; k0 < n && k0 < kMergeW; k0 += 8) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (k0 + i < n && k0 + i < kMergeW) rw[k0 + i][tid] = ex2_approx(a.pm[(first + k0 + i) * GP + g] - m);
-      }
-      mst[tid] = m;
-      rfirst[tid] = first;
-      rcount[tid] = n;
-      const int nm = __reduce_max_sync(0xffffffffu, n);
-      if (tid == 0) nmax_s = nm;
-    }
-    __syncthreads();
-    // W for (codeword c0 + c, row r): thread = (row lane, codewords warp + 8 k8).  Slots go in
-    // groups of 4 up to the pass's largest count; within a group all 8 x 4 loads are
-    // independent (predicated), so each group costs one round trip.
-    {
-      constexpr int NE = kMergeC * kMergeRows / 256;   // 8 entries per thread
-      const int rl = tid % kMergeRows, cw = tid / kMergeRows;
-      const int g = (r0 + rl) % GP, n = rcount[rl];
-      const int64_t stride = (int64_t)a.Sv * kCodebook * GP;   // one slot
-      const float* src = a.pw + (rfirst[rl] * a.Sv + s) * (int64_t)(kCodebook * GP) + (int64_t)c0 * GP + g;
-      float acc[NE];
-#pragma unroll
-      for (int k8 = 0; k8 < NE; ++k8) acc[k8] = 0.f;
-      const int nm = nmax_s;
-      for (int k0 = 0; k0 < nm; k0 += 4) {
-        float w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int k = k0 + i;
-          w[i] = k >= n ? 0.f : k < kMergeW ? rw[k][rl] : ex2_approx(a.pm[(rfirst[rl] + k) * GP + g] - mst[rl]);
-        }
-        float v[NE][4];
-#pragma unroll
-        for (int k8 = 0; k8 < NE; ++k8)
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            v[k8][i] = k0 + i < n ? src[(k0 + i) * stride + (cw + 8 * k8) * GP] : 0.f;
-#pragma unroll
-        for (int k8 = 0; k8 < NE; ++k8)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[k8] = fmaf(w[i], v[k8][i], acc[k8]);
-      }
-#pragma unroll
-      for (int k8 = 0; k8 < NE; ++k8) Ws[(cw + 8 * k8) * kMergeRows + rl] = acc[k8];
-    }
-    cp_async_wait_all();   // the codeword slice (first pass only; later a no-op)
-    __syncthreads();
-    float acc[RPT];
-#pragma unroll
-    for (int j = 0; j < RPT; ++j) acc[j] = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < kMergeC; ++c) {
-      const float cv = Cs[c * D + e];
-      const float4* w4 = reinterpret_cast<const float4*>(Ws + c * kMergeRows + grp * RPT);
-#pragma unroll
-      for (int j4 = 0; j4 < RPT / 4; ++j4) {
-        const float4 w = w4[j4];
-        acc[4 * j4 + 0] = fmaf(w.x, cv, acc[4 * j4 + 0]);
-        acc[4 * j4 + 1] = fmaf(w.y, cv, acc[4 * j4 + 1]);
-        acc[4 * j4 + 2] = fmaf(w.z, cv, acc[4 * j4 + 2]);
-        acc[4 * j4 + 3] = fmaf(w.w, cv, acc[4 * j4 + 3]);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < RPT; ++j) {
-      const int r = r0 + grp * RPT + j, b = r / GP, g = r % GP;
-      if (b < a.B) {
-        const int64_t pair = (int64_t)b * a.Hkv + kvh;
-        a.so[(((pair * a.Sv + s) * kMergeQ + qtr) * GP + g) * D + e] = acc[j];
-      }
-    }
-    __syncthreads();   // the row tables and Ws are rewritten by the next pass
-  }
-}
-
-// One block per (sequence, kv head): sum of the stage / quarter partials (rotated domain,
-// unnormalised), rotation back one head per warp, log-sum-exp merge with the window.
-template <int D, int GP>
-__global__ void __launch_bounds__(256) finalize_kernel(DecodeArgs a) {
-  constexpr int E = D / 32;
-  extern __shared__ __align__(16) unsigned char win_smem[];
-  __shared__ __align__(16) float oc[GP * D];
-  __shared__ float mstar_s[GP], lstar_s[GP];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t pair = blockIdx.x;
-  const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
-  // The window attention reads only the call's inputs (written before the table kernel, which
-  // this kernel follows on the stream): it runs before waiting for the merge.
-  window_item<D, GP>(a, b, kvh, win_smem);
-  __syncthreads();   // this block's window terms (global) are visible to all its threads
-  const int g0 = warp;
-  float mw0 = -INFINITY, lw0 = 0.f, ow0[E];
-  if (g0 < a.G) {
-    mw0 = a.wm[pair * GP + g0];
-    lw0 = a.wl[pair * GP + g0];
-#pragma unroll
-    for (int q = 0; q < E; ++q) ow0[q] = a.wo[(pair * GP + g0) * D + q * 32 + lane];
-  }
-  pdl_wait();   // stage partials of the merge
-  if (tid < GP) {
-    int64_t first, last;
-    pair_slots(a, pair, first, last);
-    const int n = last >= first ? (int)(last - first + 1) : 0;
-    const float* pmp = a.pm + (pair + first) * GP + tid;
-    const float* plp = a.pl + (pair + first) * GP + tid;
-    float m = -INFINITY, l = 0.f;
-    for (int k0 = 0; k0 < n; k0 += 8) {   // groups of 8 predicated loads
-      float v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = k0 + i < n ? pmp[(k0 + i) * GP] : -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, v[i]);
-    }
-    for (int k0 = 0; k0 < n; k0 += 8) {
-      float v[8], w[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[i] = k0 + i < n ? pmp[(k0 + i) * GP] : -INFINITY;
-        w[i] = k0 + i < n ? plp[(k0 + i) * GP] : 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) l += k0 + i < n ? ex2_approx(v[i] - m) * w[i] : 0.f;
-    }
-    mstar_s[tid] = m;
-    lstar_s[tid] = l;
-  }
-  const int nparts = a.Sv * kMergeQ;   // a multiple of 4, at most 32
-  for (int f = tid; f < GP * D; f += 256) {
-    const float* src = a.so + pair * nparts * GP * D + f;
-    float v = 0.f;
-    for (int q0 = 0; q0 < nparts; q0 += 16) {   // 16 predicated loads per round trip
-      float t[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) t[i] = q0 + i < nparts ? src[(q0 + i) * GP * D] : 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v += t[i];
-    }
-    oc[f] = v;
-  }
-  __syncthreads();
-  for (int g = warp; g < a.G; g += 8) {
-    double v[E];
-#pragma unroll
-    for (int q = 0; q < E; ++q) v[q] = (double)oc[g * D + q * 32 + lane];
-    fwht_warp_f64<D>(v, lane);
-    const float mc = mstar_s[g], lc = lstar_s[g];
-    const float mw = g == g0 ? mw0 : a.wm[pair * GP + g];
-    const float lw = g == g0 ? lw0 : a.wl[pair * GP + g];
-    const float M = fmaxf(mc, mw);
-    const float wc = (mc == -INFINITY) ? 0.f : ex2_approx(mc - M);
-    const float ww = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-    const float L = wc * lc + ww * lw;
-    const int64_t h = (int64_t)kvh * a.G + g;
-    float* o = a.out + ((int64_t)b * a.Hq + h) * D;
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
-      const int i = q * 32 + lane;
-      const float ow = g == g0 ? ow0[q] : a.wo[(pair * GP + g) * D + i];
-      o[i] = (wc * (float)(v[q] * a.rot) + ww * ow) * inv;
-    }
-    if (lane == 0 && a.lse) {
-      a.lse[(int64_t)b * a.Hq + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-    }
-  }
-}
 
 // ------------------------------------------------------------------------------------------
 // 4. Product-VQ decode (VeloxQuant "VecInfer": keys and values quantised by sub-vectors
@@ -1718,8 +1506,15 @@ __global__ void __launch_bounds__(256) pq_finalize_kernel(PqArgs a, DecodeArgs w
 // ------------------------------------------------------------------------------------------
 // Launch
 // ------------------------------------------------------------------------------------------
+// Under stream capture the record becomes an event node of the graph (so that each replay
+// records it and the caller can time the kernels between two events).
 static inline void trace(void* const* ev, int i, cudaStream_t st) {
-  if (ev && ev[i]) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), st);
+  if (!ev || !ev[i]) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) cs = cudaStreamCaptureStatusNone;
+  cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(ev[i]), st,
+                           cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                               : cudaEventRecordDefault);
 }
 
 template <int GPH, int SKP, int SVP>
@@ -1788,11 +1583,14 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
   // 1. tables and partition (with the serving step's encode in between)
   trace(ev, 0, st);
   {
-    const size_t smem = sizeof(LutSmem<D>);
+    const size_t smem = std::max(sizeof(LutSmem<D>), window_smem_bytes<D, GP>());
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
     a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
-    const int64_t blocks = (int64_t)a.n_lut_blocks + 1;   // + the partition block
+    // the window changes under the serving step's append: there it runs in the combine kernel
+    a.n_win_blocks = ap ? 0 : a.B * a.Hkv;
+    // + the partition block + one window block per (sequence, kv head)
+    const int64_t blocks = (int64_t)a.n_lut_blocks + 1 + a.n_win_blocks;
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
     // a normal launch: the caller's preceding work (which may write q) must be complete, since
     // the table blocks do not wait
@@ -1821,17 +1619,15 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     }
     if (rc != ZKV_OK) return rc;
   }
-  // 3. merge, finalize
+  // 3. value contraction and final combine (the window partials come from the table kernel, or
+  //    from one more block per pair in the serving step)
   trace(ev, 2, st);
   {
-    const size_t smem = ((size_t)kMergeC * D + (size_t)kMergeC * kMergeRows) * sizeof(float);
-    if (ensure_smem_limit(merge_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
-    const dim3 grid((unsigned)kMergeQ, (unsigned)a.Sv, (unsigned)a.Hkv);
-    if (launch_pdl(merge_kernel<D, GP>, grid, dim3(256), smem, st, a) != cudaSuccess) return ZKV_ERR_CUDA;
-    const size_t fsmem = window_smem_bytes<D, GP>();
-    if (ensure_smem_limit(finalize_kernel<D, GP>, fsmem) != cudaSuccess) return ZKV_ERR_CUDA;
-    if (launch_pdl(finalize_kernel<D, GP>, dim3((unsigned)(a.B * a.Hkv)), dim3(256), fsmem, st, a) != cudaSuccess)
-      return ZKV_ERR_CUDA;
+    const size_t smem = combine_smem_bytes(a.grid, GP, D, a.qc, ap ? window_smem_bytes<D, GP>() : 0);
+    auto* k = ap ? combine_kernel<D, GP, true> : combine_kernel<D, GP, false>;
+    if (ensure_smem_limit(k, smem) != cudaSuccess) return ZKV_ERR_CUDA;
+    const dim3 grid((unsigned)(a.Sv * a.qc + (ap ? 1 : 0)), (unsigned)(a.B * a.Hkv));
+    if (launch_pdl(k, grid, dim3(256), smem, st, a) != cudaSuccess) return ZKV_ERR_CUDA;
   }
   trace(ev, 3, st);
   return ZKV_OK;
@@ -1930,6 +1726,9 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   a.wl = reinterpret_cast<float*>(ws + pl.off_wl);
   a.wo = reinterpret_cast<float*>(ws + pl.off_wo);
   a.so = reinterpret_cast<float*>(ws + pl.off_so);
+  a.cnt = reinterpret_cast<int32_t*>(ws + pl.off_cnt);
+  a.qc = pl.qc;
+  a.n_win_blocks = 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (p->d) {
     case 64: return launch_decode_g<64>(a, pl, p->trace_events, st, ap);

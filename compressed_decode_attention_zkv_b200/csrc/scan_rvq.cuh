@@ -163,6 +163,10 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
   constexpr uint32_t KR = kS2KeyRegion, VR = kS2ValRegion;
   extern __shared__ __align__(16) unsigned char smraw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the combine kernel may be scheduled now: its blocks take the SMs this grid leaves (every
+  // block of this grid is resident, one per SM, by the time all have passed here) and stage
+  // their codebook chunks before waiting for this grid's completion
+  pdl_trigger();
   const uint32_t sbase = smem_u32(smraw);
   uint32_t dyn;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));

@@ -372,7 +372,7 @@ def rvq_decode_attn(q, k_codes, v_codes, comp_len, k_codebooks, v_codebooks, win
                     k_smooth=None, block_table=None):
     """Decode attention over the compressed prefix plus the fp16 window (see include/zkv.h).
     ``trace_events``: optional 4 torch.cuda.Event(enable_timing=True) recorded before the
-    table, scan and merge stages and after the last kernel.  ``k_smooth``: the [Hkv, d] key
+    table, scan and combine kernels and after the last one (graph nodes under capture).  ``k_smooth``: the [Hkv, d] key
     smoothing factors the prefix was encoded with.  ``block_table``: int32 [B, max_pages] for
     the paged layout (k_codes / v_codes are then page pools [n_pages, Hkv, P, S]).
     Returns (out float32 [B, Hq, d], lse float32 [B, Hq])."""
@@ -500,7 +500,7 @@ class PreparedServeStep:
                                   win_v, win_len, out, lse, max_comp_len, softmax_scale,
                                   error_flag, k_smooth, block_table)
         self._ev = None
-        if trace_events is not None:   # recorded before the tables, the scan, the merge, and last
+        if trace_events is not None:   # recorded before the tables, the scan, the combine, and last
             if len(trace_events) != 4:
                 raise ValueError("trace_events needs 4 events")
             self._ev = (c_void_p * 4)(*[e.cuda_event for e in trace_events])

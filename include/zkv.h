@@ -201,8 +201,9 @@ typedef struct {
   float* lse;
   int32_t* error_flag;
   /* Optional tracing: NULL, or 4 cudaEvent_t handles (as void*) recorded on `stream` before
-   * the lookup-table kernel, before the scan kernel, before the two merge kernels and after
-   * them. */
+   * the lookup-table kernel, before the scan kernel, before the combine kernel and after it.
+   * While `stream` is being captured into a CUDA graph they become event-record nodes of the
+   * graph (recorded at every replay). */
   void* const* trace_events;
   /* Optional float32 [Hkv][d]: the per-channel smoothing factors the compressed keys were
    * encoded with (zkv_encode_params.smooth).  The query is multiplied by them before its
