@@ -21,9 +21,8 @@
 //      sums the partial outputs (float4 loads, parts split over thread slices and added in a
 //      fixed order), rotates them back (H / sqrt(d), float64 transform rounded once), and
 //      merges with the window partial by log-sum-exp.  No block waits for another.
-// The window partial comes from the table kernel in a decode call.  In the serving step the
-// window changes under this step's append, so one more block per pair (x = Sv * QC) computes it
-// here, after the append, and takes its turn at the counter like the others.
+// The window partials come from the table kernel (complete before the scan's, and so before
+// this kernel's, wait returns).
 #pragma once
 
 constexpr int kCombineFin = 1024;   // floats of the finishing block's slice buffer
@@ -46,16 +45,12 @@ __host__ __device__ inline CombineSmem combine_layout(int grid, int GP, int d, i
   L.total = L.fin + kCombineFin;
   return L;
 }
-// At least win_bytes: the window block's tiles in the serving step.
-inline size_t combine_smem_bytes(int grid, int GP, int d, int qc, size_t win_bytes) {
-  const size_t c = (size_t)combine_layout(grid, GP, d, qc).total * sizeof(float);
-  return c > win_bytes ? c : win_bytes;
+inline size_t combine_smem_bytes(int grid, int GP, int d, int qc) {
+  return (size_t)combine_layout(grid, GP, d, qc).total * sizeof(float);
 }
 
-// WIN: the grid has the serving step's window blocks (x = Sv * QC).  Without them the kernel
-// fits four blocks per SM.
-template <int D, int GP, bool WIN>
-__global__ void __launch_bounds__(256, WIN ? 2 : 4) combine_kernel(DecodeArgs a) {
+template <int D, int GP>
+__global__ void __launch_bounds__(256, 4) combine_kernel(DecodeArgs a) {
   constexpr int E = D / 32;
   constexpr int TG = 256 / D;                       // thread groups over the head dimension
   constexpr int HPT = GP >= TG ? GP / TG : 1;       // heads per thread in the contraction
@@ -67,7 +62,6 @@ __global__ void __launch_bounds__(256, WIN ? 2 : 4) combine_kernel(DecodeArgs a)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int QC = a.qc, ncw = kCodebook / QC;
   const int s = (int)blockIdx.x / QC, qc = (int)blockIdx.x % QC;
-  const bool win_blk = WIN && s >= a.Sv;            // the serving step's window block
   const int64_t pair = blockIdx.y;
   const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
   const int c0 = qc * ncw;
@@ -79,21 +73,29 @@ __global__ void __launch_bounds__(256, WIN ? 2 : 4) combine_kernel(DecodeArgs a)
   __shared__ float Ms[GP], Ls[GP];
   __shared__ int last_s;
   // 0. the codebook chunk, in flight across the wait
-  if (!win_blk) {
+  {
     const float* cv = a.Cv + (((int64_t)kvh * a.Sv + s) * kCodebook + c0) * D;
     for (int f = tid; f < ncw * D / 4; f += 256) cp_async16(cvs + 4 * f, cv + 4 * f);
     cp_async_commit();
   }
   pdl_wait();   // the scan's partials (and, through it, the append and the table kernel)
-  if constexpr (WIN) {
-    if (win_blk) {
-      window_item<D, GP>(a, b, kvh, reinterpret_cast<unsigned char*>(csm));
-      __syncthreads();   // its shared memory is reused below
-    }
-  }
   const int64_t first = a.pfirst[pair], last = a.plast[pair];
   const int n = last >= first ? (int)(last - first + 1) : 0;
   const int64_t slot0 = pair + first;
+  // step 2's item of this thread: f0 = (c, g), g fastest (coalesced slot rows); with I < 256
+  // items, thread slice p takes the slots p, p + P, ...  Its first eight slot values are loaded
+  // now, beside the maxima (they do not depend on them).
+  const int I = ncw * GP;
+  const int P = I >= 256 ? 1 : 256 / I;
+  const int p = P == 1 ? 0 : tid / I;
+  const int64_t stride = (int64_t)a.Sv * kCodebook * GP;   // one slot
+  const float* base = a.pw + (slot0 * a.Sv + s) * (int64_t)(kCodebook * GP) + (int64_t)c0 * GP;
+  float pv[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int k = p + j * P;
+    pv[j] = k < n ? base[(int64_t)k * stride + (P == 1 ? tid : tid % I)] : 0.f;
+  }
   // 1. slot maxima -> per-head maximum (warp g) -> weights
   for (int f = tid; f < n * GP; f += 256) pmv[f] = a.pm[slot0 * GP + f];
   __syncthreads();
@@ -106,19 +108,19 @@ __global__ void __launch_bounds__(256, WIN ? 2 : 4) combine_kernel(DecodeArgs a)
   __syncthreads();
   for (int f = tid; f < n * GP; f += 256) pmv[f] = ex2_approx(pmv[f] - Ms[f % GP]);
   __syncthreads();
-  if (!win_blk) {
-    // 2. merged histogram of the chunk: item f = (c, g), g fastest (coalesced slot rows);
-    //    with I < 256 items, thread slice p takes the slots p, p + P, ...
-    const int I = ncw * GP;
-    const int P = I >= 256 ? 1 : 256 / I;
-    const int64_t stride = (int64_t)a.Sv * kCodebook * GP;   // one slot
-    const float* base = a.pw + (slot0 * a.Sv + s) * (int64_t)(kCodebook * GP) + (int64_t)c0 * GP;
-    const int p = P == 1 ? 0 : tid / I;
+  {
+    // 2. merged histogram of the chunk
     for (int f0 = (P == 1 ? tid : tid % I); f0 < I; f0 += 256) {
       const int g = f0 % GP;
       const float* src = base + f0;
       float w = 0.f;
       int k = p;
+      if (f0 < 256) {   // the first item: its first eight slots are in pv
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (p + j * P < n) w = fmaf(pmv[(p + j * P) * GP + g], pv[j], w);
+        k = p + 8 * P;
+      }
       for (; k + 7 * P < n; k += 8 * P) {   // eight independent loads per round trip
         float v[8];
 #pragma unroll
@@ -172,6 +174,14 @@ __global__ void __launch_bounds__(256, WIN ? 2 : 4) combine_kernel(DecodeArgs a)
     l = warp_sum_f32(l);
     if (lane == 0) Ls[warp] = l;
   }
+  // the window partial of warp g's head, loaded beside the partial outputs
+  float wmg = -INFINITY, wlg = 0.f, wog[E];
+  if (warp < a.G) {
+    wmg = a.wm[pair * GP + warp];
+    wlg = a.wl[pair * GP + warp];
+#pragma unroll
+    for (int q = 0; q < E; ++q) wog[q] = a.wo[(pair * GP + warp) * D + q * 32 + lane];
+  }
   // the sum of the stage / chunk partial outputs (rotated domain, unnormalised): piece f4 of
   // the parts p2, p2 + P2, ... in slice p2, then the slices in order
   float* ocb = csm + L.ocb;   // [GP][D]
@@ -211,13 +221,14 @@ __global__ void __launch_bounds__(256, WIN ? 2 : 4) combine_kernel(DecodeArgs a)
     }
   }
   __syncthreads();
-  for (int g = warp; g < a.G; g += 8) {
+  if (warp < a.G) {   // G <= 8: one head per warp
+    const int g = warp;
     double v[E];
 #pragma unroll
     for (int q = 0; q < E; ++q) v[q] = (double)ocb[g * D + q * 32 + lane];
     fwht_warp_f64<D>(v, lane);
     const float mc = Ms[g], lc = Ls[g];
-    const float mw = a.wm[pair * GP + g], lw = a.wl[pair * GP + g];
+    const float mw = wmg, lw = wlg;
     const float M = fmaxf(mc, mw);
     const float wc = (mc == -INFINITY) ? 0.f : ex2_approx(mc - M);
     const float ww = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
@@ -228,7 +239,7 @@ __global__ void __launch_bounds__(256, WIN ? 2 : 4) combine_kernel(DecodeArgs a)
 #pragma unroll
     for (int q = 0; q < E; ++q) {
       const int i = q * 32 + lane;
-      o[i] = (wc * (float)(v[q] * a.rot) + ww * a.wo[(pair * GP + g) * D + i]) * inv;
+      o[i] = (wc * (float)(v[q] * a.rot) + ww * wog[q]) * inv;
     }
     if (lane == 0 && a.lse) a.lse[(int64_t)b * a.Hq + h] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
   }

@@ -59,13 +59,15 @@ constexpr size_t kSmemMax = 227 * 1024;
 // Token-per-thread scan (scan_rvq.cuh).
 constexpr int kS2Threads = 512;
 constexpr int kS2Fix = 20;                        // value weights as integers of p * 2^20
-constexpr float kS2Headroom = 1.f;                // log2 units added to a new reference
+constexpr float kS2Headroom = 3.f;                // log2 units added to a new reference
 constexpr uint32_t kS2KeyRegion = 1u << 16;       // absolute shared address of the key tables
 constexpr uint32_t kS2ValRegion = 2u << 16;       // ... of the value histograms
-constexpr size_t kS2Smem = size_t(3) << 16;       // dynamic shared memory requested
-// Set-up cost of one scan segment (table fill, final fold and write: about 1.5K cycles) in
-// tokens of the loop (about 1.3 cycles per token and SM).
-constexpr int64_t kS2SegCost = 1200;
+constexpr uint32_t kS2ExvRegion = 3u << 16;       // ... of the listed tokens' value words
+constexpr size_t kS2Smem = (size_t(3) << 16) + 32768;   // dynamic shared memory requested
+// Set-up cost of one scan segment (table fill, the reference from the first sub-chunk, final
+// fold and write: about 8K cycles measured) in tokens of the loop (about 1.3 cycles per token
+// and SM).
+constexpr int64_t kS2SegCost = 6000;
 
 
 static int sm_count() {
@@ -104,7 +106,7 @@ struct DecodePlan {
   int64_t seg_cost;
   int64_t cap, slots;
   size_t scan_smem;
-  size_t off_lut, off_pre, off_bounds, off_vs, off_pfirst, off_plast, off_pm, off_pl, off_pw,
+  size_t off_lut, off_pre, off_bounds, off_ctap, off_vs, off_pfirst, off_plast, off_pm, off_pl, off_pw,
       off_wm, off_wl, off_wo, off_so, off_cnt, total;
   int qc;
 };
@@ -159,6 +161,7 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   pl.off_lut = o;   o = align256(o + (size_t)pairs * p->Sk * kCodebook * pl.GP * f);
   pl.off_pre = o;   o = align256(o + (size_t)(pairs + 1) * sizeof(int64_t));
   pl.off_bounds = o; o = align256(o + (size_t)(grid + 1) * sizeof(int64_t));
+  pl.off_ctap = o;  o = align256(o + (size_t)(grid + 1) * sizeof(int32_t));
   pl.off_vs = o;    o = align256(o + (size_t)(pairs + 1) * sizeof(int64_t));
   pl.off_pfirst = o; o = align256(o + (size_t)pairs * sizeof(int32_t));
   pl.off_plast = o; o = align256(o + (size_t)pairs * sizeof(int32_t));
@@ -186,12 +189,16 @@ struct DecodeArgs {
   int B, Hq, Hkv, G, GP, d, Sk, Sv, Rk, grid, n_lut_blocks;
   int64_t seg_cost;   // set-up cost of one scan segment, in tokens (partition weight)
   int qc;             // codeword chunks per value stage in the combine kernel
-  int n_win_blocks;   // window blocks of the table kernel (one per (sequence, kv head))
   // Serving step: the partition uses the lengths after this step's append (predicted from
   // the pre-step state with the append's rule), and scan block 0 stores them.  Null otherwise.
   int32_t* upd_win_len;
   int32_t* upd_win_head;
   int32_t* upd_comp_len;
+  // Serving step: the new tokens [B][Hkv][d].  The window attention runs before this step's
+  // append and attends to the window that append produces (the new token in the slot it
+  // takes).  Null otherwise.
+  const __half* new_k;
+  const __half* new_v;
   int64_t Tcap, Wcap, max_comp;
   float scale_log2;   // softmax_scale * log2(e)
   double rot;         // 1 / sqrt(d)
@@ -214,6 +221,8 @@ struct DecodeArgs {
   float* lut;        // [B][Hkv][Sk][256][GP] (heads g >= G unwritten)
   int64_t* pre;      // [B*Hkv + 1] exclusive prefix sums of compressed lengths
   int64_t* bounds;   // [grid + 1] token range of each scan CTA
+  int32_t* ctap;     // [grid + 1] the pair holding each CTA's first cut (its first segment's pair
+                     // or an earlier one with nothing left at the cut)
   int64_t* vs;       // [B*Hkv + 1] virtual start of each pair (tokens + kSegCost per nonempty pair)
   int32_t* pfirst;   // [B*Hkv] first scan CTA covering the pair (> plast when it has no tokens)
   int32_t* plast;    // [B*Hkv] last scan CTA covering the pair
@@ -237,9 +246,8 @@ __device__ __forceinline__ int64_t clamp_win_len(const DecodeArgs& a, int b) {
 }
 
 // ------------------------------------------------------------------------------------------
-// 1. Query rotation + lookup tables; length prefix sums (the partition block).  The dense
-//    window attention (window_item) runs here in a decode call and in the combine kernel in
-//    the serving step.
+// 1. Query rotation + lookup tables; length prefix sums (the partition block); the dense
+//    window attention (window_item), one block per pair.
 // ------------------------------------------------------------------------------------------
 constexpr int kLutC = 64;     // codewords per table block (one per thread and head quad)
 constexpr int kLutH = 16;     // attached query heads per table block (b * G + g)
@@ -266,38 +274,68 @@ __device__ __forceinline__ void prefetch_l2(const uint8_t* lo, const uint8_t* hi
 }
 
 // Dense attention of the GP heads of one (sequence, kv head) over its fp16 window (base-2
-// logits, online maximum over tiles).  Each tile's K and V rows are copied to shared memory
-// with cp.async in one round (64 KB); warps then take tokens and lanes split the head
-// dimension.
+// logits, online maximum over tiles).  Each tile's K and V rows (WT tokens) are copied to
+// shared memory with cp.async in one round; warps then take tokens and lanes split the head
+// dimension.  256 threads.
 template <int D>
 constexpr int win_tile() { return 16384 / D; }   // tokens per tile: K + V tiles = 64 KB
+template <int D>
+constexpr int win_tile_small() { return 4096 / D; }   // K + V tiles = 16 KB
 
-template <int D, int GP>
+// the warps' partial outputs [8][GP][D] reuse the tiles when they fit there
+template <int D, int GP, int WT>
+constexpr bool win_part_in_tiles() { return (size_t)8 * GP * D * 4 <= (size_t)2 * WT * D * 2; }
+
+template <int D, int GP, int WT = win_tile<D>()>
 constexpr size_t window_smem_bytes() {
-  return (size_t)2 * win_tile<D>() * D * sizeof(__half) + (size_t)win_tile<D>() * GP * 4 +
-         (size_t)8 * GP * 4;
+  return (size_t)2 * WT * D * sizeof(__half) + (size_t)WT * GP * 4 + (size_t)8 * GP * 4 +
+         (win_part_in_tiles<D, GP, WT>() ? 0 : (size_t)8 * GP * D * 4);
 }
 
-template <int D, int GP>
+template <int D, int GP, int WT = win_tile<D>()>
 __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* smem) {
   constexpr int PL = D / 32;        // head dims per lane
-  constexpr int WT = win_tile<D>();
   __half* kt = reinterpret_cast<__half*>(smem);                     // [WT][D]
   __half* vt = kt + WT * D;                                         // [WT][D]
   float* sc = reinterpret_cast<float*>(vt + WT * D);                // [WT][GP] scores, then p
   float* red = sc + WT * GP;                                        // [8][GP]
-  float* part = reinterpret_cast<float*>(smem);                     // [8][GP][D], after the tiles
-  static_assert((size_t)8 * GP * D * 4 <= (size_t)2 * WT * D * 2, "partials fit in the tiles");
+  float* part = win_part_in_tiles<D, GP, WT>() ? reinterpret_cast<float*>(smem)
+                                               : red + 8 * GP;      // [8][GP][D], after the tiles
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pair = (int64_t)b * a.Hkv + kvh;
-  const int64_t wl = clamp_win_len(a, b);
+  // the window's length and, in the serving step, the slot this step's append gives the new
+  // token (by the append's rule, from the pre-step state: a free slot, else the oldest one
+  // while the prefix has room); the window is a set of rows, so their order does not matter
+  int64_t wl, sub = -1;
+  if (a.new_k) {
+    const int64_t w0 = a.upd_win_len[b], hd = a.upd_win_head[b], c = a.upd_comp_len[b];
+    if (w0 >= 0 && w0 < a.Wcap) {
+      sub = w0;
+      wl = w0 + 1;
+    } else if (w0 == a.Wcap && hd >= 0 && hd < a.Wcap) {
+      wl = w0;
+      if (c >= 0 && c < a.Tcap) sub = hd;
+    } else {
+      wl = clamp_win_len(a, b);
+    }
+  } else {
+    wl = clamp_win_len(a, b);
+  }
   const __half* Kb = a.win_k + pair * a.Wcap * D;
   const __half* Vb = a.win_v + pair * a.Wcap * D;
   auto stage = [&](int64_t base) {   // rows [base, base + n) as 16-byte pieces
     const int n = (int)(wl - base < WT ? wl - base : WT);
     for (int f = tid; f < n * D / 8; f += 256) {
+      if (base + f / (D / 8) == sub) continue;
       cp_async16(kt + f * 8, Kb + base * D + f * 8);
       cp_async16(vt + f * 8, Vb + base * D + f * 8);
+    }
+    if (sub >= base && sub < base + n) {   // the new token (plain loads: no alignment assumed)
+      const int64_t ro = (sub - base) * D;
+      for (int i = tid; i < D; i += 256) {
+        kt[ro + i] = a.new_k[pair * D + i];
+        vt[ro + i] = a.new_v[pair * D + i];
+      }
     }
   };
   if (wl > 0) stage(0);   // in flight while the query is loaded
@@ -508,7 +546,10 @@ __device__ void partition_block(const DecodeArgs& a) {
   // grid is very large
   const bool wide = (double)(V + a.seg_cost + 1) * (double)grid >= 4.0e18;
   if (V == 0) {   // no compressed token at all
-    for (int c = tid; c <= grid; c += 256) a.bounds[c] = 0;
+    for (int c = tid; c <= grid; c += 256) {
+      a.bounds[c] = 0;
+      a.ctap[c] = 0;
+    }
     for (int k = tid; k < npairs; k += 256) {
       a.pfirst[k] = 1;
       a.plast[k] = 0;
@@ -518,6 +559,8 @@ __device__ void partition_block(const DecodeArgs& a) {
   if (tid == 0) {
     a.bounds[0] = 0;
     a.bounds[grid] = tot;
+    a.ctap[0] = 0;
+    a.ctap[grid] = npairs;
   }
   for (int k = tid; k < npairs; k += 256) {
     const int64_t v0 = a.vs[k], v1 = a.vs[k + 1], p0 = a.pre[k], len = a.pre[k + 1] - p0;
@@ -528,6 +571,7 @@ __device__ void partition_block(const DecodeArgs& a) {
       for (int64_t c = clo > 1 ? clo : 1; c <= chi && c < grid; ++c) {
         const int64_t off = floor_muldiv(V, c, grid, wide) - v0;
         a.bounds[c] = off < a.seg_cost ? p0 : p0 + (off - a.seg_cost < len ? off - a.seg_cost : len);
+        a.ctap[c] = k;
       }
       // the CTA holding the first token: the last cut at or before v0 + a.seg_cost (its bound is
       // p0); the one holding the last token: the last cut before v1
@@ -544,7 +588,7 @@ __device__ void partition_block(const DecodeArgs& a) {
 // head); thread (codeword cc, head quad hq) forms 4 dot products.  Block n_lut_blocks is the
 // partition block.
 template <int D, int GP>
-__global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(256, GP >= 8 ? 2 : 3) lut_kernel(DecodeArgs a) {
   constexpr int E = D / 32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -555,8 +599,9 @@ __global__ void __launch_bounds__(256) lut_kernel(DecodeArgs a) {
     return;
   }
   if ((int)blockIdx.x > a.n_lut_blocks) {
-    // dense attention over the fp16 window of one (sequence, kv head); it reads only the call's
-    // inputs, so it runs here, beside the tables and the scan's start
+    // dense attention over the fp16 window of one (sequence, kv head): it reads only the call's
+    // inputs (in the serving step it substitutes the new token for the slot the append gives
+    // it), so it runs here, beside the tables
     const int pair = (int)blockIdx.x - a.n_lut_blocks - 1;
     window_item<D, GP>(a, pair / a.Hkv, pair % a.Hkv, smem_raw);
     return;
@@ -1587,10 +1632,8 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
     a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
-    // the window changes under the serving step's append: there it runs in the combine kernel
-    a.n_win_blocks = ap ? 0 : a.B * a.Hkv;
     // + the partition block + one window block per (sequence, kv head)
-    const int64_t blocks = (int64_t)a.n_lut_blocks + 1 + a.n_win_blocks;
+    const int64_t blocks = (int64_t)a.n_lut_blocks + 1 + (int64_t)a.B * a.Hkv;
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
     // a normal launch: the caller's preceding work (which may write q) must be complete, since
     // the table blocks do not wait
@@ -1619,14 +1662,13 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
     }
     if (rc != ZKV_OK) return rc;
   }
-  // 3. value contraction and final combine (the window partials come from the table kernel, or
-  //    from one more block per pair in the serving step)
+  // 3. value contraction and the final combine with the window partials
   trace(ev, 2, st);
   {
-    const size_t smem = combine_smem_bytes(a.grid, GP, D, a.qc, ap ? window_smem_bytes<D, GP>() : 0);
-    auto* k = ap ? combine_kernel<D, GP, true> : combine_kernel<D, GP, false>;
+    const size_t smem = combine_smem_bytes(a.grid, GP, D, a.qc);
+    auto* k = combine_kernel<D, GP>;
     if (ensure_smem_limit(k, smem) != cudaSuccess) return ZKV_ERR_CUDA;
-    const dim3 grid((unsigned)(a.Sv * a.qc + (ap ? 1 : 0)), (unsigned)(a.B * a.Hkv));
+    const dim3 grid((unsigned)(a.Sv * a.qc), (unsigned)(a.B * a.Hkv));
     if (launch_pdl(k, grid, dim3(256), smem, st, a) != cudaSuccess) return ZKV_ERR_CUDA;
   }
   trace(ev, 3, st);
@@ -1701,6 +1743,8 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   a.upd_win_len = ap ? ap->win_len : nullptr;
   a.upd_win_head = ap ? ap->win_head : nullptr;
   a.upd_comp_len = ap ? ap->comp_len : nullptr;
+  a.new_k = ap ? reinterpret_cast<const __half*>(ap->new_k) : nullptr;
+  a.new_v = ap ? reinterpret_cast<const __half*>(ap->new_v) : nullptr;
   a.Tcap = p->Tcap; a.Wcap = p->Wcap; a.max_comp = p->max_comp_len;
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale : (float)(1.0 / std::sqrt((double)p->d));
   a.scale_log2 = scale * kLog2e;
@@ -1716,6 +1760,7 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   a.lut = reinterpret_cast<float*>(ws + pl.off_lut);
   a.pre = reinterpret_cast<int64_t*>(ws + pl.off_pre);
   a.bounds = reinterpret_cast<int64_t*>(ws + pl.off_bounds);
+  a.ctap = reinterpret_cast<int32_t*>(ws + pl.off_ctap);
   a.vs = reinterpret_cast<int64_t*>(ws + pl.off_vs);
   a.pfirst = reinterpret_cast<int32_t*>(ws + pl.off_pfirst);
   a.plast = reinterpret_cast<int32_t*>(ws + pl.off_plast);
@@ -1728,7 +1773,6 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   a.so = reinterpret_cast<float*>(ws + pl.off_so);
   a.cnt = reinterpret_cast<int32_t*>(ws + pl.off_cnt);
   a.qc = pl.qc;
-  a.n_win_blocks = 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (p->d) {
     case 64: return launch_decode_g<64>(a, pl, p->trace_events, st, ap);
@@ -1911,21 +1955,12 @@ namespace zkv {
 
 static __device__ __align__(256) unsigned char g_decode_scratch[ZKV_DECODE_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-static std::mutex g_scratch_mu;
-static void* g_scratch_addr[kMaxDevices];
-
-// Device address of g_decode_scratch on the current device, looked up once per device.
+// Device address of g_decode_scratch on the current device.  Looked up at every call (a
+// host-side lookup): after a device reset the module loads again, possibly at a new address.
 static void* decode_scratch_address() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_decode_scratch) != cudaSuccess) return nullptr;
-    g_scratch_addr[dev] = a;
-  }
-  return g_scratch_addr[dev];
+  void* a = nullptr;
+  if (cudaGetSymbolAddress(&a, g_decode_scratch) != cudaSuccess) return nullptr;
+  return a;
 }
 
 }  // namespace zkv

@@ -40,8 +40,11 @@
 // aggregate (plain rounding would drop the mass of the many tokens with p below 2^-21).  The sum
 // of n rounding errors has a standard deviation near 2^-20 sqrt(n / 12) of the largest p.  A word
 // collects at most one u per token of the lanes of its replica, i.e. at most 512 U / R tokens per
-// sub-chunk; the block folds the words into float32 masters at least every 8 R / U - 1
-// sub-chunks, so no word passes 2^32.
+// sub-chunk, so a run of at most 8 R / U - 1 sub-chunks cannot take a zero word past 2^32.  The
+// words are folded into float32 masters only when the next run could: every word holds at most
+// the sum of the u added since the last fold, and every thread keeps the sum of its p, so at
+// each run boundary the block knows that bound and shortens the next run, or folds, when the
+// bound plus the next run's worst case would pass 2^32.
 
 // Reference: the first sub-chunk's block maximum plus 1 (log2 units).  Sub-chunks take block i of every warp's
 // contiguous run of the segment, so that first sub-chunk samples the whole segment.  A later
@@ -87,8 +90,10 @@ struct S2Cfg {
   static constexpr int VW = U * SVP / 4;
   static constexpr int NENT = SVP * kCodebook * GPH;   // histogram entries of one pass
   static constexpr int NE = (NENT + kS2Threads - 1) / kS2Threads;
-  // a word takes <= 512 U / R tokens of <= 2^20 each per sub-chunk: fold before 2^32
-  static constexpr int FOLD_EVERY = (8 / U) * R - 1;    // sub-chunks between capacity folds
+  // a word takes <= 512 U / R tokens of <= 2^20 each per sub-chunk: runs from a zero word stay
+  // below 2^32
+  static constexpr int FOLD_EVERY = (8 / U) * R - 1;    // sub-chunks in the longest run
+  static constexpr float WSUB = (float)(kS2Threads * U / R) * 1048577.f;   // per word, sub-chunk
   static constexpr int NW = kS2Threads / 32;
   static constexpr int SUBT = kS2Threads * U;    // tokens per sub-chunk
   static constexpr int LCAP = 8192;               // exception list entries
@@ -174,11 +179,16 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
   uint32_t* redk = reinterpret_cast<uint32_t*>(smraw);                    // [2][NW][GPH] maxima
   float* reds = reinterpret_cast<float*>(smraw + 8 * C::NW * GPH);          // [NW][GPH] sums
   float* mst = reinterpret_cast<float*>(smraw + 12 * C::NW * GPH);   // masters [256][SVP][GPH]
-  // exception list: pair-local indices of tokens whose score exceeded the reference, and its count
-  uint32_t* exl = reinterpret_cast<uint32_t*>(smraw + 12 * C::NW * GPH + 4 * C::NE * kS2Threads);
-  uint32_t* exn = exl + C::LCAP;
-  const bool fits = sbase + 12u * C::NW * GPH + 4u * C::NE * kS2Threads + 4u * C::LCAP + 16u <= KR &&
-                    sbase + dyn >= VR + 65536u;
+  // exception list: the key code words of the tokens whose score exceeded the reference (each
+  // shifted so that the token's codes are its low bytes; their value words, likewise, sit at
+  // kS2ExvRegion), and its count
+  uint32_t* exk = reinterpret_cast<uint32_t*>(smraw + 12 * C::NW * GPH + 4 * C::NE * kS2Threads);
+  uint32_t* exn = exk + C::LCAP;                                // [2] counts (runs alternate)
+  float* redp = reinterpret_cast<float*>(exn + 4);              // [2][NW] warps' p sums
+  constexpr uint32_t XV = kS2ExvRegion;
+  const bool fits = sbase + 12u * C::NW * GPH + 4u * C::NE * kS2Threads + 4u * C::LCAP + 16u +
+                            8u * C::NW <= KR &&
+                    sbase + dyn >= XV + 4u * C::LCAP;
   if (fits) {
     // zero the value histograms (the final fold of every segment leaves them zero again)
     for (uint32_t o = VR + 16u * tid; o < VR + 65536u; o += 16u * kS2Threads) sts128z(o);
@@ -214,21 +224,14 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
   const int Sk = a.Sk, Sv = a.Sv, G = a.G, GP = a.GP;
   const int npairs = a.B * a.Hkv;
   const int64_t lo = a.bounds[blockIdx.x], hi = a.bounds[blockIdx.x + 1];
+  // the pair holding this CTA's cut (the partition places it with the cut); lanes hold the
+  // prefix starts of the next 32 pairs
+  const int pfirst = a.ctap[blockIdx.x];
   if (lo >= hi) return;
-  // last pair whose prefix start is <= lo (block-parallel search; pre is non-decreasing)
-  int pfirst = 0;
-  {
-    int l = 0, r = npairs;
-    while (r - l > 1) {
-      const int step = (r - l + kS2Threads - 1) / kS2Threads;
-      const int k = l + tid * step;
-      const int cnt = __syncthreads_count(k < r && a.pre[k] <= lo);
-      l = l + (cnt - 1) * step;
-      r = l + step < r ? l + step : r;
-    }
-    pfirst = l;
-  }
-
+  const int64_t pre_l = pfirst + lane <= npairs ? a.pre[pfirst + lane] : INT64_MAX;
+  auto pre_at = [&](int pr) -> int64_t {   // a.pre[pr], pr >= pfirst (uniform across the block)
+    return pr - pfirst < 32 ? __shfl_sync(0xffffffffu, pre_l, pr - pfirst) : a.pre[pr];
+  };
   // ---- per-lane constants
   const uint32_t lg = (uint32_t)lane & (GPH - 1);
   const uint32_t kcopy = (uint32_t)lane & (C::RK - 1);
@@ -276,6 +279,8 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
   const float dith = ((float)(__brev((uint32_t)lane) >> 27) + 0.5f) * (1.f / 32.f) - 0.5f;
 
   // ---- the pieces of the loop
+  // this thread's sum of the p it has added to the words since the last fold (all heads)
+  float2 ps2 = make_float2(0.f, 0.f);
   // score of token u of a group, heads rotated by lg; init = -(reference - 20) per rotated head
   auto key_score1 = [&](auto uc, const uint32_t (&wk)[C::KW], const float (&init)[GPH],
                         float (&scu)[GPH]) {
@@ -313,13 +318,17 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
     if constexpr (GPH >= 2) {
       static_for<GPH / 2>([&](auto hc) {
         constexpr int j = 2 * hc;
-        float2 e = fadd2(make_float2(ex2_ftz(scu[j]), ex2_ftz(scu[j + 1])), make_float2(dith, dith));
+        const float2 pp = make_float2(ex2_ftz(scu[j]), ex2_ftz(scu[j + 1]));
+        ps2 = fadd2(ps2, pp);
+        float2 e = fadd2(pp, make_float2(dith, dith));
         e = fadd2(e, make_float2(magic, magic));
         pu[j] = __float_as_uint(e.x) - 0x4B400000u;
         pu[j + 1] = __float_as_uint(e.y) - 0x4B400000u;
       });
     } else {
-      pu[0] = __float_as_uint((ex2_ftz(scu[0]) + dith) + magic) - 0x4B400000u;
+      const float p0 = ex2_ftz(scu[0]);
+      ps2.x += p0;
+      pu[0] = __float_as_uint((p0 + dith) + magic) - 0x4B400000u;
     }
     static_for<SVP>([&](auto ic) {
       constexpr int i = ic;
@@ -379,12 +388,9 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
         if (((uint32_t)j + lg) % GPH == (uint32_t)g) refk[g] = -init[j];
     }
   };
-  // key score (rotated heads, relative to init) of one token t of the segment, read alone
-  auto key_score_tok = [&](const PairRows& kcb_cur, uint32_t t, const float (&init)[GPH],
-                           float (&x)[GPH]) {
+  // key score (rotated heads, relative to init) of token t from its key word
+  auto key_score_w = [&](uint32_t w, uint32_t t, const float (&init)[GPH], float (&x)[GPH]) {
     const uint32_t q = t & (4u / SKP - 1u);   // the token's slot in its 32-bit code word
-    const uint8_t* row = pair_row<PAGED>(a, kcb_cur, t - q, Sk);
-    const uint32_t w = row ? __ldg(reinterpret_cast<const unsigned int*>(row)) : 0u;
 #pragma unroll
     for (int j = 0; j < GPH; ++j) x[j] = init[j];
 #pragma unroll
@@ -403,16 +409,18 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
       }
     }
   };
-  // the value side of one token t with rotated x (relative to the reference - 20)
-  auto value_red_tok = [&](const PairRows& vcb_cur, uint32_t t, const float (&x)[GPH]) {
+  // the value side of token t with rotated x (relative to the reference - 20), from its value
+  // word
+  auto value_red_w = [&](uint32_t w, uint32_t t, const float (&x)[GPH]) {
     const uint32_t q = t & (4u / SVP - 1u);
-    const uint8_t* row = pair_row<PAGED>(a, vcb_cur, t - q, Sv);
-    const uint32_t w = row ? __ldg(reinterpret_cast<const unsigned int*>(row)) : 0u;
     const float magic = 12582912.f;
     uint32_t pu[GPH];
 #pragma unroll
-    for (int j = 0; j < GPH; ++j)
-      pu[j] = __float_as_uint((ex2_ftz(x[j]) + dith) + magic) - 0x4B400000u;
+    for (int j = 0; j < GPH; ++j) {
+      const float pj = ex2_ftz(x[j]);
+      ps2.x += pj;
+      pu[j] = __float_as_uint((pj + dith) + magic) - 0x4B400000u;
+    }
 #pragma unroll
     for (int i = 0; i < SVP; ++i) {
       const uint32_t byte = q * SVP + (((uint32_t)i + lvs) & (SVP - 1));
@@ -470,14 +478,16 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
         }
       }
     }
+    ps2 = make_float2(0.f, 0.f);   // the words are zero again
     __syncthreads();
   };
 
-  for (int pr = pfirst; pr < npairs && a.pre[pr] < hi; ++pr) {
-    const int64_t seg0 = lo > a.pre[pr] ? lo : a.pre[pr];
-    const int64_t seg1 = hi < a.pre[pr + 1] ? hi : a.pre[pr + 1];
+  for (int pr = pfirst; pr < npairs && pre_at(pr) < hi; ++pr) {
+    const int64_t pr0 = pre_at(pr), pr1 = pre_at(pr + 1);
+    const int64_t seg0 = lo > pr0 ? lo : pr0;
+    const int64_t seg1 = hi < pr1 ? hi : pr1;
     if (seg0 >= seg1) continue;
-    const uint32_t s0 = (uint32_t)(seg0 - a.pre[pr]), s1 = (uint32_t)(seg1 - a.pre[pr]);
+    const uint32_t s0 = (uint32_t)(seg0 - pr0), s1 = (uint32_t)(seg1 - pr0);
     const int64_t slot = (int64_t)pr + blockIdx.x;
     PairRows kcb, vcb;
     if constexpr (PAGED) {
@@ -570,10 +580,11 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
           }
         }
       }
-      if (tid == 0) *exn = 0u;
+      if (tid < 2) exn[tid] = 0u;
       __syncthreads();   // tables ready; histograms are zero; the exception list is empty
 #pragma unroll
       for (int k = 0; k < C::NE; ++k) mst[k * kS2Threads + tid] = 0.f;   // (covers NENT)
+      ps2 = make_float2(0.f, 0.f);   // the words start at zero
       // init[j] = -(reference - 20) of the lane's rotated head j: the start of every score
       float init[GPH];
       float sc[U][GPH];
@@ -625,12 +636,16 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
         }
       }
       // Runs of sub-chunks with no block-wide step inside: a token whose score exceeds the
-      // reference is listed (and contributes nothing in the run); between runs the block folds
-      // the integer words (capacity) and, when tokens were listed, raises the reference to
-      // their maximum plus the headroom, rescales, and adds their weights.
-      int i = 0, run = C::RUN;
+      // reference is listed (and contributes nothing in the run).  Between runs the block
+      // raises the reference to the listed tokens' maximum plus the headroom when there are any
+      // (folding the words rescaled, then adding the listed tokens' weights), and otherwise
+      // folds only when the bound on the words says the next run could overflow one.  The list
+      // count and the warps' p sums alternate between two buffers, so a boundary with nothing
+      // to do costs one barrier.
+      int i = 0, run = C::RUN, pb = 0;
       while (true) {
         const int stop = i + run < nsub ? i + run : nsub;
+        uint32_t* exc = exn + pb;
         for (; i < stop; ++i) {
           if (i + 1 < nsub) {
             // token by token: the value side of sub-chunk i, then the key side of sub-chunk
@@ -654,8 +669,13 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
               float mx = sc[uc][0];
               static_for<GPH>([&](auto jc) { mx = fmaxf(mx, sc[uc][jc]); });
               if (mx > (float)kS2Fix) {   // above the reference: list it, add it later
-                const uint32_t e = atomicAdd(exn, 1u);
-                if (e < (uint32_t)C::LCAP) exl[e] = t + (uint32_t)uc;
+                constexpr int u = decltype(uc)::value;
+                const uint32_t e = atomicAdd(exc, 1u);
+                if (e < (uint32_t)C::LCAP) {   // its code words, from the registers
+                  exk[e] = kx[(u * SKP) >> 2] >> (8 * ((u * SKP) & 3));
+                  const uint32_t vw = vcur[(u * SVP) >> 2] >> (8 * ((u * SVP) & 3));
+                  asm volatile("st.shared.u32 [%0], %1;" ::"r"(XV + 4u * e), "r"(vw) : "memory");
+                }
                 static_for<GPH>([&](auto jc) { sc[uc][jc] = -INFINITY; });
               }
             });
@@ -663,15 +683,34 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
             static_for<U>([&](auto uc) { value_red1(uc, vcur, sc[uc]); });
           }
         }
-        __syncthreads();   // the run's reductions and list entries are complete
-        const uint32_t n = *exn;   // (the same for every thread)
+        {   // this warp's p sum since the last fold
+          float v = ps2.x + ps2.y;
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) redp[pb * C::NW + warp] = v;
+        }
+        __syncthreads();   // the run's reductions, list entries and p sums are complete
+        const uint32_t n = *exc;   // (the same for every thread)
         if (n > 0u) {
-          // listed tokens: their maxima set the new reference
-          float mt[GPH], m[GPH], x[GPH];
+          // listed tokens (their code words are in the list): their maxima set the new
+          // reference.  A thread's first token keeps its value word and score in registers for
+          // the second pass.
+          float mt[GPH], m[GPH], x[GPH], x0[GPH];
+          uint32_t vw0 = 0u;
+          auto exv_at = [&](uint32_t e) {
+            uint32_t w;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(XV + 4u * e) : "memory");
+            return w;
+          };
 #pragma unroll
           for (int g = 0; g < GPH; ++g) mt[g] = -INFINITY;
-          for (uint32_t e = (uint32_t)tid; e < n; e += kS2Threads) {
-            key_score_tok(kcb, exl[e], init, x);
+          if ((uint32_t)tid < n) {
+            vw0 = exv_at((uint32_t)tid);
+            key_score_w(exk[tid], 0u, init, x0);
+            unrotate_max(x0, mt);
+          }
+          for (uint32_t e = (uint32_t)tid + kS2Threads; e < n; e += kS2Threads) {
+            key_score_w(exk[e], 0u, init, x);
             unrotate_max(x, mt);
           }
           block_max_of(mt, m);
@@ -702,25 +741,39 @@ __global__ void __launch_bounds__(kS2Threads, 1) scan2_kernel(DecodeArgs a) {
           static_for<U>([&](auto uc) {
             static_for<GPH>([&](auto jc) { sc[uc][jc] -= d[jc]; });
           });
-          for (uint32_t e = (uint32_t)tid; e < n; e += kS2Threads) {
-            const uint32_t t = exl[e];
-            key_score_tok(kcb, t, init, x);
-            value_red_tok(vcb, t, x);
+          if ((uint32_t)tid < n) {
+#pragma unroll
+            for (int j = 0; j < GPH; ++j) x0[j] -= d[j];
+            value_red_w(vw0, 0u, x0);
+          }
+          for (uint32_t e = (uint32_t)tid + kS2Threads; e < n; e += kS2Threads) {
+            key_score_w(exk[e], 0u, init, x);
+            value_red_w(exv_at(e), 0u, x);
           }
           __syncthreads();   // list reads and their reductions are complete
-          if (tid == 0) *exn = 0u;
-          // the listed tokens' words count against the next run's capacity
+          if (tid == 0) *exc = 0u;
+          // the words now hold only the listed tokens (at most ceil(n / SUBT) sub-chunks' worth)
           run = C::RUN - (int)((n + C::SUBT - 1) / C::SUBT);
           if (run < 1) {
             fold(1.f);
             run = C::RUN;
           }
         } else {
-          run = C::RUN;
+          // every word holds at most 2^20 (sum of p) + (its additions) since the last fold; the
+          // next run adds at most WSUB per sub-chunk to one word
+          float T = 0.f;
+#pragma unroll
+          for (int w = 0; w < C::NW; ++w) T += redp[pb * C::NW + w];
+          const float used = T * 1048576.f * 1.001f + 16777216.f;
+          const float avail = (4294967295.f - used) * (1.f / C::WSUB);
+          run = avail >= (float)C::RUN ? C::RUN : (avail >= 1.f ? (int)avail : 0);
+          if (run < 1 && i < nsub) {
+            fold(1.f);
+            run = C::RUN;
+          }
         }
+        pb ^= 1;
         if (i >= nsub) break;
-        if (n == 0u) fold(1.f);   // capacity (the barrier above ordered every reduction)
-        else __syncthreads();      // the cleared count is visible before the next run's appends
       }
       // ---- segment partial (every reduction has landed: the last run's barrier): the last fold
       // writes the float32 histograms [slot][Sv][256][GP] (relative to the reference) straight

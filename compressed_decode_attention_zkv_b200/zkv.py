@@ -28,6 +28,7 @@ ZKV_DEVERR_COMP_LEN = 1
 ZKV_DEVERR_WIN_LEN = 2
 ZKV_DEVERR_TIMEOUT = 4
 ZKV_DEVERR_PAGE = 8
+ZKV_DEVERR_SMEM = 16
 ZKV_DTYPE_F16, ZKV_DTYPE_F32 = 0, 1
 CODEBOOK_SIZE = 256
 DECODE_SCRATCH_BYTES = 8 << 20   # ZKV_DECODE_SCRATCH_BYTES: the no-allocation decode's array

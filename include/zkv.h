@@ -13,9 +13,11 @@
  *     of the compressed part with a dense recency window.
  *
  * Conventions shared by every entry point:
- *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates
- *     nothing and keeps no state between calls.  fp16 tensors are passed as uint16_t bit
- *     patterns (IEEE binary16).
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library allocates
+ *     nothing per call.  Its state between calls is the CUDA runtime's (loaded kernels and
+ *     their attributes) plus one fixed device array per device, the scratch workspace of
+ *     zkv_rvq_decode_attn_noalloc (below); every other call works only in the caller's
+ *     buffers.  fp16 tensors are passed as uint16_t bit patterns (IEEE binary16).
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
  *     default stream).  Argument validation is synchronous and happens before any launch; a
  *     failed validation returns an error and launches nothing.  A launch failure returns
@@ -242,7 +244,8 @@ int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace, size_t work
  *   - There is ONE array per device: calls on the same device that overlap in time (different
  *     streams or host threads) race on it and give wrong results.  Order them (same stream,
  *     or events).  Calls on different devices do not interact.
- *   - The first call on each device looks up the array's device address (once) and sets
+ *   - Every call looks up the array's device address on the host (so it stays right after a
+ *     device reset).  The first call on each device loads the library's device code and sets
  *     kernel attributes; make that first call before any stream capture.
  * Errors: as zkv_rvq_decode_attn; ZKV_ERR_CUDA if the array's address cannot be obtained.
  */

@@ -46,6 +46,24 @@ def test_status_strings_and_version(L):
     assert L.zkv_version() == int(re.search(r"#define ZKV_VERSION (\d+)", text).group(1))
 
 
+def _header_define(name):
+    """The value of an integer #define (a literal or a shift of two) or enumerator in
+    include/zkv.h."""
+    text = open(os.path.join(ROOT, "include", "zkv.h")).read()
+    m = (re.search(rf"#define {name}\s+\(?\s*(\w+)\s*(?:<<\s*(\w+))?\s*\)?", text)
+         or re.search(rf"\b{name}\s*=\s*(-?\w+)()", text))   # or an enumerator
+    assert m, f"{name} not defined"
+    lit = lambda t: int(t.rstrip("uUlL"), 0)
+    return lit(m.group(1)) << (lit(m.group(2)) if m.group(2) else 0)
+
+
+def test_binding_constants_match_the_header():
+    assert zkv.DECODE_SCRATCH_BYTES == _header_define("ZKV_DECODE_SCRATCH_BYTES")
+    for name in dir(zkv):
+        if re.fullmatch(r"ZKV_(ERR|DEVERR|DTYPE)_\w+|ZKV_OK", name):
+            assert getattr(zkv, name) == _header_define(name), name
+
+
 def test_fwht_validation(L):
     assert L.zkv_fwht(None, 0, None, -1, 128, 1.0, None) == zkv.ZKV_ERR_INVALID_ARG
     assert L.zkv_fwht(None, 7, None, 4, 128, 1.0, None) == zkv.ZKV_ERR_INVALID_ARG

@@ -110,5 +110,11 @@ def test_noalloc_refusal_raises_a_clear_error_on_device():
     cb = torch.zeros((Hkv, 4, 256, d), dtype=torch.float32, device="cuda")
     w = torch.zeros((64, Hkv, 16, d), dtype=torch.float16, device="cuda")
     n = torch.zeros(64, dtype=torch.int32, device="cuda")
+    out = torch.full((64, 32, d), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((64, 32), float("nan"), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
     with pytest.raises(zkv.ZkvError, match="scratch array holds"):
-        zkv.rvq_decode_attn_noalloc(q, kc, kc, n, cb, cb, w, w, n)
+        zkv.rvq_decode_attn_noalloc(q, kc, kc, n, cb, cb, w, w, n, out=out, lse=lse)
+    torch.cuda.synchronize()
+    # the refused call launched nothing: the caller's buffers are untouched
+    assert torch.isnan(out).all() and torch.isnan(lse).all()
