@@ -35,10 +35,11 @@ METRIC = "decode-attn compressed tokens/s/GPU & HBM GB/s (% roofline); encode ve
 UNIT = "compressed tokens/s"
 WORKLOAD = "llama3_8b_32k"
 
-# DRAM bytes (read + write) of one scan2_kernel launch on this workload, from one ncu capture
-# (profiles/), valid while the scan's source (csrc/scan_rvq.cuh) is unchanged; None until a
-# capture of the current source is recorded.
-SCAN_TRAFFIC = {"scan_src_sha1": None, "bytes_per_launch": None}
+# DRAM bytes (read + write) of one scan2_kernel launch on this workload, the mean of three
+# launches of one ncu capture (profiles/scan2_kernel_llama3_8b_32k.md), valid while the scan's
+# source (csrc/scan_rvq.cuh) is unchanged.
+SCAN_TRAFFIC = {"scan_src_sha1": "89fcf79a8d2ae0c750f4cf869685082b116e67fa",
+                "bytes_per_launch": 17825280}
 
 
 def parse():
