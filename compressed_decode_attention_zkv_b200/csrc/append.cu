@@ -17,8 +17,10 @@
 // within the margin of the global minimum, so the exact argmin is always among them.  Each CTA
 // publishes, per row, its best (float64 distance, index) and after one cluster barrier every
 // CTA reduces the 8 published bests the same way (decided in float64, ties to the lowest
-// index).  Every CTA keeps an identical copy of the residuals and reads the chosen codeword
-// from its owner's shared memory.
+// index).  Within a CTA, warp r decides row r with no block-wide step (lane = local codeword);
+// each CTA writes its per-row bests into every CTA of the cluster before the barrier, so the
+// reduction after it reads local shared memory.  Every CTA keeps an identical copy of the
+// residuals and reads the chosen codeword from its owner's shared memory.
 #include <cooperative_groups.h>
 
 #include "encode_rows.cuh"
@@ -41,14 +43,10 @@ struct AppendSmem {
   double rn[kAppendR];                        // residual norms
   float dist[kAppendCw][kAppendR];            // float32 distances of this CTA's codewords
   float cnorm[kAppendCw];                     // their squared norms
-  float lmin[kAppendR];                       // this CTA's per-row minima
-  float lcmax;                                // this CTA's largest codeword norm
-  int ncand;
-  uint16_t cand[kAppendCw * kAppendR];        // (local codeword << 3) | row
-  double cand_d[kAppendCw * kAppendR];        // their float64 distances
-  double best_d[2][kAppendR];                 // published per-row best, by stage parity
-  int best_c[2][kAppendR];
-  int zsel[kAppendR];
+  // every CTA's per-row best (float64 distance, codeword), written by that CTA into every
+  // CTA of the cluster; by stage parity
+  double pub_d[2][kAppendCl][kAppendR];
+  int pub_c[2][kAppendCl][kAppendR];
   uint8_t code[kAppendR][kMaxStages];
 };
 
@@ -179,97 +177,80 @@ __global__ void __cluster_dims__(kAppendCl, 1, 1) __launch_bounds__(256)
       }
     }
     __syncthreads();
-    if (tid < kAppendR) {
-      float v = sm.dist[0][tid];
-      for (int c = 1; c < kAppendCw; ++c) v = fminf(v, sm.dist[c][tid]);
-      sm.lmin[tid] = v;
-    } else if (tid == 32) {
-      float v = sm.cnorm[0];
-      for (int c = 1; c < kAppendCw; ++c) v = fmaxf(v, sm.cnorm[c]);
-      sm.lcmax = v;
-      sm.ncand = 0;
-    }
-    __syncthreads();
-    // local candidates: within the margin of this CTA's row minimum
-    {
-      const int c = tid >> 3, r = tid & 7;
-      if ((double)sm.dist[c][r] <= (double)sm.lmin[r] + candidate_margin(sm.rn[r], sm.lcmax, D)) {
-        const int k = atomicAdd(&sm.ncand, 1);
-        sm.cand[k] = (uint16_t)((c << 3) | r);
-      }
-    }
-    __syncthreads();
-    // exact float64 distance of each candidate, one warp per candidate
-    const int nc = sm.ncand;
-    for (int k = warp; k < nc; k += 8) {
-      const int c = sm.cand[k] >> 3, r = sm.cand[k] & 7;
-      double a = 0.0;
-#pragma unroll
-      for (int q = 0; q < E; ++q) {
-        const int i = q * 32 + lane;
-        const double df = (double)sm.rows[r * LD + i] - (double)slice[c * LD + i];
-        a = fma(df, df, a);
-      }
-      a = warp_sum_f64(a);
-      if (lane == 0) sm.cand_d[k] = a;
-    }
-    __syncthreads();
-    if (tid < kAppendR) {   // this CTA's best per row, published for the cluster
-      double d = DBL_MAX;
+    // warp r decides row r among this CTA's codewords (lane = local codeword): the row minimum
+    // of the float32 distances, the candidates within the margin (taken with this slice's
+    // largest codeword norm), their float64 distances, the best (lowest index on ties); it
+    // then writes that best into every CTA of the cluster
+    static_assert(kAppendCw == 32, "one lane per local codeword");
+    if (warp < kAppendR) {
+      const int r = warp;
+      const float dr = sm.dist[lane][r];
+      const float cmax = warp_max_f32(sm.cnorm[lane]);
+      const float dmin = warp_min_f32(dr);
+      const double thr = (double)dmin + candidate_margin(sm.rn[r], cmax, D);
+      unsigned cand = __ballot_sync(0xffffffffu, (double)dr <= thr);
+      double bd = DBL_MAX;
       int bc = kCodebook;
-      for (int k = 0; k < nc; ++k) {
-        if ((sm.cand[k] & 7) != tid) continue;
-        const int c = rank * kAppendCw + (sm.cand[k] >> 3);
-        const double dd = sm.cand_d[k];
-        if (dd < d || (dd == d && c < bc)) {
-          d = dd;
-          bc = c;
+      while (cand) {
+        const int c = __ffs(cand) - 1;
+        cand &= cand - 1u;
+        double a = 0.0;
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+          const int i = q * 32 + lane;
+          const double df = (double)sm.rows[r * LD + i] - (double)slice[c * LD + i];
+          a = fma(df, df, a);
+        }
+        a = warp_sum_f64(a);
+        const int gc = rank * kAppendCw + c;
+        if (a < bd || (a == bd && gc < bc)) {
+          bd = a;
+          bc = gc;
         }
       }
-      sm.best_d[s & 1][tid] = d;
-      sm.best_c[s & 1][tid] = bc;
+      if (lane < kAppendCl) {
+        AppendSmem<D>* o = cluster.map_shared_rank(&sm, lane);
+        o->pub_d[s & 1][rank][r] = bd;
+        o->pub_c[s & 1][rank][r] = bc;
+      }
     }
-    // every CTA's bests are visible; every read of stage s-1's slices and bests is done
+    // every CTA's bests have arrived here; every read of stage s-1's slices is done
     cluster.sync();
     // the buffer of stage s-1 is free (its remote reads are done): refill it NB - 1 stages ahead
     if (s + kAppendNB - 1 < S) load_slice(s + kAppendNB - 1);
-    if (tid < kAppendR) {
-      double d[kAppendCl];
-      int c[kAppendCl];
-#pragma unroll
-      for (int k = 0; k < kAppendCl; ++k) {
-        const AppendSmem<D>* o = cluster.map_shared_rank(&sm, k);
-        d[k] = o->best_d[s & 1][tid];
-        c[k] = o->best_c[s & 1][tid];
-      }
-      double bd2 = d[0];
-      int bc2 = c[0];
-#pragma unroll
-      for (int k = 1; k < kAppendCl; ++k)
-        if (d[k] < bd2 || (d[k] == bd2 && c[k] < bc2)) {
-          bd2 = d[k];
-          bc2 = c[k];
-        }
-      // non-finite rows match no candidate; never index past the stage's codebook
-      sm.zsel[tid] = bc2 < kCodebook ? bc2 : 0;
-    }
-    __syncthreads();
-    // residual update with the chosen codeword, read from its owner's slice
+    // warp r: the cluster's best for row r (min over the 8 published bests, lowest index on
+    // ties), then the residual update with that codeword, read from its owner's slice
     if (warp < kAppendR) {
-      const int z = sm.zsel[warp];
+      const int r = warp;
+      double bd = lane < kAppendCl ? sm.pub_d[s & 1][lane][r] : DBL_MAX;
+      int bc = lane < kAppendCl ? sm.pub_c[s & 1][lane][r] : kCodebook;
+#pragma unroll
+      for (int o = 1; o < kAppendCl; o <<= 1) {
+        const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+        const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+        if (od < bd || (od == bd && oc < bc)) {
+          bd = od;
+          bc = oc;
+        }
+      }
+      // every lane of the warp holds the same choice (lanes 0-7 reduced the same set; the
+      // others take lane 0's); non-finite rows match no candidate: never index past the
+      // stage's codebook
+      bc = __shfl_sync(0xffffffffu, bc, 0);
+      const int z = bc < kCodebook ? bc : 0;
       const float* src = cluster.map_shared_rank(&sm.cb[s % kAppendNB][0], z / kAppendCw) + (z % kAppendCw) * LD;
       double ss = 0.0;
 #pragma unroll
       for (int q = 0; q < E; ++q) {
         const int i = q * 32 + lane;
-        const float nr = sm.rows[warp * LD + i] - src[i];
-        sm.rows[warp * LD + i] = nr;
+        const float nr = sm.rows[r * LD + i] - src[i];
+        sm.rows[r * LD + i] = nr;
         ss += (double)nr * (double)nr;
       }
       ss = warp_sum_f64(ss);
       if (lane == 0) {
-        sm.rn[warp] = sqrt(ss);
-        sm.code[warp][s] = (uint8_t)z;
+        sm.rn[r] = sqrt(ss);
+        sm.code[r][s] = (uint8_t)z;
       }
     }
   }
