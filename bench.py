@@ -518,7 +518,7 @@ def ragged_extra(dev, hbm_peak, R=4, steps=100):
     wl = I.workload("ragged_serving_64")
     lens = I.ragged_lengths(wl)
     comp = (lens - wl.W).astype(np.int64)
-    grow = (3 + steps + R - 1) // R + 2
+    grow = (3 + steps + 2 * R + R - 1) // R + 2
     Tcap = int((comp.max() + grow + 15) // 16 * 16)
     kc = torch.from_numpy(I.random_codes(wl, "k", Tcap)).to(dev)
     vc = torch.from_numpy(I.random_codes(wl, "v", Tcap, seed=1)).to(dev)
@@ -548,6 +548,9 @@ def ragged_extra(dev, hbm_peak, R=4, steps=100):
                                      max_comp_len=max_comp)
     wss = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(R)]
     host_comp = [int(comp.sum())] * R   # compressed tokens of all sequences, per replica
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(R)]
+    for ev in (ev for row in evs for ev in row):   # torch times only events it saw recorded
+        ev.record()
     for r in range(R):   # eager call per replica (kernel attributes before capture)
         step_fn(reps[r], wss[r], max_comp)
         host_comp[r] += wl.B
@@ -575,6 +578,30 @@ def ragged_extra(dev, hbm_peak, R=4, steps=100):
     sec = s.elapsed_time(e) / 1000.0
     assert sum(int(rep["err"].item()) for rep in reps) == 0
     del graphs
+    # per-kernel times: graphs with event nodes between the kernels, 2 rounds over the replicas
+    # (each replay appends a token to every sequence of its replica; the prefixes have room)
+    spans = None
+    try:
+        tg = []
+        for r in range(R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step_fn(reps[r], wss[r], max_comp, events=evs[r])
+            tg.append(g)
+        acc = [[], [], []]
+        for _ in range(2):
+            for r in range(R):
+                tg[r].replay()
+            torch.cuda.synchronize()
+            for r in range(R):
+                for i in range(3):
+                    acc[i].append(evs[r][i].elapsed_time(evs[r][i + 1]) * 1e3)
+        del tg
+        spans = {"tables+window+partition+append": statistics.mean(acc[0]),
+                 "scan": statistics.mean(acc[1]), "combine": statistics.mean(acc[2]),
+                 "unit": "us", "timing": "event nodes between the kernels (no overlap there)"}
+    except Exception as exc:
+        spans = {"error": f"{type(exc).__name__}: {exc}"}
     step_s = sec / steps
     tc_avg = tokens / steps
     byts = (tc_avg * wl.Hkv * (wl.Sk + wl.Sv) + wl.B * wl.Hkv * wl.W * wl.d * 2 * 2
@@ -584,6 +611,7 @@ def ragged_extra(dev, hbm_peak, R=4, steps=100):
                         "Hkv 8, d 128, Sk = Sv = 4, W 128)",
             "value": tokens / sec, "unit": UNIT, "ms_per_step": 1000.0 * step_s,
             "seq_tokens_per_s": wl.B / step_s, "compressed_tokens_per_step": tc_avg,
+            "kernels_us": spans,
             "step_gbs": byts / step_s / 1e9, "step_frac": byts / step_s / 1e9 / hbm_peak,
             "steps": steps,
             "note": f"one zkv_rvq_serve_step per step; graphs over {R} rotating replicas x "
