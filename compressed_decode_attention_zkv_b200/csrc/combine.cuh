@@ -174,13 +174,27 @@ __global__ void __launch_bounds__(256, 4) combine_kernel(DecodeArgs a) {
     l = warp_sum_f32(l);
     if (lane == 0) Ls[warp] = l;
   }
-  // the window partial of warp g's head, loaded beside the partial outputs
+  // the window partial of warp g's head: its parts merged by their maxima (log-sum-exp),
+  // loaded beside the partial outputs
   float wmg = -INFINITY, wlg = 0.f, wog[E];
-  if (warp < a.G) {
-    wmg = a.wm[pair * GP + warp];
-    wlg = a.wl[pair * GP + warp];
 #pragma unroll
-    for (int q = 0; q < E; ++q) wog[q] = a.wo[(pair * GP + warp) * D + q * 32 + lane];
+  for (int q = 0; q < E; ++q) wog[q] = 0.f;
+  if (warp < a.G) {
+    for (int pt = 0; pt < a.wparts; ++pt) {
+      const int64_t wi = (pair * a.wparts + pt) * GP + warp;
+      const float mp = a.wm[wi], lp = a.wl[wi];
+      float op[E];
+#pragma unroll
+      for (int q = 0; q < E; ++q) op[q] = a.wo[wi * D + q * 32 + lane];
+      const float mn = fmaxf(wmg, mp);
+      if (mn == -INFINITY) continue;   // both empty so far
+      const float s0 = wmg == -INFINITY ? 0.f : ex2_approx(wmg - mn);
+      const float s1 = mp == -INFINITY ? 0.f : ex2_approx(mp - mn);
+      wlg = wlg * s0 + lp * s1;
+#pragma unroll
+      for (int q = 0; q < E; ++q) wog[q] = wog[q] * s0 + op[q] * s1;
+      wmg = mn;
+    }
   }
   // the sum of the stage / chunk partial outputs (rotated domain, unnormalised): piece f4 of
   // the parts p2, p2 + P2, ... in slice p2, then the slices in order

@@ -68,6 +68,8 @@ constexpr size_t kS2Smem = (size_t(3) << 16) + 32768;   // dynamic shared memory
 // fold and write: about 8K cycles measured) in tokens of the loop (about 1.3 cycles per token
 // and SM).
 constexpr int64_t kS2SegCost = 6000;
+// tokens of one window part in the decode's table kernel (its K + V tile is 32 KB)
+inline int win_tile_part(int d) { return 8192 / d; }
 
 
 static int sm_count() {
@@ -108,7 +110,7 @@ struct DecodePlan {
   size_t scan_smem;
   size_t off_lut, off_pre, off_bounds, off_ctap, off_vs, off_pfirst, off_plast, off_pm, off_pl, off_pw,
       off_wm, off_wl, off_wo, off_so, off_cnt, total;
-  int qc;
+  int qc, wparts, wtok;
 };
 
 static size_t scan_smem_bytes(int Rk, int Sk, int Sv, int GP, const VMap& v) {
@@ -168,9 +170,12 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
   pl.off_pm = o;    o = align256(o + (size_t)pl.slots * pl.GP * f);
   pl.off_pl = o;    o = align256(o + (size_t)pl.slots * pl.GP * f);
   pl.off_pw = o;    o = align256(o + (size_t)pl.slots * p->Sv * kCodebook * pl.GP * f);
-  pl.off_wm = o;    o = align256(o + (size_t)pairs * pl.GP * f);
-  pl.off_wl = o;    o = align256(o + (size_t)pairs * pl.GP * f);
-  pl.off_wo = o;    o = align256(o + (size_t)pairs * pl.GP * p->d * f);
+  // the window in parts of one tile each, one table-kernel block per (pair, part)
+  pl.wtok = win_tile_part(p->d);
+  pl.wparts = (int)std::max<int64_t>(1, (p->Wcap + pl.wtok - 1) / pl.wtok);
+  pl.off_wm = o;    o = align256(o + (size_t)pairs * pl.wparts * pl.GP * f);
+  pl.off_wl = o;    o = align256(o + (size_t)pairs * pl.wparts * pl.GP * f);
+  pl.off_wo = o;    o = align256(o + (size_t)pairs * pl.wparts * pl.GP * p->d * f);
   // combine blocks: (pair, value stage, chunk of 256 / qc codewords); a chunk's codewords take
   // at most 32 KB of shared memory, and small problems take more chunks (up to 16 or the
   // 32 KB minimum) so that the grid covers the SMs
@@ -229,9 +234,10 @@ struct DecodeArgs {
   float* pm;         // [slots][GP] segment maxima
   float* pl;         // [slots][GP] segment sums of p
   float* pw;         // [slots][Sv][256][GP] segment histograms
-  float* wm;         // [B*Hkv][GP]
-  float* wl;         // [B*Hkv][GP]
-  float* wo;         // [B*Hkv][GP][d]
+  int wparts, wtok;  // window parts per pair, tokens per part (the part is one tile)
+  float* wm;         // [B*Hkv][wparts][GP]
+  float* wl;         // [B*Hkv][wparts][GP]
+  float* wo;         // [B*Hkv][wparts][GP][d]
   float* so;         // [B*Hkv][Sv][qc][GP][d] partial stage outputs
   int32_t* cnt;      // [B*Hkv] finished combine blocks of each pair (zeroed by the table kernel)
 };
@@ -280,7 +286,7 @@ __device__ __forceinline__ void prefetch_l2(const uint8_t* lo, const uint8_t* hi
 template <int D>
 constexpr int win_tile() { return 16384 / D; }   // tokens per tile: K + V tiles = 64 KB
 template <int D>
-constexpr int win_tile_small() { return 4096 / D; }   // K + V tiles = 16 KB
+constexpr int win_tile_part_c() { return 8192 / D; }
 
 // the warps' partial outputs [8][GP][D] reuse the tiles when they fit there
 template <int D, int GP, int WT>
@@ -292,8 +298,10 @@ constexpr size_t window_smem_bytes() {
          (win_part_in_tiles<D, GP, WT>() ? 0 : (size_t)8 * GP * D * 4);
 }
 
+// Part wpart of the window: rows [wpart wtok, (wpart + 1) wtok) of its wl rows; the partial
+// (maximum, sum, unnormalised output) goes to slot wpart of the pair's window partials.
 template <int D, int GP, int WT = win_tile<D>()>
-__device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* smem) {
+__device__ void window_item(const DecodeArgs& a, int b, int kvh, int wpart, unsigned char* smem) {
   constexpr int PL = D / 32;        // head dims per lane
   __half* kt = reinterpret_cast<__half*>(smem);                     // [WT][D]
   __half* vt = kt + WT * D;                                         // [WT][D]
@@ -321,10 +329,13 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
   } else {
     wl = clamp_win_len(a, b);
   }
+  // this part's rows
+  const int64_t t0 = (int64_t)wpart * a.wtok;
+  const int64_t t1 = wl < t0 + a.wtok ? wl : t0 + a.wtok;
   const __half* Kb = a.win_k + pair * a.Wcap * D;
   const __half* Vb = a.win_v + pair * a.Wcap * D;
   auto stage = [&](int64_t base) {   // rows [base, base + n) as 16-byte pieces
-    const int n = (int)(wl - base < WT ? wl - base : WT);
+    const int n = (int)(t1 - base < WT ? t1 - base : WT);
     for (int f = tid; f < n * D / 8; f += 256) {
       if (base + f / (D / 8) == sub) continue;
       cp_async16(kt + f * 8, Kb + base * D + f * 8);
@@ -338,7 +349,7 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
       }
     }
   };
-  if (wl > 0) stage(0);   // in flight while the query is loaded
+  if (t1 > t0) stage(t0);   // in flight while the query is loaded
   float qf[GP][PL];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
@@ -355,9 +366,9 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
 #pragma unroll
     for (int e = 0; e < PL; ++e) acc[g][e] = 0.f;
   }
-  for (int64_t base = 0; base < wl; base += WT) {
-    const int n = (int)(wl - base < WT ? wl - base : WT);
-    if (base > 0) stage(base);
+  for (int64_t base = t0; base < t1; base += WT) {
+    const int n = (int)(t1 - base < WT ? t1 - base : WT);
+    if (base > t0) stage(base);
     cp_async_wait_all();
     __syncthreads();
     // scores
@@ -450,14 +461,14 @@ __device__ void window_item(const DecodeArgs& a, int b, int kvh, unsigned char* 
 #pragma unroll
     for (int g = 0; g < GP; ++g)
       if (g == tid) mr = m_run[g];
-    a.wm[pair * GP + tid] = mr;
-    a.wl[pair * GP + tid] = l;
+    a.wm[(pair * a.wparts + wpart) * GP + tid] = mr;
+    a.wl[(pair * a.wparts + wpart) * GP + tid] = l;
   }
   for (int f = tid; f < GP * D; f += 256) {
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += part[w * GP * D + f];
-    a.wo[pair * GP * D + f] = v;
+    a.wo[(pair * a.wparts + wpart) * GP * D + f] = v;
   }
 }
 
@@ -602,8 +613,12 @@ __global__ void __launch_bounds__(256, GP >= 8 ? 2 : 3) lut_kernel(DecodeArgs a)
     // dense attention over the fp16 window of one (sequence, kv head): it reads only the call's
     // inputs (in the serving step it substitutes the new token for the slot the append gives
     // it), so it runs here, beside the tables
-    const int pair = (int)blockIdx.x - a.n_lut_blocks - 1;
-    window_item<D, GP>(a, pair / a.Hkv, pair % a.Hkv, smem_raw);
+    const int w = (int)blockIdx.x - a.n_lut_blocks - 1;   // (pair, part), part fastest
+    const int pair = w / a.wparts;
+    if (a.wparts == 1)   // the whole window in one block (64 KB tiles)
+      window_item<D, GP>(a, pair / a.Hkv, pair % a.Hkv, 0, smem_raw);
+    else                 // one tile-sized part per block
+      window_item<D, GP, win_tile_part_c<D>()>(a, pair / a.Hkv, pair % a.Hkv, w % a.wparts, smem_raw);
     return;
   }
   if ((int)blockIdx.x < a.Hkv * a.Sv && tid == 0) {
@@ -1499,7 +1514,7 @@ __global__ void __launch_bounds__(256) pq_finalize_kernel(PqArgs a, DecodeArgs w
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pair = blockIdx.x;
   const int b = (int)(pair / a.Hkv), kvh = (int)(pair % a.Hkv);
-  window_item<D, GP>(w, b, kvh, win_smem);
+  window_item<D, GP>(w, b, kvh, 0, win_smem);
   if (tid == 0) {
     const int64_t c = a.comp_len[b];
     if (c < 0 || c > a.Tcap) set_error(a.err, ZKV_DEVERR_COMP_LEN);
@@ -1628,12 +1643,21 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
   // 1. tables and partition (with the serving step's encode in between)
   trace(ev, 0, st);
   {
-    const size_t smem = std::max(sizeof(LutSmem<D>), window_smem_bytes<D, GP>());
+    // a decode call splits each pair's window into tile-sized parts (more, shorter blocks: the
+    // scan waits for this kernel); the serving step keeps one block per pair (this kernel runs
+    // beside the append, whose clusters need the SMs more)
+    if (ap) {
+      a.wparts = 1;
+      a.wtok = (int)std::min<int64_t>(a.Wcap, 0x7fffffff);
+    }
+    const size_t smem = std::max(sizeof(LutSmem<D>), a.wparts == 1
+                                                         ? window_smem_bytes<D, GP>()
+                                                         : window_smem_bytes<D, GP, win_tile_part_c<D>()>());
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
     a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
-    // + the partition block + one window block per (sequence, kv head)
-    const int64_t blocks = (int64_t)a.n_lut_blocks + 1 + (int64_t)a.B * a.Hkv;
+    // + the partition block + one window block per (sequence, kv head, window part)
+    const int64_t blocks = (int64_t)a.n_lut_blocks + 1 + (int64_t)a.B * a.Hkv * a.wparts;
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
     // a normal launch: the caller's preceding work (which may write q) must be complete, since
     // the table blocks do not wait
@@ -1770,6 +1794,8 @@ static int decode_common(const zkv_decode_params* p, void* workspace, size_t wor
   a.wm = reinterpret_cast<float*>(ws + pl.off_wm);
   a.wl = reinterpret_cast<float*>(ws + pl.off_wl);
   a.wo = reinterpret_cast<float*>(ws + pl.off_wo);
+  a.wparts = pl.wparts;
+  a.wtok = pl.wtok;
   a.so = reinterpret_cast<float*>(ws + pl.off_so);
   a.cnt = reinterpret_cast<int32_t*>(ws + pl.off_cnt);
   a.qc = pl.qc;
@@ -1927,6 +1953,8 @@ extern "C" int zkv_pq_decode_attn(const zkv_pq_decode_params* p, void* workspace
   w.wm = reinterpret_cast<float*>(ws + pl.off_wm);
   w.wl = reinterpret_cast<float*>(ws + pl.off_wl);
   w.wo = reinterpret_cast<float*>(ws + pl.off_wo);
+  w.wparts = 1;                                 // one part: the whole window, tile by tile
+  w.wtok = (int)std::min<int64_t>(p->Wcap, 0x7fffffff);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (p->d * 100 + p->m) {   // the shapes validate_pq_shapes admits
     case 6402: return launch_pq_g<64, 2>(pl.GP, a, w, st);
