@@ -192,6 +192,7 @@ static DecodePlan make_plan(const zkv_decode_params* p) {
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, GP, d, Sk, Sv, Rk, grid, n_lut_blocks;
+  int lut_cpt;        // codewords per table-kernel thread (1 or lut_cpt<D>())
   int64_t seg_cost;   // set-up cost of one scan segment, in tokens (partition weight)
   int qc;             // codeword chunks per value stage in the combine kernel
   // Serving step: the partition uses the lengths after this step's append (predicted from
@@ -255,13 +256,19 @@ __device__ __forceinline__ int64_t clamp_win_len(const DecodeArgs& a, int b) {
 // 1. Query rotation + lookup tables; length prefix sums (the partition block); the dense
 //    window attention (window_item), one block per pair.
 // ------------------------------------------------------------------------------------------
-constexpr int kLutC = 64;     // codewords per table block (one per thread and head quad)
 constexpr int kLutH = 16;     // attached query heads per table block (b * G + g)
+// codewords per table block: 64 per group of 4 heads' threads, and each thread takes lut_cpt of
+// them (two up to d = 128: six 16-byte shared loads per 32 FMAs; one at d = 256, where a
+// 128-codeword slice would leave one block per SM)
+template <int D>
+constexpr int lut_cpt() { return D >= 256 ? 1 : 2; }
+template <int D>
+constexpr int lut_c() { return 64 * lut_cpt<D>(); }
 
 template <int D>
 struct LutSmem {
   float qT[D][kLutH + 4];     // rotated queries, k-major
-  float cb[kLutC * D];        // codebook slice, row-major; 16-byte piece q of codeword c at q ^ (c & 7)
+  float cb[lut_c<D>() * D];   // codebook slice, row-major; 16-byte piece q of codeword c at q ^ (c & 7)
 };
 
 // Ask the memory system to stage [p, p + bytes) in L2 (no data returned to the SM).  p and
@@ -595,9 +602,10 @@ __device__ void partition_block(const DecodeArgs& a) {
   }
 }
 
-// Table blocks: block = (64-codeword slice, key stage, group of 16 attached query heads, kv
-// head); thread (codeword cc, head quad hq) forms 4 dot products.  Block n_lut_blocks is the
-// partition block.
+// Table blocks: block = (slice of lut_c codewords, key stage, group of 16 attached query heads,
+// kv head); thread (codewords cc + 64 u, head quad hq) forms 4 lut_cpt dot products.  Block
+// n_lut_blocks is the partition block; the blocks after it are the window blocks (one per pair
+// and window part).
 template <int D, int GP>
 __global__ void __launch_bounds__(256, GP >= 8 ? 2 : 3) lut_kernel(DecodeArgs a) {
   constexpr int E = D / 32;
@@ -631,17 +639,19 @@ __global__ void __launch_bounds__(256, GP >= 8 ? 2 : 3) lut_kernel(DecodeArgs a)
   LutSmem<D>& sm = *reinterpret_cast<LutSmem<D>*>(smem_raw);
   const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
   int rest = blockIdx.x;
-  const int cblk = rest % (kCodebook / kLutC);
-  rest /= kCodebook / kLutC;
+  constexpr int CPT = lut_cpt<D>();
+  const int cpt = a.lut_cpt, LC = 64 * cpt;
+  const int cblk = rest % (kCodebook / LC);
+  rest /= kCodebook / LC;
   const int s = rest % a.Sk;
   rest /= a.Sk;
   const int hg = rest % n_hg;
   const int kvh = rest / n_hg;
-  const int c0 = cblk * kLutC;
-  // codebook slice C[kvh][s][c0 .. c0 + kLutC)[:] -> shared memory, in flight during the rotation
+  const int c0 = cblk * LC;
+  // codebook slice C[kvh][s][c0 .. c0 + LC)[:] -> shared memory, in flight during the rotation
   {
     const float* C = a.Ck + (((size_t)kvh * a.Sk + s) * kCodebook + c0) * D;
-    for (int f = tid; f < kLutC * D / 4; f += 256) {
+    for (int f = tid; f < LC * D / 4; f += 256) {
       const int c = f / (D / 4), qq = f % (D / 4);
       cp_async16(sm.cb + c * D + 4 * (qq ^ (c & 7)), C + (size_t)c * D + 4 * qq);
     }
@@ -680,34 +690,53 @@ __global__ void __launch_bounds__(256, GP >= 8 ? 2 : 3) lut_kernel(DecodeArgs a)
   }
   cp_async_wait_all();
   __syncthreads();
-  // thread (codeword cc, heads 4 hq .. 4 hq + 3): the codeword is read as 16-byte pieces
-  // (conflict-free thanks to the swizzle), the query columns are broadcasts
-  const int cc = tid & (kLutC - 1), hq = tid / kLutC;
-  const float* row = sm.cb + cc * D;
+  // thread (codewords cc + 64 u for u < CPT, heads 4 hq .. 4 hq + 3): each codeword is read as
+  // 16-byte pieces (conflict-free thanks to the swizzle; cc + 64 u has the swizzle of cc), the
+  // query columns are broadcasts shared by the thread's codewords; every dot product is
+  // accumulated in the same order whatever CPT is
+  const int cc = tid & 63, hq = tid / 64;
   const int sw = cc & 7;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  auto dots = [&](auto nu_c) {   // nu codewords per thread (a compile-time count)
+    constexpr int NU = decltype(nu_c)::value;
+    float acc[NU][4];
+#pragma unroll
+    for (int u = 0; u < NU; ++u)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[u][k] = 0.f;
 #pragma unroll 4
-  for (int qq = 0; qq < D / 4; ++qq) {
-    const float4 c4 = *reinterpret_cast<const float4*>(row + 4 * (qq ^ sw));
-    const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+    for (int qq = 0; qq < D / 4; ++qq) {
+      float cv[NU][4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 q4 = *reinterpret_cast<const float4*>(&sm.qT[4 * qq + e][hq * 4]);
-      acc[0] = fmaf(q4.x, cv[e], acc[0]);
-      acc[1] = fmaf(q4.y, cv[e], acc[1]);
-      acc[2] = fmaf(q4.z, cv[e], acc[2]);
-      acc[3] = fmaf(q4.w, cv[e], acc[3]);
-    }
-  }
+      for (int u = 0; u < NU; ++u) {
+        const float4 c4 = *reinterpret_cast<const float4*>(sm.cb + (cc + 64 * u) * D + 4 * (qq ^ sw));
+        cv[u][0] = c4.x; cv[u][1] = c4.y; cv[u][2] = c4.z; cv[u][3] = c4.w;
+      }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int j = hg * kLutH + hq * 4 + k;
-    if (j < a.B * a.G) {
-      const int b = j / a.G, g = j % a.G;
-      a.lut[((((int64_t)b * a.Hkv + kvh) * a.Sk + s) * kCodebook + c0 + cc) * GP + g] =
-          acc[k] * a.scale_log2;
+      for (int e = 0; e < 4; ++e) {
+        const float4 q4 = *reinterpret_cast<const float4*>(&sm.qT[4 * qq + e][hq * 4]);
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          acc[u][0] = fmaf(q4.x, cv[u][e], acc[u][0]);
+          acc[u][1] = fmaf(q4.y, cv[u][e], acc[u][1]);
+          acc[u][2] = fmaf(q4.z, cv[u][e], acc[u][2]);
+          acc[u][3] = fmaf(q4.w, cv[u][e], acc[u][3]);
+        }
+      }
     }
-  }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = hg * kLutH + hq * 4 + k;
+      if (j < a.B * a.G) {
+        const int b = j / a.G, g = j % a.G;
+#pragma unroll
+        for (int u = 0; u < NU; ++u)
+          a.lut[((((int64_t)b * a.Hkv + kvh) * a.Sk + s) * kCodebook + c0 + cc + 64 * u) * GP + g] =
+              acc[u][k] * a.scale_log2;
+      }
+    }
+  };
+  if (CPT > 1 && cpt > 1) dots(std::integral_constant<int, CPT>{});
+  else dots(std::integral_constant<int, 1>{});
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1655,7 +1684,10 @@ static int launch_decode(DecodeArgs a, const DecodePlan& pl, void* const* ev, cu
                                                          : window_smem_bytes<D, GP, win_tile_part_c<D>()>());
     if (ensure_smem_limit(lut_kernel<D, GP>, smem) != cudaSuccess) return ZKV_ERR_CUDA;
     const int n_hg = (a.B * a.G + kLutH - 1) / kLutH;
-    a.n_lut_blocks = (kCodebook / kLutC) * a.Sk * a.Hkv * n_hg;
+    // two codewords per thread when that still leaves at least 64 table blocks (fewer, longer
+    // blocks cost more than they save on small problems)
+    a.lut_cpt = lut_cpt<D>() > 1 && (kCodebook / lut_c<D>()) * a.Sk * a.Hkv * n_hg >= 64 ? lut_cpt<D>() : 1;
+    a.n_lut_blocks = (kCodebook / (64 * a.lut_cpt)) * a.Sk * a.Hkv * n_hg;
     // + the partition block + one window block per (sequence, kv head, window part)
     const int64_t blocks = (int64_t)a.n_lut_blocks + 1 + (int64_t)a.B * a.Hkv * a.wparts;
     if (blocks > 0x7fffffff) return ZKV_ERR_UNSUPPORTED;
