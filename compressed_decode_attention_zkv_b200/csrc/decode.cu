@@ -11,8 +11,10 @@
 //   1. lut_kernel    q_tilde = H q / sqrt(d) (float32 transform), per stage
 //                    LUT_s[c] = (scale * log2 e) * q_tilde . Ck_s[c] -> workspace; one block
 //                    computes the prefix sums of the compressed lengths that partition the token
-//                    space among scan CTAs; one block per (sequence, kv head) takes the dense
-//                    attention over its fp16 window (partial maximum, sum and output).
+//                    space among scan CTAs; one block per (sequence, kv head) and window part
+//                    (64-token parts in a decode call, the whole window in the serving step)
+//                    takes the dense attention over its fp16 window rows (partial maximum, sum
+//                    and output).
 //   2. scan          one CTA per SM walks a contiguous range of the concatenated compressed
 //                    tokens of all (sequence, kv head) pairs.  Per pair segment it takes
 //                    score_t = sum_s LUT_s[zk_{t,s}] (base-2 logits) against a reference maximum
@@ -24,7 +26,7 @@
 //   3. combine_kernel (combine.cuh)  per (pair, value stage, codeword chunk): merges the segment
 //                    histograms by their maxima and contracts W_s with its Cv_s codewords; the
 //                    block that completes a pair sums the stage outputs, rotates back, and merges
-//                    with the window partial by log-sum-exp.
+//                    with the window parts by log-sum-exp.
 //
 // Shared-memory design of scan_kernel (shared memory bandwidth, not HBM, bounds this kernel):
 //  * key tables are replicated per lane group so that the 8 (or 16, 32) lanes of a 128-bit

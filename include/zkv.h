@@ -238,8 +238,8 @@ int zkv_rvq_decode_attn(const zkv_decode_params* p, void* workspace, size_t work
  * bytes (one per device, allocated when the library's device code is loaded; nothing is
  * allocated or freed by the call).
  *   - A call whose zkv_decode_workspace_size(p) exceeds ZKV_DECODE_SCRATCH_BYTES returns
- *     ZKV_ERR_WORKSPACE and launches nothing (8 x 32K-token GQA batches need about 6.5 MiB;
- *     64 sequences x 16K tokens need about 42 MiB and are refused).
+ *     ZKV_ERR_WORKSPACE and launches nothing (8 x 32K-token GQA batches need about 6.6 MiB;
+ *     64 sequences x 16K tokens need about 36 MiB and are refused).
  *   - Nothing in the array must start at zero: each call writes every word it reads.
  *   - There is ONE array per device: calls on the same device that overlap in time (different
  *     streams or host threads) race on it and give wrong results.  Order them (same stream,

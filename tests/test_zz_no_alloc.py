@@ -50,7 +50,7 @@ def _params(**kw):
 def test_noalloc_refuses_shapes_beyond_the_scratch_array():
     B.build()
     L = zkv.lib()
-    # 64 sequences x 16K tokens (the ragged serving batch) need ~42 MiB of workspace
+    # 64 sequences x 16K tokens (the ragged serving batch) need ~36 MiB of workspace
     p = _params(B=64, Tcap=16384, max_comp_len=16384)
     assert L.zkv_decode_workspace_size(ctypes.byref(p)) > zkv.DECODE_SCRATCH_BYTES
     assert L.zkv_rvq_decode_attn_noalloc(ctypes.byref(p), None) == zkv.ZKV_ERR_WORKSPACE
