@@ -298,9 +298,11 @@ int zkv_rvq_append(const zkv_append_params* p, void* stream);
  * Passages: VeloxQuant "Quick start" (cache.append(k, v), then cache.attend(q)); VQKV section
  * 2.3 "Local Sliding Window" and "Decoding Stage".
  * Results are identical to the two calls made in that order.  The library overlaps the
- * decode's lookup-table construction (which needs only q and the key codebooks) and its
- * partition of the token space (computed from the lengths the append will produce) with the
- * encode of the evicted tokens; the new lengths are stored by the decode's scan kernel.
+ * decode's lookup-table construction (which needs only q and the key codebooks), its partition
+ * of the token space (computed from the lengths the append will produce) and its window
+ * attention (over the window the append will produce: the pre-step rows with the new token in
+ * the slot the append gives it) with the encode of the evicted tokens; the new lengths are
+ * stored by the decode's scan kernel.
  * ap and dp describe one cache: B, Hkv, d, Sk, Sv, Tcap and Wcap must be equal, and so must
  * k_codes, v_codes, k_codebooks, v_codebooks, win_k, win_v, win_len, comp_len, k_smooth and the
  * paged layout (block_table, page_tokens, max_pages, n_pages) (else
