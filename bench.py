@@ -38,7 +38,7 @@ WORKLOAD = "llama3_8b_32k"
 # DRAM bytes (read + write) of one scan2_kernel launch on this workload, the mean of three
 # launches of one ncu capture (profiles/scan2_kernel_llama3_8b_32k.md), valid while the scan's
 # source (csrc/scan_rvq.cuh) is unchanged.
-SCAN_TRAFFIC = {"scan_src_sha1": "89fcf79a8d2ae0c750f4cf869685082b116e67fa",
+SCAN_TRAFFIC = {"scan_src_sha1": "3d61919446712b2c54318221c11f4e278f9964f3",
                 "bytes_per_launch": 17825280}
 
 

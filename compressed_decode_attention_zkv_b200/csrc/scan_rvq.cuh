@@ -5,21 +5,24 @@
 // VeloxQuant-MLX 0.5.1, "VecInfer": the rotation is absorbed into the query, so a key score is
 // a sum of per-stage table entries (q_tilde . Ck_s[z_s]).
 //
-// Every thread takes groups of four consecutive tokens of one (sequence, kv head) segment end to
-// end: the key score of each token for up to four query heads (one table gather per key stage),
-// p = 2^(score - reference) for those heads, and the value side as per-codeword weight histograms
-// W_s[c] += p (one shared-memory integer reduction per value stage and head).  No token is staged
-// through shared memory and no warp waits for another between tokens; the only block-wide
-// steps are one barrier per sub-chunk of 2048 tokens and the rare growth of the reference.
+// Every thread takes groups of U consecutive tokens (U = 2 at four heads with packed codes of at
+// least two bytes, else 4) of one (sequence, kv head) segment end to end: the key score of each
+// token for up to four query heads (one table gather per key stage), p = 2^(score - reference)
+// for those heads, and the value side as per-codeword weight histograms W_s[c] += p (one
+// shared-memory integer reduction per value stage and head).  No token is staged through shared
+// memory and no warp waits for another between tokens: sub-chunks of 512 U tokens run in
+// barrier-free runs, and the block meets only between runs.
 //
 // Shared memory (absolute addresses of the CTA's window; dynamic shared memory begins at 1 KB,
-// after the reserved system area, and this kernel asks for everything below 192 KB):
-//   [base, 64K)   block scratch (maxima, sums)
+// after the reserved system area, and this kernel asks for everything below 224 KB):
+//   [base, 64K)   block scratch: maxima, sums, float32 master histograms, the list of tokens
+//                 above the reference (their key code words), its counts, the warps' p sums
 //   [64K, 128K)   key tables: 256 rows (codewords) of 256 bytes; row c holds, for every key
 //                 stage s and table copy k, the GPH float32 entries of codeword c, stored with
 //                 the heads rotated by k mod GPH.  Entry (c, s, k) sits at 64K + 256 c +
 //                 (s RK + k) 4 GPH.
 //   [128K, 192K)  value histograms: 256 rows of 64 uint32 words; word 8/GPH... see below.
+//   [192K, 224K)  the listed tokens' value code words
 // Because every row is 256 bytes and each region starts at a multiple of 64 KB, the address
 // of a table entry is one byte permutation: [column byte | code byte | region | 0] -- the code
 // byte comes straight from the token's packed codes, the other bytes from a per-lane register.
@@ -46,14 +49,16 @@
 // each run boundary the block knows that bound and shortens the next run, or folds, when the
 // bound plus the next run's worst case would pass 2^32.
 
-// Reference: the first sub-chunk's block maximum plus 1 (log2 units).  Sub-chunks take block i of every warp's
-// contiguous run of the segment, so that first sub-chunk samples the whole segment.  A later
-// score above the reference (the interval barrier ORs a per-thread check) makes the block take
-// that sub-chunk's maximum, fold the integer words into the masters rescaled by 2^(old - new),
-// and continue with the new reference.
+// Reference: the first sub-chunk's block maximum plus a headroom (kS2Headroom, log2 units).
+// Sub-chunks take block i of every warp's contiguous run of the segment, so that first sub-chunk
+// samples the whole segment.  A later token whose score is above the reference is listed (its
+// code words copied from the registers that hold them) and contributes nothing during its run;
+// at the run's end the block takes the listed tokens' maximum plus the headroom as the new
+// reference, folds the integer words into the masters rescaled by 2^(old - new), and adds the
+// listed tokens.
 //
 // Output (one slot per (scan CTA, pair)): maxima pm = the reference (log2 units), sums pl, and
-// float32 histograms pw[slot][Sv][256][GP] relative to pm -- the partial format the merge
+// float32 histograms pw[slot][Sv][256][GP] relative to pm -- the partial format the combine
 // kernel reads.  Query-head groups larger than four are taken in passes of four heads over the
 // same segment.
 #pragma once
