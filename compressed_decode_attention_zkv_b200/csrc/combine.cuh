@@ -20,9 +20,11 @@
 //   4. an atomic counter per pair: the block that completes the pair (the last of its blocks)
 //      sums the partial outputs (float4 loads, parts split over thread slices and added in a
 //      fixed order), rotates them back (H / sqrt(d), float64 transform rounded once), and
-//      merges with the window partial by log-sum-exp.  No block waits for another.
+//      merges with the window by log-sum-exp (the window's parts merged first, by their
+//      maxima).  No block waits for another.
 // The window partials come from the table kernel (complete before the scan's, and so before
-// this kernel's, wait returns).
+// this kernel's, wait returns).  Each thread's first eight slot values of step 2 and the
+// finishing block's window parts are loaded beside the values they are combined with.
 #pragma once
 
 constexpr int kCombineFin = 1024;   // floats of the finishing block's slice buffer
