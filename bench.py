@@ -1164,9 +1164,12 @@ def run_ours(args):
 
     extras = {}
     sample4 = None
+    # the extras are single-GPU measurements: a run on several GPUs leaves them to the one-GPU
+    # run (rank 0 timing them would keep the other ranks waiting at the final barrier)
+    solo = rank == 0 and world == 1
     if rank == 0:
         del graphs, soak_graphs
-    if not args.no_encode and rank == 0:
+    if not args.no_encode and solo:
         try:
             extras["encode"] = encode_extra(dev, hbm_peak, bf16_peak)
             sample4 = extras["encode"].pop("_sample")
@@ -1175,7 +1178,7 @@ def run_ours(args):
     base_ms = 1000.0 * elapsed / args.steps
     for name, kw, skip in (("smooth", dict(smooth=True), args.no_smooth),
                            ("paged", dict(page_tokens=256), args.no_paged)):
-        if skip or rank != 0:
+        if skip or not solo:
             continue
         reps.clear()
         wss.clear()
@@ -1184,7 +1187,7 @@ def run_ours(args):
             extras[name] = variant_extra(wl, args, dev, R, base_ms, **kw)
         except Exception as exc:   # an extra never takes the main line down
             extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
-    if rank == 0 and not args.no_ragged:
+    if solo and not args.no_ragged:
         for key, kw in (("decode_only", dict(
                             name="llama3_8b_32k", R=12, calls=600,
                             label="llama3_8b_32k decode only (B 8, Hq 32 / Hkv 8, context 32768, "
@@ -1210,7 +1213,7 @@ def run_ours(args):
     for name, fn in (("pq_encode", lambda: pq_encode_extra(dev)),
                      ("pq_decode", lambda: pq_decode_extra(dev, hbm_peak)),
                      ("pq_decode_m8", lambda: pq_decode_extra(dev, hbm_peak, m=8))):
-        if args.no_encode or rank != 0:
+        if args.no_encode or not solo:
             continue
         try:
             extras[name] = fn()
